@@ -1,0 +1,310 @@
+"""The denoise step of uniform-state text diffusion, written out plainly (oracle).
+
+TEST INFRASTRUCTURE (see the package docstring).
+
+Sources (page title, section):
+  [VG]  "A Visual Guide to DiffusionGemma" (zh-CN translation, hubwiz.com):
+        3.2 uniform-state diffusion; 5.1 self-conditioning; 5.2 multi-canvas
+        sampling; 5.3 scheduler (step budget, logits temperature schedule,
+        adaptive stop); 5.4 entropy-bounded sampler (canvas initialisation,
+        token acceptance, token re-noising).
+  [DP]  "DiffusionGemma: from autoregressive to diffusion denoising" (blog,
+        vatt-ghern.pages.dev): the diffusion decode loop pseudocode
+        (canvas = random_tokens(256); for step: logits = model(canvas);
+        conf = confidence(logits); canvas = update(...)).
+  [WS]  local-deploy workshop (yomxxx.com): "scheduler" (temperature high early,
+        low late; stop when either stability or confidence holds; entropy below
+        0.005) and "entropy-constrained sampler" (sort by entropy ascending,
+        accept while the cumulative entropy stays within the threshold,
+        re-noise the rest); generate(..., temperature_schedule="cosine").
+  [EX]  "DiffusionGemma explained" (ai.google.dev, ja; zh-TW translation on
+        gemma.gh.miniasp.com): self-conditioning multiplies the probability
+        matrix by the token embedding table; 256-token canvases, block by block.
+
+Readings where the pages are silent or garbled (each also listed in the design doc):
+  * The acceptance formula is lost in extraction ([VG] 5.4 ends "based on the
+    following formula:"). Default rule (accept_rule 0): accept the sorted
+    prefix whose inclusive running entropy sum is <= tau ([WS]). Rule 1 reads
+    [VG]'s "sum so far minus the maximum entropy": in ascending order the
+    maximum so far is the current entry, so a position is accepted when the sum
+    of the entries before it is <= tau (always accepts at least one).
+  * Tokens are chosen by argmax (the most likely token per position, [VG] 3.2);
+    ties go to the lowest vocabulary index.
+  * Logits temperature: T_t = T_end + (T_start - T_end) * (1 + cos(pi t/(S-1)))/2,
+    t = 0..S-1 (the cosine schedule of [WS]; lower temperature at later steps,
+    [VG] 5.3); S = 1 gives T_start.
+  * Entropy in nats, H = -sum p log p, clamped at 0.
+  * Entropy sort ties: lower position first (stable).
+  * Adaptive stop (stop_rule 0): the canvas unchanged for N consecutive steps,
+    OR all entropies < stop_entropy, OR the step budget reached. stop_rule 1
+    compares the argmax predictions of consecutive steps instead.
+  * A finished block emits the final step's argmax at every position.
+  * Self-conditioning feeds sc = softmax(z) E of the tempered logits straight
+    into the next step's stand-in hidden state (the small FFNN of [VG] 5.1
+    needs trained weights and is left out).
+
+Precision: fp64 throughout. Decisions that turn floats into integers are taken
+in fp32, the precision the CUDA kernels take them in: argmax over fp32-rounded
+logits, the sort over fp32-rounded entropies, sequential fp32 prefix sums of
+the sorted entropies compared with fp32(tau), and H_fp32 < fp32(stop_entropy).
+For bf16 workloads the stand-in hidden state is rounded to bf16
+(round-to-nearest-even) before the dot products, as the kernels see it.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+from . import rng
+
+_VOCAB_CHUNK = 8192
+
+
+# ----------------------------------------------------------------------------
+# Scheduler: cosine logits temperature ([VG] 5.3, [WS] scheduler).
+# ----------------------------------------------------------------------------
+def temperature(t: int, S: int, T_start: float, T_end: float) -> float:
+    if S <= 1:
+        return float(T_start)
+    return T_end + (T_start - T_end) * 0.5 * (1.0 + math.cos(math.pi * t / (S - 1)))
+
+
+# ----------------------------------------------------------------------------
+# bf16 rounding (round to nearest, ties to even), done on fp64 values directly.
+# ----------------------------------------------------------------------------
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                     # x = m * 2**e, 0.5 <= |m| < 1
+    # bf16 keeps 8 significant bits; below 2**-126 the quantum is fixed.
+    e = np.maximum(e, -125)
+    q = np.ldexp(np.rint(np.ldexp(x, 8 - e)), e - 8)
+    return np.where(x == 0.0, x, q)
+
+
+# ----------------------------------------------------------------------------
+# Canvas initialisation ([VG] 5.4) and the stand-in backbone.
+# ----------------------------------------------------------------------------
+def init_block(w, block: int):
+    """Targets and initial canvas of one block: uniform tokens keyed on seed+block."""
+    pos = np.arange(w.C, dtype=np.uint64)
+    s = (w.seed + block) & ((1 << 64) - 1)
+    target = rng.tokens(s, 0, rng.TAG_TARGET, pos, w.V)
+    canvas = rng.tokens(s, 0, rng.TAG_INIT_CANVAS, pos, w.V)
+    return target, canvas
+
+
+def standin_hidden(w, E: np.ndarray, target, canvas, sc_prev, block: int, t: int):
+    """h_i = A E[target_i] + B E[canvas_i] + sc_prev_i + eps_i, eps ~ N(0, (noise_var_d/d) I).
+
+    Replaces the bidirectional denoiser, which needs trained weights. The
+    self-conditioning vector of the previous step enters additively ([VG] 5.1).
+    """
+    C, d = w.C, w.d
+    idx = (np.arange(C, dtype=np.uint64)[:, None] * np.uint64(d)
+           + np.arange(d, dtype=np.uint64)[None, :])
+    eps = rng.gaussian(w.seed, block, rng.TAG_NOISE + t, idx) * math.sqrt(w.noise_var_d / d)
+    Et = E[np.asarray(target)].astype(np.float64)
+    Ec = E[np.asarray(canvas)].astype(np.float64)
+    h = w.coef_target * Et + w.coef_canvas * Ec + np.asarray(sc_prev, np.float64) + eps
+    if w.dtype == "bf16":
+        h = bf16_round(h)
+    return h
+
+
+# ----------------------------------------------------------------------------
+# Logits -> probabilities, entropy, argmax, self-conditioning vector.
+# ----------------------------------------------------------------------------
+def logits(h: np.ndarray, E: np.ndarray, scale: float) -> np.ndarray:
+    """z[i, v] = scale * <h_i, E_v>, fp64, materialised as [rows, V]."""
+    h = np.asarray(h, dtype=np.float64)
+    V = E.shape[0]
+    z = np.empty((h.shape[0], V), dtype=np.float64)
+    for v0 in range(0, V, _VOCAB_CHUNK):
+        Ec = E[v0:v0 + _VOCAB_CHUNK].astype(np.float64)
+        z[:, v0:v0 + Ec.shape[0]] = scale * (h @ Ec.T)
+    return z
+
+
+@dataclasses.dataclass
+class Attention:
+    argmax: np.ndarray      # int64 [rows]; decided on fp32-rounded logits
+    H: np.ndarray           # fp64 [rows]; entropy in nats, >= 0
+    sc: np.ndarray          # fp64 [rows, d]; sum_v p_v E_v
+    zmax: np.ndarray        # fp64 [rows]; largest logit
+    margin: np.ndarray      # fp64 [rows]; gap between the two largest logits
+
+
+def vocab_attention(h: np.ndarray, E: np.ndarray, scale: float) -> Attention:
+    """Per position: softmax of the tempered logits, its entropy, argmax and p.E.
+
+    The probability of each vocabulary token is the softmax of the logits
+    divided by the temperature ([VG] 5.3 logits scheduler); confidence is the
+    entropy of that distribution ([VG] 5.3 adaptive stop, 5.4 acceptance); the
+    self-conditioning vector is the probability row times the embedding table
+    ([VG] 5.1, [EX] self-conditioning).
+    """
+    z = logits(h, E, scale)
+    rows = z.shape[0]
+    zmax = z.max(axis=1)
+    z32 = z.astype(np.float32)
+    argmax = np.argmax(z32, axis=1).astype(np.int64)        # first index of max
+    top2 = np.partition(z, -2, axis=1)[:, -2:] if z.shape[1] > 1 else np.stack([zmax, zmax], 1)
+    margin = np.abs(top2[:, 1] - top2[:, 0])
+    logZ = np.empty(rows)
+    H = np.empty(rows)
+    p = np.empty_like(z)
+    for i in range(rows):
+        shifted = z[i] - zmax[i]
+        e = np.exp(shifted)
+        Z = e.sum()
+        logZ[i] = math.log(Z)
+        p[i] = e / Z
+        logp = shifted - logZ[i]
+        H[i] = max(0.0, float(-(p[i] * logp).sum()))
+    d = E.shape[1]
+    sc = np.zeros((rows, d), dtype=np.float64)
+    for v0 in range(0, E.shape[0], _VOCAB_CHUNK):
+        Ec = E[v0:v0 + _VOCAB_CHUNK].astype(np.float64)
+        sc += p[:, v0:v0 + Ec.shape[0]] @ Ec
+    return Attention(argmax=argmax, H=H, sc=sc, zmax=zmax, margin=margin)
+
+
+# ----------------------------------------------------------------------------
+# Entropy-bounded sampler ([VG] 5.4, [WS] entropy-constrained sampler).
+# ----------------------------------------------------------------------------
+@dataclasses.dataclass
+class Acceptance:
+    order: np.ndarray       # positions sorted by (H_fp32, position)
+    accepted: np.ndarray    # bool [C]
+    k: int                  # number accepted
+    prefix: np.ndarray      # fp32 inclusive prefix sums in sorted order
+
+
+def entropy_bounded_accept(H32: np.ndarray, tau: float, rule: int) -> Acceptance:
+    """Sort positions from lowest to highest entropy and walk the list.
+
+    rule 0: accept while the running sum including this entry is <= tau.
+    rule 1: accept while the running sum minus the largest entropy seen so far
+            (the current entry, in ascending order) is <= tau.
+    Sums are sequential fp32 additions in sorted order, compared with fp32(tau).
+    """
+    H32 = np.asarray(H32, dtype=np.float32)
+    C = H32.shape[0]
+    order = np.argsort(H32, kind="stable")
+    tau32 = np.float32(tau)
+    prefix = np.zeros(C, dtype=np.float32)
+    run = np.float32(0.0)
+    accepted = np.zeros(C, dtype=bool)
+    k = 0
+    stopped = False
+    for j in range(C):
+        before = run
+        run = np.float32(run + H32[order[j]])
+        prefix[j] = run
+        ok = (run <= tau32) if rule == 0 else (before <= tau32)
+        if ok and not stopped:
+            accepted[order[j]] = True
+            k += 1
+        else:
+            stopped = True
+    return Acceptance(order=order, accepted=accepted, k=k, prefix=prefix)
+
+
+def renoise(w, accepted, argmax, block: int, t: int) -> np.ndarray:
+    """Accepted positions take the argmax; every rejected one a fresh uniform token."""
+    noise = rng.tokens(w.seed, block, t, np.arange(w.C, dtype=np.uint64), w.V)
+    return np.where(accepted, argmax, noise).astype(np.int64)
+
+
+# ----------------------------------------------------------------------------
+# One step and the block loop ([DP] decode loop; [VG] 5.2, 5.3).
+# ----------------------------------------------------------------------------
+@dataclasses.dataclass
+class State:
+    block: int
+    t: int
+    target: np.ndarray
+    canvas: np.ndarray
+    sc: np.ndarray
+    unchanged: int = 0
+    argmax_prev: np.ndarray | None = None
+    done: bool = False
+    steps_done: int = 0
+
+
+@dataclasses.dataclass
+class StepRecord:
+    t: int
+    temperature: float
+    h: np.ndarray
+    att: Attention
+    acc: Acceptance
+    canvas_in: np.ndarray
+    canvas_out: np.ndarray
+    noise: np.ndarray
+    unchanged: int
+    all_confident: bool
+    done: bool
+
+
+def begin_block(w, block: int) -> State:
+    target, canvas = init_block(w, block)
+    return State(block=block, t=0, target=target, canvas=canvas,
+                 sc=np.zeros((w.C, w.d), dtype=np.float64))
+
+
+def step(w, E: np.ndarray, st: State, h: np.ndarray | None = None) -> StepRecord:
+    """One denoise step from state st (mutated in place). h overrides the stand-in."""
+    t = st.t
+    T = temperature(t, w.max_steps, w.T_start, w.T_end)
+    if h is None:
+        h = standin_hidden(w, E, st.target, st.canvas, st.sc, st.block, t)
+    att = vocab_attention(h, E, w.logit_scale / T)
+    H32 = att.H.astype(np.float32)
+    acc = entropy_bounded_accept(H32, w.tau, w.accept_rule)
+    noise = rng.tokens(w.seed, st.block, t, np.arange(w.C, dtype=np.uint64), w.V)
+    canvas_out = np.where(acc.accepted, att.argmax, noise).astype(np.int64)
+    all_conf = bool(np.all(H32 < np.float32(w.stop_entropy)))
+    if w.stop_rule == 0:
+        same = bool(np.array_equal(canvas_out, st.canvas))
+    else:
+        same = st.argmax_prev is not None and bool(np.array_equal(att.argmax, st.argmax_prev))
+    unchanged = st.unchanged + 1 if same else 0
+    last = (t + 1 >= w.max_steps)
+    if w.fixed_steps:
+        done = last
+    else:
+        done = last or all_conf or unchanged >= w.stop_unchanged
+    rec = StepRecord(t=t, temperature=T, h=h, att=att, acc=acc, canvas_in=st.canvas.copy(),
+                     canvas_out=canvas_out, noise=noise, unchanged=unchanged,
+                     all_confident=all_conf, done=done)
+    st.canvas = canvas_out
+    st.sc = att.sc
+    st.unchanged = unchanged
+    st.argmax_prev = att.argmax
+    st.t = t + 1
+    st.done = done
+    st.steps_done = t + 1
+    return rec
+
+
+def denoise_block(w, E: np.ndarray, block: int):
+    """Run one canvas to its stop; returns (final argmax, steps, per-step records)."""
+    st = begin_block(w, block)
+    records = []
+    while not st.done:
+        records.append(step(w, E, st))
+    return records[-1].att.argmax.copy(), st.steps_done, records
+
+
+def generate(w, E: np.ndarray):
+    """Blocks 0..blocks-1 in sequence; each block's final argmax is emitted."""
+    out = np.zeros(w.blocks * w.C, dtype=np.int64)
+    steps = []
+    for b in range(w.blocks):
+        tokens, n, _ = denoise_block(w, E, b)
+        out[b * w.C:(b + 1) * w.C] = tokens
+        steps.append(n)
+    return out, steps
