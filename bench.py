@@ -1,0 +1,345 @@
+#!/usr/bin/env python
+"""Benchmark of the denoise step: steps/s and canvas tokens/s, roofline fraction.
+
+One bench "step" is one denoise step of the whole hot path (stand-in hidden
+state, vocabulary attention, entropy sort, acceptance, re-noise, stop test) on
+the headline canvas C=256, V=262144, d=2048 (bf16 E, fp32 accumulation), in
+the fixed-step timing mode (adaptive stop off; each block runs its S=32 steps
+and the next block starts). E (1.07 GB) is larger than L2 and is streamed from
+HBM every step, so no L2 flush is needed between steps.
+
+  value  device-timed throughput with inputs resident (CUDA events around K
+         steps on the context's stream, max over ranks).
+  e2e    the same metric through dg_denoise_step_h: every step copies that
+         step's hidden state from pinned host memory and reads the updated
+         canvas and loop state back to the host.
+  roofline  the vocabulary-attention kernels (the dominant kernel) against the
+         tensor roofline: 4*C*d*V flops per step over their event-timed duration.
+  cpu_baseline  the CPU oracle (fp64 numpy) on a bounded sample of rows.
+
+--impl reference runs the CPU oracle as the reference arm.
+Multi-GPU (torchrun): independent canvases per rank (replicas, seed = rank),
+no collective on the data path; value sums all ranks' steps over the slowest
+rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+METRIC = "denoise steps/s & canvas tok/s at C=256,V=262k,d=2048; % of step roofline"
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), tflops=float(p["bf16_tflops"]),
+                    tflops_sustained=float(p["bf16_tflops_sustained"]), src="measured")
+    except Exception:
+        return dict(hbm=6650.0, tflops=1590.0, tflops_sustained=1400.0, src="fallback")
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.index), "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_baseline(w, E32, rows: int, seed_steps: int = 1):
+    """The oracle, as it stands, on `rows` canvas rows of one step; scaled to steps/s."""
+    from oracle import method as M
+
+    st = M.begin_block(w, 0)
+    h = M.standin_hidden(w, E32, st.target, st.canvas, st.sc, 0, 0)
+    T = M.temperature(0, w.max_steps, w.T_start, w.T_end)
+    t0 = time.perf_counter()
+    for _ in range(seed_steps):
+        att = M.vocab_attention(h[:rows], E32, w.logit_scale / T)
+        M.entropy_bounded_accept(att.H.astype(np.float32), w.tau, w.accept_rule)
+    dt = (time.perf_counter() - t0) / seed_steps
+    step_s = dt * w.C / rows
+    threads = int(os.environ.get("OPENBLAS_NUM_THREADS", len(os.sched_getaffinity(0))))
+    return {"value": 1.0 / step_s, "unit": "steps/s", "cores": threads, "kind": "oracle",
+            "sample": f"{rows} of {w.C} canvas rows of one step (fp64 numpy, {dt:.1f} s), "
+                      f"scaled by {w.C}/{rows}",
+            "tok_per_s": w.C / step_s}
+
+
+def roofline_time(w, pk, sustained=True):
+    flops = 4.0 * w.C * w.d * w.V
+    t_c = flops / ((pk["tflops_sustained"] if sustained else pk["tflops"]) * 1e12)
+    t_m = 2.0 * w.V * w.d * 2 / (pk["hbm"] * 1e9)
+    return max(t_c, t_m), flops
+
+
+def run_reference(args, w):
+    """Reference arm: the CPU oracle on the host cores, same metric and config."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    E32 = synthetic.make_embedding_f32(w.V, w.d, w.e_seed)
+    if w.dtype == "bf16":
+        import torch
+        E32 = torch.from_numpy(E32).to(torch.bfloat16).float().numpy()
+    rows = max(1, min(w.C, args.ref_rows))
+    times = []
+    if args.warmup > 0:
+        cpu_baseline(w, E32, rows)
+    for _ in range(args.steps):
+        times.append(1.0 / cpu_baseline(w, E32, rows)["value"])
+    step_s = float(np.mean(times))
+    cb = cpu_baseline(w, E32, rows)
+    val = 1.0 / step_s
+    line = {"metric": METRIC, "value": val, "unit": "steps/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "tok_per_s": w.C * val,
+            "config": {"workload": w.name, "C": w.C, "V": w.V, "d": w.d, "mode": "fixed_steps"},
+            "cpu_baseline": {"value": val, "unit": "steps/s", "cores": cb["cores"],
+                             "kind": "oracle", "sample": cb["sample"]},
+            "e2e": {"value": val, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=synthetic.HEADLINE.name, choices=sorted(synthetic.WORKLOADS))
+    ap.add_argument("--kernels", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--cpu-rows", type=int, default=32, help="rows of the oracle baseline sample")
+    ap.add_argument("--ref-rows", type=int, default=16, help="rows per reference-arm step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    w = synthetic.WORKLOADS[args.workload].replace(fixed_steps=1)
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import uniform_state_text_b200 as dg
+    from uniform_state_text_b200 import build as dgbuild
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        if world == 1 and args.gpus > 1:
+            print(f"--gpus {args.gpus} needs torchrun with {args.gpus} processes", file=sys.stderr)
+            return 2
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    if rank == 0:
+        dgbuild.build()
+    if dist:
+        dist.barrier()
+    dg.lib()
+    w = w.replace(seed=rank)
+    impl = {"auto": dg.DG_IMPL_AUTO, "simt": dg.DG_IMPL_SIMT, "tc": dg.DG_IMPL_TC}[args.kernels]
+
+    E_cpu = synthetic.make_embedding(w)
+    E = E_cpu.to(f"cuda:{local}")
+    den = dg.Denoiser(w, E, impl=impl)
+    stream = den.stream
+    S = w.max_steps
+
+    state = {"t": 0, "block": 0}
+
+    def one_step():
+        if state["t"] == S:
+            state["block"] += 1
+            den.begin_block(state["block"])
+            state["t"] = 0
+        den.step()
+        state["t"] += 1
+
+    for _ in range(args.warmup):
+        one_step()
+    stream.synchronize()
+
+    # --- device-timed region -------------------------------------------------
+    clocks = Clocks(local)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    dg.dg_profile(den.ctx, True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        one_step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    attn_ms, attn_steps, launches = dg.dg_profile_read(den.ctx)
+    dg.dg_profile(den.ctx, False)
+    clk = clocks.stop()
+    st = den.state()
+    if st["status"] != 0:
+        raise RuntimeError(f"device status {st['status']}")
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    total_steps = args.steps * world
+    value = total_steps / (ms / 1e3)
+    ms_per_step = ms / args.steps
+
+    # --- end to end through host buffers ----------------------------------------
+    e2e = None
+    if not args.no_e2e:
+        den.begin_block(0)
+        den.step()
+        h_host = den.read(dg.DG_HIDDEN).cpu().pin_memory()
+        canvas_host = torch.empty(w.C, dtype=torch.int32).pin_memory()
+        den.begin_block(0)
+        n_e2e = max(8, args.steps // 2)
+        for _ in range(3):
+            den.step_h(h_host, canvas_host=canvas_host, want_done=True)
+        den.begin_block(0)
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        done_steps = 0
+        for i in range(n_e2e):
+            if done_steps == S:
+                den.begin_block(0)
+                done_steps = 0
+            den.step_h(h_host, canvas_host=canvas_host, want_done=True)
+            done_steps += 1
+        torch.cuda.synchronize()
+        el = time.perf_counter() - t0
+        if dist:
+            t = torch.tensor([el], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            el = float(t.item())
+        e2e = {"value": n_e2e * world / el, "unit": "steps/s",
+               "h2d_bytes_per_step": int(h_host.numel() * h_host.element_size()),
+               "d2h_bytes_per_step": int(w.C * 4 + 64),
+               "tok_per_s": w.C * n_e2e * world / el,
+               "path": "dg_denoise_step_h, hidden state from pinned host memory"}
+
+    pk = measured_peaks()
+    t_roof, flops = roofline_time(w, pk, sustained=True)
+    attn_s = (attn_ms / 1e3) / max(attn_steps, 1)
+    achieved_tflops = flops / attn_s / 1e12
+    peak = pk["tflops_sustained"]
+    roof = {"bound": "tensor", "achieved": achieved_tflops, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved_tflops / peak, "traffic": None,
+            "kernel": "vocabulary attention (" + ("tcgen05" if den.impl == dg.DG_IMPL_TC else "CUDA-core") + ")",
+            "kernel_ms_per_step": attn_s * 1e3,
+            "peak_src": f"{pk['src']} bf16 sustained (kernel timed inside a long step loop)",
+            "algorithmic_flops_per_step": flops,
+            "step_roofline_pct": 100.0 * t_roof / (ms_per_step / 1e3),
+            "step_roofline_us": t_roof * 1e6}
+
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        E32 = synthetic.embedding_as_f32(E_cpu)
+        cb = cpu_baseline(w, E32, max(1, min(w.C, args.cpu_rows)))
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16" if w.dtype == "bf16" else "f32",
+                "data": "synthetic (seeded E ~ N(0, I/d), stand-in hidden state)",
+                "tok_per_s": w.C * value,
+                "roofline_pct": roof["step_roofline_pct"],
+                "config": {"workload": w.name, "C": w.C, "V": w.V, "d": w.d,
+                           "max_steps": S, "mode": "fixed_steps (adaptive stop off)",
+                           "kernels": "tc" if den.impl == dg.DG_IMPL_TC else "simt",
+                           "l2": "no flush: E (%.2f GB) exceeds the 126 MB L2 and is streamed every step" % (w.e_bytes / 1e9),
+                           "parallelism": f"replicas x{world}"},
+                "roofline": roof, "e2e": e2e, "gpu_launches": launches,
+                "clocks": clk, "cpu_baseline": cb}
+        print(json.dumps(line), flush=True)
+    den.close()
+    if dist:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

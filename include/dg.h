@@ -1,0 +1,206 @@
+/*
+ * dg.h -- C ABI of the uniform-state text-diffusion denoise step (B200, sm_100a).
+ *
+ * The calls follow the decode loop of uniform-state text diffusion: start a
+ * canvas of uniformly random tokens, run denoise steps (score every position
+ * against the vocabulary, accept the most confident predictions within an
+ * entropy budget, re-noise the rest, test for an adaptive stop), then emit the
+ * canvas and start the next block.
+ *
+ * Sources (page title, section):
+ *   [VG] "A Visual Guide to DiffusionGemma": 3.2 uniform-state diffusion;
+ *        5.1 self-conditioning; 5.2 multi-canvas sampling (block diffusion);
+ *        5.3 scheduler (step budget, logits temperature, adaptive stop);
+ *        5.4 entropy-bounded sampler (canvas initialisation, token acceptance,
+ *        token re-noising).
+ *   [DP] "DiffusionGemma: from autoregressive to diffusion denoising"
+ *        (vatt-ghern.pages.dev), the diffusion decode-loop pseudocode.
+ *   [WS] local-deploy workshop (yomxxx.com): scheduler and
+ *        entropy-constrained sampler; generate(diffusion_steps, canvas_size,
+ *        temperature_schedule="cosine").
+ *   [EX] "DiffusionGemma explained" (ai.google.dev): self-conditioning as the
+ *        probability matrix times the token embedding table.
+ *
+ * Conventions for every call:
+ *   - Device pointers are CUDA global-memory addresses on the device that is
+ *     current when dg_init runs; host pointers are ordinary process memory.
+ *   - The caller owns E, the workspace, every output buffer and the stream.
+ *     The library allocates no device memory and frees nothing it was given.
+ *   - All calls are asynchronous on the context's stream unless they return a
+ *     value through a host pointer (then they synchronise that stream).
+ *   - Return value: DG_OK (0) or a negative DG_E* code; dg_last_error() gives
+ *     a message. A context is not thread-safe; use one per stream.
+ *   - Layouts are row-major. E is [V][d] (d contiguous). Hidden states and
+ *     self-conditioning vectors are [C][d].
+ */
+#ifndef DG_H
+#define DG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+#define DG_OK            0
+#define DG_EINVAL       -1   /* bad argument or unsupported configuration     */
+#define DG_ENOMEM       -2   /* workspace smaller than dg_workspace_bytes()   */
+#define DG_ECUDA        -3   /* a CUDA runtime/driver call failed             */
+#define DG_ETIMEOUT     -4   /* a bounded device wait ran out (kernel status) */
+#define DG_EUNSUPPORTED -5   /* shape not supported by the requested kernels  */
+#define DG_ESTATE       -6   /* device status word reported an error          */
+
+/* Element types of E and of the hidden state h. */
+#define DG_F32   0
+#define DG_BF16  1
+
+/* Adaptive-stability rule ([VG] 5.3 "stability"). */
+#define DG_STOP_CANVAS  0    /* canvas unchanged for stop_unchanged steps     */
+#define DG_STOP_ARGMAX  1    /* argmax predictions unchanged for that many    */
+
+/* Token-acceptance rule ([VG] 5.4 "token acceptance"). */
+#define DG_ACCEPT_CUMSUM    0  /* inclusive running entropy sum <= tau         */
+#define DG_ACCEPT_MINUS_MAX 1  /* running sum minus the largest so far <= tau  */
+
+/* Kernel family for the vocabulary-attention step. */
+#define DG_IMPL_AUTO  0      /* tensor-core path when the shape allows it     */
+#define DG_IMPL_SIMT  1      /* CUDA-core kernels (any shape, f32 or bf16)    */
+#define DG_IMPL_TC    2      /* tcgen05/TMEM kernels (bf16; see dg_init)      */
+
+typedef struct dg_config {
+  int32_t  C;               /* canvas positions, 1..1024 ([VG] 5.2: 256)       */
+  int32_t  V;               /* vocabulary size, power of two, >= 64            */
+  int32_t  d;               /* hidden width, multiple of 8                     */
+  int32_t  dtype;           /* DG_F32 or DG_BF16 (E and h)                     */
+  int32_t  max_steps;       /* S, step budget per block ([VG] 5.3), >= 1       */
+  float    T_start, T_end;  /* cosine logits temperature, T_t over t=0..S-1    */
+  float    tau;             /* entropy bound of the sampler, nats ([VG] 5.4)   */
+  float    logit_scale;     /* L in z = L h.E^T / T_t                          */
+  float    coef_target;     /* stand-in A: h = A E[target] + ...               */
+  float    coef_canvas;     /* stand-in B: ... + B E[canvas] + sc + noise      */
+  float    noise_var_d;     /* stand-in noise variance times d                 */
+  float    stop_entropy;    /* confidence stop: every H < this ([VG] 5.3)      */
+  int32_t  stop_unchanged;  /* stability stop after this many unchanged steps  */
+  int32_t  stop_rule;       /* DG_STOP_*                                       */
+  int32_t  accept_rule;     /* DG_ACCEPT_*                                     */
+  int32_t  fixed_steps;     /* 1: ignore adaptive stop, run exactly S steps    */
+  int32_t  impl;            /* DG_IMPL_*                                       */
+  int32_t  reserved0;
+  uint64_t seed;            /* keys every draw: key(seed, block, step, index)  */
+} dg_config;
+
+typedef struct dg_ctx dg_ctx;
+
+/* What dg_read / dg_write transfer (device buffers of the stated type/size). */
+#define DG_CANVAS    0   /* int32 [C]   current canvas                          */
+#define DG_ARGMAX    1   /* int32 [C]   argmax of the last step                 */
+#define DG_ENTROPY   2   /* float [C]   entropy (nats) of the last step         */
+#define DG_ACCEPT    3   /* int32 [C]   1 = accepted in the last step           */
+#define DG_SC        4   /* float [C*d] self-conditioning vector p.E            */
+#define DG_HIDDEN    5   /* dtype [C*d] hidden state h of the last step         */
+#define DG_TARGET    6   /* int32 [C]   stand-in targets of the current block   */
+#define DG_ORDER     7   /* int32 [C]   positions sorted by (entropy, position) */
+#define DG_PREFIX    8   /* float [C]   fp32 running entropy sums, sorted order */
+#define DG_STATE     9   /* int32 [16]  see DG_ST_* below                       */
+#define DG_MREF     10   /* float [C]   tensor-core path: per-row logit reference */
+
+/* Indices into the DG_STATE array. */
+#define DG_ST_T          0  /* next step index within the block               */
+#define DG_ST_BLOCK      1  /* current block index                             */
+#define DG_ST_UNCHANGED  2  /* consecutive unchanged steps                     */
+#define DG_ST_DONE       3  /* 1 once the block has stopped                    */
+#define DG_ST_STEPS      4  /* steps run in this block                         */
+#define DG_ST_K          5  /* positions accepted in the last step             */
+#define DG_ST_STATUS     6  /* 0, or a DG_E* code raised on the device         */
+#define DG_ST_HASPREV    7  /* 1 once an argmax of a previous step exists      */
+#define DG_ST_REDO       8  /* rows recomputed because the reference was low   */
+
+/*
+ * Bytes of device workspace the configuration needs (0 if it is invalid).
+ * The workspace holds the canvas state, the hidden state, the
+ * self-conditioning vector and the kernels' per-tile partial results.
+ */
+size_t dg_workspace_bytes(const dg_config* cfg);
+
+/*
+ * Create a context.
+ *   cfg       configuration (copied).
+ *   E         device, [V][d] of cfg->dtype, the tied vocabulary embedding;
+ *             read-only and caller-owned; must outlive the context.
+ *   workspace device, >= dg_workspace_bytes(cfg) bytes, 256-byte aligned,
+ *             caller-owned; its contents are managed by the library.
+ *   stream    a cudaStream_t (NULL = legacy default stream).
+ *   out       receives the context (NULL on failure).
+ * Errors: DG_EINVAL (bad config or pointer), DG_ENOMEM (workspace too small),
+ * DG_EUNSUPPORTED (cfg->impl = DG_IMPL_TC with a shape the tensor-core path
+ * does not cover: it needs dtype bf16, C = 128 or 256, d a multiple of 256,
+ * V a multiple of 256), DG_ECUDA. The context starts at block 0 (as if
+ * dg_begin_block(ctx, 0) had run).
+ */
+int dg_init(const dg_config* cfg, const void* E, void* workspace, size_t ws_bytes,
+            void* stream, dg_ctx** out);
+
+/*
+ * Start block `block` ([VG] 5.4 canvas initialisation; 5.2 multi-canvas):
+ * targets and the initial canvas are uniform tokens keyed on (seed + block),
+ * sc := 0, unchanged := 0, t := 0.
+ */
+int dg_begin_block(dg_ctx* ctx, int32_t block);
+
+/*
+ * One denoise step ([DP] loop body; [VG] 5.1, 5.3, 5.4): stand-in hidden
+ * state, tempered logits against E, per-position argmax, entropy and
+ * self-conditioning vector, entropy sort, acceptance, re-noise, stop test.
+ * No-op once the block is done. done_host: NULL = stay asynchronous;
+ * otherwise the stream is synchronised and *done_host receives the done flag.
+ */
+int dg_denoise_step(dg_ctx* ctx, int32_t* done_host);
+
+/*
+ * The same step with the hidden state supplied by the caller instead of the
+ * stand-in backbone: h_src holds [C][d] of cfg->dtype, in host memory when
+ * h_on_host != 0 (pinned memory keeps the copy asynchronous) or device memory
+ * otherwise. canvas_host (nullable) receives the updated canvas, int32 [C];
+ * done_host (nullable) the done flag. A non-NULL host output synchronises.
+ */
+int dg_denoise_step_h(dg_ctx* ctx, const void* h_src, int32_t h_on_host,
+                      int32_t* canvas_host, int32_t* done_host);
+
+/*
+ * A whole block ([VG] 5.2): dg_begin_block, then denoise steps until the
+ * adaptive stop or the step budget (one CUDA graph launch with a device-side
+ * loop), then the final step's argmax is written to out_dev (device, int32 [C]).
+ * steps_host (nullable) receives the number of steps run (synchronises).
+ */
+int dg_denoise_block(dg_ctx* ctx, int32_t block, int32_t* out_dev, int32_t* steps_host);
+
+/* Copy one piece of state to / from a caller device buffer (see DG_CANVAS...). */
+int dg_read(dg_ctx* ctx, int32_t what, void* dst_dev);
+int dg_write(dg_ctx* ctx, int32_t what, const void* src_dev);
+
+/*
+ * Per-step timing of the vocabulary-attention kernels, for measurement:
+ * enable != 0 records CUDA events around them on the context's stream in every
+ * dg_denoise_step / dg_denoise_step_h and resets the counters;
+ * dg_profile_read synchronises and returns the total milliseconds and number
+ * of steps timed, and the number of kernels the library launched, since the
+ * last dg_profile call (any output pointer may be NULL).
+ */
+int dg_profile(dg_ctx* ctx, int32_t enable);
+int dg_profile_read(dg_ctx* ctx, double* ms_total, int32_t* steps, int64_t* launches);
+
+/* Which kernel family the context runs (DG_IMPL_SIMT or DG_IMPL_TC). */
+int dg_impl(const dg_ctx* ctx);
+
+/* Release the context (host memory and graph objects only). */
+int dg_free(dg_ctx* ctx);
+
+/* Message for the last error on ctx (or of the last failed dg_init if NULL). */
+const char* dg_last_error(const dg_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DG_H */

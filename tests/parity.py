@@ -1,0 +1,106 @@
+"""Comparison of the CUDA path's step outputs with the oracle (test helper).
+
+Tolerances (from the method's stated bar): token ids, accept masks, noise
+tokens and step counts bit-exact, except positions that sit on a near-tie --
+top-2 logit margin < 1e-3, entropy within 1e-3 of a rank neighbour, or a
+running entropy sum within 1e-3 of tau at the acceptance boundary -- which are
+counted and must stay <= 0.1% of all compared positions; entropies within 1e-3
+absolute; self-conditioning vectors within 2e-2 relative L2 per position.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+
+from oracle import method as M
+from oracle import rng
+
+H_ATOL = 1e-3
+SC_RTOL = 2e-2
+TIE = 1e-3
+TIE_BUDGET = 1e-3
+
+
+@dataclasses.dataclass
+class Tally:
+    positions: int = 0
+    tie_mismatch: int = 0
+    worst_H: float = 0.0
+    worst_sc: float = 0.0
+    steps: int = 0
+
+    def check_budget(self):
+        assert self.tie_mismatch <= TIE_BUDGET * max(self.positions, 1), (
+            f"{self.tie_mismatch} near-tie mismatches over {self.positions} positions")
+
+
+def near_tie_flags(att, acc, tau: float, rule: int) -> np.ndarray:
+    """Per position: argmax margin, entropy-rank gap or acceptance boundary within TIE."""
+    C = att.H.shape[0]
+    H = att.H.astype(np.float64)
+    flags = att.margin < TIE
+    order = acc.order
+    Hs = H[order]
+    gap = np.full(C, np.inf)
+    if C > 1:
+        dif = np.abs(np.diff(Hs))
+        gap[order[:-1]] = np.minimum(gap[order[:-1]], dif)
+        gap[order[1:]] = np.minimum(gap[order[1:]], dif)
+    flags |= gap < TIE
+    pref = np.cumsum(Hs)
+    ref = pref if rule == 0 else np.concatenate([[0.0], pref[:-1]])
+    boundary = np.abs(ref - tau) < TIE
+    flags[order[boundary]] = True
+    return flags
+
+
+def sc_rel_err(sc_gpu: np.ndarray, sc_ref: np.ndarray) -> np.ndarray:
+    num = np.linalg.norm(sc_gpu - sc_ref, axis=1)
+    den = np.maximum(np.linalg.norm(sc_ref, axis=1), 1e-30)
+    return num / den
+
+
+def compare_attention(tally: Tally, att, H_gpu, argmax_gpu, sc_gpu, flags, rows=None):
+    """H, argmax and sc of the GPU against the oracle's attention for the same h."""
+    H_gpu = np.asarray(H_gpu, np.float64)
+    err = np.abs(H_gpu - att.H)
+    tally.worst_H = max(tally.worst_H, float(err.max()))
+    assert err.max() <= H_ATOL, f"entropy error {err.max()} at row {int(err.argmax())}"
+    mism = np.flatnonzero(np.asarray(argmax_gpu) != att.argmax)
+    bad = [int(i) for i in mism if not flags[i]]
+    assert not bad, f"argmax mismatch off a near-tie at rows {bad[:8]} (margins {att.margin[bad[:8]]})"
+    tally.tie_mismatch += len(mism)
+    r = sc_rel_err(np.asarray(sc_gpu, np.float64), att.sc)
+    tally.worst_sc = max(tally.worst_sc, float(r.max()))
+    assert r.max() <= SC_RTOL, f"sc relative error {r.max()} at row {int(r.argmax())}"
+
+
+def check_sampler_exact(w, block, t, H_gpu, argmax_gpu, canvas_in, out):
+    """The sampler given the GPU's own entropies and argmax must agree bit for bit."""
+    H32 = np.asarray(H_gpu, np.float32)
+    acc = M.entropy_bounded_accept(H32, w.tau, w.accept_rule)
+    noise = rng.tokens(w.seed, block, t, np.arange(w.C, dtype=np.uint64), w.V)
+    want_canvas = np.where(acc.accepted, np.asarray(argmax_gpu), noise)
+    assert np.array_equal(out["order"], acc.order), "sort order differs"
+    assert np.array_equal(out["prefix"], acc.prefix), "prefix sums differ"
+    assert np.array_equal(out["accept"].astype(bool), acc.accepted), "accept mask differs"
+    assert np.array_equal(out["canvas"], want_canvas), "canvas update differs"
+    assert out["state"]["k"] == acc.k
+    return acc
+
+
+def h_agreement(w, h_gpu, h_orc) -> float:
+    """Fraction of hidden-state elements that differ (bf16: by more than nothing)."""
+    h_gpu = np.asarray(h_gpu, np.float64)
+    if w.dtype == "bf16":
+        diff = h_gpu != h_orc
+        if diff.any():
+            # any difference must be one bf16 ulp (fp32 vs fp64 evaluation before rounding)
+            e = np.frexp(np.abs(h_orc))[1]
+            two_ulp = np.ldexp(1.0, e - 7)
+            assert np.all(np.abs(h_gpu - h_orc)[diff] <= two_ulp[diff])
+        return float(diff.mean())
+    rel = np.abs(h_gpu - h_orc) / np.maximum(np.abs(h_orc), 1e-3)
+    assert rel.max() < 1e-5
+    return 0.0

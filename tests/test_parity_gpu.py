@@ -1,0 +1,288 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, on a B200.
+
+Teacher-forced step parity: before each GPU step the canvas, sc and step index
+are read back; the oracle recomputes the stand-in hidden state from them
+(compared element by element), then the vocabulary attention from the GPU's
+own hidden state (entropy, argmax, sc) and the sampler twice: from the GPU's
+entropies (must agree bit for bit) and from its own (near-tie budget).
+Trajectory parity runs whole blocks through the CUDA-graph loop.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synthetic
+import uniform_state_text_b200 as dg
+from oracle import method as M
+from parity import (Tally, check_sampler_exact, compare_attention, h_agreement,
+                    near_tie_flags)
+
+pytestmark = pytest.mark.gpu
+
+IMPLS = [dg.DG_IMPL_SIMT, dg.DG_IMPL_TC]
+_E_CACHE = {}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from uniform_state_text_b200 import build
+    build.build()
+    dg.lib()
+
+
+def embedding(w):
+    key = (w.V, w.d, w.dtype, w.e_seed)
+    if key not in _E_CACHE:
+        _E_CACHE.clear()
+        E = synthetic.make_embedding(w)
+        _E_CACHE[key] = (E.cuda(), synthetic.embedding_as_f32(E))
+    return _E_CACHE[key]
+
+
+def supported(w, impl):
+    return dg.dg_workspace_bytes(dg.make_config(w, impl)) > 0
+
+
+def make(w, impl):
+    if not supported(w, impl):
+        pytest.skip(f"impl {impl} does not cover {w.name}")
+    Eg, E32 = embedding(w)
+    den = dg.Denoiser(w, Eg, impl=impl)
+    assert den.impl == impl
+    return den, E32
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy() if t.dtype in (torch.bfloat16, torch.float32) \
+        else t.detach().cpu().numpy()
+
+
+def step_and_compare(den, w, E32, tally: Tally, prev_amax=None):
+    st0 = den.state()
+    if st0["done"]:
+        return False
+    canvas_in = _np(den.read(dg.DG_CANVAS)).astype(np.int64)
+    sc_in = _np(den.read(dg.DG_SC)).astype(np.float64)
+    target = _np(den.read(dg.DG_TARGET)).astype(np.int64)
+    den.step()
+    h = _np(den.read(dg.DG_HIDDEN)).astype(np.float64)
+    H = _np(den.read(dg.DG_ENTROPY))
+    amax = _np(den.read(dg.DG_ARGMAX)).astype(np.int64)
+    sc = _np(den.read(dg.DG_SC)).astype(np.float64)
+    out = dict(accept=_np(den.read(dg.DG_ACCEPT)), canvas=_np(den.read(dg.DG_CANVAS)),
+               order=_np(den.read(dg.DG_ORDER)), prefix=_np(den.read(dg.DG_PREFIX)))
+    st1 = den.state()
+    out["state"] = st1
+    assert st1["status"] == 0
+    t, b = st0["t"], st0["block"]
+    h_orc = M.standin_hidden(w, E32, target, canvas_in, sc_in, b, t)
+    assert h_agreement(w, h, h_orc) < 2e-3
+    T = M.temperature(t, w.max_steps, w.T_start, w.T_end)
+    att = M.vocab_attention(h, E32, w.logit_scale / T)
+    acc_orc = M.entropy_bounded_accept(att.H.astype(np.float32), w.tau, w.accept_rule)
+    flags = near_tie_flags(att, acc_orc, w.tau, w.accept_rule)
+    compare_attention(tally, att, H, amax, sc, flags)
+    check_sampler_exact(w, b, t, H, amax, canvas_in, out)
+    mism = np.flatnonzero(acc_orc.accepted != out["accept"].astype(bool))
+    bad = [int(i) for i in mism if not flags[i]]
+    assert not bad, f"accept mismatch off a near-tie at {bad[:8]}"
+    tally.tie_mismatch += len(mism)
+    tally.positions += w.C
+    tally.steps += 1
+    # adaptive stop from the same outputs
+    same = np.array_equal(out["canvas"], canvas_in) if w.stop_rule == 0 else \
+        (st0["has_prev"] == 1 and np.array_equal(amax, prev_amax))
+    unchanged = st0["unchanged"] + 1 if same else 0
+    conf = bool(np.all(H.astype(np.float32) < np.float32(w.stop_entropy)))
+    last = t + 1 >= w.max_steps
+    done = last if w.fixed_steps else (last or conf or unchanged >= w.stop_unchanged)
+    assert st1["unchanged"] == unchanged and st1["done"] == int(done) and st1["t"] == t + 1
+    return True
+
+
+def run_teacher_forced(den, w, E32, max_steps=None):
+    tally = Tally()
+    n = 0
+    while max_steps is None or n < max_steps:
+        if den.state()["done"]:
+            break
+        pre = _np(den.read(dg.DG_ARGMAX)).astype(np.int64) if den.state()["has_prev"] else None
+        if not step_and_compare(den, w, E32, tally, pre):
+            break
+        n += 1
+    tally.check_budget()
+    return tally
+
+
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("impl", IMPLS)
+def test_tiny_block_trajectory(impl):
+    w = synthetic.TINY
+    den, E32 = make(w, impl)
+    out, steps = den.block(0)
+    want, want_steps, _ = M.denoise_block(w, E32, 0)
+    assert steps == want_steps
+    assert np.array_equal(_np(out), want)
+    den.close()
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("variant", ["fixed", "stress", "minus_max", "argmax_stop", "tau0"])
+def test_tiny_teacher_forced(impl, variant):
+    base = synthetic.TINY.replace(coef_target=0.5, coef_canvas=0.5, logit_scale=1.5, tau=2.0)
+    w = {"fixed": base.replace(fixed_steps=1),
+         "stress": base,
+         "minus_max": base.replace(accept_rule=1, fixed_steps=1),
+         "argmax_stop": base.replace(stop_rule=1),
+         "tau0": base.replace(tau=0.0, max_steps=4)}[variant]
+    den, E32 = make(w, impl)
+    tally = run_teacher_forced(den, w, E32)
+    assert tally.steps >= 1
+    den.close()
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("name", ["canvas_c256_v32768_d1024_bf16",
+                                  "stress_partial_c256_v32768_d1024_bf16",
+                                  "stress_ties_c256_v32768_d1024_bf16"])
+def test_small_teacher_forced(impl, name):
+    w = synthetic.WORKLOADS[name]
+    if name.startswith("stress_ties"):
+        w = w.replace(max_steps=4, fixed_steps=1)
+    den, E32 = make(w, impl)
+    tally = run_teacher_forced(den, w, E32)
+    print(name, impl, tally)
+    den.close()
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_small_fixed_steps_sampled(impl):
+    """The timing mode (adaptive stop off) over all 16 steps, compared at every step."""
+    w = synthetic.SMALL.replace(fixed_steps=1)
+    den, E32 = make(w, impl)
+    tally = run_teacher_forced(den, w, E32)
+    assert tally.steps == w.max_steps
+    den.close()
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("name", ["canvas_c256_v262144_d2048_bf16",
+                                  "canvas_c128_v262144_d2816_bf16"])
+def test_full_size_two_fixed_steps(impl, name):
+    """Full-size shapes in the timed configuration: two steps, every row compared."""
+    w = synthetic.WORKLOADS[name].replace(fixed_steps=1)
+    den, E32 = make(w, impl)
+    tally = run_teacher_forced(den, w, E32, max_steps=2)
+    assert tally.steps == 2
+    den.close()
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_graph_loop_equals_stepwise(impl):
+    w = synthetic.STRESS_PARTIAL
+    den, E32 = make(w, impl)
+    out, steps = den.block(0)
+    g_out = _np(out)
+    den.begin_block(0)
+    n = 0
+    while not den.step(want_done=True):
+        n += 1
+    n += 1
+    assert n == steps
+    assert np.array_equal(_np(den.read(dg.DG_ARGMAX)), g_out)
+    den.close()
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_block_diffusion_small(impl):
+    """Four sequential canvases; each block is independent and emits its final argmax."""
+    w = synthetic.SMALL.replace(blocks=4, max_steps=24)
+    den, E32 = make(w, impl)
+    want, want_steps = M.generate(w, E32)
+    got = []
+    for b in range(w.blocks):
+        out, steps = den.block(b)
+        assert steps == want_steps[b]
+        got.append(_np(out))
+    assert np.array_equal(np.concatenate(got), want)
+    den.close()
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_block_diffusion_full_size(impl):
+    w = synthetic.BLOCKS
+    den, E32 = make(w, impl)
+    buf = torch.empty(w.blocks * w.C, dtype=torch.int32, device="cuda")
+    steps = []
+    for b in range(w.blocks):
+        _, s = den.block(b, out=buf[b * w.C:(b + 1) * w.C])
+        steps.append(s)
+    want, want_steps = M.generate(w, E32)
+    assert steps == want_steps
+    assert np.array_equal(_np(buf), want)
+    den.close()
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_external_hidden_state_from_host(impl):
+    """dg_denoise_step_h with the hidden state in pinned host memory equals the stand-in step."""
+    w = synthetic.SMALL
+    den, E32 = make(w, impl)
+    den.step()
+    h = den.read(dg.DG_HIDDEN)
+    ref = {k: _np(den.read(k)) for k in (dg.DG_ENTROPY, dg.DG_ARGMAX, dg.DG_CANVAS, dg.DG_SC)}
+    den.begin_block(0)
+    host_h = h.cpu().pin_memory()
+    canvas_host = torch.empty(w.C, dtype=torch.int32).pin_memory()
+    done = den.step_h(host_h, canvas_host=canvas_host, want_done=True)
+    assert done in (0, 1)
+    assert np.array_equal(canvas_host.numpy(), ref[dg.DG_CANVAS])
+    assert np.array_equal(_np(den.read(dg.DG_ARGMAX)), ref[dg.DG_ARGMAX])
+    np.testing.assert_array_equal(_np(den.read(dg.DG_ENTROPY)), ref[dg.DG_ENTROPY])
+    den.close()
+
+
+@pytest.mark.parametrize("shape", [(37, 128, 24), (1, 64, 8), (200, 1024, 72), (256, 512, 64)])
+def test_ragged_shapes_simt(shape):
+    C, V, d = shape
+    w = synthetic.TINY.replace(C=C, V=V, d=d, tau=0.5 * C * 0.693, coef_target=1.0,
+                               coef_canvas=0.5, logit_scale=2.0, max_steps=5, fixed_steps=1)
+    den, E32 = make(w, dg.DG_IMPL_SIMT)
+    run_teacher_forced(den, w, E32)
+    den.close()
+
+
+def test_workspace_too_small_is_rejected():
+    w = synthetic.TINY
+    Eg, _ = embedding(w)
+    cfg = dg.make_config(w)
+    n = dg.dg_workspace_bytes(cfg)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    with pytest.raises(dg.DgError) as e:
+        dg.dg_init(cfg, Eg.data_ptr(), ws.data_ptr(), n - 256, torch.cuda.Stream().cuda_stream)
+    assert e.value.code == dg.DG_ENOMEM
+
+
+def test_device_status_word_is_reported():
+    """A status raised on the device (injected from the host) fails the next synchronising call."""
+    w = synthetic.TINY
+    den, _ = make(w, dg.DG_IMPL_SIMT)
+    st = den.read(dg.DG_STATE)
+    st[dg.DG_ST_STATUS] = dg.DG_ETIMEOUT
+    den.write(dg.DG_STATE, st)
+    with pytest.raises(dg.DgError) as e:
+        den.step(want_done=True)
+    assert e.value.code == dg.DG_ETIMEOUT
+    den.close()
+
+
+def test_block_loop_needs_a_stream():
+    w = synthetic.TINY
+    Eg, _ = embedding(w)
+    den = dg.Denoiser(w, Eg, stream=torch.cuda.default_stream())
+    with pytest.raises(dg.DgError) as e:
+        den.block(0)
+    assert e.value.code == dg.DG_EINVAL
+    den.close()

@@ -1,0 +1,276 @@
+"""Python binding of the denoise-step C ABI declared in include/dg.h.
+
+Argument marshalling only: every step of the path runs in libdg.so's CUDA
+kernels. The functions keep the C names (dg_init, dg_denoise_step, ...), take
+raw pointers as Python ints, and raise DgError on a non-zero return code.
+`Denoiser` is a convenience owner of the device buffers (allocated with torch,
+which here only provides memory and streams).
+
+The library must be built first (uniform_state_text_b200.build.build(), nvcc
+for sm_100a); without it every call raises, there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libdg.so")
+
+DG_OK, DG_EINVAL, DG_ENOMEM, DG_ECUDA, DG_ETIMEOUT, DG_EUNSUPPORTED, DG_ESTATE = 0, -1, -2, -3, -4, -5, -6
+DG_F32, DG_BF16 = 0, 1
+DG_STOP_CANVAS, DG_STOP_ARGMAX = 0, 1
+DG_ACCEPT_CUMSUM, DG_ACCEPT_MINUS_MAX = 0, 1
+DG_IMPL_AUTO, DG_IMPL_SIMT, DG_IMPL_TC = 0, 1, 2
+(DG_CANVAS, DG_ARGMAX, DG_ENTROPY, DG_ACCEPT, DG_SC, DG_HIDDEN, DG_TARGET, DG_ORDER, DG_PREFIX,
+ DG_STATE, DG_MREF) = range(11)
+DG_ST_T, DG_ST_BLOCK, DG_ST_UNCHANGED, DG_ST_DONE, DG_ST_STEPS, DG_ST_K, DG_ST_STATUS, \
+    DG_ST_HASPREV, DG_ST_REDO = range(9)
+
+
+class dg_config(ctypes.Structure):
+    _fields_ = [
+        ("C", ctypes.c_int32), ("V", ctypes.c_int32), ("d", ctypes.c_int32),
+        ("dtype", ctypes.c_int32), ("max_steps", ctypes.c_int32),
+        ("T_start", ctypes.c_float), ("T_end", ctypes.c_float), ("tau", ctypes.c_float),
+        ("logit_scale", ctypes.c_float), ("coef_target", ctypes.c_float),
+        ("coef_canvas", ctypes.c_float), ("noise_var_d", ctypes.c_float),
+        ("stop_entropy", ctypes.c_float), ("stop_unchanged", ctypes.c_int32),
+        ("stop_rule", ctypes.c_int32), ("accept_rule", ctypes.c_int32),
+        ("fixed_steps", ctypes.c_int32), ("impl", ctypes.c_int32), ("reserved0", ctypes.c_int32),
+        ("seed", ctypes.c_uint64),
+    ]
+
+
+class DgError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"dg error {code}: {msg}")
+        self.code = code
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+
+
+def lib():
+    """Load libdg.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "uniform_state_text_b200.build.build() (nvcc, sm_100a)")
+    L = ctypes.CDLL(LIB_PATH)
+    cfgp = ctypes.POINTER(dg_config)
+    L.dg_workspace_bytes.argtypes = [cfgp]
+    L.dg_workspace_bytes.restype = ctypes.c_size_t
+    L.dg_init.argtypes = [cfgp, _P, _P, ctypes.c_size_t, _P, ctypes.POINTER(_P)]
+    L.dg_begin_block.argtypes = [_P, _I]
+    L.dg_denoise_step.argtypes = [_P, ctypes.POINTER(_I)]
+    L.dg_denoise_step_h.argtypes = [_P, _P, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]
+    L.dg_denoise_block.argtypes = [_P, _I, _P, ctypes.POINTER(_I)]
+    L.dg_read.argtypes = [_P, _I, _P]
+    L.dg_write.argtypes = [_P, _I, _P]
+    L.dg_profile.argtypes = [_P, _I]
+    L.dg_profile_read.argtypes = [_P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I),
+                                  ctypes.POINTER(ctypes.c_int64)]
+    L.dg_impl.argtypes = [_P]
+    L.dg_free.argtypes = [_P]
+    L.dg_last_error.argtypes = [_P]
+    L.dg_last_error.restype = ctypes.c_char_p
+    for name in ("dg_init", "dg_begin_block", "dg_denoise_step", "dg_denoise_step_h",
+                 "dg_denoise_block", "dg_read", "dg_write", "dg_profile", "dg_profile_read",
+                 "dg_impl", "dg_free"):
+        getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _check(rc: int, ctx) -> int:
+    if rc < 0:
+        raise DgError(rc, dg_last_error(ctx))
+    return rc
+
+
+def make_config(w, impl: int = DG_IMPL_AUTO) -> dg_config:
+    """dg_config from a synthetic.Workload-like object (same field names)."""
+    return dg_config(C=w.C, V=w.V, d=w.d, dtype=DG_BF16 if w.dtype == "bf16" else DG_F32,
+                     max_steps=w.max_steps, T_start=w.T_start, T_end=w.T_end, tau=w.tau,
+                     logit_scale=w.logit_scale, coef_target=w.coef_target,
+                     coef_canvas=w.coef_canvas, noise_var_d=w.noise_var_d,
+                     stop_entropy=w.stop_entropy, stop_unchanged=w.stop_unchanged,
+                     stop_rule=w.stop_rule, accept_rule=w.accept_rule,
+                     fixed_steps=w.fixed_steps, impl=impl, reserved0=0, seed=w.seed)
+
+
+# ----------------------------------------------------------------------------
+# The C ABI, same names.
+# ----------------------------------------------------------------------------
+def dg_workspace_bytes(cfg: dg_config) -> int:
+    return int(lib().dg_workspace_bytes(ctypes.byref(cfg)))
+
+
+def dg_init(cfg: dg_config, E_ptr: int, ws_ptr: int, ws_bytes: int, stream_ptr: int):
+    out = _P()
+    rc = lib().dg_init(ctypes.byref(cfg), _P(E_ptr), _P(ws_ptr), ws_bytes, _P(stream_ptr),
+                       ctypes.byref(out))
+    _check(rc, None)
+    return out
+
+
+def dg_begin_block(ctx, block: int) -> None:
+    _check(lib().dg_begin_block(ctx, block), ctx)
+
+
+def dg_denoise_step(ctx, want_done: bool = False):
+    if not want_done:
+        _check(lib().dg_denoise_step(ctx, None), ctx)
+        return None
+    done = _I()
+    _check(lib().dg_denoise_step(ctx, ctypes.byref(done)), ctx)
+    return int(done.value)
+
+
+def dg_denoise_step_h(ctx, h_ptr: int, on_host: bool, canvas_host_ptr: int | None = None,
+                      want_done: bool = False):
+    done = _I()
+    cptr = ctypes.cast(canvas_host_ptr, ctypes.POINTER(_I)) if canvas_host_ptr else None
+    _check(lib().dg_denoise_step_h(ctx, _P(h_ptr), 1 if on_host else 0, cptr,
+                                   ctypes.byref(done) if want_done else None), ctx)
+    return int(done.value) if want_done else None
+
+
+def dg_denoise_block(ctx, block: int, out_ptr: int, want_steps: bool = True):
+    steps = _I()
+    _check(lib().dg_denoise_block(ctx, block, _P(out_ptr),
+                                  ctypes.byref(steps) if want_steps else None), ctx)
+    return int(steps.value) if want_steps else None
+
+
+def dg_read(ctx, what: int, dst_ptr: int) -> None:
+    _check(lib().dg_read(ctx, what, _P(dst_ptr)), ctx)
+
+
+def dg_write(ctx, what: int, src_ptr: int) -> None:
+    _check(lib().dg_write(ctx, what, _P(src_ptr)), ctx)
+
+
+def dg_profile(ctx, enable: bool) -> None:
+    _check(lib().dg_profile(ctx, 1 if enable else 0), ctx)
+
+
+def dg_profile_read(ctx):
+    """(milliseconds in the vocabulary-attention kernels, steps timed, kernels launched)."""
+    ms = ctypes.c_double()
+    n = _I()
+    nl = ctypes.c_int64()
+    _check(lib().dg_profile_read(ctx, ctypes.byref(ms), ctypes.byref(n), ctypes.byref(nl)), ctx)
+    return float(ms.value), int(n.value), int(nl.value)
+
+
+def dg_impl(ctx) -> int:
+    return _check(lib().dg_impl(ctx), ctx)
+
+
+def dg_free(ctx) -> None:
+    lib().dg_free(ctx)
+
+
+def dg_last_error(ctx) -> str:
+    msg = lib().dg_last_error(ctx)
+    return msg.decode() if msg else ""
+
+
+# ----------------------------------------------------------------------------
+# Convenience owner of device buffers.
+# ----------------------------------------------------------------------------
+class Denoiser:
+    """One context with its workspace; E must be a CUDA tensor [V, d] of the workload dtype."""
+
+    def __init__(self, w, E, stream=None, impl: int = DG_IMPL_AUTO):
+        import torch
+
+        self.w = w
+        self.cfg = make_config(w, impl)
+        if not E.is_cuda or not E.is_contiguous():
+            raise ValueError("E must be a contiguous CUDA tensor")
+        self.E = E
+        self.device = E.device
+        self.stream = stream if stream is not None else torch.cuda.Stream(device=self.device)
+        nbytes = dg_workspace_bytes(self.cfg)
+        if nbytes == 0:
+            raise DgError(DG_EINVAL, "invalid configuration: " + dg_last_error(None))
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        self.ctx = dg_init(self.cfg, E.data_ptr(), self.ws.data_ptr(), nbytes,
+                           self.stream.cuda_stream)
+        self.impl = dg_impl(self.ctx)
+        self._dtype = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    # state -----------------------------------------------------------------
+    def _shape(self, what):
+        import torch
+
+        C, d = self.w.C, self.w.d
+        return {DG_CANVAS: ((C,), torch.int32), DG_ARGMAX: ((C,), torch.int32),
+                DG_ENTROPY: ((C,), torch.float32), DG_ACCEPT: ((C,), torch.int32),
+                DG_SC: ((C, d), torch.float32), DG_HIDDEN: ((C, d), self._dtype),
+                DG_TARGET: ((C,), torch.int32), DG_ORDER: ((C,), torch.int32),
+                DG_PREFIX: ((C,), torch.float32), DG_STATE: ((16,), torch.int32),
+                DG_MREF: ((C,), torch.float32)}[what]
+
+    def read(self, what):
+        import torch
+
+        shape, dt = self._shape(what)
+        out = torch.empty(shape, dtype=dt, device=self.device)
+        dg_read(self.ctx, what, out.data_ptr())
+        self.stream.synchronize()
+        return out
+
+    def write(self, what, tensor):
+        shape, dt = self._shape(what)
+        t = tensor.to(device=self.device, dtype=dt).contiguous()
+        if tuple(t.shape) != shape:
+            raise ValueError(f"expected shape {shape}")
+        dg_write(self.ctx, what, t.data_ptr())
+        self.stream.synchronize()
+
+    def state(self) -> dict:
+        s = self.read(DG_STATE).cpu().tolist()
+        return dict(t=s[DG_ST_T], block=s[DG_ST_BLOCK], unchanged=s[DG_ST_UNCHANGED],
+                    done=s[DG_ST_DONE], steps=s[DG_ST_STEPS], k=s[DG_ST_K],
+                    status=s[DG_ST_STATUS], has_prev=s[DG_ST_HASPREV], redo=s[DG_ST_REDO])
+
+    # loop ------------------------------------------------------------------
+    def begin_block(self, block: int) -> None:
+        dg_begin_block(self.ctx, block)
+
+    def step(self, want_done: bool = False):
+        return dg_denoise_step(self.ctx, want_done)
+
+    def step_h(self, h, canvas_host=None, want_done: bool = False):
+        on_host = not h.is_cuda
+        return dg_denoise_step_h(self.ctx, h.data_ptr(), on_host,
+                                 canvas_host.data_ptr() if canvas_host is not None else None,
+                                 want_done)
+
+    def block(self, block: int, out=None):
+        import torch
+
+        if out is None:
+            out = torch.empty(self.w.C, dtype=torch.int32, device=self.device)
+        steps = dg_denoise_block(self.ctx, block, out.data_ptr())
+        return out, steps
+
+    def close(self) -> None:
+        if getattr(self, "ctx", None) is not None:
+            self.stream.synchronize()
+            dg_free(self.ctx)
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

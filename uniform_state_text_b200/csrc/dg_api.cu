@@ -1,0 +1,499 @@
+// C ABI of the denoise step (declared in include/dg.h): configuration checks,
+// workspace layout, step orchestration and the CUDA-graph block loop.
+//
+// The loop follows the decode pseudocode of "DiffusionGemma: from
+// autoregressive to diffusion denoising" (canvas = random tokens; for each
+// step: logits = model(canvas); confidence; update) with the scheduler and
+// sampler of "A Visual Guide to DiffusionGemma" (5.3, 5.4) and block-by-block
+// canvases (5.2).
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "../../include/dg.h"
+#include "dg_common.cuh"
+#include "dg_kernels.h"
+#include "dg_tc.h"
+
+using namespace dg;
+
+namespace {
+
+thread_local char g_init_err[512] = "";
+
+constexpr size_t kAlign = 256;
+constexpr float kRedoGap = 64.0f;   // largest logit minus reference that P may carry
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Layout {
+  int impl = 0;
+  int ntiles = 0;      // vocabulary tiles carrying per-row statistics
+  int nsplit = 0;      // CUDA-core path: vocabulary splits of sc
+  size_t state = 0, scale = 0, target = 0, canvas = 0, argmax = 0, argmax_prev = 0, accept = 0,
+         order = 0, prefix = 0, H = 0, mref = 0, rowstat = 0, redo_rows = 0, h = 0, sc = 0,
+         tstats = 0, zbuf = 0, partial = 0, O = 0, tc = 0, total = 0;
+  size_t tc_bytes = 0;
+};
+
+bool is_pow2(long long v) { return v > 0 && (v & (v - 1)) == 0; }
+
+int check_config(const dg_config* c, char* why, size_t n) {
+  if (!c) { snprintf(why, n, "config is NULL"); return DG_EINVAL; }
+  if (c->C < 1 || c->C > 1024) { snprintf(why, n, "C=%d outside 1..1024", c->C); return DG_EINVAL; }
+  if (!is_pow2(c->V) || c->V < 64 || c->V > (1 << 30)) {
+    snprintf(why, n, "V=%d must be a power of two in 64..2^30", c->V); return DG_EINVAL;
+  }
+  if (c->d < 8 || c->d > 65536 || c->d % 8) {
+    snprintf(why, n, "d=%d must be a multiple of 8 in 8..65536", c->d); return DG_EINVAL;
+  }
+  if (c->dtype != DG_F32 && c->dtype != DG_BF16) { snprintf(why, n, "bad dtype"); return DG_EINVAL; }
+  if (c->max_steps < 1 || c->max_steps > (1 << 20)) { snprintf(why, n, "bad max_steps"); return DG_EINVAL; }
+  if (!(c->T_start > 0.f) || !(c->T_end > 0.f) || !std::isfinite(c->T_start) ||
+      !std::isfinite(c->T_end)) { snprintf(why, n, "temperatures must be finite and > 0"); return DG_EINVAL; }
+  if (!(c->tau >= 0.f) || !std::isfinite(c->tau)) { snprintf(why, n, "tau must be finite, >= 0"); return DG_EINVAL; }
+  if (!std::isfinite(c->logit_scale) || !std::isfinite(c->coef_target) ||
+      !std::isfinite(c->coef_canvas) || !(c->noise_var_d >= 0.f) ||
+      !std::isfinite(c->noise_var_d) || !std::isfinite(c->stop_entropy)) {
+    snprintf(why, n, "non-finite coefficient"); return DG_EINVAL;
+  }
+  if (c->stop_unchanged < 1) { snprintf(why, n, "stop_unchanged must be >= 1"); return DG_EINVAL; }
+  if (c->stop_rule != DG_STOP_CANVAS && c->stop_rule != DG_STOP_ARGMAX) { snprintf(why, n, "bad stop_rule"); return DG_EINVAL; }
+  if (c->accept_rule != DG_ACCEPT_CUMSUM && c->accept_rule != DG_ACCEPT_MINUS_MAX) { snprintf(why, n, "bad accept_rule"); return DG_EINVAL; }
+  if (c->impl < DG_IMPL_AUTO || c->impl > DG_IMPL_TC) { snprintf(why, n, "bad impl"); return DG_EINVAL; }
+  return DG_OK;
+}
+
+int resolve_impl(const dg_config* c, char* why, size_t n) {
+  const bool tc_ok = c->dtype == DG_BF16 && tc_supported(c->C, c->V, c->d);
+  if (c->impl == DG_IMPL_TC) {
+    if (!tc_ok) {
+      snprintf(why, n, "tensor-core path needs bf16, C in {128, 256}, d %% 256 == 0, V %% 256 == 0");
+      return -1;
+    }
+    return DG_IMPL_TC;
+  }
+  if (c->impl == DG_IMPL_SIMT) return DG_IMPL_SIMT;
+  return tc_ok ? DG_IMPL_TC : DG_IMPL_SIMT;
+}
+
+int make_layout(const dg_config* c, Layout* L, char* why, size_t n) {
+  int rc = check_config(c, why, n);
+  if (rc) return rc;
+  const int impl = resolve_impl(c, why, n);
+  if (impl < 0) return DG_EUNSUPPORTED;
+  const size_t C = (size_t)c->C, V = (size_t)c->V, d = (size_t)c->d;
+  const size_t esz = c->dtype == DG_F32 ? 4 : 2;
+  L->impl = impl;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes); return o; };
+  L->state = take(sizeof(DevState));
+  L->scale = take(sizeof(float) * (size_t)c->max_steps);
+  L->target = take(4 * C);
+  L->canvas = take(4 * C);
+  L->argmax = take(4 * C);
+  L->argmax_prev = take(4 * C);
+  L->accept = take(4 * C);
+  L->order = take(4 * C);
+  L->prefix = take(4 * C);
+  L->H = take(4 * C);
+  L->mref = take(4 * C);
+  L->rowstat = take(sizeof(RowStat) * C);
+  L->redo_rows = take(4 * C);
+  L->h = take(esz * C * d);
+  L->sc = take(4 * C * d);
+  if (impl == DG_IMPL_SIMT) {
+    L->ntiles = (int)(V / 64);
+    const size_t rt = (C + 63) / 64, dt = (d + 63) / 64;
+    size_t ns = 1;
+    while (ns * rt * dt < 1184 && ns * 2 <= V / 32) ns *= 2;
+    L->nsplit = (int)ns;
+    L->tstats = take(sizeof(TileStat) * C * L->ntiles);
+    L->zbuf = take(4 * C * V);
+    L->partial = take(4 * ns * C * d);
+  } else {
+    L->ntiles = tc_stat_tiles(c->C, c->V, c->d);
+    L->tstats = take(sizeof(TileStat) * C * L->ntiles);
+    L->O = take(4 * C * d);
+    L->tc_bytes = tc_workspace_bytes(c->C, c->V, c->d);
+    L->tc = take(L->tc_bytes);
+  }
+  L->total = off;
+  return DG_OK;
+}
+
+}  // namespace
+
+struct dg_ctx {
+  dg_config cfg;
+  Layout L;
+  const void* E = nullptr;
+  char* ws = nullptr;
+  cudaStream_t stream = nullptr;
+  int device = 0;
+  // pointers into the workspace
+  DevState* st = nullptr;
+  float* scale_tab = nullptr;
+  int32_t *target = nullptr, *canvas = nullptr, *argmax = nullptr, *argmax_prev = nullptr,
+          *accept = nullptr, *order = nullptr, *redo_rows = nullptr;
+  float *prefix = nullptr, *H = nullptr, *mref = nullptr, *sc = nullptr, *zbuf = nullptr,
+        *partial = nullptr, *O = nullptr;
+  RowStat* rowstat = nullptr;
+  TileStat* tstats = nullptr;
+  void* h = nullptr;
+  void* tc = nullptr;
+  TcPlan tc_plan;
+  // block-loop graph
+  bool graph_ready = false;
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t graph_exec = nullptr;
+  cudaGraphConditionalHandle cond = 0;
+  // profiling
+  bool prof = false;
+  std::vector<cudaEvent_t> ev;
+  size_t ev_used = 0;
+  long long launches = 0;   // kernels launched since the last dg_profile call
+  char err[512] = "";
+};
+
+namespace {
+
+int fail(dg_ctx* ctx, int code, const char* fmt, ...) {
+  char* buf = ctx ? ctx->err : g_init_err;
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, 512, fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+#define DG_CK(call)                                                                   \
+  do {                                                                                \
+    cudaError_t e_ = (call);                                                          \
+    if (e_ != cudaSuccess)                                                            \
+      return fail(ctx, DG_ECUDA, "%s failed: %s", #call, cudaGetErrorString(e_));    \
+  } while (0)
+
+template <typename T> T* at(dg_ctx* c, size_t off) { return reinterpret_cast<T*>(c->ws + off); }
+
+int launch_step(dg_ctx* ctx, bool standin, bool use_cond) {
+  const dg_config& c = ctx->cfg;
+  cudaStream_t s = ctx->stream;
+  const float sigma = (float)std::sqrt((double)c.noise_var_d / (double)c.d);
+  const bool tc = ctx->L.impl == DG_IMPL_TC;
+  DG_CK(launch_prologue(s, c.dtype, ctx->st, ctx->E, ctx->target, ctx->canvas, ctx->sc, ctx->h,
+                        c.C, c.V, c.d, c.seed, c.coef_target, c.coef_canvas, sigma, standin ? 1 : 0,
+                        ctx->scale_tab, c.max_steps, ctx->argmax_prev, tc ? ctx->mref : nullptr));
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  if (ctx->prof && !use_cond) {
+    if (ctx->ev_used + 2 > ctx->ev.size()) {
+      for (int j = 0; j < 64; ++j) {
+        cudaEvent_t e;
+        DG_CK(cudaEventCreate(&e));
+        ctx->ev.push_back(e);
+      }
+    }
+    e0 = ctx->ev[ctx->ev_used++];
+    e1 = ctx->ev[ctx->ev_used++];
+    DG_CK(cudaEventRecord(e0, s));
+  }
+  ctx->launches += 2 + (tc ? 2 + tc_launches(ctx->tc_plan) : 4);
+  if (tc) {
+    DG_CK(launch_tc_attention(s, ctx->tc_plan, ctx->st, ctx->h, ctx->E, ctx->mref, ctx->scale_tab,
+                              ctx->tstats, ctx->O, ctx->tc));
+    DG_CK(launch_merge(s, ctx->st, ctx->tstats, ctx->L.ntiles, ctx->rowstat, ctx->H, ctx->argmax,
+                       c.C, ctx->O, ctx->mref, ctx->sc, c.d, ctx->redo_rows, kRedoGap));
+    DG_CK(launch_tc_redo(s, ctx->tc_plan, ctx->st, ctx->h, ctx->E, ctx->scale_tab, ctx->rowstat,
+                         ctx->redo_rows, ctx->sc));
+  } else {
+    DG_CK(launch_simt_attention(s, c.dtype, ctx->st, ctx->h, ctx->E, ctx->zbuf, ctx->tstats,
+                                ctx->rowstat, ctx->partial, ctx->H, ctx->argmax, ctx->sc, c.C,
+                                c.V, c.d, ctx->L.nsplit, ctx->scale_tab, c.max_steps));
+  }
+  if (e1) DG_CK(cudaEventRecord(e1, s));
+  DG_CK(launch_sampler(s, ctx->st, ctx->H, ctx->argmax, ctx->canvas, ctx->argmax_prev,
+                       ctx->accept, ctx->order, ctx->prefix, c.C, c.V, c.seed, c.tau,
+                       c.stop_entropy, c.stop_unchanged, c.stop_rule, c.accept_rule,
+                       c.fixed_steps, c.max_steps, ctx->cond, use_cond ? 1 : 0));
+  return DG_OK;
+}
+
+int read_state(dg_ctx* ctx, DevState* hs) {
+  DG_CK(cudaMemcpyAsync(hs, ctx->st, sizeof(DevState), cudaMemcpyDeviceToHost, ctx->stream));
+  DG_CK(cudaStreamSynchronize(ctx->stream));
+  if (hs->status != 0)
+    return fail(ctx, hs->status == DG_ETIMEOUT ? DG_ETIMEOUT : DG_ESTATE,
+                "device status word reports %d", hs->status);
+  return DG_OK;
+}
+
+int build_graph(dg_ctx* ctx) {
+  if (ctx->stream == nullptr)
+    return fail(ctx, DG_EINVAL, "dg_denoise_block needs a non-default stream (graph capture)");
+  DG_CK(cudaGraphCreate(&ctx->graph, 0));
+  DG_CK(cudaGraphConditionalHandleCreate(&ctx->cond, ctx->graph, 1, cudaGraphCondAssignDefault));
+  cudaGraphNodeParams p = {};
+  p.type = cudaGraphNodeTypeConditional;
+  p.conditional.handle = ctx->cond;
+  p.conditional.type = cudaGraphCondTypeWhile;
+  p.conditional.size = 1;
+  cudaGraphNode_t node;
+  DG_CK(cudaGraphAddNode(&node, ctx->graph, nullptr, 0, &p));
+  cudaGraph_t body = p.conditional.phGraph_out[0];
+  DG_CK(cudaStreamBeginCaptureToGraph(ctx->stream, body, nullptr, nullptr, 0,
+                                      cudaStreamCaptureModeThreadLocal));
+  int rc = launch_step(ctx, true, true);
+  cudaGraph_t captured = nullptr;
+  cudaError_t e = cudaStreamEndCapture(ctx->stream, &captured);
+  if (rc) return rc;
+  if (e != cudaSuccess) return fail(ctx, DG_ECUDA, "capture failed: %s", cudaGetErrorString(e));
+  DG_CK(cudaGraphInstantiate(&ctx->graph_exec, ctx->graph, 0));
+  ctx->graph_ready = true;
+  return DG_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dg_workspace_bytes(const dg_config* cfg) {
+  Layout L;
+  char why[256];
+  if (make_layout(cfg, &L, why, sizeof(why)) != DG_OK) return 0;
+  return L.total;
+}
+
+int dg_init(const dg_config* cfg, const void* E, void* workspace, size_t ws_bytes, void* stream,
+            dg_ctx** out) {
+  if (out) *out = nullptr;
+  if (!out) return fail(nullptr, DG_EINVAL, "out is NULL");
+  Layout L;
+  char why[256] = "";
+  int rc = make_layout(cfg, &L, why, sizeof(why));
+  if (rc) return fail(nullptr, rc, "%s", why);
+  if (!E || !workspace) return fail(nullptr, DG_EINVAL, "E and workspace must be device pointers");
+  if (((uintptr_t)workspace) % kAlign) return fail(nullptr, DG_EINVAL, "workspace must be 256-byte aligned");
+  if (ws_bytes < L.total)
+    return fail(nullptr, DG_ENOMEM, "workspace has %zu bytes, needs %zu", ws_bytes, L.total);
+  cudaPointerAttributes pa;
+  if (cudaPointerGetAttributes(&pa, E) != cudaSuccess || pa.type != cudaMemoryTypeDevice) {
+    cudaGetLastError();
+    return fail(nullptr, DG_EINVAL, "E is not a device pointer");
+  }
+  if (cudaPointerGetAttributes(&pa, workspace) != cudaSuccess || pa.type != cudaMemoryTypeDevice) {
+    cudaGetLastError();
+    return fail(nullptr, DG_EINVAL, "workspace is not a device pointer");
+  }
+  dg_ctx* ctx = new dg_ctx();
+  ctx->cfg = *cfg;
+  ctx->L = L;
+  ctx->E = E;
+  ctx->ws = static_cast<char*>(workspace);
+  ctx->stream = static_cast<cudaStream_t>(stream);
+  cudaGetDevice(&ctx->device);
+  ctx->st = at<DevState>(ctx, L.state);
+  ctx->scale_tab = at<float>(ctx, L.scale);
+  ctx->target = at<int32_t>(ctx, L.target);
+  ctx->canvas = at<int32_t>(ctx, L.canvas);
+  ctx->argmax = at<int32_t>(ctx, L.argmax);
+  ctx->argmax_prev = at<int32_t>(ctx, L.argmax_prev);
+  ctx->accept = at<int32_t>(ctx, L.accept);
+  ctx->order = at<int32_t>(ctx, L.order);
+  ctx->prefix = at<float>(ctx, L.prefix);
+  ctx->H = at<float>(ctx, L.H);
+  ctx->mref = at<float>(ctx, L.mref);
+  ctx->rowstat = at<RowStat>(ctx, L.rowstat);
+  ctx->redo_rows = at<int32_t>(ctx, L.redo_rows);
+  ctx->h = at<void>(ctx, L.h);
+  ctx->sc = at<float>(ctx, L.sc);
+  ctx->tstats = at<TileStat>(ctx, L.tstats);
+  if (L.impl == DG_IMPL_SIMT) {
+    ctx->zbuf = at<float>(ctx, L.zbuf);
+    ctx->partial = at<float>(ctx, L.partial);
+  } else {
+    ctx->O = at<float>(ctx, L.O);
+    ctx->tc = at<void>(ctx, L.tc);
+    rc = tc_plan_init(&ctx->tc_plan, cfg->C, cfg->V, cfg->d, E, ctx->h, ctx->O, ctx->tstats,
+                      ctx->tc, ctx->err, sizeof(ctx->err));
+    if (rc) {
+      snprintf(g_init_err, sizeof(g_init_err), "%s", ctx->err);
+      delete ctx;
+      return rc;
+    }
+  }
+  // Logit scale per step: L / T_t with the cosine temperature schedule.
+  std::vector<float> tab(cfg->max_steps);
+  const int S = cfg->max_steps;
+  for (int t = 0; t < S; ++t) {
+    const double T = S <= 1 ? (double)cfg->T_start
+                            : (double)cfg->T_end + ((double)cfg->T_start - (double)cfg->T_end) *
+                                  0.5 * (1.0 + std::cos(M_PI * (double)t / (double)(S - 1)));
+    tab[t] = (float)((double)cfg->logit_scale / T);
+  }
+  cudaError_t e = cudaMemcpyAsync(ctx->scale_tab, tab.data(), sizeof(float) * S,
+                                  cudaMemcpyHostToDevice, ctx->stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->stream);
+  if (e != cudaSuccess) {
+    fail(nullptr, DG_ECUDA, "scale table upload: %s", cudaGetErrorString(e));
+    delete ctx;
+    return DG_ECUDA;
+  }
+  rc = dg_begin_block(ctx, 0);
+  if (rc) {
+    snprintf(g_init_err, sizeof(g_init_err), "%s", ctx->err);
+    delete ctx;
+    return rc;
+  }
+  *out = ctx;
+  return DG_OK;
+}
+
+int dg_begin_block(dg_ctx* ctx, int32_t block) {
+  if (!ctx) return fail(nullptr, DG_EINVAL, "ctx is NULL");
+  if (block < 0) return fail(ctx, DG_EINVAL, "block must be >= 0");
+  const dg_config& c = ctx->cfg;
+  DG_CK(launch_begin_block(ctx->stream, ctx->st, ctx->target, ctx->canvas, ctx->sc, c.C, c.d, c.V,
+                           c.seed, block));
+  ctx->launches += 1;
+  return DG_OK;
+}
+
+int dg_denoise_step(dg_ctx* ctx, int32_t* done_host) {
+  if (!ctx) return fail(nullptr, DG_EINVAL, "ctx is NULL");
+  int rc = launch_step(ctx, true, false);
+  if (rc) return rc;
+  if (done_host) {
+    DevState hs;
+    rc = read_state(ctx, &hs);
+    if (rc) return rc;
+    *done_host = hs.done;
+  }
+  return DG_OK;
+}
+
+int dg_denoise_step_h(dg_ctx* ctx, const void* h_src, int32_t h_on_host, int32_t* canvas_host,
+                      int32_t* done_host) {
+  if (!ctx) return fail(nullptr, DG_EINVAL, "ctx is NULL");
+  if (!h_src) return fail(ctx, DG_EINVAL, "h_src is NULL");
+  const dg_config& c = ctx->cfg;
+  const size_t bytes = (size_t)c.C * c.d * (c.dtype == DG_F32 ? 4 : 2);
+  DG_CK(cudaMemcpyAsync(ctx->h, h_src, bytes,
+                        h_on_host ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice,
+                        ctx->stream));
+  int rc = launch_step(ctx, false, false);
+  if (rc) return rc;
+  if (canvas_host)
+    DG_CK(cudaMemcpyAsync(canvas_host, ctx->canvas, sizeof(int32_t) * c.C, cudaMemcpyDeviceToHost,
+                          ctx->stream));
+  if (canvas_host || done_host) {
+    DevState hs;
+    rc = read_state(ctx, &hs);
+    if (rc) return rc;
+    if (done_host) *done_host = hs.done;
+  }
+  return DG_OK;
+}
+
+int dg_denoise_block(dg_ctx* ctx, int32_t block, int32_t* out_dev, int32_t* steps_host) {
+  if (!ctx) return fail(nullptr, DG_EINVAL, "ctx is NULL");
+  if (!out_dev) return fail(ctx, DG_EINVAL, "out_dev is NULL");
+  int rc = dg_begin_block(ctx, block);
+  if (rc) return rc;
+  if (!ctx->graph_ready && (rc = build_graph(ctx))) return rc;
+  DG_CK(cudaGraphLaunch(ctx->graph_exec, ctx->stream));
+  DG_CK(cudaMemcpyAsync(out_dev, ctx->argmax, sizeof(int32_t) * ctx->cfg.C,
+                        cudaMemcpyDeviceToDevice, ctx->stream));
+  if (steps_host) {
+    DevState hs;
+    rc = read_state(ctx, &hs);
+    if (rc) return rc;
+    *steps_host = hs.steps;
+  }
+  return DG_OK;
+}
+
+int dg_read(dg_ctx* ctx, int32_t what, void* dst) {
+  if (!ctx) return fail(nullptr, DG_EINVAL, "ctx is NULL");
+  if (!dst) return fail(ctx, DG_EINVAL, "dst is NULL");
+  const dg_config& c = ctx->cfg;
+  const size_t C = c.C, Cd = (size_t)c.C * c.d;
+  const void* src = nullptr;
+  size_t bytes = 0;
+  switch (what) {
+    case DG_CANVAS: src = ctx->canvas; bytes = 4 * C; break;
+    case DG_ARGMAX: src = ctx->argmax; bytes = 4 * C; break;
+    case DG_ENTROPY: src = ctx->H; bytes = 4 * C; break;
+    case DG_ACCEPT: src = ctx->accept; bytes = 4 * C; break;
+    case DG_SC: src = ctx->sc; bytes = 4 * Cd; break;
+    case DG_HIDDEN: src = ctx->h; bytes = Cd * (c.dtype == DG_F32 ? 4 : 2); break;
+    case DG_TARGET: src = ctx->target; bytes = 4 * C; break;
+    case DG_ORDER: src = ctx->order; bytes = 4 * C; break;
+    case DG_PREFIX: src = ctx->prefix; bytes = 4 * C; break;
+    case DG_STATE: src = ctx->st; bytes = 64; break;
+    case DG_MREF: src = ctx->mref; bytes = 4 * C; break;
+    default: return fail(ctx, DG_EINVAL, "unknown item %d", what);
+  }
+  DG_CK(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, ctx->stream));
+  return DG_OK;
+}
+
+int dg_write(dg_ctx* ctx, int32_t what, const void* src) {
+  if (!ctx) return fail(nullptr, DG_EINVAL, "ctx is NULL");
+  if (!src) return fail(ctx, DG_EINVAL, "src is NULL");
+  const dg_config& c = ctx->cfg;
+  const size_t C = c.C, Cd = (size_t)c.C * c.d;
+  void* dst = nullptr;
+  size_t bytes = 0;
+  switch (what) {
+    case DG_CANVAS: dst = ctx->canvas; bytes = 4 * C; break;
+    case DG_ARGMAX: dst = ctx->argmax_prev; bytes = 4 * C; break;
+    case DG_SC: dst = ctx->sc; bytes = 4 * Cd; break;
+    case DG_HIDDEN: dst = ctx->h; bytes = Cd * (c.dtype == DG_F32 ? 4 : 2); break;
+    case DG_TARGET: dst = ctx->target; bytes = 4 * C; break;
+    case DG_STATE: dst = ctx->st; bytes = 64; break;
+    default: return fail(ctx, DG_EINVAL, "item %d is not writable", what);
+  }
+  DG_CK(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, ctx->stream));
+  return DG_OK;
+}
+
+int dg_profile(dg_ctx* ctx, int32_t enable) {
+  if (!ctx) return fail(nullptr, DG_EINVAL, "ctx is NULL");
+  ctx->prof = enable != 0;
+  ctx->ev_used = 0;
+  ctx->launches = 0;
+  return DG_OK;
+}
+
+int dg_profile_read(dg_ctx* ctx, double* ms_total, int32_t* steps, int64_t* launches) {
+  if (!ctx) return fail(nullptr, DG_EINVAL, "ctx is NULL");
+  DG_CK(cudaStreamSynchronize(ctx->stream));
+  double tot = 0.0;
+  for (size_t j = 0; j + 1 < ctx->ev_used; j += 2) {
+    float ms = 0.f;
+    DG_CK(cudaEventElapsedTime(&ms, ctx->ev[j], ctx->ev[j + 1]));
+    tot += ms;
+  }
+  if (ms_total) *ms_total = tot;
+  if (steps) *steps = (int32_t)(ctx->ev_used / 2);
+  if (launches) *launches = ctx->launches;
+  return DG_OK;
+}
+
+int dg_impl(const dg_ctx* ctx) { return ctx ? ctx->L.impl : DG_EINVAL; }
+
+int dg_free(dg_ctx* ctx) {
+  if (!ctx) return DG_OK;
+  if (ctx->graph_exec) cudaGraphExecDestroy(ctx->graph_exec);
+  if (ctx->graph) cudaGraphDestroy(ctx->graph);
+  for (cudaEvent_t e : ctx->ev) cudaEventDestroy(e);
+  tc_plan_free(&ctx->tc_plan);
+  delete ctx;
+  return DG_OK;
+}
+
+const char* dg_last_error(const dg_ctx* ctx) { return ctx ? ctx->err : g_init_err; }
+
+}  // extern "C"

@@ -1,0 +1,35 @@
+// Host launchers of the denoise-step kernels (CUDA-core path and shared kernels).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include "dg_common.cuh"
+
+namespace dg {
+
+cudaError_t launch_begin_block(cudaStream_t s, DevState* st, int32_t* target, int32_t* canvas,
+                               float* sc, int C, int d, int V, uint64_t seed, int block);
+
+cudaError_t launch_prologue(cudaStream_t s, int dtype, const DevState* st, const void* E,
+                            const int32_t* target, const int32_t* canvas, const float* sc,
+                            void* h, int C, int V, int d, uint64_t seed, float A, float B, float sigma,
+                            int standin, const float* scale_tab, int S,
+                            const int32_t* argmax_prev, float* mref);
+
+cudaError_t launch_simt_attention(cudaStream_t s, int dtype, DevState* st, const void* h,
+                                  const void* E, float* zbuf, TileStat* tstats, RowStat* rowstat,
+                                  float* partial, float* H, int32_t* argmax, float* sc, int C,
+                                  int V, int d, int nsplit, const float* scale_tab, int S);
+
+cudaError_t launch_merge(cudaStream_t s, DevState* st, const TileStat* tstats, int ntiles,
+                         RowStat* rowstat, float* H, int32_t* argmax, int C, const float* O,
+                         const float* mref, float* sc, int d, int32_t* redo_rows,
+                         float redo_gap);
+
+cudaError_t launch_sampler(cudaStream_t s, DevState* st, const float* H, const int32_t* argmax,
+                           int32_t* canvas, int32_t* argmax_prev, int32_t* accept,
+                           int32_t* order, float* prefix, int C, int V, uint64_t seed, float tau,
+                           float stop_entropy, int stop_unchanged, int stop_rule,
+                           int accept_rule, int fixed_steps, int S,
+                           cudaGraphConditionalHandle cond, int use_cond);
+
+}  // namespace dg

@@ -1,0 +1,34 @@
+// Tensor-core (tcgen05/TMEM) vocabulary-attention path: host interface.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+#include "dg_common.cuh"
+
+namespace dg {
+
+// Plan of the tensor-core kernels for one context (tensor maps, tile counts).
+struct TcPlan {
+  int C = 0, V = 0, d = 0;
+  bool ready = false;
+  alignas(64) unsigned char maps[8][128];   // CUtensorMap objects
+  int num_sms = 0;
+  int grid = 0;
+  void* ws = nullptr;
+};
+
+bool tc_supported(int C, int V, int d);
+int tc_stat_tiles(int C, int V, int d);
+size_t tc_workspace_bytes(int C, int V, int d);
+int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, float* O,
+                 TileStat* tstats, void* ws, char* err, size_t errn);
+void tc_plan_free(TcPlan* p);
+int tc_launches(const TcPlan& p);   // kernels per launch_tc_attention call
+cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& p, DevState* st, const void* h,
+                                const void* E, const float* mref, const float* scale_tab,
+                                TileStat* tstats, float* O, void* ws);
+cudaError_t launch_tc_redo(cudaStream_t s, const TcPlan& p, DevState* st, const void* h,
+                           const void* E, const float* scale_tab, const RowStat* rowstat,
+                           const int32_t* redo_rows, float* sc);
+
+}  // namespace dg
