@@ -96,11 +96,14 @@ def h_agreement(w, h_gpu, h_orc) -> float:
     if w.dtype == "bf16":
         diff = h_gpu != h_orc
         if diff.any():
-            # any difference must be one bf16 ulp (fp32 vs fp64 evaluation before rounding)
+            # a difference comes from evaluating the sum in fp32 rather than fp64 before
+            # rounding: one bf16 ulp, or, where the terms cancel to a tiny value, the fp32
+            # absolute error of the summands (magnitude <~ 2)
             e = np.frexp(np.abs(h_orc))[1]
-            two_ulp = np.ldexp(1.0, e - 7)
-            assert np.all(np.abs(h_gpu - h_orc)[diff] <= two_ulp[diff])
+            tol = np.maximum(np.ldexp(1.0, e - 7), 2e-6)
+            assert np.all(np.abs(h_gpu - h_orc)[diff] <= tol[diff])
         return float(diff.mean())
-    rel = np.abs(h_gpu - h_orc) / np.maximum(np.abs(h_orc), 1e-3)
-    assert rel.max() < 1e-5
+    # fp32 evaluation of four summands of magnitude <~ 2: a few fp32 ulps absolute
+    err = np.abs(h_gpu - h_orc)
+    assert err.max() < 2e-6, err.max()
     return 0.0
