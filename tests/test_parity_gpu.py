@@ -117,6 +117,39 @@ def run_teacher_forced(den, w, E32, max_steps=None):
 
 
 # ----------------------------------------------------------------------------
+@pytest.mark.parametrize("shape", [(128, 4096, 256), (256, 8192, 512), (128, 16384, 768)])
+def test_tc_small_shapes(shape):
+    """The tensor-core kernel on small shapes (one range group up to several), 3 steps."""
+    C, V, d = shape
+    w = synthetic.SMALL.replace(C=C, V=V, d=d, tau=0.5 * C * np.log(2), max_steps=3,
+                                fixed_steps=1, coef_target=1.0, coef_canvas=0.5, logit_scale=2.0)
+    den, E32 = make(w, dg.DG_IMPL_TC)
+    tally = run_teacher_forced(den, w, E32)
+    assert tally.steps == 3
+    assert den.state()["redo"] == 0
+    den.close()
+
+
+def test_tc_reference_too_low_is_recomputed():
+    """Hidden states whose best logit far exceeds the per-row reference take the exact fix-up path."""
+    w = synthetic.SMALL.replace(C=128, V=8192, d=512, tau=40.0, max_steps=2, fixed_steps=1)
+    den, E32 = make(w, dg.DG_IMPL_TC)
+    Eg, _ = embedding(w)
+    canvas = _np(den.read(dg.DG_CANVAS)).astype(np.int64)
+    tok = (canvas * 7 + 3) % w.V
+    h = (30.0 * Eg[torch.from_numpy(tok).cuda()].float()).to(torch.bfloat16).contiguous()
+    den.step_h(h)
+    st = den.state()
+    assert st["status"] == 0 and st["redo"] > 0
+    att = M.vocab_attention(_np(h).astype(np.float64), E32, w.logit_scale / w.T_start)
+    acc = M.entropy_bounded_accept(att.H.astype(np.float32), w.tau, w.accept_rule)
+    flags = near_tie_flags(att, acc, w.tau, w.accept_rule)
+    tally = Tally()
+    compare_attention(tally, att, _np(den.read(dg.DG_ENTROPY)), _np(den.read(dg.DG_ARGMAX)),
+                      _np(den.read(dg.DG_SC)).astype(np.float64), flags)
+    den.close()
+
+
 @pytest.mark.parametrize("impl", IMPLS)
 def test_tiny_block_trajectory(impl):
     w = synthetic.TINY

@@ -183,9 +183,13 @@ int launch_step(dg_ctx* ctx, bool standin, bool use_cond) {
   cudaStream_t s = ctx->stream;
   const float sigma = (float)std::sqrt((double)c.noise_var_d / (double)c.d);
   const bool tc = ctx->L.impl == DG_IMPL_TC;
+  unsigned* zero = nullptr;
+  int nzero = 0;
+  if (tc) tc_counters(ctx->tc_plan, &zero, &nzero);
   DG_CK(launch_prologue(s, c.dtype, ctx->st, ctx->E, ctx->target, ctx->canvas, ctx->sc, ctx->h,
                         c.C, c.V, c.d, c.seed, c.coef_target, c.coef_canvas, sigma, standin ? 1 : 0,
-                        ctx->scale_tab, c.max_steps, ctx->argmax_prev, tc ? ctx->mref : nullptr));
+                        ctx->scale_tab, c.max_steps, ctx->argmax_prev, tc ? ctx->mref : nullptr,
+                        zero, nzero));
   cudaEvent_t e0 = nullptr, e1 = nullptr;
   if (ctx->prof && !use_cond) {
     if (ctx->ev_used + 2 > ctx->ev.size()) {
@@ -202,11 +206,14 @@ int launch_step(dg_ctx* ctx, bool standin, bool use_cond) {
   ctx->launches += 2 + (tc ? 2 + tc_launches(ctx->tc_plan) : 4);
   if (tc) {
     DG_CK(launch_tc_attention(s, ctx->tc_plan, ctx->st, ctx->h, ctx->E, ctx->mref, ctx->scale_tab,
-                              ctx->tstats, ctx->O, ctx->tc));
+                              c.max_steps, ctx->tstats, ctx->O, ctx->tc));
+    const float* Opart = nullptr;
+    int nO = 0;
+    tc_partials(ctx->tc_plan, &Opart, &nO);
     DG_CK(launch_merge(s, ctx->st, ctx->tstats, ctx->L.ntiles, ctx->rowstat, ctx->H, ctx->argmax,
-                       c.C, ctx->O, ctx->mref, ctx->sc, c.d, ctx->redo_rows, kRedoGap));
-    DG_CK(launch_tc_redo(s, ctx->tc_plan, ctx->st, ctx->h, ctx->E, ctx->scale_tab, ctx->rowstat,
-                         ctx->redo_rows, ctx->sc));
+                       c.C, Opart, nO, ctx->mref, ctx->sc, c.d, ctx->redo_rows, kRedoGap));
+    DG_CK(launch_tc_redo(s, ctx->tc_plan, ctx->st, ctx->h, ctx->E, ctx->scale_tab, c.max_steps,
+                         ctx->rowstat, ctx->redo_rows, ctx->H, ctx->sc));
   } else {
     DG_CK(launch_simt_attention(s, c.dtype, ctx->st, ctx->h, ctx->E, ctx->zbuf, ctx->tstats,
                                 ctx->rowstat, ctx->partial, ctx->H, ctx->argmax, ctx->sc, c.C,

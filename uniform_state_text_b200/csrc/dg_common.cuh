@@ -74,9 +74,9 @@ struct TileStat {
 
 // Per-row merged statistics used by the sampler and the sc normalisation.
 struct RowStat {
-  float m;      // largest logit
+  float m;      // reference the partition sum is taken against
   float Z;      // sum e^(z - m)
-  float pad[2];
+  float pad[2]; // pad[0]: the row's largest logit
 };
 
 // Total order used for argmax: larger value first, then lower index.

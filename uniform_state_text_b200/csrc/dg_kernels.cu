@@ -58,8 +58,10 @@ template <typename T>
 __global__ void __launch_bounds__(256) k_prologue(const DevState* st, const T* E,
     const int32_t* target, const int32_t* canvas, const float* sc, T* h, int C, int V, int d,
     uint64_t seed, float A, float B, float sigma, int standin, const float* scale_tab, int S,
-    const int32_t* argmax_prev, float* mref) {
+    const int32_t* argmax_prev, float* mref, unsigned* zero, int nzero) {
   if (st->done) return;
+  if (zero && blockIdx.x == 0)
+    for (int j = threadIdx.x; j < nzero; j += blockDim.x) zero[j] = 0u;
   const int i = blockIdx.x;
   const int t = st->t;
   const int ts = min(max(t, 0), S - 1);
@@ -216,8 +218,8 @@ __global__ void __launch_bounds__(256) k_simt_logits(const DevState* st, const T
 // sc = O e^(mref - m) / Z and flags rows whose logit reference was too low.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_merge(DevState* st, const TileStat* tstats, int ntiles,
-    RowStat* rowstat, float* H, int32_t* argmax, int C, const float* O, const float* mref,
-    float* sc, int d, int32_t* redo_rows, float redo_gap) {
+    RowStat* rowstat, float* H, int32_t* argmax, int C, const float* O, int nO,
+    const float* mref, float* sc, int d, int32_t* redo_rows, float redo_gap) {
   if (st->done) return;
   const int i = blockIdx.x;
   Stat s;
@@ -240,11 +242,11 @@ __global__ void __launch_bounds__(256) k_merge(DevState* st, const TileStat* tst
     const float Hv = logf(r.Z) - r.S1 / r.Z;
     H[i] = fmaxf(Hv, 0.f);
     argmax[i] = r.arg;
-    RowStat rs; rs.m = r.m; rs.Z = r.Z; rs.pad[0] = rs.pad[1] = 0.f;
+    RowStat rs; rs.m = r.m; rs.Z = r.Z; rs.pad[0] = r.best; rs.pad[1] = 0.f;
     rowstat[i] = rs;
     int redo = 0;
     if (O) {
-      const float gap = r.m - mref[i];
+      const float gap = r.best - mref[i];
       redo = !(gap <= redo_gap);   // also catches NaN
       sh_scale = __expf(mref[i] - r.m) / r.Z;
       if (redo) { redo_rows[atomicAdd(&st->redo, 1)] = i; }
@@ -255,7 +257,12 @@ __global__ void __launch_bounds__(256) k_merge(DevState* st, const TileStat* tst
   __syncthreads();
   if (sh_redo) return;
   const float f = sh_scale;
-  for (int k = threadIdx.x; k < d; k += blockDim.x) sc[(size_t)i * d + k] = O[(size_t)i * d + k] * f;
+  const size_t pstride = (size_t)C * d;
+  for (int k = threadIdx.x; k < d; k += blockDim.x) {
+    float acc = 0.f;
+    for (int g = 0; g < nO; ++g) acc += O[g * pstride + (size_t)i * d + k];
+    sc[(size_t)i * d + k] = acc * f;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -424,15 +431,16 @@ cudaError_t launch_prologue(cudaStream_t s, int dtype, const DevState* st, const
                             const int32_t* target, const int32_t* canvas, const float* sc,
                             void* h, int C, int V, int d, uint64_t seed, float A, float B, float sigma,
                             int standin, const float* scale_tab, int S,
-                            const int32_t* argmax_prev, float* mref) {
+                            const int32_t* argmax_prev, float* mref, unsigned* zero, int nzero) {
   if (dtype == 0)
     k_prologue<float><<<C, 256, 0, s>>>(st, (const float*)E, target, canvas, sc, (float*)h, C, V, d,
                                         seed, A, B, sigma, standin, scale_tab, S, argmax_prev,
-                                        mref);
+                                        mref, zero, nzero);
   else
     k_prologue<__nv_bfloat16><<<C, 256, 0, s>>>(st, (const __nv_bfloat16*)E, target, canvas, sc,
                                                 (__nv_bfloat16*)h, C, V, d, seed, A, B, sigma,
-                                                standin, scale_tab, S, argmax_prev, mref);
+                                                standin, scale_tab, S, argmax_prev, mref, zero,
+                                                nzero);
   return cudaGetLastError();
 }
 
@@ -450,8 +458,8 @@ cudaError_t launch_simt_attention(cudaStream_t s, int dtype, DevState* st, const
                                                      d, scale_tab, S);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_merge<<<C, 256, 0, s>>>(st, tstats, V / ST, rowstat, H, argmax, C, nullptr, nullptr, nullptr,
-                            d, nullptr, 0.f);
+  k_merge<<<C, 256, 0, s>>>(st, tstats, V / ST, rowstat, H, argmax, C, nullptr, 0, nullptr,
+                            nullptr, d, nullptr, 0.f);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   dim3 g2((d + ST - 1) / ST, (C + ST - 1) / ST, nsplit);
   if (dtype == 0)
@@ -470,10 +478,10 @@ cudaError_t launch_simt_attention(cudaStream_t s, int dtype, DevState* st, const
 
 cudaError_t launch_merge(cudaStream_t s, DevState* st, const TileStat* tstats, int ntiles,
                          RowStat* rowstat, float* H, int32_t* argmax, int C, const float* O,
-                         const float* mref, float* sc, int d, int32_t* redo_rows,
+                         int nO, const float* mref, float* sc, int d, int32_t* redo_rows,
                          float redo_gap) {
-  k_merge<<<C, 256, 0, s>>>(st, tstats, ntiles, rowstat, H, argmax, C, O, mref, sc, d, redo_rows,
-                            redo_gap);
+  k_merge<<<C, 256, 0, s>>>(st, tstats, ntiles, rowstat, H, argmax, C, O, nO, mref, sc, d,
+                            redo_rows, redo_gap);
   return cudaGetLastError();
 }
 

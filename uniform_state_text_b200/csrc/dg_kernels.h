@@ -13,7 +13,8 @@ cudaError_t launch_prologue(cudaStream_t s, int dtype, const DevState* st, const
                             const int32_t* target, const int32_t* canvas, const float* sc,
                             void* h, int C, int V, int d, uint64_t seed, float A, float B, float sigma,
                             int standin, const float* scale_tab, int S,
-                            const int32_t* argmax_prev, float* mref);
+                            const int32_t* argmax_prev, float* mref, unsigned* zero = nullptr,
+                            int nzero = 0);
 
 cudaError_t launch_simt_attention(cudaStream_t s, int dtype, DevState* st, const void* h,
                                   const void* E, float* zbuf, TileStat* tstats, RowStat* rowstat,
@@ -22,7 +23,7 @@ cudaError_t launch_simt_attention(cudaStream_t s, int dtype, DevState* st, const
 
 cudaError_t launch_merge(cudaStream_t s, DevState* st, const TileStat* tstats, int ntiles,
                          RowStat* rowstat, float* H, int32_t* argmax, int C, const float* O,
-                         const float* mref, float* sc, int d, int32_t* redo_rows,
+                         int nO, const float* mref, float* sc, int d, int32_t* redo_rows,
                          float redo_gap);
 
 cudaError_t launch_sampler(cudaStream_t s, DevState* st, const float* H, const int32_t* argmax,

@@ -1,25 +1,739 @@
-// Tensor-core vocabulary-attention path (placeholder until the tcgen05 kernels land).
+// Tensor-core vocabulary attention for sm_100a (tcgen05 MMA, TMEM accumulators,
+// TMA-staged operands).
+//
+// What it computes ("A Visual Guide to DiffusionGemma", 5.1 self-conditioning,
+// 5.3 logits temperature, 5.4 entropy): for every canvas row i and vocabulary
+// entry v the tempered logit z = (L/T) <h_i, E_v>; per row the softmax
+// statistics (partition sum, entropy sum, argmax) and sc_i = sum_v p_v E_v,
+// without ever storing the C x V logits.
+//
+// Design (B200):
+//   * Both contractions run on tcgen05 (bf16 in, fp32 accumulate in TMEM).
+//   * A fixed per-row logit reference m_ref (the larger of the logits of the
+//     row's current canvas token and of its previous argmax, computed by the
+//     prologue) replaces the running maximum: probabilities are
+//     P = exp(z - m_ref). With no running maximum there is nothing to agree on
+//     between CTAs, so the P.E contraction can run on other SMs than the h.E^T
+//     contraction. The exact maximum is tracked alongside; a row whose maximum
+//     exceeds m_ref by more than 64 (P could overflow) is recomputed exactly by
+//     the fix-up kernels below. Entropy and argmax never depend on m_ref.
+//   * One persistent cooperative kernel, two CTA roles:
+//       G1 CTAs: S = h E_tile^T for 128 rows x 256 vocabulary entries (K = d)
+//                into a double-buffered TMEM accumulator; the epilogue warps
+//                turn S into per-tile statistics and bf16 P, written into an
+//                L2-resident ring of vocabulary ranges (KV2 entries per range).
+//       G2 CTAs: each owns (row block, 256-column slice of d, range group) and
+//                accumulates O = P E over its ranges in TMEM, then writes one
+//                partial; the merge kernel sums the partials in fixed order.
+//     Hand-off: per-range "ready" and "consumed" counters in global memory
+//     (release/acquire); every wait is bounded by %globaltimer and aborts the
+//     whole kernel through a flag, after draining its in-flight copies.
+//   * Warp roles per CTA (192 threads): warp 0 TMA producer, warp 1 TMEM
+//     allocator + MMA issuer, warps 2-5 epilogue (one TMEM lane per thread).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
 #include "dg_tc.h"
 
 namespace dg {
+namespace tc {
 
-bool tc_supported(int, int, int) { return false; }
-int tc_stat_tiles(int, int V, int) { return V / 256; }
-size_t tc_workspace_bytes(int, int, int) { return 0; }
-int tc_plan_init(TcPlan*, int, int, int, const void*, void*, float*, TileStat*, void*, char* err,
-                 size_t errn) {
-  if (err && errn) err[0] = 0;
-  return -5;
+constexpr int BM = 128;        // canvas rows per CTA (MMA M)
+constexpr int BN = 256;        // MMA N: vocabulary entries (G1) or columns of d (G2)
+constexpr int BK = 64;         // K per pipeline stage (one 128-byte swizzle row of bf16)
+constexpr int STAGES = 4;
+constexpr int KV2 = 4096;      // vocabulary entries per P range
+constexpr int RING = 4;        // P ranges resident at once
+constexpr int THREADS = 192;
+constexpr int RSPLIT = 16;     // vocabulary splits of the fix-up kernels
+constexpr uint32_t A_BYTES = BM * BK * 2;
+constexpr uint32_t B_BYTES = BN * BK * 2;
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+constexpr unsigned long long TIMEOUT_NS = 2000000000ull;   // 2 s
+
+struct Params {
+  int C, V, d, RB, n_vt, n_ranges, n_dt, G, n1, tiles_per_range, S;
+  const float* mref;
+  const float* scale_tab;
+  TileStat* tstats;
+  float* Opart;              // [G][C][d]
+  __nv_bfloat16* P;          // [RING][C][KV2]
+  unsigned* ready;           // [n_ranges]
+  unsigned* consumed;        // [n_ranges]
+  int* abort_flag;
+  DevState* st;
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
 }
-void tc_plan_free(TcPlan*) {}
-int tc_launches(const TcPlan&) { return 1; }
-cudaError_t launch_tc_attention(cudaStream_t, const TcPlan&, DevState*, const void*, const void*,
-                                const float*, const float*, TileStat*, float*, void*) {
-  return cudaErrorNotSupported;
+__device__ __forceinline__ uint64_t gtimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
 }
-cudaError_t launch_tc_redo(cudaStream_t, const TcPlan&, DevState*, const void*, const void*,
-                           const float*, const RowStat*, const int32_t*, float*) {
-  return cudaErrorNotSupported;
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ void raise_abort(const Params& p) {
+  atomicExch(p.abort_flag, 1);
+  atomicCAS(&p.st->status, 0, -4 /* DG_ETIMEOUT */);
+}
+
+// Bounded wait on an mbarrier phase. Returns false on abort (own timeout or
+// another warp's). With check_abort = false only the time limit applies (used
+// to drain copies that are certain to complete).
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Params& p,
+                                       bool check_abort = true) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = gtimer();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try(bar, parity)) return true;
+    if ((n & 63) == 0) {
+      if (check_abort && *(volatile int*)p.abort_flag) return false;
+      if (gtimer() - t0 > TIMEOUT_NS) { raise_abort(p); return false; }
+    }
+  }
+}
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* ptr) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_add(unsigned* ptr, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Bounded wait until a global counter reaches target.
+__device__ __noinline__ bool counter_wait(const unsigned* ptr, unsigned target, const Params& p) {
+  if (ld_acquire(ptr) >= target) return true;
+  const uint64_t t0 = gtimer();
+  for (uint32_t n = 1;; ++n) {
+    if (ld_acquire(ptr) >= target) return true;
+    __nanosleep(64);
+    if ((n & 15) == 0) {
+      if (*(volatile int*)p.abort_flag) return false;
+      if (gtimer() - t0 > TIMEOUT_NS) { raise_abort(p); return false; }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
+}
+// Instruction descriptor: bf16 x bf16 -> f32, A K-major, B K- or MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn_major << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::
+                   "r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// 32 lanes x 32 columns of fp32 from TMEM: thread t of the warp gets its lane's columns.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// ---------------------------------------------------------------------------
+// The persistent kernel.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(THREADS, 1)
+    k_vocab_attention(const __grid_constant__ CUtensorMap tm_h,
+                      const __grid_constant__ CUtensorMap tm_ek,
+                      const __grid_constant__ CUtensorMap tm_emn,
+                      const __grid_constant__ CUtensorMap tm_p, const Params p) {
+  if (p.st->done) return;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* full = bars;                 // [STAGES]
+  uint64_t* empty = bars + STAGES;       // [STAGES]
+  uint64_t* acc_full = bars + 2 * STAGES;   // [2]
+  uint64_t* acc_empty = acc_full + 2;       // [2]
+  uint64_t* fin = acc_empty + 2;            // [1]
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(fin + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool is_g1 = (int)blockIdx.x < p.n1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 4); }
+    mbar_init(fin, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::
+                     "r"(smem_u32(tmem_base_slot)), "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_slot;
+
+  // Work description.
+  const int n_items1 = p.RB * p.n_vt;
+  const int nk1 = p.d / BK;               // K stages per G1 item
+  const int nk2 = KV2 / BK;               // K stages per G2 range
+  int o = 0, g = 0, rb2 = 0, dt = 0;
+  if (!is_g1) {
+    o = blockIdx.x - p.n1;
+    g = o / (p.RB * p.n_dt);
+    const int rem = o % (p.RB * p.n_dt);
+    rb2 = rem / p.n_dt;
+    dt = rem % p.n_dt;
+  }
+  const unsigned ready_target = (unsigned)(p.RB * p.tiles_per_range * 4);
+  const unsigned consumed_target = (unsigned)(p.RB * p.n_dt);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      long issued = 0;
+      bool ok = true;
+      if (is_g1) {
+        for (int it = blockIdx.x; ok && it < n_items1; it += p.n1) {
+          const int vt = it / p.RB, rb = it % p.RB;
+          const int r = vt / p.tiles_per_range;
+          if (r >= RING && !counter_wait(&p.consumed[r - RING], consumed_target, p)) { ok = false; break; }
+          for (int kc = 0; kc < nk1; ++kc) {
+            if (!mbar_wait(&empty[s], ph ^ 1, p)) { ok = false; break; }
+            unsigned char* st = smem + s * STAGE_BYTES;
+            mbar_expect_tx(&full[s], STAGE_BYTES);
+            tma_load_2d(st, &tm_h, &full[s], kc * BK, rb * BM);
+            tma_load_2d(st + A_BYTES, &tm_ek, &full[s], kc * BK, vt * BN);
+            ++issued;
+            if (++s == STAGES) { s = 0; ph ^= 1; }
+          }
+        }
+      } else {
+        for (int r = g; ok && r < p.n_ranges; r += p.G) {
+          if (!counter_wait(&p.ready[r], ready_target, p)) { ok = false; break; }
+          fence_proxy_async_global();
+          const int slot = r % RING;
+          for (int kc = 0; kc < nk2; ++kc) {
+            if (!mbar_wait(&empty[s], ph ^ 1, p)) { ok = false; break; }
+            unsigned char* st = smem + s * STAGE_BYTES;
+            mbar_expect_tx(&full[s], STAGE_BYTES);
+            tma_load_2d(st, &tm_p, &full[s], kc * BK, slot * p.C + rb2 * BM);
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d(st + A_BYTES + j * (64 * BK * 2), &tm_emn, &full[s], dt * BN + j * 64,
+                          r * KV2 + kc * BK);
+            ++issued;
+            if (++s == STAGES) { s = 0; ph ^= 1; }
+          }
+        }
+      }
+      // Drain: every issued copy must land before the CTA can exit.
+      for (long k = (issued > STAGES ? issued - STAGES : 0); k < issued; ++k) {
+        const int ss = (int)(k % STAGES);
+        const uint32_t pp = (uint32_t)((k / STAGES) & 1);
+        mbar_wait(&full[ss], pp, p, false);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      bool issued_any = false;
+      if (is_g1) {
+        const uint32_t idesc = idesc_bf16(BM, BN, 0);
+        int n = 0;
+        for (int it = blockIdx.x; ok && it < n_items1; it += p.n1, ++n) {
+          const int buf = n & 1;
+          if (!mbar_wait(&acc_empty[buf], ((n >> 1) & 1) ^ 1, p)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem + buf * BN;
+          for (int kc = 0; kc < nk1; ++kc) {
+            if (!mbar_wait(&full[s], ph, p)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
+            const uint32_t b0 = a0 + A_BYTES;
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k) {
+              const uint64_t ad = sdesc(a0 + k * 32, 16, 1024);
+              const uint64_t bd = sdesc(b0 + k * 32, 16, 1024);
+              mma_bf16(d_tmem, ad, bd, idesc, (kc | k) ? 1u : 0u);
+            }
+            issued_any = true;
+            mma_commit(&empty[s]);
+            if (++s == STAGES) { s = 0; ph ^= 1; }
+          }
+          if (!ok) break;
+          mma_commit(&acc_full[buf]);
+        }
+      } else {
+        const uint32_t idesc = idesc_bf16(BM, BN, 1);
+        bool first = true;
+        for (int r = g; ok && r < p.n_ranges; r += p.G) {
+          for (int kc = 0; kc < nk2; ++kc) {
+            if (!mbar_wait(&full[s], ph, p)) { ok = false; break; }
+            tc_fence_after();
+            if (kc == nk2 - 1) red_release_add(&p.consumed[r], 1u);   // P range is in smem
+            const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
+            const uint32_t b0 = a0 + A_BYTES;
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k) {
+              const uint64_t ad = sdesc(a0 + k * 32, 16, 1024);
+              // MN-major B: 64-column blocks 8 KB apart (LBO), 8-row K groups 1 KB apart (SBO)
+              const uint64_t bd = sdesc(b0 + k * (16 * 128), 64 * BK * 2, 1024);
+              mma_bf16(tmem, ad, bd, idesc, first ? 0u : 1u);
+              first = false;
+            }
+            issued_any = true;
+            mma_commit(&empty[s]);
+            if (++s == STAGES) { s = 0; ph ^= 1; }
+          }
+        }
+        if (ok) mma_commit(&acc_full[0]);
+      }
+      // All MMAs this thread issued must finish before TMEM is released.
+      if (issued_any) {
+        mma_commit(fin);
+        mbar_wait(fin, 0, p, false);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                 // TMEM lane quarter of this warp
+    const int r_local = q * 32 + lane;      // row within the CTA's 128
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    if (is_g1) {
+      const float scale = p.scale_tab[min(max(p.st->t, 0), p.S - 1)];
+      int n = 0;
+      for (int it = blockIdx.x; it < n_items1; it += p.n1, ++n) {
+        const int vt = it / p.RB, rb = it % p.RB;
+        const int r = vt / p.tiles_per_range;
+        const int buf = n & 1;
+        if (!mbar_wait(&acc_full[buf], (n >> 1) & 1, p)) break;
+        tc_fence_after();
+        const int row = rb * BM + r_local;
+        const float mref = p.mref[row];
+        float Z = 0.f, S1 = 0.f, best = -INFINITY;
+        int arg = 0x7fffffff;
+        __nv_bfloat16* prow = p.P + ((size_t)((r % RING) * p.C + row)) * KV2 +
+                              (size_t)(vt % p.tiles_per_range) * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          tmem_ld32(tmem + lane_addr + buf * BN + c * 32, v);
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float z0 = v[j] * scale, z1 = v[j + 1] * scale;
+            if (z0 > best) { best = z0; arg = vt * BN + c * 32 + j; }
+            if (z1 > best) { best = z1; arg = vt * BN + c * 32 + j + 1; }
+            const float d0 = z0 - mref, d1 = z1 - mref;
+            const float e0 = __expf(d0), e1 = __expf(d1);
+            Z += e0 + e1;
+            S1 = fmaf(e0, d0, fmaf(e1, d1, S1));
+            pk[j >> 1] = pack_bf16(e0, e1);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(prow + c * 32);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        }
+        // This warp is done reading the accumulator buffer.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        TileStat ts;
+        ts.m = mref; ts.Z = Z; ts.S1 = S1; ts.best = best; ts.arg = arg;
+        ts.pad[0] = ts.pad[1] = ts.pad[2] = 0;
+        p.tstats[(size_t)row * p.n_vt + vt] = ts;
+        // Publish this warp's rows of the P tile: generic-proxy stores, read later by
+        // TMA on other SMs. Each of the 4 epilogue warps counts once per item.
+        fence_proxy_async_global();
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence();
+          red_release_add(&p.ready[r], 1u);
+        }
+      }
+    } else {
+      const bool has_work = g < p.n_ranges;
+      const int row = rb2 * BM + r_local;
+      float* orow = p.Opart + ((size_t)g * p.C + row) * p.d + (size_t)dt * BN;
+      bool ok = true;
+      if (has_work) {
+        ok = mbar_wait(&acc_full[0], 0, p);
+        tc_fence_after();
+      }
+      if (ok) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          if (has_work) tmem_ld32(tmem + lane_addr + c * 32, v);
+          else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.f;
+          }
+          float4* dst = reinterpret_cast<float4*>(orow + c * 32);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
+      }
+      tc_fence_before();
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Exact recomputation of rows whose logit maximum exceeded the reference.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_redo_partial(const DevState* st,
+    const __nv_bfloat16* h, const __nv_bfloat16* E, const float* scale_tab, int S,
+    const RowStat* rowstat, const int32_t* redo_rows, float* part, int C, int V, int d) {
+  if (st->done || (int)blockIdx.y >= st->redo) return;
+  extern __shared__ float sacc[];           // [d]
+  __shared__ float wz[8], ws1[8];
+  const int row = redo_rows[blockIdx.y];
+  const float scale = scale_tab[min(max(st->t, 0), S - 1)];
+  const float m = rowstat[row].pad[0];        // exact maximum logit
+  for (int k = threadIdx.x; k < d; k += blockDim.x) sacc[k] = 0.f;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int vlen = V / RSPLIT, v0 = blockIdx.x * vlen;
+  const __nv_bfloat16* hr = h + (size_t)row * d;
+  float Z = 0.f, S1 = 0.f;
+  for (int v = v0 + warp; v < v0 + vlen; v += 8) {
+    const __nv_bfloat16* ev = E + (size_t)v * d;
+    float dot = 0.f;
+    for (int k = lane; k < d; k += 32) dot = fmaf(__bfloat162float(hr[k]), __bfloat162float(ev[k]), dot);
+    for (int off = 16; off; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+    const float dz = dot * scale - m;
+    const float e = expf(dz);
+    Z += e;
+    S1 = fmaf(e, dz, S1);
+    if (e > 0.f)
+      for (int k = lane; k < d; k += 32) atomicAdd(&sacc[k], e * __bfloat162float(ev[k]));
+  }
+  if (lane == 0) { wz[warp] = Z; ws1[warp] = S1; }
+  __syncthreads();
+  float* out = part + ((size_t)blockIdx.x * C + row) * (size_t)(d + 4);
+  for (int k = threadIdx.x; k < d; k += blockDim.x) out[k] = sacc[k];
+  if (threadIdx.x == 0) {
+    float a = 0.f, b = 0.f;
+    for (int j = 0; j < 8; ++j) { a += wz[j]; b += ws1[j]; }
+    out[d] = a;
+    out[d + 1] = b;
+  }
+}
+
+__global__ void __launch_bounds__(256) k_redo_finish(const DevState* st, const int32_t* redo_rows,
+    const float* part, float* H, float* sc, int C, int d) {
+  if (st->done || (int)blockIdx.x >= st->redo) return;
+  const int row = redo_rows[blockIdx.x];
+  __shared__ float sZ;
+  if (threadIdx.x == 0) {
+    float Z = 0.f, S1 = 0.f;
+    for (int s = 0; s < RSPLIT; ++s) {
+      const float* q = part + ((size_t)s * C + row) * (size_t)(d + 4);
+      Z += q[d];
+      S1 += q[d + 1];
+    }
+    H[row] = fmaxf(logf(Z) - S1 / Z, 0.f);
+    sZ = Z;
+  }
+  __syncthreads();
+  const float inv = 1.0f / sZ;
+  for (int k = threadIdx.x; k < d; k += blockDim.x) {
+    float acc = 0.f;
+    for (int s = 0; s < RSPLIT; ++s) acc += part[((size_t)s * C + row) * (size_t)(d + 4) + k];
+    sc[(size_t)row * d + k] = acc * inv;
+  }
+}
+
+}  // namespace tc
+
+// ---------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct TcLayout {
+  size_t counters = 0, P = 0, Opart = 0, redo = 0, total = 0;
+  int RB = 0, n_vt = 0, n_ranges = 0, n_dt = 0, G = 0, n1 = 0, n2 = 0;
+};
+
+size_t al(size_t x) { return (x + 255) / 256 * 256; }
+
+int device_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+    return n;
+  cudaGetLastError();
+  return 148;
+}
+
+TcLayout tc_layout(int C, int V, int d, int sms) {
+  TcLayout L;
+  L.RB = C / tc::BM;
+  L.n_vt = V / tc::BN;
+  L.n_ranges = V / tc::KV2;
+  L.n_dt = d / tc::BN;
+  // Choose the number of range groups G: G2 CTAs = RB * n_dt * G, G1 CTAs take
+  // the rest; minimise the larger of the two roles' per-CTA work.
+  const double u1 = (double)tc::BM * tc::BN * d;                 // one G1 item
+  const double u2 = (double)tc::BM * tc::BN * tc::KV2;           // one G2 range
+  const int per_g = L.RB * L.n_dt;
+  double best = 1e300;
+  for (int G = 1; G <= L.n_ranges; ++G) {
+    const int n2 = per_g * G;
+    const int items = L.RB * L.n_vt;
+    int n1 = sms - n2;
+    if (n1 < 1) break;
+    if (n1 > items) n1 = items;
+    const double t1 = std::ceil((double)items / n1) * u1;
+    const double t2 = std::ceil((double)L.n_ranges / G) * u2;
+    const double t = t1 > t2 ? t1 : t2;
+    if (t < best) { best = t; L.G = G; L.n1 = n1; L.n2 = n2; }
+  }
+  size_t off = 0;
+  L.counters = off; off = al(off + sizeof(unsigned) * (2 * (size_t)L.n_ranges + 64));
+  L.P = off; off = al(off + (size_t)tc::RING * C * tc::KV2 * 2);
+  L.Opart = off; off = al(off + (size_t)(L.G > 0 ? L.G : 1) * C * d * 4);
+  L.redo = off; off = al(off + (size_t)tc::RSPLIT * C * (d + 4) * 4);
+  L.total = off;
+  return L;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    else
+      cudaGetLastError();
+  }
+  return fn;
+}
+
+bool encode(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+            uint32_t box_outer) {
+  auto fn = get_encoder();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool tc_supported(int C, int V, int d) {
+  return (C == 128 || C == 256) && d % 256 == 0 && d >= 256 && d <= 8192 && V % tc::KV2 == 0 &&
+         V >= tc::KV2 && V <= (1 << 24);
+}
+
+int tc_stat_tiles(int, int V, int) { return V / tc::BN; }
+
+size_t tc_workspace_bytes(int C, int V, int d) { return tc_layout(C, V, d, device_sms()).total; }
+
+int tc_launches(const TcPlan&) { return 3; }
+
+int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, float* O,
+                 TileStat* tstats, void* ws, char* err, size_t errn) {
+  (void)O;
+  (void)tstats;
+  p->C = C; p->V = V; p->d = d;
+  p->num_sms = device_sms();
+  TcLayout L = tc_layout(C, V, d, p->num_sms);
+  p->grid = L.n1 + L.n2;
+  p->ws = ws;
+  char* base = static_cast<char*>(ws);
+  static_assert(sizeof(CUtensorMap) <= 128, "tensor map size");
+  CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(p->maps);
+  bool ok = encode(&maps[0], h, (uint64_t)d, (uint64_t)C, tc::BK, tc::BM) &&
+            encode(&maps[1], E, (uint64_t)d, (uint64_t)V, tc::BK, tc::BN) &&
+            encode(&maps[2], E, (uint64_t)d, (uint64_t)V, tc::BK, 64) &&
+            encode(&maps[3], base + L.P, (uint64_t)tc::KV2, (uint64_t)tc::RING * C, tc::BK, tc::BM);
+  if (!ok) {
+    snprintf(err, errn, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
+    return -3;
+  }
+  cudaError_t e = cudaFuncSetAttribute(tc::k_vocab_attention,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)tc::SMEM_BYTES);
+  if (e != cudaSuccess) {
+    snprintf(err, errn, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    return -3;
+  }
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tc::k_vocab_attention, tc::THREADS,
+                                                    tc::SMEM_BYTES);
+  if (e != cudaSuccess || per_sm < 1 || p->grid > per_sm * p->num_sms) {
+    snprintf(err, errn, "tensor-core kernel cannot be co-resident (%d per SM, grid %d)", per_sm,
+             p->grid);
+    return -5;
+  }
+  p->ready = true;
+  return 0;
+}
+
+void tc_plan_free(TcPlan* p) { p->ready = false; }
+
+void tc_counters(const TcPlan& p, unsigned** ptr, int* count) {
+  TcLayout L = tc_layout(p.C, p.V, p.d, p.num_sms);
+  *ptr = reinterpret_cast<unsigned*>(static_cast<char*>(p.ws) + L.counters);
+  *count = 2 * L.n_ranges + 64;
+}
+
+cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, const void* h,
+                                const void* E, const float* mref, const float* scale_tab,
+                                int S, TileStat* tstats, float* O, void* ws) {
+  (void)h; (void)E; (void)O;
+  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
+  char* base = static_cast<char*>(ws);
+  tc::Params prm;
+  prm.C = pl.C; prm.V = pl.V; prm.d = pl.d; prm.RB = L.RB; prm.n_vt = L.n_vt;
+  prm.n_ranges = L.n_ranges; prm.n_dt = L.n_dt; prm.G = L.G; prm.n1 = L.n1;
+  prm.tiles_per_range = tc::KV2 / tc::BN; prm.S = S;
+  prm.mref = mref; prm.scale_tab = scale_tab; prm.tstats = tstats;
+  prm.Opart = reinterpret_cast<float*>(base + L.Opart);
+  prm.P = reinterpret_cast<__nv_bfloat16*>(base + L.P);
+  unsigned* ctr = reinterpret_cast<unsigned*>(base + L.counters);
+  prm.ready = ctr;
+  prm.consumed = ctr + L.n_ranges;
+  prm.abort_flag = reinterpret_cast<int*>(ctr + 2 * L.n_ranges);
+  prm.st = st;
+  const CUtensorMap* maps = reinterpret_cast<const CUtensorMap*>(pl.maps);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(L.n1 + L.n2);
+  cfg.blockDim = dim3(tc::THREADS);
+  cfg.dynamicSmemBytes = tc::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc::k_vocab_attention, maps[0], maps[1], maps[2], maps[3], prm);
+}
+
+void tc_partials(const TcPlan& pl, const float** Opart, int* nO) {
+  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
+  *Opart = reinterpret_cast<const float*>(static_cast<const char*>(pl.ws) + L.Opart);
+  *nO = L.G;
+}
+
+cudaError_t launch_tc_redo(cudaStream_t s, const TcPlan& pl, DevState* st, const void* h,
+                           const void* E, const float* scale_tab, int S, const RowStat* rowstat,
+                           const int32_t* redo_rows, float* H, float* sc) {
+  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
+  float* part = reinterpret_cast<float*>(static_cast<char*>(pl.ws) + L.redo);
+  dim3 g1(tc::RSPLIT, pl.C);
+  tc::k_redo_partial<<<g1, 256, sizeof(float) * pl.d, s>>>(
+      st, static_cast<const __nv_bfloat16*>(h), static_cast<const __nv_bfloat16*>(E), scale_tab, S,
+      rowstat, redo_rows, part, pl.C, pl.V, pl.d);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  tc::k_redo_finish<<<pl.C, 256, 0, s>>>(st, redo_rows, part, H, sc, pl.C, pl.d);
+  return cudaGetLastError();
 }
 
 }  // namespace dg

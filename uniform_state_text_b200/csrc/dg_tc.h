@@ -26,9 +26,13 @@ void tc_plan_free(TcPlan* p);
 int tc_launches(const TcPlan& p);   // kernels per launch_tc_attention call
 cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& p, DevState* st, const void* h,
                                 const void* E, const float* mref, const float* scale_tab,
-                                TileStat* tstats, float* O, void* ws);
+                                int S, TileStat* tstats, float* O, void* ws);
 cudaError_t launch_tc_redo(cudaStream_t s, const TcPlan& p, DevState* st, const void* h,
-                           const void* E, const float* scale_tab, const RowStat* rowstat,
-                           const int32_t* redo_rows, float* sc);
+                           const void* E, const float* scale_tab, int S, const RowStat* rowstat,
+                           const int32_t* redo_rows, float* H, float* sc);
+// Hand-off counters the prologue zeroes before every step.
+void tc_counters(const TcPlan& p, unsigned** ptr, int* count);
+// Per-range-group partials of O = P E that the merge sums.
+void tc_partials(const TcPlan& p, const float** Opart, int* nO);
 
 }  // namespace dg
