@@ -103,8 +103,12 @@ STRESS_PARTIAL = SMALL.replace(name="stress_partial_c256_v32768_d1024_bf16",
 STRESS_TIES = SMALL.replace(name="stress_ties_c256_v32768_d1024_bf16",
                             coef_target=0.5, coef_canvas=0.5, logit_scale=1.0)
 
+# Headline shapes with a quarter of the vocabulary (E = 268 MB, still larger than
+# L2): small enough for a multi-pass profiler capture of one step.
+PROFILE = HEADLINE.replace(name="profile_c256_v65536_d2048_bf16", V=65536)
+
 WORKLOADS = {w.name: w for w in (TINY, SMALL, HEADLINE, LATENCY, BLOCKS,
-                                 STRESS_PARTIAL, STRESS_TIES)}
+                                 STRESS_PARTIAL, STRESS_TIES, PROFILE)}
 
 
 def _chunk(args):

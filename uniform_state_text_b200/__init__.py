@@ -15,7 +15,8 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libdg.so")
+# DG_LIBRARY selects another build of the same library (e.g. an instrumented one).
+LIB_PATH = os.environ.get("DG_LIBRARY") or os.path.join(HERE, "libdg.so")
 
 DG_OK, DG_EINVAL, DG_ENOMEM, DG_ECUDA, DG_ETIMEOUT, DG_EUNSUPPORTED, DG_ESTATE = 0, -1, -2, -3, -4, -5, -6
 DG_F32, DG_BF16 = 0, 1

@@ -21,11 +21,11 @@
 //       G1 CTAs: S = h E_tile^T for 128 rows x 256 vocabulary entries (K = d)
 //                into a double-buffered TMEM accumulator; the epilogue warps
 //                turn S into per-tile statistics and bf16 P, written into an
-//                L2-resident ring of vocabulary ranges (KV2 entries per range).
+//                L2-resident ring of P tiles.
 //       G2 CTAs: each owns (row block, 256-column slice of d, range group) and
 //                accumulates O = P E over its ranges in TMEM, then writes one
 //                partial; the merge kernel sums the partials in fixed order.
-//     Hand-off: per-range "ready" and "consumed" counters in global memory
+//     Hand-off: per-tile "ready" and "consumed" counters in global memory
 //     (release/acquire); every wait is bounded by %globaltimer and aborts the
 //     whole kernel through a flag, after draining its in-flight copies.
 //   * Warp roles per CTA (192 threads): warp 0 TMA producer, warp 1 TMEM
@@ -46,8 +46,8 @@ constexpr int BM = 128;        // canvas rows per CTA (MMA M)
 constexpr int BN = 256;        // MMA N: vocabulary entries (G1) or columns of d (G2)
 constexpr int BK = 64;         // K per pipeline stage (one 128-byte swizzle row of bf16)
 constexpr int STAGES = 4;
-constexpr int KV2 = 4096;      // vocabulary entries per P range
-constexpr int RING = 4;        // P ranges resident at once
+constexpr int KV2 = 1024;      // vocabulary entries per range (unit of G2 ownership)
+constexpr int RING = 64;       // P tiles (256 vocabulary entries each) resident at once
 constexpr int THREADS = 192;
 constexpr int RSPLIT = 16;     // vocabulary splits of the fix-up kernels
 constexpr uint32_t A_BYTES = BM * BK * 2;
@@ -62,12 +62,27 @@ struct Params {
   const float* scale_tab;
   TileStat* tstats;
   float* Opart;              // [G][C][d]
-  __nv_bfloat16* P;          // [RING][C][KV2]
-  unsigned* ready;           // [n_ranges]
-  unsigned* consumed;        // [n_ranges]
+  __nv_bfloat16* P;          // [RING][C][BN]: ring of P tiles
+  unsigned* ready;           // [n_vt]: epilogue warps that finished a tile
+  unsigned* consumed;        // [n_vt]: G2 CTAs that finished loading a tile
   int* abort_flag;
   DevState* st;
+  unsigned long long* trace;   // [grid][32] wait-time counters (DG_TC_TRACE builds only)
 };
+
+// Per-CTA wait-time tracing, compiled in only with -DDG_TC_TRACE (measurement
+// builds); slots: 0 start, 1 end, 2 producer waits on empty stages, 3 producer
+// waits on counters, 4 MMA waits on full stages, 5 MMA waits on free
+// accumulators, 6 epilogue waits on full accumulators, 7 items, 8 epilogue busy.
+#ifdef DG_TC_TRACE
+#define TRACE_T0() const unsigned long long tr_t0_ = gtimer()
+#define TRACE_ADD(slot) (p.trace[blockIdx.x * 32 + (slot)] += gtimer() - tr_t0_)
+#define TRACE_SET(slot, v) (p.trace[blockIdx.x * 32 + (slot)] = (v))
+#else
+#define TRACE_T0() ((void)0)
+#define TRACE_ADD(slot) ((void)0)
+#define TRACE_SET(slot, v) ((void)0)
+#endif
 
 // ---------------------------------------------------------------------------
 // PTX wrappers.
@@ -235,6 +250,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool is_g1 = (int)blockIdx.x < p.n1;
+  if (threadIdx.x == 0) TRACE_SET(0, gtimer());
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -265,7 +281,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     rb2 = rem / p.n_dt;
     dt = rem % p.n_dt;
   }
-  const unsigned ready_target = (unsigned)(p.RB * p.tiles_per_range * 4);
+  const unsigned ready_target = (unsigned)(p.RB * 4);
   const unsigned consumed_target = (unsigned)(p.RB * p.n_dt);
 
   if (warp == 0) {
@@ -278,10 +294,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (is_g1) {
         for (int it = blockIdx.x; ok && it < n_items1; it += p.n1) {
           const int vt = it / p.RB, rb = it % p.RB;
-          const int r = vt / p.tiles_per_range;
-          if (r >= RING && !counter_wait(&p.consumed[r - RING], consumed_target, p)) { ok = false; break; }
+          {
+            TRACE_T0();
+            if (vt >= RING && !counter_wait(&p.consumed[vt - RING], consumed_target, p)) { ok = false; break; }
+            TRACE_ADD(3);
+          }
           for (int kc = 0; kc < nk1; ++kc) {
+            TRACE_T0();
             if (!mbar_wait(&empty[s], ph ^ 1, p)) { ok = false; break; }
+            TRACE_ADD(2);
             unsigned char* st = smem + s * STAGE_BYTES;
             mbar_expect_tx(&full[s], STAGE_BYTES);
             tma_load_2d(st, &tm_h, &full[s], kc * BK, rb * BM);
@@ -292,14 +313,20 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       } else {
         for (int r = g; ok && r < p.n_ranges; r += p.G) {
-          if (!counter_wait(&p.ready[r], ready_target, p)) { ok = false; break; }
-          fence_proxy_async_global();
-          const int slot = r % RING;
           for (int kc = 0; kc < nk2; ++kc) {
+            const int vt = r * p.tiles_per_range + kc / (BN / BK);
+            if (kc % (BN / BK) == 0) {
+              TRACE_T0();
+              if (!counter_wait(&p.ready[vt], ready_target, p)) { ok = false; break; }
+              TRACE_ADD(3);
+              fence_proxy_async_global();
+            }
+            TRACE_T0();
             if (!mbar_wait(&empty[s], ph ^ 1, p)) { ok = false; break; }
+            TRACE_ADD(2);
             unsigned char* st = smem + s * STAGE_BYTES;
             mbar_expect_tx(&full[s], STAGE_BYTES);
-            tma_load_2d(st, &tm_p, &full[s], kc * BK, slot * p.C + rb2 * BM);
+            tma_load_2d(st, &tm_p, &full[s], (kc % (BN / BK)) * BK, (vt % RING) * p.C + rb2 * BM);
 #pragma unroll
             for (int j = 0; j < BN / 64; ++j)
               tma_load_2d(st + A_BYTES + j * (64 * BK * 2), &tm_emn, &full[s], dt * BN + j * 64,
@@ -328,11 +355,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         int n = 0;
         for (int it = blockIdx.x; ok && it < n_items1; it += p.n1, ++n) {
           const int buf = n & 1;
-          if (!mbar_wait(&acc_empty[buf], ((n >> 1) & 1) ^ 1, p)) { ok = false; break; }
+          {
+            TRACE_T0();
+            if (!mbar_wait(&acc_empty[buf], ((n >> 1) & 1) ^ 1, p)) { ok = false; break; }
+            TRACE_ADD(5);
+          }
           tc_fence_after();
           const uint32_t d_tmem = tmem + buf * BN;
           for (int kc = 0; kc < nk1; ++kc) {
+            TRACE_T0();
             if (!mbar_wait(&full[s], ph, p)) { ok = false; break; }
+            TRACE_ADD(4);
             tc_fence_after();
             const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
             const uint32_t b0 = a0 + A_BYTES;
@@ -354,9 +387,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         bool first = true;
         for (int r = g; ok && r < p.n_ranges; r += p.G) {
           for (int kc = 0; kc < nk2; ++kc) {
+            TRACE_T0();
             if (!mbar_wait(&full[s], ph, p)) { ok = false; break; }
+            TRACE_ADD(4);
             tc_fence_after();
-            if (kc == nk2 - 1) red_release_add(&p.consumed[r], 1u);   // P range is in smem
+            if (kc % (BN / BK) == BN / BK - 1)      // the tile's P is now in shared memory
+              red_release_add(&p.consumed[r * p.tiles_per_range + kc / (BN / BK)], 1u);
             const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
             const uint32_t b0 = a0 + A_BYTES;
 #pragma unroll
@@ -390,16 +426,19 @@ __global__ void __launch_bounds__(THREADS, 1)
       int n = 0;
       for (int it = blockIdx.x; it < n_items1; it += p.n1, ++n) {
         const int vt = it / p.RB, rb = it % p.RB;
-        const int r = vt / p.tiles_per_range;
         const int buf = n & 1;
-        if (!mbar_wait(&acc_full[buf], (n >> 1) & 1, p)) break;
+        {
+          TRACE_T0();
+          if (!mbar_wait(&acc_full[buf], (n >> 1) & 1, p)) break;
+          if (threadIdx.x == 64) TRACE_ADD(6);
+        }
+        TRACE_T0();
         tc_fence_after();
         const int row = rb * BM + r_local;
         const float mref = p.mref[row];
         float Z = 0.f, S1 = 0.f, best = -INFINITY;
         int arg = 0x7fffffff;
-        __nv_bfloat16* prow = p.P + ((size_t)((r % RING) * p.C + row)) * KV2 +
-                              (size_t)(vt % p.tiles_per_range) * BN;
+        __nv_bfloat16* prow = p.P + ((size_t)((vt % RING) * p.C + row)) * BN;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           float v[32];
@@ -435,8 +474,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
         if (lane == 0) {
           __threadfence();
-          red_release_add(&p.ready[r], 1u);
+          red_release_add(&p.ready[vt], 1u);
         }
+        if (threadIdx.x == 64) { TRACE_ADD(8); TRACE_SET(7, (unsigned long long)(n + 1)); }
       }
     } else {
       const bool has_work = g < p.n_ranges;
@@ -466,6 +506,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 
   __syncthreads();
+  if (threadIdx.x == 0) TRACE_SET(1, gtimer());
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
@@ -547,7 +588,7 @@ __global__ void __launch_bounds__(256) k_redo_finish(const DevState* st, const i
 namespace {
 
 struct TcLayout {
-  size_t counters = 0, P = 0, Opart = 0, redo = 0, total = 0;
+  size_t counters = 0, P = 0, Opart = 0, redo = 0, trace = 0, total = 0;
   int RB = 0, n_vt = 0, n_ranges = 0, n_dt = 0, G = 0, n1 = 0, n2 = 0;
 };
 
@@ -586,10 +627,11 @@ TcLayout tc_layout(int C, int V, int d, int sms) {
     if (t < best) { best = t; L.G = G; L.n1 = n1; L.n2 = n2; }
   }
   size_t off = 0;
-  L.counters = off; off = al(off + sizeof(unsigned) * (2 * (size_t)L.n_ranges + 64));
-  L.P = off; off = al(off + (size_t)tc::RING * C * tc::KV2 * 2);
+  L.counters = off; off = al(off + sizeof(unsigned) * (2 * (size_t)L.n_vt + 64));
+  L.P = off; off = al(off + (size_t)tc::RING * C * tc::BN * 2);
   L.Opart = off; off = al(off + (size_t)(L.G > 0 ? L.G : 1) * C * d * 4);
   L.redo = off; off = al(off + (size_t)tc::RSPLIT * C * (d + 4) * 4);
+  L.trace = off; off = al(off + (size_t)256 * 32 * 8);
   L.total = off;
   return L;
 }
@@ -651,7 +693,7 @@ int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, float* 
   bool ok = encode(&maps[0], h, (uint64_t)d, (uint64_t)C, tc::BK, tc::BM) &&
             encode(&maps[1], E, (uint64_t)d, (uint64_t)V, tc::BK, tc::BN) &&
             encode(&maps[2], E, (uint64_t)d, (uint64_t)V, tc::BK, 64) &&
-            encode(&maps[3], base + L.P, (uint64_t)tc::KV2, (uint64_t)tc::RING * C, tc::BK, tc::BM);
+            encode(&maps[3], base + L.P, (uint64_t)tc::BN, (uint64_t)tc::RING * C, tc::BK, tc::BM);
   if (!ok) {
     snprintf(err, errn, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
     return -3;
@@ -680,7 +722,7 @@ void tc_plan_free(TcPlan* p) { p->ready = false; }
 void tc_counters(const TcPlan& p, unsigned** ptr, int* count) {
   TcLayout L = tc_layout(p.C, p.V, p.d, p.num_sms);
   *ptr = reinterpret_cast<unsigned*>(static_cast<char*>(p.ws) + L.counters);
-  *count = 2 * L.n_ranges + 64;
+  *count = 2 * L.n_vt + 64;
 }
 
 cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, const void* h,
@@ -698,9 +740,10 @@ cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, 
   prm.P = reinterpret_cast<__nv_bfloat16*>(base + L.P);
   unsigned* ctr = reinterpret_cast<unsigned*>(base + L.counters);
   prm.ready = ctr;
-  prm.consumed = ctr + L.n_ranges;
-  prm.abort_flag = reinterpret_cast<int*>(ctr + 2 * L.n_ranges);
+  prm.consumed = ctr + L.n_vt;
+  prm.abort_flag = reinterpret_cast<int*>(ctr + 2 * L.n_vt);
   prm.st = st;
+  prm.trace = reinterpret_cast<unsigned long long*>(base + L.trace);
   const CUtensorMap* maps = reinterpret_cast<const CUtensorMap*>(pl.maps);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(L.n1 + L.n2);
