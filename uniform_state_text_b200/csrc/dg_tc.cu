@@ -45,15 +45,18 @@ namespace tc {
 constexpr int BM = 128;        // canvas rows per CTA (MMA M)
 constexpr int BN = 256;        // MMA N: vocabulary entries (G1) or columns of d (G2)
 constexpr int BK = 64;         // K per pipeline stage (one 128-byte swizzle row of bf16)
-constexpr int STAGES = 4;
 constexpr int KV2 = 1024;      // vocabulary entries per range (unit of G2 ownership)
 constexpr int RING = 64;       // P tiles (256 vocabulary entries each) resident at once
 constexpr int THREADS = 192;
 constexpr int RSPLIT = 16;     // vocabulary splits of the fix-up kernels
 constexpr uint32_t A_BYTES = BM * BK * 2;
 constexpr uint32_t B_BYTES = BN * BK * 2;
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+// Pipeline depth per CTA-group size: the same ~192 KB of stages either way.
+template <int CG> struct Pipe {
+  static constexpr int STAGES = CG == 2 ? 6 : 4;
+  static constexpr uint32_t STAGE = A_BYTES + B_BYTES / CG;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 256;
+};
 constexpr unsigned long long TIMEOUT_NS = 2000000000ull;   // 2 s
 
 struct Params {
@@ -229,60 +232,145 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 }
 
 // ---------------------------------------------------------------------------
-// The persistent kernel.
+// CTA-pair helpers (CG = 2: two CTAs of a cluster share one MMA of M = 256).
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+}
+// Address of the same shared variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+// TMA load whose completion is counted on the pair leader's barrier.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar) & 0xFEFFFFFFu), "r"(x), "r"(y)
+      : "memory");
+}
+template <int CG>
+__device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                         int y) {
+  if constexpr (CG == 2) tma_load_2d_pair(dst, map, bar, x, y);
+  else tma_load_2d(dst, map, bar, x, y);
+}
+template <int CG>
+__device__ __forceinline__ void mma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                    uint32_t accumulate) {
+  if constexpr (CG == 2) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    mma_bf16(d_tmem, a, b, idesc, accumulate);
+  }
+}
+// Arrive on `bar` in every CTA of the group once this thread's MMAs complete.
+template <int CG>
+__device__ __forceinline__ void commit(uint64_t* bar) {
+  if constexpr (CG == 2) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(smem_u32(bar)), "h"((uint16_t)3)
+        : "memory");
+  } else {
+    mma_commit(bar);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The persistent kernel. CG = 1: one CTA per MMA (M = 128 rows).
+// CG = 2: CTA pairs, M = 256 rows (both row blocks), each CTA stages its own
+// 128 rows of A and half of B; the pair leader (rank 0) issues the MMAs.
+// ---------------------------------------------------------------------------
+template <int CG>
 __global__ void __launch_bounds__(THREADS, 1)
     k_vocab_attention(const __grid_constant__ CUtensorMap tm_h,
                       const __grid_constant__ CUtensorMap tm_ek,
                       const __grid_constant__ CUtensorMap tm_emn,
                       const __grid_constant__ CUtensorMap tm_p, const Params p) {
-  if (p.st->done) return;
+  constexpr int STAGES = Pipe<CG>::STAGES;
+  constexpr uint32_t STAGE_CTA = Pipe<CG>::STAGE;       // A + this CTA's share of B
+  constexpr uint32_t STAGE_BYTES = STAGE_CTA;
+  constexpr int NB_ROWS = BN / CG;                      // B rows (G1) / columns (G2) per CTA
+  if (p.st->done) return;                               // uniform over the grid
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  uint64_t* full = bars;                 // [STAGES]
-  uint64_t* empty = bars + STAGES;       // [STAGES]
+  uint64_t* full = bars;                    // [STAGES] (leader's counts both CTAs' bytes)
+  uint64_t* empty = bars + STAGES;          // [STAGES]
   uint64_t* acc_full = bars + 2 * STAGES;   // [2]
-  uint64_t* acc_empty = acc_full + 2;       // [2]
+  uint64_t* acc_empty = acc_full + 2;       // [2] (leader's counts both CTAs' epilogues)
   uint64_t* fin = acc_empty + 2;            // [1]
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(fin + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool is_g1 = (int)blockIdx.x < p.n1;
+  const uint32_t rank = CG == 2 ? cluster_rank() : 0u;
+  const bool leader = rank == 0;
+  const int unit = blockIdx.x / CG;                    // pair (or CTA) index
+  const bool is_g1 = unit < p.n1;
   if (threadIdx.x == 0) TRACE_SET(0, gtimer());
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 4); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 4 * CG); }
     mbar_init(fin, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::
-                     "r"(smem_u32(tmem_base_slot)), "r"(512)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if constexpr (CG == 2) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::
+                       "r"(smem_u32(tmem_base_slot)), "r"(512)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::
+                       "r"(smem_u32(tmem_base_slot)), "r"(512)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (CG == 2) cluster_sync();   // peer barriers initialised before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_base_slot;
 
-  // Work description.
-  const int n_items1 = p.RB * p.n_vt;
-  const int nk1 = p.d / BK;               // K stages per G1 item
-  const int nk2 = KV2 / BK;               // K stages per G2 range
-  int o = 0, g = 0, rb2 = 0, dt = 0;
+  // Work description. RB: row blocks per MMA group is 1 for CG = 2 (the pair
+  // covers both), p.RB for CG = 1 (items iterate over row blocks).
+  const int RBI = CG == 2 ? 1 : p.RB;
+  const int n_items1 = RBI * p.n_vt;
+  const int nk1 = p.d / BK;
+  const int nk2 = KV2 / BK;
+  int g = 0, rb2 = 0, dt = 0;
   if (!is_g1) {
-    o = blockIdx.x - p.n1;
-    g = o / (p.RB * p.n_dt);
-    const int rem = o % (p.RB * p.n_dt);
-    rb2 = rem / p.n_dt;
+    const int o = unit - p.n1;
+    g = o / (RBI * p.n_dt);
+    const int rem = o % (RBI * p.n_dt);
+    rb2 = CG == 2 ? (int)rank : rem / p.n_dt;
     dt = rem % p.n_dt;
   }
   const unsigned ready_target = (unsigned)(p.RB * 4);
-  const unsigned consumed_target = (unsigned)(p.RB * p.n_dt);
+  const unsigned consumed_target = (unsigned)(RBI * p.n_dt);
+  bool aborted = false;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -292,8 +380,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       long issued = 0;
       bool ok = true;
       if (is_g1) {
-        for (int it = blockIdx.x; ok && it < n_items1; it += p.n1) {
-          const int vt = it / p.RB, rb = it % p.RB;
+        for (int it = unit; ok && it < n_items1; it += p.n1) {
+          const int vt = it / RBI;
+          const int rb = CG == 2 ? (int)rank : it % RBI;
           {
             TRACE_T0();
             if (vt >= RING && !counter_wait(&p.consumed[vt - RING], consumed_target, p)) { ok = false; break; }
@@ -304,9 +393,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (!mbar_wait(&empty[s], ph ^ 1, p)) { ok = false; break; }
             TRACE_ADD(2);
             unsigned char* st = smem + s * STAGE_BYTES;
-            mbar_expect_tx(&full[s], STAGE_BYTES);
-            tma_load_2d(st, &tm_h, &full[s], kc * BK, rb * BM);
-            tma_load_2d(st + A_BYTES, &tm_ek, &full[s], kc * BK, vt * BN);
+            if (leader) mbar_expect_tx(&full[s], STAGE_CTA * CG);
+            tma_load<CG>(st, &tm_h, &full[s], kc * BK, rb * BM);
+            tma_load<CG>(st + A_BYTES, &tm_ek, &full[s], kc * BK, vt * BN + (int)rank * NB_ROWS);
             ++issued;
             if (++s == STAGES) { s = 0; ph ^= 1; }
           }
@@ -325,35 +414,36 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (!mbar_wait(&empty[s], ph ^ 1, p)) { ok = false; break; }
             TRACE_ADD(2);
             unsigned char* st = smem + s * STAGE_BYTES;
-            mbar_expect_tx(&full[s], STAGE_BYTES);
-            tma_load_2d(st, &tm_p, &full[s], (kc % (BN / BK)) * BK, (vt % RING) * p.C + rb2 * BM);
+            if (leader) mbar_expect_tx(&full[s], STAGE_CTA * CG);
+            tma_load<CG>(st, &tm_p, &full[s], (kc % (BN / BK)) * BK, (vt % RING) * p.C + rb2 * BM);
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j)
-              tma_load_2d(st + A_BYTES + j * (64 * BK * 2), &tm_emn, &full[s], dt * BN + j * 64,
-                          r * KV2 + kc * BK);
+            for (int j = 0; j < NB_ROWS / 64; ++j)
+              tma_load<CG>(st + A_BYTES + j * (64 * BK * 2), &tm_emn, &full[s],
+                           dt * BN + (int)rank * NB_ROWS + j * 64, r * KV2 + kc * BK);
             ++issued;
             if (++s == STAGES) { s = 0; ph ^= 1; }
           }
         }
       }
-      // Drain: every issued copy must land before the CTA can exit.
-      for (long k = (issued > STAGES ? issued - STAGES : 0); k < issued; ++k) {
-        const int ss = (int)(k % STAGES);
-        const uint32_t pp = (uint32_t)((k / STAGES) & 1);
-        mbar_wait(&full[ss], pp, p, false);
+      aborted = !ok;
+      if (CG == 1 || leader) {
+        // Drain: every issued copy must land before the CTA can exit.
+        for (long k = (issued > STAGES ? issued - STAGES : 0); k < issued; ++k)
+          mbar_wait(&full[(int)(k % STAGES)], (uint32_t)((k / STAGES) & 1), p, false);
+      } else if (aborted) {
+        __nanosleep(100000);   // the peer's copies complete on the leader's barrier
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      bool issued_any = false;
       if (is_g1) {
-        const uint32_t idesc = idesc_bf16(BM, BN, 0);
+        const uint32_t idesc = idesc_bf16(BM * CG, BN, 0);
         int n = 0;
-        for (int it = blockIdx.x; ok && it < n_items1; it += p.n1, ++n) {
+        for (int it = unit; ok && it < n_items1; it += p.n1, ++n) {
           const int buf = n & 1;
           {
             TRACE_T0();
@@ -373,17 +463,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int k = 0; k < BK / 16; ++k) {
               const uint64_t ad = sdesc(a0 + k * 32, 16, 1024);
               const uint64_t bd = sdesc(b0 + k * 32, 16, 1024);
-              mma_bf16(d_tmem, ad, bd, idesc, (kc | k) ? 1u : 0u);
+              mma<CG>(d_tmem, ad, bd, idesc, (kc | k) ? 1u : 0u);
             }
-            issued_any = true;
-            mma_commit(&empty[s]);
+            commit<CG>(&empty[s]);
             if (++s == STAGES) { s = 0; ph ^= 1; }
           }
           if (!ok) break;
-          mma_commit(&acc_full[buf]);
+          commit<CG>(&acc_full[buf]);
         }
       } else {
-        const uint32_t idesc = idesc_bf16(BM, BN, 1);
+        const uint32_t idesc = idesc_bf16(BM * CG, BN, 1);
         bool first = true;
         for (int r = g; ok && r < p.n_ranges; r += p.G) {
           for (int kc = 0; kc < nk2; ++kc) {
@@ -400,32 +489,33 @@ __global__ void __launch_bounds__(THREADS, 1)
               const uint64_t ad = sdesc(a0 + k * 32, 16, 1024);
               // MN-major B: 64-column blocks 8 KB apart (LBO), 8-row K groups 1 KB apart (SBO)
               const uint64_t bd = sdesc(b0 + k * (16 * 128), 64 * BK * 2, 1024);
-              mma_bf16(tmem, ad, bd, idesc, first ? 0u : 1u);
+              mma<CG>(tmem, ad, bd, idesc, first ? 0u : 1u);
               first = false;
             }
-            issued_any = true;
-            mma_commit(&empty[s]);
+            commit<CG>(&empty[s]);
             if (++s == STAGES) { s = 0; ph ^= 1; }
           }
         }
-        if (ok) mma_commit(&acc_full[0]);
+        if (ok) commit<CG>(&acc_full[0]);
       }
-      // All MMAs this thread issued must finish before TMEM is released.
-      if (issued_any) {
-        mma_commit(fin);
-        mbar_wait(fin, 0, p, false);
-      }
+      // Every MMA this thread issued completes before TMEM is released (in both CTAs).
+      commit<CG>(fin);
     }
+    if (lane == 0) mbar_wait(fin, 0, p, false);
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                 // TMEM lane quarter of this warp
     const int r_local = q * 32 + lane;      // row within the CTA's 128
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    // Where this warp reports that it has read an accumulator buffer.
+    const uint32_t acc_empty_leader = CG == 2 ? mapa(smem_u32(acc_empty), 0) : smem_u32(acc_empty);
     if (is_g1) {
       const float scale = p.scale_tab[min(max(p.st->t, 0), p.S - 1)];
       int n = 0;
-      for (int it = blockIdx.x; it < n_items1; it += p.n1, ++n) {
-        const int vt = it / p.RB, rb = it % p.RB;
+      for (int it = unit; it < n_items1; it += p.n1, ++n) {
+        const int vt = it / RBI;
+        const int rb = CG == 2 ? (int)rank : it % RBI;
         const int buf = n & 1;
         {
           TRACE_T0();
@@ -463,13 +553,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         // This warp is done reading the accumulator buffer.
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        if (lane == 0) {
+          if (CG == 2) mbar_arrive_remote(acc_empty_leader + buf * 8);
+          else mbar_arrive(&acc_empty[buf]);
+        }
         TileStat ts;
         ts.m = mref; ts.Z = Z; ts.S1 = S1; ts.best = best; ts.arg = arg;
         ts.pad[0] = ts.pad[1] = ts.pad[2] = 0;
         p.tstats[(size_t)row * p.n_vt + vt] = ts;
-        // Publish this warp's rows of the P tile: generic-proxy stores, read later by
-        // TMA on other SMs. Each of the 4 epilogue warps counts once per item.
+        // Publish this warp's rows of the P tile: generic-proxy stores, read later
+        // by TMA on other SMs. Each epilogue warp counts once per tile.
         fence_proxy_async_global();
         __syncwarp();
         if (lane == 0) {
@@ -504,13 +597,19 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
     }
   }
+  (void)aborted;
 
   __syncthreads();
+  if constexpr (CG == 2) cluster_sync();    // no remote arrivals after this point
   if (threadIdx.x == 0) TRACE_SET(1, gtimer());
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
-                 : "memory");
+    if constexpr (CG == 2)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
+                   : "memory");
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
+                   : "memory");
   }
 }
 
@@ -589,7 +688,8 @@ namespace {
 
 struct TcLayout {
   size_t counters = 0, P = 0, Opart = 0, redo = 0, trace = 0, total = 0;
-  int RB = 0, n_vt = 0, n_ranges = 0, n_dt = 0, G = 0, n1 = 0, n2 = 0;
+  int CG = 1;              // CTAs per MMA group (2: CTA pairs, M = 256)
+  int RB = 0, n_vt = 0, n_ranges = 0, n_dt = 0, G = 0, n1 = 0, n2 = 0;   // n1, n2 in groups
 };
 
 size_t al(size_t x) { return (x + 255) / 256 * 256; }
@@ -605,20 +705,23 @@ int device_sms() {
 
 TcLayout tc_layout(int C, int V, int d, int sms) {
   TcLayout L;
+  L.CG = C == 256 ? 2 : 1;
   L.RB = C / tc::BM;
   L.n_vt = V / tc::BN;
   L.n_ranges = V / tc::KV2;
   L.n_dt = d / tc::BN;
-  // Choose the number of range groups G: G2 CTAs = RB * n_dt * G, G1 CTAs take
-  // the rest; minimise the larger of the two roles' per-CTA work.
+  // Choose the number of range groups G: G2 units = RBI * n_dt * G, G1 units take
+  // the rest; minimise the larger of the two roles' per-unit work.
+  const int units = sms / L.CG;
+  const int RBI = L.CG == 2 ? 1 : L.RB;
   const double u1 = (double)tc::BM * tc::BN * d;                 // one G1 item
   const double u2 = (double)tc::BM * tc::BN * tc::KV2;           // one G2 range
-  const int per_g = L.RB * L.n_dt;
+  const int per_g = RBI * L.n_dt;
   double best = 1e300;
   for (int G = 1; G <= L.n_ranges; ++G) {
     const int n2 = per_g * G;
-    const int items = L.RB * L.n_vt;
-    int n1 = sms - n2;
+    const int items = RBI * L.n_vt;
+    int n1 = units - n2;
     if (n1 < 1) break;
     if (n1 > items) n1 = items;
     const double t1 = std::ceil((double)items / n1) * u1;
@@ -678,6 +781,66 @@ size_t tc_workspace_bytes(int C, int V, int d) { return tc_layout(C, V, d, devic
 
 int tc_launches(const TcPlan&) { return 3; }
 
+template <int CG>
+cudaError_t launch_kernel(cudaStream_t s, int units, const CUtensorMap* maps, const tc::Params& prm) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(units * CG);
+  cfg.blockDim = dim3(tc::THREADS);
+  cfg.dynamicSmemBytes = tc::Pipe<CG>::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (CG == 2) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+  } else {
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc::k_vocab_attention<CG>, maps[0], maps[1], maps[2], maps[3], prm);
+}
+
+// Every unit of the persistent grid must be resident at once (they wait on one another).
+template <int CG>
+int check_residency(int units, int sms, char* err, size_t errn) {
+  cudaError_t e = cudaFuncSetAttribute(tc::k_vocab_attention<CG>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)tc::Pipe<CG>::SMEM);
+  if (e != cudaSuccess) {
+    snprintf(err, errn, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    return -3;
+  }
+  int fit = 0;
+  if (CG == 2) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(units * CG);
+    cfg.blockDim = dim3(tc::THREADS);
+    cfg.dynamicSmemBytes = tc::Pipe<CG>::SMEM;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaOccupancyMaxActiveClusters(&fit, tc::k_vocab_attention<CG>, &cfg);
+  } else {
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tc::k_vocab_attention<CG>,
+                                                      tc::THREADS, tc::Pipe<CG>::SMEM);
+    fit = per_sm * sms;
+  }
+  if (e != cudaSuccess || fit < units) {
+    if (e != cudaSuccess) cudaGetLastError();
+    snprintf(err, errn, "tensor-core kernel cannot be co-resident (%d of %d units fit)", fit, units);
+    return -5;
+  }
+  return 0;
+}
+
 int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, float* O,
                  TileStat* tstats, void* ws, char* err, size_t errn) {
   (void)O;
@@ -691,28 +854,16 @@ int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, float* 
   static_assert(sizeof(CUtensorMap) <= 128, "tensor map size");
   CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(p->maps);
   bool ok = encode(&maps[0], h, (uint64_t)d, (uint64_t)C, tc::BK, tc::BM) &&
-            encode(&maps[1], E, (uint64_t)d, (uint64_t)V, tc::BK, tc::BN) &&
+            encode(&maps[1], E, (uint64_t)d, (uint64_t)V, tc::BK, tc::BN / L.CG) &&
             encode(&maps[2], E, (uint64_t)d, (uint64_t)V, tc::BK, 64) &&
             encode(&maps[3], base + L.P, (uint64_t)tc::BN, (uint64_t)tc::RING * C, tc::BK, tc::BM);
   if (!ok) {
     snprintf(err, errn, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
     return -3;
   }
-  cudaError_t e = cudaFuncSetAttribute(tc::k_vocab_attention,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)tc::SMEM_BYTES);
-  if (e != cudaSuccess) {
-    snprintf(err, errn, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    return -3;
-  }
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tc::k_vocab_attention, tc::THREADS,
-                                                    tc::SMEM_BYTES);
-  if (e != cudaSuccess || per_sm < 1 || p->grid > per_sm * p->num_sms) {
-    snprintf(err, errn, "tensor-core kernel cannot be co-resident (%d per SM, grid %d)", per_sm,
-             p->grid);
-    return -5;
-  }
+  const int rc = L.CG == 2 ? check_residency<2>(p->grid, p->num_sms, err, errn)
+                           : check_residency<1>(p->grid, p->num_sms, err, errn);
+  if (rc) return rc;
   p->ready = true;
   return 0;
 }
@@ -745,17 +896,8 @@ cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, 
   prm.st = st;
   prm.trace = reinterpret_cast<unsigned long long*>(base + L.trace);
   const CUtensorMap* maps = reinterpret_cast<const CUtensorMap*>(pl.maps);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(L.n1 + L.n2);
-  cfg.blockDim = dim3(tc::THREADS);
-  cfg.dynamicSmemBytes = tc::SMEM_BYTES;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, tc::k_vocab_attention, maps[0], maps[1], maps[2], maps[3], prm);
+  return L.CG == 2 ? launch_kernel<2>(s, L.n1 + L.n2, maps, prm)
+                   : launch_kernel<1>(s, L.n1 + L.n2, maps, prm);
 }
 
 void tc_partials(const TcPlan& pl, const float** Opart, int* nO) {
