@@ -116,7 +116,6 @@ int make_layout(const dg_config* c, Layout* L, char* why, size_t n) {
   } else {
     L->ntiles = tc_stat_tiles(c->C, c->V, c->d);
     L->tstats = take(sizeof(TileStat) * C * L->ntiles);
-    L->O = take(4 * C * d);
     L->tc_bytes = tc_workspace_bytes(c->C, c->V, c->d);
     L->tc = take(L->tc_bytes);
   }
@@ -207,11 +206,8 @@ int launch_step(dg_ctx* ctx, bool standin, bool use_cond) {
   if (tc) {
     DG_CK(launch_tc_attention(s, ctx->tc_plan, ctx->st, ctx->h, ctx->E, ctx->mref, ctx->scale_tab,
                               c.max_steps, ctx->tstats, ctx->O, ctx->tc));
-    const float* Opart = nullptr;
-    int nO = 0;
-    tc_partials(ctx->tc_plan, &Opart, &nO);
-    DG_CK(launch_merge(s, ctx->st, ctx->tstats, ctx->L.ntiles, ctx->rowstat, ctx->H, ctx->argmax,
-                       c.C, Opart, nO, ctx->mref, ctx->sc, c.d, ctx->redo_rows, kRedoGap));
+    DG_CK(launch_tc_merge(s, ctx->tc_plan, ctx->st, ctx->tstats, ctx->mref, ctx->rowstat, ctx->H,
+                          ctx->argmax, ctx->sc, ctx->redo_rows, kRedoGap));
     DG_CK(launch_tc_redo(s, ctx->tc_plan, ctx->st, ctx->h, ctx->E, ctx->scale_tab, c.max_steps,
                          ctx->rowstat, ctx->redo_rows, ctx->H, ctx->sc));
   } else {

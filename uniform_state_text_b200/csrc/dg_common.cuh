@@ -72,6 +72,14 @@ struct TileStat {
   int32_t pad[3];
 };
 
+// Tensor-core path: per-(row, half tile) statistics, all taken against the
+// row's logit reference m_ref: Z = sum e^(z - m_ref), S1 = sum e^(z - m_ref)
+// (z - m_ref), and the best logit with its vocabulary index.
+struct TcStat {
+  float Z, S1, best;
+  int32_t arg;
+};
+
 // Per-row merged statistics used by the sampler and the sc normalisation.
 struct RowStat {
   float m;      // reference the partition sum is taken against

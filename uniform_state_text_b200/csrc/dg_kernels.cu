@@ -342,6 +342,7 @@ __global__ void __launch_bounds__(1024) k_sampler(DevState* st, const float* H,
     int stop_unchanged, int stop_rule, int accept_rule, int fixed_steps, int S,
     cudaGraphConditionalHandle cond, int use_cond) {
   __shared__ float sH[1024];
+  __shared__ float sSorted[1024];
   __shared__ int32_t sOrder[1024];
   __shared__ int sk;
   const int i = threadIdx.x;
@@ -362,21 +363,33 @@ __global__ void __launch_bounds__(1024) k_sampler(DevState* st, const float* H,
       rank += (Hj < Hi) || (Hj == Hi && j < i);
     }
     sOrder[rank] = i;
+    sSorted[rank] = Hi;
   }
   __syncthreads();
-  // Sequential fp32 running sums in sorted order (a fixed summation order).
-  if (i == 0) {
+  // Running entropy sums in sorted order, added one at a time in fp32 (a fixed
+  // summation order): warp 0 holds the sorted entropies, lane l the entries
+  // [l*per, (l+1)*per), and passes the running sum from lane to lane.
+  if (i < 32) {
+    const int per = (C + 31) / 32;
     float run = 0.f;
     int k = 0;
-    bool stopped = false;
-    for (int j = 0; j < C; ++j) {
-      const float before = run;
-      run = __fadd_rn(run, sH[sOrder[j]]);
-      prefix[j] = run;
-      const bool ok = accept_rule == 0 ? (run <= tau) : (before <= tau);
-      if (ok && !stopped) ++k; else stopped = true;
+    for (int src = 0; src < 32; ++src) {
+      if (i == src) {
+        for (int e = 0; e < per; ++e) {
+          const int j = src * per + e;
+          if (j >= C) break;
+          const float before = run;
+          run = __fadd_rn(run, sSorted[j]);
+          prefix[j] = run;
+          // prefix sums of non-negative terms never decrease, so the accepted
+          // positions are a prefix of the sorted order
+          k += (accept_rule == 0 ? (run <= tau) : (before <= tau)) ? 1 : 0;
+        }
+      }
+      run = __shfl_sync(0xffffffffu, run, src);
     }
-    sk = k;
+    for (int o = 16; o; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
+    if (i == 0) sk = k;
   }
   __syncthreads();
   const int k = sk;

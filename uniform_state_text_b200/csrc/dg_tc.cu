@@ -45,9 +45,12 @@ namespace tc {
 constexpr int BM = 128;        // canvas rows per CTA (MMA M)
 constexpr int BN = 256;        // MMA N: vocabulary entries (G1) or columns of d (G2)
 constexpr int BK = 64;         // K per pipeline stage (one 128-byte swizzle row of bf16)
-constexpr int KV2 = 1024;      // vocabulary entries per range (unit of G2 ownership)
-constexpr int RING = 64;       // P tiles (256 vocabulary entries each) resident at once
-constexpr int THREADS = 192;
+constexpr int KV2 = 256;       // vocabulary entries per range (unit of G2 ownership): one tile,
+                               // so range group g owns tiles g, g+G, ... and all groups
+                               // advance through the ring together
+constexpr int RING = 96;       // P tiles (256 vocabulary entries each) resident at once
+constexpr int THREADS = 320;    // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+constexpr int EPI_WARPS = 8;
 constexpr int RSPLIT = 16;     // vocabulary splits of the fix-up kernels
 constexpr uint32_t A_BYTES = BM * BK * 2;
 constexpr uint32_t B_BYTES = BN * BK * 2;
@@ -63,7 +66,6 @@ struct Params {
   int C, V, d, RB, n_vt, n_ranges, n_dt, G, n1, tiles_per_range, S;
   const float* mref;
   const float* scale_tab;
-  TileStat* tstats;
   float* Opart;              // [G][C][d]
   __nv_bfloat16* P;          // [RING][C][BN]: ring of P tiles
   unsigned* ready;           // [n_vt]: epilogue warps that finished a tile
@@ -71,20 +73,24 @@ struct Params {
   int* abort_flag;
   DevState* st;
   unsigned long long* trace;   // [grid][32] wait-time counters (DG_TC_TRACE builds only)
+  TcStat* tstats2;             // [C][2 * n_vt] half-tile statistics
 };
 
 // Per-CTA wait-time tracing, compiled in only with -DDG_TC_TRACE (measurement
-// builds); slots: 0 start, 1 end, 2 producer waits on empty stages, 3 producer
-// waits on counters, 4 MMA waits on full stages, 5 MMA waits on free
-// accumulators, 6 epilogue waits on full accumulators, 7 items, 8 epilogue busy.
+// builds). Each role accumulates in registers and stores once at its end.
+// Slots: 0 start, 1 end, 2 producer waits on free stages, 3 producer waits on
+// counters, 4 MMA waits on full stages, 5 MMA waits on free accumulators,
+// 6 epilogue waits on full accumulators, 7 items, 8 epilogue busy.
 #ifdef DG_TC_TRACE
-#define TRACE_T0() const unsigned long long tr_t0_ = gtimer()
-#define TRACE_ADD(slot) (p.trace[blockIdx.x * 32 + (slot)] += gtimer() - tr_t0_)
-#define TRACE_SET(slot, v) (p.trace[blockIdx.x * 32 + (slot)] = (v))
+#define TR_DECL(v) unsigned long long v = 0
+#define TR_T0() const unsigned long long tr_t0_ = gtimer()
+#define TR_ADD(v) (v += gtimer() - tr_t0_)
+#define TR_STORE(slot, v) (p.trace[blockIdx.x * 32 + (slot)] = (v))
 #else
-#define TRACE_T0() ((void)0)
-#define TRACE_ADD(slot) ((void)0)
-#define TRACE_SET(slot, v) ((void)0)
+#define TR_DECL(v) ((void)0)
+#define TR_T0() ((void)0)
+#define TR_ADD(v) ((void)0)
+#define TR_STORE(slot, v) ((void)0)
 #endif
 
 // ---------------------------------------------------------------------------
@@ -148,6 +154,11 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* ptr) {
 }
 __device__ __forceinline__ void red_release_add(unsigned* ptr, unsigned v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+// Relaxed add: for counters whose only meaning is "my reads of this data have
+// completed" (the reads finished before the add is issued), no release needed.
+__device__ __forceinline__ void red_relaxed_add(unsigned* ptr, unsigned v) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
@@ -300,6 +311,12 @@ __device__ __forceinline__ void commit(uint64_t* bar) {
 // CG = 2: CTA pairs, M = 256 rows (both row blocks), each CTA stages its own
 // 128 rows of A and half of B; the pair leader (rank 0) issues the MMAs.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <int CG>
 __global__ void __launch_bounds__(THREADS, 1)
     k_vocab_attention(const __grid_constant__ CUtensorMap tm_h,
@@ -307,9 +324,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                       const __grid_constant__ CUtensorMap tm_emn,
                       const __grid_constant__ CUtensorMap tm_p, const Params p) {
   constexpr int STAGES = Pipe<CG>::STAGES;
-  constexpr uint32_t STAGE_CTA = Pipe<CG>::STAGE;       // A + this CTA's share of B
-  constexpr uint32_t STAGE_BYTES = STAGE_CTA;
+  constexpr uint32_t STAGE_BYTES = Pipe<CG>::STAGE;     // A + this CTA's share of B
   constexpr int NB_ROWS = BN / CG;                      // B rows (G1) / columns (G2) per CTA
+  constexpr int HALF = BN / 2;                          // columns per epilogue warp
   if (p.st->done) return;                               // uniform over the grid
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
@@ -327,11 +344,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   const bool leader = rank == 0;
   const int unit = blockIdx.x / CG;                    // pair (or CTA) index
   const bool is_g1 = unit < p.n1;
-  if (threadIdx.x == 0) TRACE_SET(0, gtimer());
+  if (threadIdx.x == 0) TR_STORE(0, gtimer());
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 4 * CG); }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], EPI_WARPS * CG);
+    }
     mbar_init(fin, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -354,8 +374,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_base_slot;
 
-  // Work description. RB: row blocks per MMA group is 1 for CG = 2 (the pair
-  // covers both), p.RB for CG = 1 (items iterate over row blocks).
+  // Work description. RBI: row blocks iterated by G1 items (1 for pairs, which
+  // cover both row blocks with M = 256).
   const int RBI = CG == 2 ? 1 : p.RB;
   const int n_items1 = RBI * p.n_vt;
   const int nk1 = p.d / BK;
@@ -368,13 +388,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     rb2 = CG == 2 ? (int)rank : rem / p.n_dt;
     dt = rem % p.n_dt;
   }
-  const unsigned ready_target = (unsigned)(p.RB * 4);
+  const unsigned ready_target = (unsigned)(p.RB * EPI_WARPS);
   const unsigned consumed_target = (unsigned)(RBI * p.n_dt);
-  bool aborted = false;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      TR_DECL(w_empty);
+      TR_DECL(w_ctr);
       int s = 0;
       uint32_t ph = 0;
       long issued = 0;
@@ -383,17 +404,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int it = unit; ok && it < n_items1; it += p.n1) {
           const int vt = it / RBI;
           const int rb = CG == 2 ? (int)rank : it % RBI;
-          {
-            TRACE_T0();
-            if (vt >= RING && !counter_wait(&p.consumed[vt - RING], consumed_target, p)) { ok = false; break; }
-            TRACE_ADD(3);
+          if (vt >= RING) {
+            TR_T0();
+            if (!counter_wait(&p.consumed[vt - RING], consumed_target, p)) { ok = false; break; }
+            TR_ADD(w_ctr);
           }
           for (int kc = 0; kc < nk1; ++kc) {
-            TRACE_T0();
+            TR_T0();
             if (!mbar_wait(&empty[s], ph ^ 1, p)) { ok = false; break; }
-            TRACE_ADD(2);
+            TR_ADD(w_empty);
             unsigned char* st = smem + s * STAGE_BYTES;
-            if (leader) mbar_expect_tx(&full[s], STAGE_CTA * CG);
+            if (leader) mbar_expect_tx(&full[s], STAGE_BYTES * CG);
             tma_load<CG>(st, &tm_h, &full[s], kc * BK, rb * BM);
             tma_load<CG>(st + A_BYTES, &tm_ek, &full[s], kc * BK, vt * BN + (int)rank * NB_ROWS);
             ++issued;
@@ -405,16 +426,16 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int kc = 0; kc < nk2; ++kc) {
             const int vt = r * p.tiles_per_range + kc / (BN / BK);
             if (kc % (BN / BK) == 0) {
-              TRACE_T0();
+              TR_T0();
               if (!counter_wait(&p.ready[vt], ready_target, p)) { ok = false; break; }
-              TRACE_ADD(3);
+              TR_ADD(w_ctr);
               fence_proxy_async_global();
             }
-            TRACE_T0();
+            TR_T0();
             if (!mbar_wait(&empty[s], ph ^ 1, p)) { ok = false; break; }
-            TRACE_ADD(2);
+            TR_ADD(w_empty);
             unsigned char* st = smem + s * STAGE_BYTES;
-            if (leader) mbar_expect_tx(&full[s], STAGE_CTA * CG);
+            if (leader) mbar_expect_tx(&full[s], STAGE_BYTES * CG);
             tma_load<CG>(st, &tm_p, &full[s], (kc % (BN / BK)) * BK, (vt % RING) * p.C + rb2 * BM);
 #pragma unroll
             for (int j = 0; j < NB_ROWS / 64; ++j)
@@ -425,18 +446,21 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
-      aborted = !ok;
       if (CG == 1 || leader) {
         // Drain: every issued copy must land before the CTA can exit.
         for (long k = (issued > STAGES ? issued - STAGES : 0); k < issued; ++k)
           mbar_wait(&full[(int)(k % STAGES)], (uint32_t)((k / STAGES) & 1), p, false);
-      } else if (aborted) {
+      } else if (!ok) {
         __nanosleep(100000);   // the peer's copies complete on the leader's barrier
       }
+      TR_STORE(2, w_empty);
+      TR_STORE(3, w_ctr);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && leader) {
+      TR_DECL(w_full);
+      TR_DECL(w_acc);
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -446,16 +470,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int it = unit; ok && it < n_items1; it += p.n1, ++n) {
           const int buf = n & 1;
           {
-            TRACE_T0();
+            TR_T0();
             if (!mbar_wait(&acc_empty[buf], ((n >> 1) & 1) ^ 1, p)) { ok = false; break; }
-            TRACE_ADD(5);
+            TR_ADD(w_acc);
           }
           tc_fence_after();
           const uint32_t d_tmem = tmem + buf * BN;
           for (int kc = 0; kc < nk1; ++kc) {
-            TRACE_T0();
+            TR_T0();
             if (!mbar_wait(&full[s], ph, p)) { ok = false; break; }
-            TRACE_ADD(4);
+            TR_ADD(w_full);
             tc_fence_after();
             const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
             const uint32_t b0 = a0 + A_BYTES;
@@ -476,12 +500,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         bool first = true;
         for (int r = g; ok && r < p.n_ranges; r += p.G) {
           for (int kc = 0; kc < nk2; ++kc) {
-            TRACE_T0();
+            TR_T0();
             if (!mbar_wait(&full[s], ph, p)) { ok = false; break; }
-            TRACE_ADD(4);
+            TR_ADD(w_full);
             tc_fence_after();
             if (kc % (BN / BK) == BN / BK - 1)      // the tile's P is now in shared memory
-              red_release_add(&p.consumed[r * p.tiles_per_range + kc / (BN / BK)], 1u);
+              red_relaxed_add(&p.consumed[r * p.tiles_per_range + kc / (BN / BK)], 1u);
             const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
             const uint32_t b0 = a0 + A_BYTES;
 #pragma unroll
@@ -500,49 +524,66 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       // Every MMA this thread issued completes before TMEM is released (in both CTAs).
       commit<CG>(fin);
+      TR_STORE(4, w_full);
+      TR_STORE(5, w_acc);
     }
     if (lane == 0) mbar_wait(fin, 0, p, false);
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;                 // TMEM lane quarter of this warp
+    // Warps 2..9: TMEM lane quarter (warp % 4), column half ((warp - 2) / 4).
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int r_local = q * 32 + lane;      // row within the CTA's 128
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    const int c0 = half * HALF;             // first column of this warp
     // Where this warp reports that it has read an accumulator buffer.
     const uint32_t acc_empty_leader = CG == 2 ? mapa(smem_u32(acc_empty), 0) : smem_u32(acc_empty);
+    TR_DECL(w_acc);
+    TR_DECL(busy);
     if (is_g1) {
       const float scale = p.scale_tab[min(max(p.st->t, 0), p.S - 1)];
+      const float k1 = scale * 1.4426950408889634f;           // logit scale in log2 units
       int n = 0;
       for (int it = unit; it < n_items1; it += p.n1, ++n) {
         const int vt = it / RBI;
         const int rb = CG == 2 ? (int)rank : it % RBI;
         const int buf = n & 1;
         {
-          TRACE_T0();
+          TR_T0();
           if (!mbar_wait(&acc_full[buf], (n >> 1) & 1, p)) break;
-          if (threadIdx.x == 64) TRACE_ADD(6);
+          TR_ADD(w_acc);
         }
-        TRACE_T0();
+        TR_T0();
         tc_fence_after();
         const int row = rb * BM + r_local;
         const float mref = p.mref[row];
-        float Z = 0.f, S1 = 0.f, best = -INFINITY;
+        const float k0 = -mref * 1.4426950408889634f;
+        // P = 2^(k1 v + k0) = e^(z - mref); Z = sum P; S2 = sum P (z - mref) log2(e).
+        float Z = 0.f, S2 = 0.f, vbest = -INFINITY;
         int arg = 0x7fffffff;
-        __nv_bfloat16* prow = p.P + ((size_t)((vt % RING) * p.C + row)) * BN;
+        __nv_bfloat16* prow = p.P + ((size_t)((vt % RING) * p.C + row)) * BN + c0;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < HALF / 32; ++c) {
           float v[32];
-          tmem_ld32(tmem + lane_addr + buf * BN + c * 32, v);
+          tmem_ld32(tmem + lane_addr + buf * BN + c0 + c * 32, v);
+          float cm = v[0];
+#pragma unroll
+          for (int j = 1; j < 32; ++j) cm = fmaxf(cm, v[j]);
+          if (cm > vbest) {            // first position of the new maximum
+            int jj = 31;
+#pragma unroll
+            for (int j = 31; j >= 0; --j) jj = (v[j] == cm) ? j : jj;
+            vbest = cm;
+            arg = vt * BN + c0 + c * 32 + jj;
+          }
           uint32_t pk[16];
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
-            const float z0 = v[j] * scale, z1 = v[j + 1] * scale;
-            if (z0 > best) { best = z0; arg = vt * BN + c * 32 + j; }
-            if (z1 > best) { best = z1; arg = vt * BN + c * 32 + j + 1; }
-            const float d0 = z0 - mref, d1 = z1 - mref;
-            const float e0 = __expf(d0), e1 = __expf(d1);
+            const float x0 = fmaf(v[j], k1, k0), x1 = fmaf(v[j + 1], k1, k0);
+            const float e0 = ex2(x0), e1 = ex2(x1);
             Z += e0 + e1;
-            S1 = fmaf(e0, d0, fmaf(e1, d1, S1));
+            S2 = fmaf(e0, x0, fmaf(e1, x1, S2));
             pk[j >> 1] = pack_bf16(e0, e1);
           }
           uint4* dst = reinterpret_cast<uint4*>(prow + c * 32);
@@ -557,24 +598,24 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (CG == 2) mbar_arrive_remote(acc_empty_leader + buf * 8);
           else mbar_arrive(&acc_empty[buf]);
         }
-        TileStat ts;
-        ts.m = mref; ts.Z = Z; ts.S1 = S1; ts.best = best; ts.arg = arg;
-        ts.pad[0] = ts.pad[1] = ts.pad[2] = 0;
-        p.tstats[(size_t)row * p.n_vt + vt] = ts;
-        // Publish this warp's rows of the P tile: generic-proxy stores, read later
+        TcStat ts;
+        ts.Z = Z;
+        ts.S1 = S2 * 0.6931471805599453f;
+        ts.best = vbest * scale;
+        ts.arg = arg;
+        p.tstats2[(size_t)row * (2 * p.n_vt) + 2 * vt + half] = ts;
+        // Publish this warp's part of the P tile: generic-proxy stores, read later
         // by TMA on other SMs. Each epilogue warp counts once per tile.
         fence_proxy_async_global();
-        __syncwarp();
-        if (lane == 0) {
-          __threadfence();
-          red_release_add(&p.ready[vt], 1u);
-        }
-        if (threadIdx.x == 64) { TRACE_ADD(8); TRACE_SET(7, (unsigned long long)(n + 1)); }
+        __syncwarp();                              // orders the warp's stores before lane 0's release
+        if (lane == 0) red_release_add(&p.ready[vt], 1u);
+        TR_ADD(busy);
       }
+      if (threadIdx.x == 64) { TR_STORE(6, w_acc); TR_STORE(8, busy); TR_STORE(7, (unsigned long long)n); }
     } else {
       const bool has_work = g < p.n_ranges;
       const int row = rb2 * BM + r_local;
-      float* orow = p.Opart + ((size_t)g * p.C + row) * p.d + (size_t)dt * BN;
+      float* orow = p.Opart + ((size_t)g * p.C + row) * p.d + (size_t)dt * BN + c0;
       bool ok = true;
       if (has_work) {
         ok = mbar_wait(&acc_full[0], 0, p);
@@ -582,9 +623,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (ok) {
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < HALF / 32; ++c) {
           float v[32];
-          if (has_work) tmem_ld32(tmem + lane_addr + c * 32, v);
+          if (has_work) tmem_ld32(tmem + lane_addr + c0 + c * 32, v);
           else {
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = 0.f;
@@ -597,11 +638,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
     }
   }
-  (void)aborted;
 
   __syncthreads();
   if constexpr (CG == 2) cluster_sync();    // no remote arrivals after this point
-  if (threadIdx.x == 0) TRACE_SET(1, gtimer());
+  if (threadIdx.x == 0) TR_STORE(1, gtimer());
   if (warp == 1) {
     tc_fence_after();
     if constexpr (CG == 2)
@@ -614,15 +654,80 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Per-row merge of the half-tile statistics (one CTA per row, fixed order):
+// H = log Z - S1/Z, argmax, sc = (sum of the G2 partials) / Z; rows whose
+// largest logit exceeds the reference by more than redo_gap are listed for the
+// exact recomputation instead.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_merge_tc(DevState* st, const TcStat* ts, int nts,
+    const float* mref, const float* Opart, int nO, int C, int d, RowStat* rowstat, float* H,
+    int32_t* argmax, float* sc, int32_t* redo_rows, float redo_gap) {
+  if (st->done) return;
+  const int i = blockIdx.x;
+  float Z = 0.f, S1 = 0.f, best = -INFINITY;
+  int arg = 0x7fffffff;
+  for (int j = threadIdx.x; j < nts; j += blockDim.x) {
+    const TcStat t = ts[(size_t)i * nts + j];
+    Z += t.Z;
+    S1 += t.S1;
+    if (better(t.best, t.arg, best, arg)) { best = t.best; arg = t.arg; }
+  }
+  for (int o = 16; o; o >>= 1) {
+    Z += __shfl_xor_sync(0xffffffffu, Z, o);
+    S1 += __shfl_xor_sync(0xffffffffu, S1, o);
+    const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+    const int oa = __shfl_xor_sync(0xffffffffu, arg, o);
+    if (better(ob, oa, best, arg)) { best = ob; arg = oa; }
+  }
+  __shared__ float sZ[8], sS[8], sB[8];
+  __shared__ int sA[8];
+  __shared__ float sh_inv;
+  __shared__ int sh_redo;
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) { sZ[w] = Z; sS[w] = S1; sB[w] = best; sA[w] = arg; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    Z = sZ[0]; S1 = sS[0]; best = sB[0]; arg = sA[0];
+    for (int j = 1; j < (int)(blockDim.x >> 5); ++j) {
+      Z += sZ[j];
+      S1 += sS[j];
+      if (better(sB[j], sA[j], best, arg)) { best = sB[j]; arg = sA[j]; }
+    }
+    H[i] = fmaxf(logf(Z) - S1 / Z, 0.f);
+    argmax[i] = arg;
+    RowStat rs;
+    rs.m = mref[i]; rs.Z = Z; rs.pad[0] = best; rs.pad[1] = 0.f;
+    rowstat[i] = rs;
+    const float gap = best - mref[i];
+    const int redo = !(gap <= redo_gap) || !(Z > 0.f) || !(Z < INFINITY);
+    if (redo) redo_rows[atomicAdd(&st->redo, 1)] = i;
+    sh_redo = redo;
+    sh_inv = 1.0f / Z;
+  }
+  __syncthreads();
+  if (sh_redo) return;
+  const float inv = sh_inv;
+  const size_t pstride = (size_t)C * d;
+  for (int k = threadIdx.x; k < d; k += blockDim.x) {
+    float acc = 0.f;
+    for (int g = 0; g < nO; ++g) acc += Opart[g * pstride + (size_t)i * d + k];
+    sc[(size_t)i * d + k] = acc * inv;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Exact recomputation of rows whose logit maximum exceeded the reference.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_redo_partial(const DevState* st,
     const __nv_bfloat16* h, const __nv_bfloat16* E, const float* scale_tab, int S,
     const RowStat* rowstat, const int32_t* redo_rows, float* part, int C, int V, int d) {
-  if (st->done || (int)blockIdx.y >= st->redo) return;
+  if (st->done) return;
   extern __shared__ float sacc[];           // [d]
   __shared__ float wz[8], ws1[8];
-  const int row = redo_rows[blockIdx.y];
+  const int nrow = st->redo;
+  for (int y = blockIdx.y; y < nrow; y += gridDim.y) {
+  const int row = redo_rows[y];
+  __syncthreads();
   const float scale = scale_tab[min(max(st->t, 0), S - 1)];
   const float m = rowstat[row].pad[0];        // exact maximum logit
   for (int k = threadIdx.x; k < d; k += blockDim.x) sacc[k] = 0.f;
@@ -653,13 +758,17 @@ __global__ void __launch_bounds__(256) k_redo_partial(const DevState* st,
     out[d] = a;
     out[d + 1] = b;
   }
+  }
 }
 
 __global__ void __launch_bounds__(256) k_redo_finish(const DevState* st, const int32_t* redo_rows,
     const float* part, float* H, float* sc, int C, int d) {
-  if (st->done || (int)blockIdx.x >= st->redo) return;
-  const int row = redo_rows[blockIdx.x];
+  if (st->done) return;
   __shared__ float sZ;
+  const int nrow = st->redo;
+  for (int y = blockIdx.x; y < nrow; y += gridDim.x) {
+  const int row = redo_rows[y];
+  __syncthreads();
   if (threadIdx.x == 0) {
     float Z = 0.f, S1 = 0.f;
     for (int s = 0; s < RSPLIT; ++s) {
@@ -676,6 +785,7 @@ __global__ void __launch_bounds__(256) k_redo_finish(const DevState* st, const i
     float acc = 0.f;
     for (int s = 0; s < RSPLIT; ++s) acc += part[((size_t)s * C + row) * (size_t)(d + 4) + k];
     sc[(size_t)row * d + k] = acc * inv;
+  }
   }
 }
 
@@ -886,7 +996,8 @@ cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, 
   prm.C = pl.C; prm.V = pl.V; prm.d = pl.d; prm.RB = L.RB; prm.n_vt = L.n_vt;
   prm.n_ranges = L.n_ranges; prm.n_dt = L.n_dt; prm.G = L.G; prm.n1 = L.n1;
   prm.tiles_per_range = tc::KV2 / tc::BN; prm.S = S;
-  prm.mref = mref; prm.scale_tab = scale_tab; prm.tstats = tstats;
+  prm.mref = mref; prm.scale_tab = scale_tab;
+  prm.tstats2 = reinterpret_cast<TcStat*>(tstats);
   prm.Opart = reinterpret_cast<float*>(base + L.Opart);
   prm.P = reinterpret_cast<__nv_bfloat16*>(base + L.P);
   unsigned* ctr = reinterpret_cast<unsigned*>(base + L.counters);
@@ -900,6 +1011,17 @@ cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, 
                    : launch_kernel<1>(s, L.n1 + L.n2, maps, prm);
 }
 
+cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& pl, DevState* st, const TileStat* tstats,
+                            const float* mref, RowStat* rowstat, float* H, int32_t* argmax,
+                            float* sc, int32_t* redo_rows, float redo_gap) {
+  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
+  const float* Opart = reinterpret_cast<const float*>(static_cast<const char*>(pl.ws) + L.Opart);
+  tc::k_merge_tc<<<pl.C, 256, 0, s>>>(st, reinterpret_cast<const TcStat*>(tstats), 2 * L.n_vt,
+                                      mref, Opart, L.G, pl.C, pl.d, rowstat, H, argmax, sc,
+                                      redo_rows, redo_gap);
+  return cudaGetLastError();
+}
+
 void tc_partials(const TcPlan& pl, const float** Opart, int* nO) {
   TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
   *Opart = reinterpret_cast<const float*>(static_cast<const char*>(pl.ws) + L.Opart);
@@ -911,13 +1033,13 @@ cudaError_t launch_tc_redo(cudaStream_t s, const TcPlan& pl, DevState* st, const
                            const int32_t* redo_rows, float* H, float* sc) {
   TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
   float* part = reinterpret_cast<float*>(static_cast<char*>(pl.ws) + L.redo);
-  dim3 g1(tc::RSPLIT, pl.C);
+  dim3 g1(tc::RSPLIT, pl.C < 16 ? pl.C : 16);
   tc::k_redo_partial<<<g1, 256, sizeof(float) * pl.d, s>>>(
       st, static_cast<const __nv_bfloat16*>(h), static_cast<const __nv_bfloat16*>(E), scale_tab, S,
       rowstat, redo_rows, part, pl.C, pl.V, pl.d);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  tc::k_redo_finish<<<pl.C, 256, 0, s>>>(st, redo_rows, part, H, sc, pl.C, pl.d);
+  tc::k_redo_finish<<<pl.C < 16 ? pl.C : 16, 256, 0, s>>>(st, redo_rows, part, H, sc, pl.C, pl.d);
   return cudaGetLastError();
 }
 
