@@ -51,6 +51,7 @@ constexpr int KV2 = 256;       // vocabulary entries per range (unit of G2 owner
 constexpr int RING = 96;       // P tiles (256 vocabulary entries each) resident at once
 constexpr int THREADS = 320;    // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr int EPI_WARPS = 8;
+constexpr int QN = 8;          // G1 item queue depth (tile indices handed to the CTA's warps)
 constexpr int RSPLIT = 16;     // vocabulary splits of the fix-up kernels
 constexpr uint32_t A_BYTES = BM * BK * 2;
 constexpr uint32_t B_BYTES = BN * BK * 2;
@@ -58,7 +59,7 @@ constexpr uint32_t B_BYTES = BN * BK * 2;
 template <int CG> struct Pipe {
   static constexpr int STAGES = CG == 2 ? 6 : 4;
   static constexpr uint32_t STAGE = A_BYTES + B_BYTES / CG;
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 256;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 512;
 };
 constexpr unsigned long long TIMEOUT_NS = 2000000000ull;   // 2 s
 
@@ -71,6 +72,7 @@ struct Params {
   unsigned* ready;           // [n_vt]: epilogue warps that finished a tile
   unsigned* consumed;        // [n_vt]: G2 CTAs that finished loading a tile
   int* abort_flag;
+  unsigned* g1_next;         // next G1 item to hand out (dynamic schedule)
   DevState* st;
   unsigned long long* trace;   // [grid][32] wait-time counters (DG_TC_TRACE builds only)
   TcStat* tstats2;             // [C][2 * n_vt] half-tile statistics
@@ -260,8 +262,10 @@ __device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
 }
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+// Relaxed arrive: signals only that this warp's TMEM reads are done (ordered by
+// tcgen05.fence::before_thread_sync), without waiting for its global stores.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
 }
 // TMA load whose completion is counted on the pair leader's barrier.
@@ -317,6 +321,43 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// G1 items are handed out dynamically: the producer of the pair leader (or of
+// the single CTA) takes the next item from a global counter and publishes it
+// in slot n % QN of every CTA's item queue; every consumer of the CTA reads the
+// slot and reports on the leader's item_empty barrier.
+template <int CG>
+__device__ __forceinline__ bool item_publish(int n, int item, uint64_t* item_full,
+                                             uint64_t* item_empty, int* item_q, const Params& p) {
+  const int q = n % QN;
+  if (!mbar_wait(&item_empty[q], ((n / QN) & 1) ^ 1, p)) return false;
+  item_q[q] = item;
+  if constexpr (CG == 2) {
+    const uint32_t rq = mapa(smem_u32(&item_q[q]), 1);
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(rq), "r"(item) : "memory");
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::
+                     "r"(mapa(smem_u32(&item_full[q]), 1))
+                 : "memory");
+  }
+  mbar_arrive(&item_full[q]);
+  return true;
+}
+// Returns false on abort; *item < 0 means no more items.
+template <int CG>
+__device__ __forceinline__ bool item_take(int n, int* item, uint64_t* item_full,
+                                          uint64_t* item_empty, const int* item_q, bool leader,
+                                          const Params& p) {
+  const int q = n % QN;
+  if (!mbar_wait(&item_full[q], (n / QN) & 1, p)) return false;
+  *item = ((volatile const int*)item_q)[q];
+  if (CG == 2 && !leader)
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::
+                     "r"(mapa(smem_u32(&item_empty[q]), 0))
+                 : "memory");
+  else
+    mbar_arrive(&item_empty[q]);
+  return true;
+}
+
 template <int CG>
 __global__ void __launch_bounds__(THREADS, 1)
     k_vocab_attention(const __grid_constant__ CUtensorMap tm_h,
@@ -338,6 +379,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* acc_empty = acc_full + 2;       // [2] (leader's counts both CTAs' epilogues)
   uint64_t* fin = acc_empty + 2;            // [1]
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(fin + 1);
+  uint64_t* item_full = fin + 2;            // [QN] item index written
+  uint64_t* item_empty = item_full + QN;    // [QN] item index read by every consumer (leader's)
+  int* item_q = reinterpret_cast<int*>(item_empty + QN);   // [QN]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = CG == 2 ? cluster_rank() : 0u;
@@ -353,6 +397,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&acc_empty[b], EPI_WARPS * CG);
     }
     mbar_init(fin, 1);
+    for (int q = 0; q < QN; ++q) {
+      mbar_init(&item_full[q], 1);
+      // consumers: the MMA thread and the epilogue warps (and, for pairs, the
+      // peer's producer and epilogue warps)
+      mbar_init(&item_empty[q], CG == 2 ? 2 + 2 * EPI_WARPS : 1 + EPI_WARPS);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -401,7 +451,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       long issued = 0;
       bool ok = true;
       if (is_g1) {
-        for (int it = unit; ok && it < n_items1; it += p.n1) {
+        for (int n = 0; ok; ++n) {
+          int it;
+          if (leader) {
+            const unsigned got = atomicAdd(p.g1_next, 1u);
+            it = got < (unsigned)n_items1 ? (int)got : -1;
+            if (!item_publish<CG>(n, it, item_full, item_empty, item_q, p)) { ok = false; break; }
+          } else if (!item_take<CG>(n, &it, item_full, item_empty, item_q, leader, p)) {
+            ok = false;
+            break;
+          }
+          if (it < 0) break;
           const int vt = it / RBI;
           const int rb = CG == 2 ? (int)rank : it % RBI;
           if (vt >= RING) {
@@ -466,8 +526,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool ok = true;
       if (is_g1) {
         const uint32_t idesc = idesc_bf16(BM * CG, BN, 0);
-        int n = 0;
-        for (int it = unit; ok && it < n_items1; it += p.n1, ++n) {
+        for (int n = 0; ok; ++n) {
+          int it;
+          if (!item_take<CG>(n, &it, item_full, item_empty, item_q, true, p)) { ok = false; break; }
+          if (it < 0) break;
           const int buf = n & 1;
           {
             TR_T0();
@@ -537,15 +599,26 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int r_local = q * 32 + lane;      // row within the CTA's 128
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     const int c0 = half * HALF;             // first column of this warp
-    // Where this warp reports that it has read an accumulator buffer.
-    const uint32_t acc_empty_leader = CG == 2 ? mapa(smem_u32(acc_empty), 0) : smem_u32(acc_empty);
+    // Where this warp reports that it has read an accumulator buffer (the pair
+    // leader's barrier; for CG = 1 the CTA's own).
+    const uint32_t acc_empty_addr = CG == 2 ? mapa(smem_u32(acc_empty), 0) : smem_u32(acc_empty);
     TR_DECL(w_acc);
     TR_DECL(busy);
+    TR_DECL(t_ld);
+    TR_DECL(t_math);
+    TR_DECL(t_st);
+    TR_DECL(t_pub);
     if (is_g1) {
       const float scale = p.scale_tab[min(max(p.st->t, 0), p.S - 1)];
       const float k1 = scale * 1.4426950408889634f;           // logit scale in log2 units
       int n = 0;
-      for (int it = unit; it < n_items1; it += p.n1, ++n) {
+      for (;; ++n) {
+        int it = 0;
+        bool took = true;
+        if (lane == 0) took = item_take<CG>(n, &it, item_full, item_empty, item_q, leader, p);
+        took = __shfl_sync(0xffffffffu, took ? 1 : 0, 0) != 0;
+        it = __shfl_sync(0xffffffffu, it, 0);
+        if (!took || it < 0) break;
         const int vt = it / RBI;
         const int rb = CG == 2 ? (int)rank : it % RBI;
         const int buf = n & 1;
@@ -566,7 +639,18 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
         for (int c = 0; c < HALF / 32; ++c) {
           float v[32];
-          tmem_ld32(tmem + lane_addr + buf * BN + c0 + c * 32, v);
+          {
+            TR_T0();
+            tmem_ld32(tmem + lane_addr + buf * BN + c0 + c * 32, v);
+            TR_ADD(t_ld);
+          }
+          if (c == HALF / 32 - 1) {
+            // Last read of this accumulator buffer: hand it back to the MMA warp.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote_relaxed(acc_empty_addr + buf * 8);
+          }
+          TR_T0();
           float cm = v[0];
 #pragma unroll
           for (int j = 1; j < 32; ++j) cm = fmaxf(cm, v[j]);
@@ -586,17 +670,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             S2 = fmaf(e0, x0, fmaf(e1, x1, S2));
             pk[j >> 1] = pack_bf16(e0, e1);
           }
-          uint4* dst = reinterpret_cast<uint4*>(prow + c * 32);
+          TR_ADD(t_math);
+          {
+            TR_T0();
+            uint4* dst = reinterpret_cast<uint4*>(prow + c * 32);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-        }
-        // This warp is done reading the accumulator buffer.
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          if (CG == 2) mbar_arrive_remote(acc_empty_leader + buf * 8);
-          else mbar_arrive(&acc_empty[buf]);
+            for (int j = 0; j < 4; ++j)
+              dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            TR_ADD(t_st);
+          }
         }
         TcStat ts;
         ts.Z = Z;
@@ -606,12 +688,19 @@ __global__ void __launch_bounds__(THREADS, 1)
         p.tstats2[(size_t)row * (2 * p.n_vt) + 2 * vt + half] = ts;
         // Publish this warp's part of the P tile: generic-proxy stores, read later
         // by TMA on other SMs. Each epilogue warp counts once per tile.
-        fence_proxy_async_global();
-        __syncwarp();                              // orders the warp's stores before lane 0's release
-        if (lane == 0) red_release_add(&p.ready[vt], 1u);
+        {
+          TR_T0();
+          fence_proxy_async_global();
+          __syncwarp();                            // orders the warp's stores before lane 0's release
+          if (lane == 0) red_release_add(&p.ready[vt], 1u);
+          TR_ADD(t_pub);
+        }
         TR_ADD(busy);
       }
-      if (threadIdx.x == 64) { TR_STORE(6, w_acc); TR_STORE(8, busy); TR_STORE(7, (unsigned long long)n); }
+      if (threadIdx.x == 64) {
+        TR_STORE(6, w_acc); TR_STORE(8, busy); TR_STORE(7, (unsigned long long)n);
+        TR_STORE(9, t_ld); TR_STORE(10, t_math); TR_STORE(11, t_st); TR_STORE(12, t_pub);
+      }
     } else {
       const bool has_work = g < p.n_ranges;
       const int row = rb2 * BM + r_local;
@@ -824,7 +913,9 @@ TcLayout tc_layout(int C, int V, int d, int sms) {
   // the rest; minimise the larger of the two roles' per-unit work.
   const int units = sms / L.CG;
   const int RBI = L.CG == 2 ? 1 : L.RB;
-  const double u1 = (double)tc::BM * tc::BN * d;                 // one G1 item
+  // One G1 item costs about 1.3x a G2 range of the same MMA work (measured on
+  // B200: the softmax epilogue and the HBM-side fill); weight it accordingly.
+  const double u1 = 1.3 * tc::BM * tc::BN * d;                   // one G1 item
   const double u2 = (double)tc::BM * tc::BN * tc::KV2;           // one G2 range
   const int per_g = RBI * L.n_dt;
   double best = 1e300;
@@ -1004,6 +1095,7 @@ cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, 
   prm.ready = ctr;
   prm.consumed = ctr + L.n_vt;
   prm.abort_flag = reinterpret_cast<int*>(ctr + 2 * L.n_vt);
+  prm.g1_next = ctr + 2 * L.n_vt + 1;
   prm.st = st;
   prm.trace = reinterpret_cast<unsigned long long*>(base + L.trace);
   const CUtensorMap* maps = reinterpret_cast<const CUtensorMap*>(pl.maps);
