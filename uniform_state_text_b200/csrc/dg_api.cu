@@ -202,14 +202,13 @@ int launch_step(dg_ctx* ctx, bool standin, bool use_cond) {
     e1 = ctx->ev[ctx->ev_used++];
     DG_CK(cudaEventRecord(e0, s));
   }
-  ctx->launches += 2 + (tc ? 2 + tc_launches(ctx->tc_plan) : 4);
+  ctx->launches += 2 + (tc ? 1 + tc_launches(ctx->tc_plan) : 4);
   if (tc) {
     DG_CK(launch_tc_attention(s, ctx->tc_plan, ctx->st, ctx->h, ctx->E, ctx->mref, ctx->scale_tab,
                               c.max_steps, ctx->tstats, ctx->O, ctx->tc));
     DG_CK(launch_tc_merge(s, ctx->tc_plan, ctx->st, ctx->tstats, ctx->mref, ctx->rowstat, ctx->H,
-                          ctx->argmax, ctx->sc, ctx->redo_rows, kRedoGap));
-    DG_CK(launch_tc_redo(s, ctx->tc_plan, ctx->st, ctx->h, ctx->E, ctx->scale_tab, c.max_steps,
-                         ctx->rowstat, ctx->redo_rows, ctx->H, ctx->sc));
+                          ctx->argmax, ctx->sc, ctx->redo_rows, kRedoGap, ctx->h, ctx->E,
+                          ctx->scale_tab, c.max_steps));
   } else {
     DG_CK(launch_simt_attention(s, c.dtype, ctx->st, ctx->h, ctx->E, ctx->zbuf, ctx->tstats,
                                 ctx->rowstat, ctx->partial, ctx->H, ctx->argmax, ctx->sc, c.C,

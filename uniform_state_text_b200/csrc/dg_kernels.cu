@@ -74,6 +74,7 @@ __global__ void __launch_bounds__(256) k_prologue(const DevState* st, const T* E
   const T* Ec = E + (size_t)can * d;
   const T* Ep = E + (size_t)prev * d;
   float dc = 0.f, dp = 0.f;
+#pragma unroll 4
   for (int k = threadIdx.x; k < d; k += blockDim.x) {
     T hv;
     if (standin) {
@@ -367,26 +368,38 @@ __global__ void __launch_bounds__(1024) k_sampler(DevState* st, const float* H,
   }
   __syncthreads();
   // Running entropy sums in sorted order, added one at a time in fp32 (a fixed
-  // summation order): warp 0 holds the sorted entropies, lane l the entries
-  // [l*per, (l+1)*per), and passes the running sum from lane to lane.
+  // summation order): warp 0 holds the sorted entropies in registers, lane l
+  // the entries [l*per, (l+1)*per), and relays the running sum lane to lane.
   if (i < 32) {
-    const int per = (C + 31) / 32;
-    float run = 0.f;
-    int k = 0;
+    const int per = (C + 31) / 32;   // <= 32
+    float v[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int j = i * per + e;
+      v[e] = (e < per && j < C) ? sSorted[j] : 0.f;
+    }
+    float run = 0.f, start = 0.f;
     for (int src = 0; src < 32; ++src) {
       if (i == src) {
-        for (int e = 0; e < per; ++e) {
-          const int j = src * per + e;
-          if (j >= C) break;
-          const float before = run;
-          run = __fadd_rn(run, sSorted[j]);
-          prefix[j] = run;
-          // prefix sums of non-negative terms never decrease, so the accepted
-          // positions are a prefix of the sorted order
-          k += (accept_rule == 0 ? (run <= tau) : (before <= tau)) ? 1 : 0;
-        }
+        start = run;
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (e < per) { run = __fadd_rn(run, v[e]); v[e] = run; }
       }
       run = __shfl_sync(0xffffffffu, run, src);
+    }
+    // prefix sums of non-negative terms never decrease, so the accepted
+    // positions are a prefix of the sorted order: count them
+    int k = 0;
+    float before = start;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int j = i * per + e;
+      if (e < per && j < C) {
+        prefix[j] = v[e];
+        k += (accept_rule == 0 ? (v[e] <= tau) : (before <= tau)) ? 1 : 0;
+        before = v[e];
+      }
     }
     for (int o = 16; o; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
     if (i == 0) sk = k;

@@ -52,7 +52,6 @@ constexpr int RING = 96;       // P tiles (256 vocabulary entries each) resident
 constexpr int THREADS = 320;    // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr int EPI_WARPS = 8;
 constexpr int QN = 8;          // G1 item queue depth (tile indices handed to the CTA's warps)
-constexpr int RSPLIT = 16;     // vocabulary splits of the fix-up kernels
 constexpr uint32_t A_BYTES = BM * BK * 2;
 constexpr uint32_t B_BYTES = BN * BK * 2;
 // Pipeline depth per CTA-group size: the same ~192 KB of stages either way.
@@ -189,6 +188,28 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// L2 eviction policies for TMA loads: G1 marks the E tiles (and h) it reads as
+// evict_last so that they are still in L2 when the G2 CTAs read the same
+// tiles; G2 reads them evict_first (they are dead afterwards).
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int x, int y, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(pol)
+      : "memory");
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
 __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
@@ -277,11 +298,20 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar) & 0xFEFFFFFFu), "r"(x), "r"(y)
       : "memory");
 }
+__device__ __forceinline__ void tma_load_2d_pair_hint(void* dst, const CUtensorMap* map,
+                                                      uint64_t* bar, int x, int y, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar) & 0xFEFFFFFFu), "r"(x), "r"(y),
+      "l"(pol)
+      : "memory");
+}
 template <int CG>
 __device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
-                                         int y) {
-  if constexpr (CG == 2) tma_load_2d_pair(dst, map, bar, x, y);
-  else tma_load_2d(dst, map, bar, x, y);
+                                         int y, uint64_t pol) {
+  if constexpr (CG == 2) tma_load_2d_pair_hint(dst, map, bar, x, y, pol);
+  else tma_load_2d_hint(dst, map, bar, x, y, pol);
 }
 template <int CG>
 __device__ __forceinline__ void mma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
@@ -450,6 +480,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t ph = 0;
       long issued = 0;
       bool ok = true;
+      const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
       if (is_g1) {
         for (int n = 0; ok; ++n) {
           int it;
@@ -475,8 +506,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             TR_ADD(w_empty);
             unsigned char* st = smem + s * STAGE_BYTES;
             if (leader) mbar_expect_tx(&full[s], STAGE_BYTES * CG);
-            tma_load<CG>(st, &tm_h, &full[s], kc * BK, rb * BM);
-            tma_load<CG>(st + A_BYTES, &tm_ek, &full[s], kc * BK, vt * BN + (int)rank * NB_ROWS);
+            tma_load<CG>(st, &tm_h, &full[s], kc * BK, rb * BM, keep);
+            tma_load<CG>(st + A_BYTES, &tm_ek, &full[s], kc * BK, vt * BN + (int)rank * NB_ROWS, keep);
             ++issued;
             if (++s == STAGES) { s = 0; ph ^= 1; }
           }
@@ -496,11 +527,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             TR_ADD(w_empty);
             unsigned char* st = smem + s * STAGE_BYTES;
             if (leader) mbar_expect_tx(&full[s], STAGE_BYTES * CG);
-            tma_load<CG>(st, &tm_p, &full[s], (kc % (BN / BK)) * BK, (vt % RING) * p.C + rb2 * BM);
+            tma_load<CG>(st, &tm_p, &full[s], (kc % (BN / BK)) * BK, (vt % RING) * p.C + rb2 * BM,
+                         keep);
 #pragma unroll
             for (int j = 0; j < NB_ROWS / 64; ++j)
               tma_load<CG>(st + A_BYTES + j * (64 * BK * 2), &tm_emn, &full[s],
-                           dt * BN + (int)rank * NB_ROWS + j * 64, r * KV2 + kc * BK);
+                           dt * BN + (int)rank * NB_ROWS + j * 64, r * KV2 + kc * BK, drop);
             ++issued;
             if (++s == STAGES) { s = 0; ph ^= 1; }
           }
@@ -744,17 +776,20 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 // ---------------------------------------------------------------------------
 // Per-row merge of the half-tile statistics (one CTA per row, fixed order):
-// H = log Z - S1/Z, argmax, sc = (sum of the G2 partials) / Z; rows whose
-// largest logit exceeds the reference by more than redo_gap are listed for the
-// exact recomputation instead.
+// H = log Z - S1/Z, argmax, sc = (sum of the G2 partials) / Z. A row whose
+// largest logit exceeds its reference by more than redo_gap (its P could have
+// overflowed) is recomputed here exactly against its true maximum.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_merge_tc(DevState* st, const TcStat* ts, int nts,
-    const float* mref, const float* Opart, int nO, int C, int d, RowStat* rowstat, float* H,
-    int32_t* argmax, float* sc, int32_t* redo_rows, float redo_gap) {
+    const float* mref, const float* Opart, int nO, int C, int V, int d, RowStat* rowstat,
+    float* H, int32_t* argmax, float* sc, float redo_gap, const __nv_bfloat16* h,
+    const __nv_bfloat16* E, const float* scale_tab, int S) {
   if (st->done) return;
+  extern __shared__ float sacc[];   // [d], exact recomputation only
   const int i = blockIdx.x;
   float Z = 0.f, S1 = 0.f, best = -INFINITY;
   int arg = 0x7fffffff;
+#pragma unroll 4
   for (int j = threadIdx.x; j < nts; j += blockDim.x) {
     const TcStat t = ts[(size_t)i * nts + j];
     Z += t.Z;
@@ -770,7 +805,7 @@ __global__ void __launch_bounds__(256) k_merge_tc(DevState* st, const TcStat* ts
   }
   __shared__ float sZ[8], sS[8], sB[8];
   __shared__ int sA[8];
-  __shared__ float sh_inv;
+  __shared__ float sh_inv, sh_best;
   __shared__ int sh_redo;
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
   if (l == 0) { sZ[w] = Z; sS[w] = S1; sB[w] = best; sA[w] = arg; }
@@ -789,93 +824,56 @@ __global__ void __launch_bounds__(256) k_merge_tc(DevState* st, const TcStat* ts
     rowstat[i] = rs;
     const float gap = best - mref[i];
     const int redo = !(gap <= redo_gap) || !(Z > 0.f) || !(Z < INFINITY);
-    if (redo) redo_rows[atomicAdd(&st->redo, 1)] = i;
+    if (redo) atomicAdd(&st->redo, 1);
     sh_redo = redo;
     sh_inv = 1.0f / Z;
+    sh_best = best;
   }
   __syncthreads();
-  if (sh_redo) return;
-  const float inv = sh_inv;
-  const size_t pstride = (size_t)C * d;
-  for (int k = threadIdx.x; k < d; k += blockDim.x) {
-    float acc = 0.f;
-    for (int g = 0; g < nO; ++g) acc += Opart[g * pstride + (size_t)i * d + k];
-    sc[(size_t)i * d + k] = acc * inv;
+  if (!sh_redo) {
+    const float inv = sh_inv;
+    const size_t pstride = (size_t)C * d;
+#pragma unroll 2
+    for (int k = threadIdx.x; k < d; k += blockDim.x) {
+      float acc = 0.f;
+#pragma unroll 4
+      for (int g = 0; g < nO; ++g) acc += Opart[g * pstride + (size_t)i * d + k];
+      sc[(size_t)i * d + k] = acc * inv;
+    }
+    return;
   }
-}
-
-// ---------------------------------------------------------------------------
-// Exact recomputation of rows whose logit maximum exceeded the reference.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_redo_partial(const DevState* st,
-    const __nv_bfloat16* h, const __nv_bfloat16* E, const float* scale_tab, int S,
-    const RowStat* rowstat, const int32_t* redo_rows, float* part, int C, int V, int d) {
-  if (st->done) return;
-  extern __shared__ float sacc[];           // [d]
-  __shared__ float wz[8], ws1[8];
-  const int nrow = st->redo;
-  for (int y = blockIdx.y; y < nrow; y += gridDim.y) {
-  const int row = redo_rows[y];
-  __syncthreads();
+  // Exact recomputation against the true maximum m: Z = sum e^(z-m),
+  // S1 = sum e^(z-m)(z-m), sc = sum e^(z-m) E_v / Z. One warp per vocabulary
+  // entry at a time; sc accumulates in shared memory.
   const float scale = scale_tab[min(max(st->t, 0), S - 1)];
-  const float m = rowstat[row].pad[0];        // exact maximum logit
+  const float m = sh_best;
   for (int k = threadIdx.x; k < d; k += blockDim.x) sacc[k] = 0.f;
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int vlen = V / RSPLIT, v0 = blockIdx.x * vlen;
-  const __nv_bfloat16* hr = h + (size_t)row * d;
-  float Z = 0.f, S1 = 0.f;
-  for (int v = v0 + warp; v < v0 + vlen; v += 8) {
+  const __nv_bfloat16* hr = h + (size_t)i * d;
+  float Zl = 0.f, S1l = 0.f;
+  for (int v = w; v < V; v += 8) {
     const __nv_bfloat16* ev = E + (size_t)v * d;
     float dot = 0.f;
-    for (int k = lane; k < d; k += 32) dot = fmaf(__bfloat162float(hr[k]), __bfloat162float(ev[k]), dot);
-    for (int off = 16; off; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+    for (int k = l; k < d; k += 32) dot = fmaf(__bfloat162float(hr[k]), __bfloat162float(ev[k]), dot);
+    for (int o = 16; o; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
     const float dz = dot * scale - m;
     const float e = expf(dz);
-    Z += e;
-    S1 = fmaf(e, dz, S1);
+    Zl += e;
+    S1l = fmaf(e, dz, S1l);
     if (e > 0.f)
-      for (int k = lane; k < d; k += 32) atomicAdd(&sacc[k], e * __bfloat162float(ev[k]));
+      for (int k = l; k < d; k += 32) atomicAdd(&sacc[k], e * __bfloat162float(ev[k]));
   }
-  if (lane == 0) { wz[warp] = Z; ws1[warp] = S1; }
   __syncthreads();
-  float* out = part + ((size_t)blockIdx.x * C + row) * (size_t)(d + 4);
-  for (int k = threadIdx.x; k < d; k += blockDim.x) out[k] = sacc[k];
+  if (l == 0) { sZ[w] = Zl; sS[w] = S1l; }
+  __syncthreads();
   if (threadIdx.x == 0) {
     float a = 0.f, b = 0.f;
-    for (int j = 0; j < 8; ++j) { a += wz[j]; b += ws1[j]; }
-    out[d] = a;
-    out[d + 1] = b;
-  }
-  }
-}
-
-__global__ void __launch_bounds__(256) k_redo_finish(const DevState* st, const int32_t* redo_rows,
-    const float* part, float* H, float* sc, int C, int d) {
-  if (st->done) return;
-  __shared__ float sZ;
-  const int nrow = st->redo;
-  for (int y = blockIdx.x; y < nrow; y += gridDim.x) {
-  const int row = redo_rows[y];
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float Z = 0.f, S1 = 0.f;
-    for (int s = 0; s < RSPLIT; ++s) {
-      const float* q = part + ((size_t)s * C + row) * (size_t)(d + 4);
-      Z += q[d];
-      S1 += q[d + 1];
-    }
-    H[row] = fmaxf(logf(Z) - S1 / Z, 0.f);
-    sZ = Z;
+    for (int j = 0; j < 8; ++j) { a += sZ[j]; b += sS[j]; }
+    H[i] = fmaxf(logf(a) - b / a, 0.f);
+    sh_inv = 1.0f / a;
   }
   __syncthreads();
-  const float inv = 1.0f / sZ;
-  for (int k = threadIdx.x; k < d; k += blockDim.x) {
-    float acc = 0.f;
-    for (int s = 0; s < RSPLIT; ++s) acc += part[((size_t)s * C + row) * (size_t)(d + 4) + k];
-    sc[(size_t)row * d + k] = acc * inv;
-  }
-  }
+  for (int k = threadIdx.x; k < d; k += blockDim.x) sc[(size_t)i * d + k] = sacc[k] * sh_inv;
 }
 
 }  // namespace tc
@@ -886,7 +884,7 @@ __global__ void __launch_bounds__(256) k_redo_finish(const DevState* st, const i
 namespace {
 
 struct TcLayout {
-  size_t counters = 0, P = 0, Opart = 0, redo = 0, trace = 0, total = 0;
+  size_t counters = 0, P = 0, Opart = 0, trace = 0, total = 0;
   int CG = 1;              // CTAs per MMA group (2: CTA pairs, M = 256)
   int RB = 0, n_vt = 0, n_ranges = 0, n_dt = 0, G = 0, n1 = 0, n2 = 0;   // n1, n2 in groups
 };
@@ -934,7 +932,6 @@ TcLayout tc_layout(int C, int V, int d, int sms) {
   L.counters = off; off = al(off + sizeof(unsigned) * (2 * (size_t)L.n_vt + 64));
   L.P = off; off = al(off + (size_t)tc::RING * C * tc::BN * 2);
   L.Opart = off; off = al(off + (size_t)(L.G > 0 ? L.G : 1) * C * d * 4);
-  L.redo = off; off = al(off + (size_t)tc::RSPLIT * C * (d + 4) * 4);
   L.trace = off; off = al(off + (size_t)256 * 32 * 8);
   L.total = off;
   return L;
@@ -980,7 +977,7 @@ int tc_stat_tiles(int, int V, int) { return V / tc::BN; }
 
 size_t tc_workspace_bytes(int C, int V, int d) { return tc_layout(C, V, d, device_sms()).total; }
 
-int tc_launches(const TcPlan&) { return 3; }
+int tc_launches(const TcPlan&) { return 1; }
 
 template <int CG>
 cudaError_t launch_kernel(cudaStream_t s, int units, const CUtensorMap* maps, const tc::Params& prm) {
@@ -1105,12 +1102,15 @@ cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, 
 
 cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& pl, DevState* st, const TileStat* tstats,
                             const float* mref, RowStat* rowstat, float* H, int32_t* argmax,
-                            float* sc, int32_t* redo_rows, float redo_gap) {
+                            float* sc, int32_t* redo_rows, float redo_gap, const void* h,
+                            const void* E, const float* scale_tab, int S) {
   TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
   const float* Opart = reinterpret_cast<const float*>(static_cast<const char*>(pl.ws) + L.Opart);
-  tc::k_merge_tc<<<pl.C, 256, 0, s>>>(st, reinterpret_cast<const TcStat*>(tstats), 2 * L.n_vt,
-                                      mref, Opart, L.G, pl.C, pl.d, rowstat, H, argmax, sc,
-                                      redo_rows, redo_gap);
+  (void)redo_rows;
+  tc::k_merge_tc<<<pl.C, 256, sizeof(float) * pl.d, s>>>(
+      st, reinterpret_cast<const TcStat*>(tstats), 2 * L.n_vt, mref, Opart, L.G, pl.C, pl.V, pl.d,
+      rowstat, H, argmax, sc, redo_gap, static_cast<const __nv_bfloat16*>(h),
+      static_cast<const __nv_bfloat16*>(E), scale_tab, S);
   return cudaGetLastError();
 }
 
@@ -1118,21 +1118,6 @@ void tc_partials(const TcPlan& pl, const float** Opart, int* nO) {
   TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
   *Opart = reinterpret_cast<const float*>(static_cast<const char*>(pl.ws) + L.Opart);
   *nO = L.G;
-}
-
-cudaError_t launch_tc_redo(cudaStream_t s, const TcPlan& pl, DevState* st, const void* h,
-                           const void* E, const float* scale_tab, int S, const RowStat* rowstat,
-                           const int32_t* redo_rows, float* H, float* sc) {
-  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
-  float* part = reinterpret_cast<float*>(static_cast<char*>(pl.ws) + L.redo);
-  dim3 g1(tc::RSPLIT, pl.C < 16 ? pl.C : 16);
-  tc::k_redo_partial<<<g1, 256, sizeof(float) * pl.d, s>>>(
-      st, static_cast<const __nv_bfloat16*>(h), static_cast<const __nv_bfloat16*>(E), scale_tab, S,
-      rowstat, redo_rows, part, pl.C, pl.V, pl.d);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  tc::k_redo_finish<<<pl.C < 16 ? pl.C : 16, 256, 0, s>>>(st, redo_rows, part, H, sc, pl.C, pl.d);
-  return cudaGetLastError();
 }
 
 }  // namespace dg

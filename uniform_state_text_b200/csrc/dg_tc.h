@@ -27,13 +27,12 @@ int tc_launches(const TcPlan& p);   // kernels per launch_tc_attention call
 cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& p, DevState* st, const void* h,
                                 const void* E, const float* mref, const float* scale_tab,
                                 int S, TileStat* tstats, float* O, void* ws);
-cudaError_t launch_tc_redo(cudaStream_t s, const TcPlan& p, DevState* st, const void* h,
-                           const void* E, const float* scale_tab, int S, const RowStat* rowstat,
-                           const int32_t* redo_rows, float* H, float* sc);
-// Per-row merge of the kernel's statistics and partials (sc, H, argmax, redo list).
+// Per-row merge of the kernel's statistics and partials into sc, H and argmax;
+// rows whose maximum overshot the reference are recomputed exactly.
 cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& p, DevState* st, const TileStat* tstats,
                             const float* mref, RowStat* rowstat, float* H, int32_t* argmax,
-                            float* sc, int32_t* redo_rows, float redo_gap);
+                            float* sc, int32_t* redo_rows, float redo_gap, const void* h,
+                            const void* E, const float* scale_tab, int S);
 // Hand-off counters the prologue zeroes before every step.
 void tc_counters(const TcPlan& p, unsigned** ptr, int* count);
 // Per-range-group partials of O = P E that the merge sums.
