@@ -194,6 +194,36 @@ int dg_profile_read(dg_ctx* ctx, double* ms_total, int32_t* steps, int64_t* laun
 /* Which kernel family the context runs (DG_IMPL_SIMT or DG_IMPL_TC). */
 int dg_impl(const dg_ctx* ctx);
 
+/*
+ * Vocabulary attention without any allocation. The pages have no counterpart:
+ * this entry point exists for callers that cannot call cudaMalloc (code inside
+ * a host callback, a plugin whose host framework owns every device allocation,
+ * a process that must not grow its device footprint after start-up).
+ *
+ * Computes, for each of the C rows of h, the tempered logits z = scale h.E^T
+ * over the V vocabulary rows of E, and writes the entropy H (nats, float [C]),
+ * the argmax (int32 [C], lowest index on ties) and the self-conditioning
+ * vector sc = softmax(z).E (float [C*d]) -- the same CUDA-core kernels a
+ * DG_IMPL_SIMT context runs, with scratch taken from one file-scope device
+ * array of DG_STATIC_SCRATCH_BYTES instead of a caller workspace.
+ *   E, h     device, [V][d] and [C][d] of dtype (DG_F32 or DG_BF16).
+ *   H, argmax, sc  device outputs, caller-owned.
+ *   stream   cudaStream_t (NULL = legacy default stream); asynchronous.
+ * The array is held by every GPU that loads the library until the process
+ * exits. All calls share it and it keeps the last call's contents (this call
+ * writes every scratch word before reading it); calls whose kernels overlap on
+ * the GPU race on it, so serialise them. The first call on each device looks
+ * up the array's address (cudaGetSymbolAddress, that device current); make it
+ * before capturing a stream into a graph. No cudaMalloc or cudaFree is called.
+ * Errors: DG_EINVAL (bad shape, dtype or NULL pointer), DG_EUNSUPPORTED (the
+ * shape needs more than DG_STATIC_SCRATCH_BYTES of scratch, about
+ * 4.5*C*V + 4*C*d bytes), DG_ECUDA; dg_last_error(NULL) gives the message.
+ */
+#define DG_STATIC_SCRATCH_BYTES (32u << 20)
+int dg_vocab_attention_static(int32_t C, int32_t V, int32_t d, int32_t dtype, float scale,
+                              const void* E, const void* h, float* H, int32_t* argmax,
+                              float* sc, void* stream);
+
 /* Release the context (host memory and graph objects only). */
 int dg_free(dg_ctx* ctx);
 

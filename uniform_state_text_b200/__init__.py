@@ -77,12 +77,13 @@ def lib():
     L.dg_profile_read.argtypes = [_P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I),
                                   ctypes.POINTER(ctypes.c_int64)]
     L.dg_impl.argtypes = [_P]
+    L.dg_vocab_attention_static.argtypes = [_I, _I, _I, _I, ctypes.c_float, _P, _P, _P, _P, _P, _P]
     L.dg_free.argtypes = [_P]
     L.dg_last_error.argtypes = [_P]
     L.dg_last_error.restype = ctypes.c_char_p
     for name in ("dg_init", "dg_begin_block", "dg_denoise_step", "dg_denoise_step_h",
                  "dg_denoise_block", "dg_read", "dg_write", "dg_profile", "dg_profile_read",
-                 "dg_impl", "dg_free"):
+                 "dg_impl", "dg_free", "dg_vocab_attention_static"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -168,6 +169,14 @@ def dg_profile_read(ctx):
     nl = ctypes.c_int64()
     _check(lib().dg_profile_read(ctx, ctypes.byref(ms), ctypes.byref(n), ctypes.byref(nl)), ctx)
     return float(ms.value), int(n.value), int(nl.value)
+
+
+def dg_vocab_attention_static(C: int, V: int, d: int, dtype: int, scale: float, E_ptr: int,
+                              h_ptr: int, H_ptr: int, argmax_ptr: int, sc_ptr: int,
+                              stream_ptr: int) -> None:
+    """Vocabulary attention with the library's static scratch (no allocation)."""
+    _check(lib().dg_vocab_attention_static(C, V, d, dtype, scale, _P(E_ptr), _P(h_ptr), _P(H_ptr),
+                                           _P(argmax_ptr), _P(sc_ptr), _P(stream_ptr)), None)
 
 
 def dg_impl(ctx) -> int:

@@ -125,6 +125,10 @@ int make_layout(const dg_config* c, Layout* L, char* why, size_t n) {
 
 }  // namespace
 
+namespace dg {
+void set_last_error(const char* msg) { snprintf(g_init_err, sizeof(g_init_err), "%s", msg); }
+}  // namespace dg
+
 struct dg_ctx {
   dg_config cfg;
   Layout L;
