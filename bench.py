@@ -129,6 +129,21 @@ def cpu_baseline(w, E32, rows: int, seed_steps: int = 1):
             "tok_per_s": w.C / step_s}
 
 
+def max_over_ranks(x: float, dist=None, device="cpu") -> float:
+    """The largest value of x over all ranks (x itself without a process group)."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(steps_per_rank: int, world: int, slowest_ms: float) -> float:
+    """Weak scaling: every rank runs its own canvases; units of all ranks over the slowest rank's time."""
+    return steps_per_rank * world / (slowest_ms / 1e3)
+
+
 def roofline_time(w, pk, sustained=True):
     flops = 4.0 * w.C * w.d * w.V
     t_c = flops / ((pk["tflops_sustained"] if sustained else pk["tflops"]) * 1e12)
@@ -257,12 +272,8 @@ def main():
     st = den.state()
     if st["status"] != 0:
         raise RuntimeError(f"device status {st['status']}")
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    total_steps = args.steps * world
-    value = total_steps / (ms / 1e3)
+    ms = max_over_ranks(ms, dist, "cuda")
+    value = whole_job_rate(args.steps, world, ms)
     ms_per_step = ms / args.steps
 
     # --- end to end through host buffers ----------------------------------------
@@ -290,10 +301,7 @@ def main():
             done_steps += 1
         torch.cuda.synchronize()
         el = time.perf_counter() - t0
-        if dist:
-            t = torch.tensor([el], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            el = float(t.item())
+        el = max_over_ranks(el, dist, "cuda")
         e2e = {"value": n_e2e * world / el, "unit": "steps/s",
                "h2d_bytes_per_step": int(h_host.numel() * h_host.element_size()),
                "d2h_bytes_per_step": int(w.C * 4 + 64),
