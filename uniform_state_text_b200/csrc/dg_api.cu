@@ -12,7 +12,7 @@
 #include <cstring>
 #include <vector>
 
-#include "../../include/dg.h"
+#include "dg.h"
 #include "dg_common.cuh"
 #include "dg_kernels.h"
 #include "dg_tc.h"

@@ -21,7 +21,7 @@
 #include <cstdio>
 #include <mutex>
 
-#include "../../include/dg.h"
+#include "dg.h"
 #include "dg_common.cuh"
 #include "dg_kernels.h"
 
