@@ -181,7 +181,9 @@ int dg_read(dg_ctx* ctx, int32_t what, void* dst_dev);
 int dg_write(dg_ctx* ctx, int32_t what, const void* src_dev);
 
 /*
- * Per-step timing of the vocabulary-attention kernels, for measurement:
+ * Per-step timing of the vocabulary-attention kernel(s) (the tensor-core
+ * kernel alone on that path; the CUDA-core attention kernels otherwise), for
+ * measurement:
  * enable != 0 records CUDA events around them on the context's stream in every
  * dg_denoise_step / dg_denoise_step_h and resets the counters;
  * dg_profile_read synchronises and returns the total milliseconds and number

@@ -206,23 +206,29 @@ int launch_step(dg_ctx* ctx, bool standin, bool use_cond) {
     e1 = ctx->ev[ctx->ev_used++];
     DG_CK(cudaEventRecord(e0, s));
   }
-  ctx->launches += 2 + (tc ? 1 + tc_launches(ctx->tc_plan) : 4);
+  ctx->launches += tc ? 2 + tc_launches(ctx->tc_plan) : 6;
+  const SamplerArgs sa = make_sampler_args(
+      ctx->st, ctx->H, ctx->argmax, ctx->canvas, ctx->argmax_prev, ctx->accept, ctx->order,
+      ctx->prefix, c.C, c.V, c.seed, c.tau, c.stop_entropy, c.stop_unchanged, c.stop_rule,
+      c.accept_rule, c.fixed_steps, c.max_steps, ctx->cond, use_cond ? 1 : 0);
   if (tc) {
     DG_CK(launch_tc_attention(s, ctx->tc_plan, ctx->st, ctx->h, ctx->E, ctx->mref, ctx->scale_tab,
                               c.max_steps, ctx->tstats, ctx->O, ctx->tc));
+    if (e1) DG_CK(cudaEventRecord(e1, s));
+    // merge, then (inside the same kernel) the sampler and stop test
     DG_CK(launch_tc_merge(s, ctx->tc_plan, ctx->st, ctx->tstats, ctx->mref, ctx->rowstat, ctx->H,
                           ctx->argmax, ctx->sc, ctx->redo_rows, kRedoGap, ctx->h, ctx->E,
-                          ctx->scale_tab, c.max_steps));
+                          ctx->scale_tab, c.max_steps, sa));
   } else {
     DG_CK(launch_simt_attention(s, c.dtype, ctx->st, ctx->h, ctx->E, ctx->zbuf, ctx->tstats,
                                 ctx->rowstat, ctx->partial, ctx->H, ctx->argmax, ctx->sc, c.C,
                                 c.V, c.d, ctx->L.nsplit, ctx->scale_tab, c.max_steps));
+    if (e1) DG_CK(cudaEventRecord(e1, s));
+    DG_CK(launch_sampler(s, ctx->st, ctx->H, ctx->argmax, ctx->canvas, ctx->argmax_prev,
+                         ctx->accept, ctx->order, ctx->prefix, c.C, c.V, c.seed, c.tau,
+                         c.stop_entropy, c.stop_unchanged, c.stop_rule, c.accept_rule,
+                         c.fixed_steps, c.max_steps, ctx->cond, use_cond ? 1 : 0));
   }
-  if (e1) DG_CK(cudaEventRecord(e1, s));
-  DG_CK(launch_sampler(s, ctx->st, ctx->H, ctx->argmax, ctx->canvas, ctx->argmax_prev,
-                       ctx->accept, ctx->order, ctx->prefix, c.C, c.V, c.seed, c.tau,
-                       c.stop_entropy, c.stop_unchanged, c.stop_rule, c.accept_rule,
-                       c.fixed_steps, c.max_steps, ctx->cond, use_cond ? 1 : 0));
   return DG_OK;
 }
 

@@ -17,6 +17,7 @@
 //   k_sampler       entropy sort, acceptance, re-noise, adaptive stop.
 #include "dg_common.cuh"
 #include "dg_kernels.h"
+#include "dg_sampler.cuh"
 
 namespace dg {
 
@@ -335,109 +336,16 @@ __global__ void k_simt_reduce(const DevState* st, const float* partial, float* s
 }
 
 // ---------------------------------------------------------------------------
-// Entropy-bounded sampler and adaptive stop, one CTA (blockDim >= C).
+// Entropy-bounded sampler and adaptive stop: one CTA (blockDim >= C). The body
+// (sample_and_stop) lives in dg_sampler.cuh; the tensor-core merge runs it too.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(1024) k_sampler(DevState* st, const float* H,
-    const int32_t* argmax, int32_t* canvas, int32_t* argmax_prev, int32_t* accept,
-    int32_t* order, float* prefix, int C, int V, uint64_t seed, float tau, float stop_entropy,
-    int stop_unchanged, int stop_rule, int accept_rule, int fixed_steps, int S,
-    cudaGraphConditionalHandle cond, int use_cond) {
-  __shared__ float sH[1024];
-  __shared__ float sSorted[1024];
-  __shared__ int32_t sOrder[1024];
-  __shared__ int sk;
-  const int i = threadIdx.x;
-  const bool valid = i < C;
-  if (st->done) {
-    if (use_cond && i == 0) cudaGraphSetConditional(cond, 0);
+__global__ void __launch_bounds__(1024) k_sampler(SamplerArgs a) {
+  __shared__ SamplerSmem sm;
+  if (a.st->done) {
+    if (a.use_cond && threadIdx.x == 0) cudaGraphSetConditional(a.cond, 0);
     return;
   }
-  const int t = st->t;
-  const float Hi = valid ? H[i] : 0.f;
-  if (valid) sH[i] = Hi;
-  __syncthreads();
-  // Stable rank by (entropy, position).
-  int rank = 0;
-  if (valid) {
-    for (int j = 0; j < C; ++j) {
-      const float Hj = sH[j];
-      rank += (Hj < Hi) || (Hj == Hi && j < i);
-    }
-    sOrder[rank] = i;
-    sSorted[rank] = Hi;
-  }
-  __syncthreads();
-  // Running entropy sums in sorted order, added one at a time in fp32 (a fixed
-  // summation order): warp 0 holds the sorted entropies in registers, lane l
-  // the entries [l*per, (l+1)*per), and relays the running sum lane to lane.
-  if (i < 32) {
-    const int per = (C + 31) / 32;   // <= 32
-    float v[32];
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int j = i * per + e;
-      v[e] = (e < per && j < C) ? sSorted[j] : 0.f;
-    }
-    float run = 0.f, start = 0.f;
-    for (int src = 0; src < 32; ++src) {
-      if (i == src) {
-        start = run;
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (e < per) { run = __fadd_rn(run, v[e]); v[e] = run; }
-      }
-      run = __shfl_sync(0xffffffffu, run, src);
-    }
-    // prefix sums of non-negative terms never decrease, so the accepted
-    // positions are a prefix of the sorted order: count them
-    int k = 0;
-    float before = start;
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int j = i * per + e;
-      if (e < per && j < C) {
-        prefix[j] = v[e];
-        k += (accept_rule == 0 ? (v[e] <= tau) : (before <= tau)) ? 1 : 0;
-        before = v[e];
-      }
-    }
-    for (int o = 16; o; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
-    if (i == 0) sk = k;
-  }
-  __syncthreads();
-  const int k = sk;
-  int32_t am = 0, old = 0, nw = 0;
-  bool acc = false;
-  if (valid) {
-    order[i] = sOrder[i];
-    am = argmax[i];
-    old = canvas[i];
-    acc = rank < k;
-    const uint64_t pre = key_prefix(seed, (uint64_t)(uint32_t)st->block, (uint64_t)t);
-    const int32_t noise = (int32_t)(sm64(pre ^ (uint64_t)i) & (uint64_t)(V - 1));
-    nw = acc ? am : noise;
-  }
-  const int all_conf = __syncthreads_and(!valid || Hi < stop_entropy);
-  int same;
-  if (stop_rule == 0) same = __syncthreads_and(!valid || nw == old);
-  else same = __syncthreads_and(!valid || am == argmax_prev[i]) && st->has_prev;
-  if (valid) {
-    canvas[i] = nw;
-    accept[i] = acc ? 1 : 0;
-    argmax_prev[i] = am;
-  }
-  if (i == 0) {
-    const int unchanged = same ? st->unchanged + 1 : 0;
-    const bool last = t + 1 >= S;
-    const bool done = fixed_steps ? last : (last || all_conf || unchanged >= stop_unchanged);
-    st->unchanged = unchanged;
-    st->k = k;
-    st->t = t + 1;
-    st->steps = t + 1;
-    st->has_prev = 1;
-    st->done = done ? 1 : 0;
-    if (use_cond) cudaGraphSetConditional(cond, done ? 0u : 1u);
-  }
+  sample_and_stop(a, sm);
 }
 
 // ---------------------------------------------------------------------------
@@ -518,9 +426,10 @@ cudaError_t launch_sampler(cudaStream_t s, DevState* st, const float* H, const i
                            int accept_rule, int fixed_steps, int S,
                            cudaGraphConditionalHandle cond, int use_cond) {
   const int threads = ((C + 31) / 32) * 32;
-  k_sampler<<<1, threads, 0, s>>>(st, H, argmax, canvas, argmax_prev, accept, order, prefix, C, V,
-                                  seed, tau, stop_entropy, stop_unchanged, stop_rule, accept_rule,
-                                  fixed_steps, S, cond, use_cond);
+  SamplerArgs a = make_sampler_args(st, H, argmax, canvas, argmax_prev, accept, order, prefix, C, V,
+                                    seed, tau, stop_entropy, stop_unchanged, stop_rule,
+                                    accept_rule, fixed_steps, S, cond, use_cond);
+  k_sampler<<<1, threads, 0, s>>>(a);
   return cudaGetLastError();
 }
 

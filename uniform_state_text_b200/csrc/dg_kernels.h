@@ -6,6 +6,41 @@
 
 namespace dg {
 
+// Everything the entropy-bounded sampler and the stop test need for one step.
+struct SamplerArgs {
+  DevState* st;
+  const float* H;
+  const int32_t* argmax;
+  int32_t *canvas, *argmax_prev, *accept, *order;
+  float* prefix;
+  int C, V;
+  uint64_t seed;
+  float tau, stop_entropy;
+  int stop_unchanged, stop_rule, accept_rule, fixed_steps, S;
+  cudaGraphConditionalHandle cond;
+  int use_cond;
+};
+struct SamplerSmem {
+  float H[1024];
+  float sorted[1024];
+  int32_t order[1024];
+  int k;
+};
+inline SamplerArgs make_sampler_args(DevState* st, const float* H, const int32_t* argmax,
+                                     int32_t* canvas, int32_t* argmax_prev, int32_t* accept,
+                                     int32_t* order, float* prefix, int C, int V, uint64_t seed,
+                                     float tau, float stop_entropy, int stop_unchanged,
+                                     int stop_rule, int accept_rule, int fixed_steps, int S,
+                                     cudaGraphConditionalHandle cond, int use_cond) {
+  SamplerArgs a;
+  a.st = st; a.H = H; a.argmax = argmax; a.canvas = canvas; a.argmax_prev = argmax_prev;
+  a.accept = accept; a.order = order; a.prefix = prefix; a.C = C; a.V = V; a.seed = seed;
+  a.tau = tau; a.stop_entropy = stop_entropy; a.stop_unchanged = stop_unchanged;
+  a.stop_rule = stop_rule; a.accept_rule = accept_rule; a.fixed_steps = fixed_steps; a.S = S;
+  a.cond = cond; a.use_cond = use_cond;
+  return a;
+}
+
 cudaError_t launch_begin_block(cudaStream_t s, DevState* st, int32_t* target, int32_t* canvas,
                                float* sc, int C, int d, int V, uint64_t seed, int block);
 

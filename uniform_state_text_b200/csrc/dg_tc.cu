@@ -38,6 +38,7 @@
 #include <cstring>
 
 #include "dg_tc.h"
+#include "dg_sampler.cuh"
 
 namespace dg {
 namespace tc {
@@ -780,11 +781,55 @@ __global__ void __launch_bounds__(THREADS, 1)
 // largest logit exceeds its reference by more than redo_gap (its P could have
 // overflowed) is recomputed here exactly against its true maximum.
 // ---------------------------------------------------------------------------
+// Exact recomputation against the true maximum m: Z = sum e^(z-m),
+// S1 = sum e^(z-m)(z-m), sc = sum e^(z-m) E_v / Z. One warp per vocabulary
+// entry at a time; sc accumulates in shared memory.
+__device__ __noinline__ void merge_recompute(int i, int V, int d, const __nv_bfloat16* h,
+                                            const __nv_bfloat16* E, const float* scale_tab, int S,
+                                            const DevState* st, float m, float* H, float* sc,
+                                            float* sacc) {
+  __shared__ float sZ[8], sS[8], sInv;
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  const float scale = scale_tab[min(max(st->t, 0), S - 1)];
+  for (int k = threadIdx.x; k < d; k += blockDim.x) sacc[k] = 0.f;
+  __syncthreads();
+  const __nv_bfloat16* hr = h + (size_t)i * d;
+  float Zl = 0.f, S1l = 0.f;
+  for (int v = w; v < V; v += 8) {
+    const __nv_bfloat16* ev = E + (size_t)v * d;
+    float dot = 0.f;
+    for (int k = l; k < d; k += 32) dot = fmaf(__bfloat162float(hr[k]), __bfloat162float(ev[k]), dot);
+    for (int o = 16; o; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    const float dz = dot * scale - m;
+    const float e = expf(dz);
+    Zl += e;
+    S1l = fmaf(e, dz, S1l);
+    if (e > 0.f)
+      for (int k = l; k < d; k += 32) atomicAdd(&sacc[k], e * __bfloat162float(ev[k]));
+  }
+  __syncthreads();
+  if (l == 0) { sZ[w] = Zl; sS[w] = S1l; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float a = 0.f, b = 0.f;
+    for (int j = 0; j < 8; ++j) { a += sZ[j]; b += sS[j]; }
+    H[i] = fmaxf(logf(a) - b / a, 0.f);
+    sInv = 1.0f / a;
+  }
+  __syncthreads();
+  for (int k = threadIdx.x; k < d; k += blockDim.x) sc[(size_t)i * d + k] = sacc[k] * sInv;
+}
+
 __global__ void __launch_bounds__(256) k_merge_tc(DevState* st, const TcStat* ts, int nts,
     const float* mref, const float* Opart, int nO, int C, int V, int d, RowStat* rowstat,
     float* H, int32_t* argmax, float* sc, float redo_gap, const __nv_bfloat16* h,
-    const __nv_bfloat16* E, const float* scale_tab, int S) {
-  if (st->done) return;
+    const __nv_bfloat16* E, const float* scale_tab, int S, unsigned* ticket,
+    const SamplerArgs sa) {
+  if (st->done) {
+    if (sa.use_cond && blockIdx.x == 0 && threadIdx.x == 0) cudaGraphSetConditional(sa.cond, 0);
+    return;
+  }
+  __shared__ SamplerSmem sm;
   extern __shared__ float sacc[];   // [d], exact recomputation only
   const int i = blockIdx.x;
   float Z = 0.f, S1 = 0.f, best = -INFINITY;
@@ -840,41 +885,23 @@ __global__ void __launch_bounds__(256) k_merge_tc(DevState* st, const TcStat* ts
       for (int g = 0; g < nO; ++g) acc += Opart[g * pstride + (size_t)i * d + k];
       sc[(size_t)i * d + k] = acc * inv;
     }
-    return;
+  } else {
+    merge_recompute(i, V, d, h, E, scale_tab, S, st, sh_best, H, sc, sacc);
   }
-  // Exact recomputation against the true maximum m: Z = sum e^(z-m),
-  // S1 = sum e^(z-m)(z-m), sc = sum e^(z-m) E_v / Z. One warp per vocabulary
-  // entry at a time; sc accumulates in shared memory.
-  const float scale = scale_tab[min(max(st->t, 0), S - 1)];
-  const float m = sh_best;
-  for (int k = threadIdx.x; k < d; k += blockDim.x) sacc[k] = 0.f;
-  __syncthreads();
-  const __nv_bfloat16* hr = h + (size_t)i * d;
-  float Zl = 0.f, S1l = 0.f;
-  for (int v = w; v < V; v += 8) {
-    const __nv_bfloat16* ev = E + (size_t)v * d;
-    float dot = 0.f;
-    for (int k = l; k < d; k += 32) dot = fmaf(__bfloat162float(hr[k]), __bfloat162float(ev[k]), dot);
-    for (int o = 16; o; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-    const float dz = dot * scale - m;
-    const float e = expf(dz);
-    Zl += e;
-    S1l = fmaf(e, dz, S1l);
-    if (e > 0.f)
-      for (int k = l; k < d; k += 32) atomicAdd(&sacc[k], e * __bfloat162float(ev[k]));
-  }
-  __syncthreads();
-  if (l == 0) { sZ[w] = Zl; sS[w] = S1l; }
+  // The last row to finish runs the sampler for the whole canvas (its H and
+  // argmax inputs are final once every row has passed this point).
+  __shared__ unsigned sh_ticket;
   __syncthreads();
   if (threadIdx.x == 0) {
-    float a = 0.f, b = 0.f;
-    for (int j = 0; j < 8; ++j) { a += sZ[j]; b += sS[j]; }
-    H[i] = fmaxf(logf(a) - b / a, 0.f);
-    sh_inv = 1.0f / a;
+    __threadfence();
+    sh_ticket = atomicAdd(ticket, 1u);
   }
   __syncthreads();
-  for (int k = threadIdx.x; k < d; k += blockDim.x) sc[(size_t)i * d + k] = sacc[k] * sh_inv;
+  if (sh_ticket != (unsigned)(C - 1)) return;
+  __threadfence();
+  sample_and_stop(sa, sm);
 }
+
 
 }  // namespace tc
 
@@ -1103,14 +1130,16 @@ cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, 
 cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& pl, DevState* st, const TileStat* tstats,
                             const float* mref, RowStat* rowstat, float* H, int32_t* argmax,
                             float* sc, int32_t* redo_rows, float redo_gap, const void* h,
-                            const void* E, const float* scale_tab, int S) {
+                            const void* E, const float* scale_tab, int S,
+                            const SamplerArgs& sa) {
   TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
   const float* Opart = reinterpret_cast<const float*>(static_cast<const char*>(pl.ws) + L.Opart);
   (void)redo_rows;
   tc::k_merge_tc<<<pl.C, 256, sizeof(float) * pl.d, s>>>(
       st, reinterpret_cast<const TcStat*>(tstats), 2 * L.n_vt, mref, Opart, L.G, pl.C, pl.V, pl.d,
       rowstat, H, argmax, sc, redo_gap, static_cast<const __nv_bfloat16*>(h),
-      static_cast<const __nv_bfloat16*>(E), scale_tab, S);
+      static_cast<const __nv_bfloat16*>(E), scale_tab, S,
+      reinterpret_cast<unsigned*>(static_cast<char*>(pl.ws) + L.counters) + 2 * L.n_vt + 2, sa);
   return cudaGetLastError();
 }
 
