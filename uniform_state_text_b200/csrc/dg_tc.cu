@@ -56,15 +56,20 @@ constexpr int QN = 8;          // G1 item queue depth (tile indices handed to th
 constexpr uint32_t A_BYTES = BM * BK * 2;
 constexpr uint32_t B_BYTES = BN * BK * 2;
 // Pipeline depth per CTA-group size: the same ~192 KB of stages either way.
+// G2 units with two accumulators (W2 = 2, pairs only) stage twice the B per
+// K step, in four 48 KB stages (also 192 KB).
 template <int CG> struct Pipe {
   static constexpr int STAGES = CG == 2 ? 6 : 4;
   static constexpr uint32_t STAGE = A_BYTES + B_BYTES / CG;
+  static constexpr int STAGES_W2 = 4;
+  static constexpr uint32_t STAGE_W2 = A_BYTES + 2 * (B_BYTES / CG);
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 512;
 };
 constexpr unsigned long long TIMEOUT_NS = 2000000000ull;   // 2 s
 
 struct Params {
   int C, V, d, RB, n_vt, n_ranges, n_dt, G, n1, tiles_per_range, S;
+  int W2;                    // G2 accumulators per CTA: a G2 unit owns W2*256 columns of d
   const float* mref;
   const float* scale_tab;
   float* Opart;              // [G][C][d]
@@ -389,24 +394,32 @@ __device__ __forceinline__ bool item_take(int n, int* item, uint64_t* item_full,
   return true;
 }
 
+__device__ __forceinline__ bool is_g1_unit(const Params& p, int CG) {
+  return (int)(blockIdx.x / CG) < p.n1;
+}
+
 template <int CG>
 __global__ void __launch_bounds__(THREADS, 1)
     k_vocab_attention(const __grid_constant__ CUtensorMap tm_h,
                       const __grid_constant__ CUtensorMap tm_ek,
                       const __grid_constant__ CUtensorMap tm_emn,
                       const __grid_constant__ CUtensorMap tm_p, const Params p) {
-  constexpr int STAGES = Pipe<CG>::STAGES;
-  constexpr uint32_t STAGE_BYTES = Pipe<CG>::STAGE;     // A + this CTA's share of B
+  constexpr int NSTAGE_MAX = Pipe<CG>::STAGES;         // barrier array size
   constexpr int NB_ROWS = BN / CG;                      // B rows (G1) / columns (G2) per CTA
-  constexpr int HALF = BN / 2;                          // columns per epilogue warp
+  // G1 CTAs and single-accumulator G2 CTAs: Pipe::STAGES stages of A + B/CG;
+  // two-accumulator G2 CTAs: Pipe::STAGES_W2 stages of A + 2B/CG.
+  const bool w2 = (int)(blockIdx.x / CG) >= p.n1 && p.W2 == 2;
+  const int STAGES = w2 ? Pipe<CG>::STAGES_W2 : Pipe<CG>::STAGES;
+  const uint32_t STAGE_BYTES = w2 ? Pipe<CG>::STAGE_W2 : Pipe<CG>::STAGE;
+  const int HALF = (is_g1_unit(p, CG) ? BN : BN * p.W2) / 2;   // columns per epilogue warp
   if (p.st->done) return;                               // uniform over the grid
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  uint64_t* full = bars;                    // [STAGES] (leader's counts both CTAs' bytes)
-  uint64_t* empty = bars + STAGES;          // [STAGES]
-  uint64_t* acc_full = bars + 2 * STAGES;   // [2]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Pipe<CG>::STAGES * Pipe<CG>::STAGE);
+  uint64_t* full = bars;                        // [STAGES] (leader's counts both CTAs' bytes)
+  uint64_t* empty = bars + NSTAGE_MAX;          // [STAGES]
+  uint64_t* acc_full = bars + 2 * NSTAGE_MAX;   // [2]
   uint64_t* acc_empty = acc_full + 2;       // [2] (leader's counts both CTAs' epilogues)
   uint64_t* fin = acc_empty + 2;            // [1]
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(fin + 1);
@@ -467,7 +480,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     g = o / (RBI * p.n_dt);
     const int rem = o % (RBI * p.n_dt);
     rb2 = CG == 2 ? (int)rank : rem / p.n_dt;
-    dt = rem % p.n_dt;
+    dt = rem % p.n_dt;                  // slice of W2*256 columns of d
   }
   const unsigned ready_target = (unsigned)(p.RB * EPI_WARPS);
   const unsigned consumed_target = (unsigned)(RBI * p.n_dt);
@@ -530,10 +543,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (leader) mbar_expect_tx(&full[s], STAGE_BYTES * CG);
             tma_load<CG>(st, &tm_p, &full[s], (kc % (BN / BK)) * BK, (vt % RING) * p.C + rb2 * BM,
                          keep);
+            for (int b = 0; b < p.W2; ++b)
 #pragma unroll
-            for (int j = 0; j < NB_ROWS / 64; ++j)
-              tma_load<CG>(st + A_BYTES + j * (64 * BK * 2), &tm_emn, &full[s],
-                           dt * BN + (int)rank * NB_ROWS + j * 64, r * KV2 + kc * BK, drop);
+              for (int j = 0; j < NB_ROWS / 64; ++j)
+                tma_load<CG>(st + A_BYTES + (b * (NB_ROWS / 64) + j) * (64 * BK * 2), &tm_emn,
+                             &full[s], (dt * p.W2 + b) * BN + (int)rank * NB_ROWS + j * 64,
+                             r * KV2 + kc * BK, drop);
             ++issued;
             if (++s == STAGES) { s = 0; ph ^= 1; }
           }
@@ -606,9 +621,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k) {
               const uint64_t ad = sdesc(a0 + k * 32, 16, 1024);
-              // MN-major B: 64-column blocks 8 KB apart (LBO), 8-row K groups 1 KB apart (SBO)
-              const uint64_t bd = sdesc(b0 + k * (16 * 128), 64 * BK * 2, 1024);
-              mma<CG>(tmem, ad, bd, idesc, first ? 0u : 1u);
+              for (int b = 0; b < p.W2; ++b) {
+                // MN-major B: 64-column blocks 8 KB apart (LBO), 8-row K groups 1 KB apart (SBO)
+                const uint64_t bd = sdesc(b0 + b * (NB_ROWS / 64) * (64 * BK * 2) + k * (16 * 128),
+                                          64 * BK * 2, 1024);
+                mma<CG>(tmem + b * BN, ad, bd, idesc, first ? 0u : 1u);
+              }
               first = false;
             }
             commit<CG>(&empty[s]);
@@ -737,7 +755,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else {
       const bool has_work = g < p.n_ranges;
       const int row = rb2 * BM + r_local;
-      float* orow = p.Opart + ((size_t)g * p.C + row) * p.d + (size_t)dt * BN + c0;
+      float* orow = p.Opart + ((size_t)g * p.C + row) * p.d + (size_t)dt * BN * p.W2 + c0;
       bool ok = true;
       if (has_work) {
         ok = mbar_wait(&acc_full[0], 0, p);
@@ -913,6 +931,7 @@ namespace {
 struct TcLayout {
   size_t counters = 0, P = 0, Opart = 0, trace = 0, total = 0;
   int CG = 1;              // CTAs per MMA group (2: CTA pairs, M = 256)
+  int W2 = 1;              // accumulators per G2 unit (2: a 512-column slice of d)
   int RB = 0, n_vt = 0, n_ranges = 0, n_dt = 0, G = 0, n1 = 0, n2 = 0;   // n1, n2 in groups
 };
 
@@ -930,10 +949,11 @@ int device_sms() {
 TcLayout tc_layout(int C, int V, int d, int sms) {
   TcLayout L;
   L.CG = C == 256 ? 2 : 1;
+  L.W2 = (L.CG == 2 && d % (2 * tc::BN) == 0) ? 2 : 1;
   L.RB = C / tc::BM;
   L.n_vt = V / tc::BN;
   L.n_ranges = V / tc::KV2;
-  L.n_dt = d / tc::BN;
+  L.n_dt = d / (tc::BN * L.W2);
   // Choose the number of range groups G: G2 units = RBI * n_dt * G, G1 units take
   // the rest; minimise the larger of the two roles' per-unit work.
   const int units = sms / L.CG;
@@ -941,7 +961,7 @@ TcLayout tc_layout(int C, int V, int d, int sms) {
   // One G1 item costs about 1.3x a G2 range of the same MMA work (measured on
   // B200: the softmax epilogue and the HBM-side fill); weight it accordingly.
   const double u1 = 1.3 * tc::BM * tc::BN * d;                   // one G1 item
-  const double u2 = (double)tc::BM * tc::BN * tc::KV2;           // one G2 range
+  const double u2 = (double)L.W2 * tc::BM * tc::BN * tc::KV2;    // one G2 range
   const int per_g = RBI * L.n_dt;
   double best = 1e300;
   for (int G = 1; G <= L.n_ranges; ++G) {
@@ -1109,7 +1129,7 @@ cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, 
   char* base = static_cast<char*>(ws);
   tc::Params prm;
   prm.C = pl.C; prm.V = pl.V; prm.d = pl.d; prm.RB = L.RB; prm.n_vt = L.n_vt;
-  prm.n_ranges = L.n_ranges; prm.n_dt = L.n_dt; prm.G = L.G; prm.n1 = L.n1;
+  prm.n_ranges = L.n_ranges; prm.n_dt = L.n_dt; prm.G = L.G; prm.n1 = L.n1; prm.W2 = L.W2;
   prm.tiles_per_range = tc::KV2 / tc::BN; prm.S = S;
   prm.mref = mref; prm.scale_tab = scale_tab;
   prm.tstats2 = reinterpret_cast<TcStat*>(tstats);
