@@ -128,7 +128,8 @@ size_t dg_workspace_bytes(const dg_config* cfg);
  * Create a context.
  *   cfg       configuration (copied).
  *   E         device, [V][d] of cfg->dtype, the tied vocabulary embedding;
- *             read-only and caller-owned; must outlive the context.
+ *             16-byte aligned, read-only and caller-owned; must outlive the
+ *             context.
  *   workspace device, >= dg_workspace_bytes(cfg) bytes, 256-byte aligned,
  *             caller-owned; its contents are managed by the library.
  *   stream    a cudaStream_t (NULL = legacy default stream).

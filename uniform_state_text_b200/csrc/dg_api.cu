@@ -286,6 +286,7 @@ int dg_init(const dg_config* cfg, const void* E, void* workspace, size_t ws_byte
   int rc = make_layout(cfg, &L, why, sizeof(why));
   if (rc) return fail(nullptr, rc, "%s", why);
   if (!E || !workspace) return fail(nullptr, DG_EINVAL, "E and workspace must be device pointers");
+  if (((uintptr_t)E) % 16) return fail(nullptr, DG_EINVAL, "E must be 16-byte aligned");
   if (((uintptr_t)workspace) % kAlign) return fail(nullptr, DG_EINVAL, "workspace must be 256-byte aligned");
   if (ws_bytes < L.total)
     return fail(nullptr, DG_ENOMEM, "workspace has %zu bytes, needs %zu", ws_bytes, L.total);

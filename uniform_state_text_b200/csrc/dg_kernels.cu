@@ -55,42 +55,92 @@ __global__ void k_begin_block(DevState* st, int32_t* target, int32_t* canvas, fl
 // Stand-in hidden state and per-row logit reference.
 // One CTA per canvas row.
 // ---------------------------------------------------------------------------
+// Eight consecutive elements of E, sc or h (16-byte aligned for bf16, 32 for fp32).
+__device__ __forceinline__ void load8(const float* p, float v[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float v[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    v[2 * j] = __uint_as_float(w[j] << 16);
+    v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void store8(float* p, const float v[8]) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float v[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+    w[j] = *reinterpret_cast<const uint32_t*>(&b2);
+  }
+  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) k_prologue(const DevState* st, const T* E,
     const int32_t* target, const int32_t* canvas, const float* sc, T* h, int C, int V, int d,
     uint64_t seed, float A, float B, float sigma, int standin, const float* scale_tab, int S,
     const int32_t* argmax_prev, float* mref, unsigned* zero, int nzero) {
+  // Programmatic dependent launch: the previous step's kernels are complete
+  // after this wait; the attention kernel may start its set-up meanwhile.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
+  const int i = blockIdx.x;
+  // Token ids index rows of E; masking keeps caller-written ids in range
+  // (V is a power of two, valid ids are unchanged). All three are read before
+  // the loop state so that the loads overlap.
+  const int tgt = target[i] & (V - 1), can = canvas[i] & (V - 1);
+  const int prev_raw = argmax_prev[i] & (V - 1);
   if (st->done) return;
   if (zero && blockIdx.x == 0)
     for (int j = threadIdx.x; j < nzero; j += blockDim.x) zero[j] = 0u;
-  const int i = blockIdx.x;
   const int t = st->t;
   const int ts = min(max(t, 0), S - 1);
-  // Token ids index rows of E; masking keeps caller-written ids in range
-  // (V is a power of two, valid ids are unchanged).
-  const int tgt = target[i] & (V - 1), can = canvas[i] & (V - 1);
-  const int prev = st->has_prev ? (argmax_prev[i] & (V - 1)) : can;
+  const int prev = st->has_prev ? prev_raw : can;
   const uint64_t pre = key_prefix(seed, (uint64_t)(uint32_t)st->block, kTagNoise + (uint64_t)t);
   const T* Et = E + (size_t)tgt * d;
   const T* Ec = E + (size_t)can * d;
   const T* Ep = E + (size_t)prev * d;
+  T* hrow = h + (size_t)i * d;
+  const float* scrow = sc + (size_t)i * d;
   float dc = 0.f, dp = 0.f;
-#pragma unroll 4
-  for (int k = threadIdx.x; k < d; k += blockDim.x) {
-    T hv;
+  for (int k0 = threadIdx.x * 8; k0 < d; k0 += blockDim.x * 8) {
+    float ec[8], hv[8];
+    load8(Ec + k0, ec);
     if (standin) {
-      float v = A * to_f32(Et[k]) + B * to_f32(Ec[k]);
-      v = v + sc[(size_t)i * d + k];
-      v = v + sigma * gauss_from_key(sm64(pre ^ ((uint64_t)i * (uint64_t)d + (uint64_t)k)));
-      hv = from_f32<T>(v);
-      h[(size_t)i * d + k] = hv;
+      float et[8], s8[8];
+      load8(Et + k0, et);
+      load8(scrow + k0, s8);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint64_t idx = (uint64_t)i * (uint64_t)d + (uint64_t)(k0 + j);
+        float v = A * et[j] + B * ec[j];
+        v = v + s8[j];
+        v = v + sigma * gauss_from_key(sm64(pre ^ idx));
+        hv[j] = v;
+      }
+      store8(hrow + k0, hv);
+      // what the contraction reads is the stored (rounded) value
+#pragma unroll
+      for (int j = 0; j < 8; ++j) hv[j] = to_f32(from_f32<T>(hv[j]));
     } else {
-      hv = h[(size_t)i * d + k];
+      load8(hrow + k0, hv);
     }
     if (mref) {
-      const float hf = to_f32(hv);
-      dc = fmaf(hf, to_f32(Ec[k]), dc);
-      dp = fmaf(hf, to_f32(Ep[k]), dp);
+      float ep[8];
+      load8(Ep + k0, ep);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        dc = fmaf(hv[j], ec[j], dc);
+        dp = fmaf(hv[j], ep[j], dp);
+      }
     }
   }
   if (!mref) return;
@@ -366,16 +416,22 @@ cudaError_t launch_prologue(cudaStream_t s, int dtype, const DevState* st, const
                             void* h, int C, int V, int d, uint64_t seed, float A, float B, float sigma,
                             int standin, const float* scale_tab, int S,
                             const int32_t* argmax_prev, float* mref, unsigned* zero, int nzero) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(C);
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (dtype == 0)
-    k_prologue<float><<<C, 256, 0, s>>>(st, (const float*)E, target, canvas, sc, (float*)h, C, V, d,
-                                        seed, A, B, sigma, standin, scale_tab, S, argmax_prev,
-                                        mref, zero, nzero);
-  else
-    k_prologue<__nv_bfloat16><<<C, 256, 0, s>>>(st, (const __nv_bfloat16*)E, target, canvas, sc,
-                                                (__nv_bfloat16*)h, C, V, d, seed, A, B, sigma,
-                                                standin, scale_tab, S, argmax_prev, mref, zero,
-                                                nzero);
-  return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, k_prologue<float>, st, (const float*)E, target, canvas, sc,
+                              (float*)h, C, V, d, seed, A, B, sigma, standin, scale_tab, S,
+                              argmax_prev, mref, zero, nzero);
+  return cudaLaunchKernelEx(&cfg, k_prologue<__nv_bfloat16>, st, (const __nv_bfloat16*)E, target,
+                            canvas, sc, (__nv_bfloat16*)h, C, V, d, seed, A, B, sigma, standin,
+                            scale_tab, S, argmax_prev, mref, zero, nzero);
 }
 
 cudaError_t launch_simt_attention(cudaStream_t s, int dtype, DevState* st, const void* h,

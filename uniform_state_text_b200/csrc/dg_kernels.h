@@ -21,10 +21,10 @@ struct SamplerArgs {
   int use_cond;
 };
 struct SamplerSmem {
-  float H[1024];
-  float sorted[1024];
-  int32_t order[1024];
-  int k;
+  unsigned long long key[1024];   // (entropy bits, position); padded with ~0
+  float sorted[1024];             // entropies in rank order
+  float prefix[1024];             // their running sums
+  int32_t order[1024];            // positions in rank order
 };
 inline SamplerArgs make_sampler_args(DevState* st, const float* H, const int32_t* argmax,
                                      int32_t* canvas, int32_t* argmax_prev, int32_t* accept,

@@ -15,94 +15,85 @@ namespace dg {
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void sample_and_stop(const SamplerArgs& a, SamplerSmem& sm) {
   DevState* st = a.st;
-  const float* H = a.H;
-  const int32_t* argmax = a.argmax;
-  int32_t* canvas = a.canvas;
-  int32_t* argmax_prev = a.argmax_prev;
   const int C = a.C, V = a.V, accept_rule = a.accept_rule, stop_rule = a.stop_rule;
   const float tau = a.tau;
-  float* sH = sm.H;
-  float* sSorted = sm.sorted;
-  int32_t* sOrder = sm.order;
-  int& sk = sm.k;
   const int i = threadIdx.x;
   const bool valid = i < C;
+  // Every global input is read up front (one round trip): the loop state and
+  // this position's entropy, argmax, canvas token and previous argmax.
   const int t = st->t;
-  const float Hi = valid ? H[i] : 0.f;
-  if (valid) sH[i] = Hi;
+  const int blk = st->block;
+  const int has_prev = st->has_prev;
+  const int unchanged_before = st->unchanged;
+  float Hi = 0.f;
+  int32_t am = 0, old = 0, am_prev = 0;
+  if (valid) {
+    Hi = a.H[i];
+    am = a.argmax[i];
+    old = a.canvas[i];
+    am_prev = a.argmax_prev[i];
+  }
+  // Stable rank by (entropy, position) as one 64-bit key: entropies are >= 0,
+  // so their bit patterns order like their values (-0 is taken as +0).
+  const unsigned long long key =
+      ((unsigned long long)(Hi == 0.f ? 0u : __float_as_uint(Hi)) << 32) | (unsigned)i;
+  const int C2 = (C + 1) & ~1;
+  if (valid) sm.key[i] = key;
+  else if (i < C2) sm.key[i] = ~0ull;    // padding never ranks below a real entry
   __syncthreads();
-  // Stable rank by (entropy, position).
   int rank = 0;
   if (valid) {
-    for (int j = 0; j < C; ++j) {
-      const float Hj = sH[j];
-      rank += (Hj < Hi) || (Hj == Hi && j < i);
+    const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(sm.key);
+#pragma unroll 8
+    for (int j2 = 0; j2 < C2 / 2; ++j2) {
+      const ulonglong2 q = k2[j2];
+      rank += (q.x < key) + (q.y < key);
     }
-    sOrder[rank] = i;
-    sSorted[rank] = Hi;
+    sm.order[rank] = i;
+    sm.sorted[rank] = Hi;
   }
   __syncthreads();
   // Running entropy sums in sorted order, added one at a time in fp32 (a fixed
-  // summation order): warp 0 holds the sorted entropies in registers, lane l
-  // the entries [l*per, (l+1)*per), and relays the running sum lane to lane.
-  if (i < 32) {
-    const int per = (C + 31) / 32;   // <= 32
-    float v[32];
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int j = i * per + e;
-      v[e] = (e < per && j < C) ? sSorted[j] : 0.f;
+  // summation order) by one thread.
+  if (i == 0) {
+    float run = 0.f;
+#pragma unroll 16
+    for (int j = 0; j < C; ++j) {
+      run = __fadd_rn(run, sm.sorted[j]);
+      sm.prefix[j] = run;
     }
-    float run = 0.f, start = 0.f;
-    for (int src = 0; src < 32; ++src) {
-      if (i == src) {
-        start = run;
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (e < per) { run = __fadd_rn(run, v[e]); v[e] = run; }
-      }
-      run = __shfl_sync(0xffffffffu, run, src);
-    }
-    // prefix sums of non-negative terms never decrease, so the accepted
-    // positions are a prefix of the sorted order: count them
-    int k = 0;
-    float before = start;
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int j = i * per + e;
-      if (e < per && j < C) {
-        a.prefix[j] = v[e];
-        k += (accept_rule == 0 ? (v[e] <= tau) : (before <= tau)) ? 1 : 0;
-        before = v[e];
-      }
-    }
-    for (int o = 16; o; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
-    if (i == 0) sk = k;
   }
   __syncthreads();
-  const int k = sk;
-  int32_t am = 0, old = 0, nw = 0;
+  // Running sums of non-negative terms never decrease, so the accepted
+  // positions are a prefix of the sorted order: count them.
+  bool take = false;
+  if (valid) {
+    const float pj = sm.prefix[i];
+    a.prefix[i] = pj;
+    a.order[i] = sm.order[i];
+    const float before = i ? sm.prefix[i - 1] : 0.f;
+    take = accept_rule == 0 ? (pj <= tau) : (before <= tau);
+  }
+  const int k = __syncthreads_count(take);
+  int32_t nw = 0;
   bool acc = false;
   if (valid) {
-    a.order[i] = sOrder[i];
-    am = argmax[i];
-    old = canvas[i];
     acc = rank < k;
-    const uint64_t pre = key_prefix(a.seed, (uint64_t)(uint32_t)st->block, (uint64_t)t);
+    const uint64_t pre = key_prefix(a.seed, (uint64_t)(uint32_t)blk, (uint64_t)t);
     const int32_t noise = (int32_t)(sm64(pre ^ (uint64_t)i) & (uint64_t)(V - 1));
     nw = acc ? am : noise;
   }
   const int all_conf = __syncthreads_and(!valid || Hi < a.stop_entropy);
   int same;
   if (stop_rule == 0) same = __syncthreads_and(!valid || nw == old);
-  else same = __syncthreads_and(!valid || am == argmax_prev[i]) && st->has_prev;
+  else same = __syncthreads_and(!valid || am == am_prev) && has_prev;
   if (valid) {
-    canvas[i] = nw;
+    a.canvas[i] = nw;
     a.accept[i] = acc ? 1 : 0;
-    argmax_prev[i] = am;
+    a.argmax_prev[i] = am;
   }
   if (i == 0) {
-    const int unchanged = same ? st->unchanged + 1 : 0;
+    const int unchanged = same ? unchanged_before + 1 : 0;
     const bool last = t + 1 >= a.S;
     const bool done = a.fixed_steps ? last : (last || all_conf || unchanged >= a.stop_unchanged);
     st->unchanged = unchanged;

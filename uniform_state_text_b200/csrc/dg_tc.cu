@@ -412,7 +412,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int STAGES = w2 ? Pipe<CG>::STAGES_W2 : Pipe<CG>::STAGES;
   const uint32_t STAGE_BYTES = w2 ? Pipe<CG>::STAGE_W2 : Pipe<CG>::STAGE;
   const int HALF = (is_g1_unit(p, CG) ? BN : BN * p.W2) / 2;   // columns per epilogue warp
-  if (p.st->done) return;                               // uniform over the grid
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -467,6 +466,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   if constexpr (CG == 2) cluster_sync();   // peer barriers initialised before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_base_slot;
+  // Programmatic dependent launch: the set-up above overlapped the prologue;
+  // its outputs (h, m_ref, zeroed counters, loop state) are visible after the
+  // wait. The merge kernel may then start its own set-up.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
+  const bool skip = p.st->done != 0;                     // uniform over the grid
 
   // Work description. RBI: row blocks iterated by G1 items (1 for pairs, which
   // cover both row blocks with M = 256).
@@ -485,7 +490,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   const unsigned ready_target = (unsigned)(p.RB * EPI_WARPS);
   const unsigned consumed_target = (unsigned)(RBI * p.n_dt);
 
-  if (warp == 0) {
+  if (skip) {
+    // the block has stopped: no work this step
+  } else if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       TR_DECL(w_empty);
@@ -794,26 +801,33 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Per-row merge of the half-tile statistics (one CTA per row, fixed order):
-// H = log Z - S1/Z, argmax, sc = (sum of the G2 partials) / Z. A row whose
-// largest logit exceeds its reference by more than redo_gap (its P could have
-// overflowed) is recomputed here exactly against its true maximum.
+// Merge of the half-tile statistics, two canvas rows per CTA (256 threads
+// per row, fixed summation order): H = log Z - S1/Z, argmax, and
+// sc = (sum of the G2 partials) / Z. A row whose largest logit exceeds its
+// reference by more than redo_gap (its P could have overflowed) is recomputed
+// exactly against its true maximum. C/2 CTAs fit on the GPU at once, so the
+// last row to finish -- the one that runs the sampler -- is not held back by a
+// second wave.
 // ---------------------------------------------------------------------------
-// Exact recomputation against the true maximum m: Z = sum e^(z-m),
-// S1 = sum e^(z-m)(z-m), sc = sum e^(z-m) E_v / Z. One warp per vocabulary
-// entry at a time; sc accumulates in shared memory.
+constexpr int kMergeRows = 2;
+constexpr int kMergeThreadsPerRow = 256;
+
+// Exact recomputation of row i against its true maximum m by the whole CTA:
+// Z = sum e^(z-m), S1 = sum e^(z-m)(z-m), sc = sum e^(z-m) E_v / Z. One warp
+// per vocabulary entry at a time; sc accumulates in shared memory.
 __device__ __noinline__ void merge_recompute(int i, int V, int d, const __nv_bfloat16* h,
                                             const __nv_bfloat16* E, const float* scale_tab, int S,
                                             const DevState* st, float m, float* H, float* sc,
                                             float* sacc) {
-  __shared__ float sZ[8], sS[8], sInv;
+  __shared__ float sZ[32], sS[32], sInv;
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  const int nw = blockDim.x >> 5;
   const float scale = scale_tab[min(max(st->t, 0), S - 1)];
   for (int k = threadIdx.x; k < d; k += blockDim.x) sacc[k] = 0.f;
   __syncthreads();
   const __nv_bfloat16* hr = h + (size_t)i * d;
   float Zl = 0.f, S1l = 0.f;
-  for (int v = w; v < V; v += 8) {
+  for (int v = w; v < V; v += nw) {
     const __nv_bfloat16* ev = E + (size_t)v * d;
     float dot = 0.f;
     for (int k = l; k < d; k += 32) dot = fmaf(__bfloat162float(hr[k]), __bfloat162float(ev[k]), dot);
@@ -830,34 +844,48 @@ __device__ __noinline__ void merge_recompute(int i, int V, int d, const __nv_bfl
   __syncthreads();
   if (threadIdx.x == 0) {
     float a = 0.f, b = 0.f;
-    for (int j = 0; j < 8; ++j) { a += sZ[j]; b += sS[j]; }
+    for (int j = 0; j < nw; ++j) { a += sZ[j]; b += sS[j]; }
     H[i] = fmaxf(logf(a) - b / a, 0.f);
     sInv = 1.0f / a;
   }
   __syncthreads();
   for (int k = threadIdx.x; k < d; k += blockDim.x) sc[(size_t)i * d + k] = sacc[k] * sInv;
+  __syncthreads();
 }
 
-__global__ void __launch_bounds__(256) k_merge_tc(DevState* st, const TcStat* ts, int nts,
-    const float* mref, const float* Opart, int nO, int C, int V, int d, RowStat* rowstat,
-    float* H, int32_t* argmax, float* sc, float redo_gap, const __nv_bfloat16* h,
-    const __nv_bfloat16* E, const float* scale_tab, int S, unsigned* ticket,
-    const SamplerArgs sa) {
+__global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(DevState* st,
+    const TcStat* ts, int nts, const float* mref, const float* Opart, int nO, int C, int V, int d,
+    RowStat* rowstat, float* H, int32_t* argmax, float* sc, float redo_gap,
+    const __nv_bfloat16* h, const __nv_bfloat16* E, const float* scale_tab, int S,
+    unsigned* ticket, const SamplerArgs sa) {
+  // Programmatic dependent launch: wait for the attention kernel's results,
+  // then let the next step's prologue be scheduled (it waits for this grid).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
   if (st->done) {
     if (sa.use_cond && blockIdx.x == 0 && threadIdx.x == 0) cudaGraphSetConditional(sa.cond, 0);
     return;
   }
   __shared__ SamplerSmem sm;
   extern __shared__ float sacc[];   // [d], exact recomputation only
-  const int i = blockIdx.x;
+  const int r = threadIdx.x / kMergeThreadsPerRow;      // row of this CTA
+  const int tid = threadIdx.x % kMergeThreadsPerRow;
+  const int i0 = blockIdx.x * kMergeRows;
+  const int i = i0 + r;
+  const bool row_ok = i < C;
+  const float mref_i = row_ok ? mref[i] : 0.f;
   float Z = 0.f, S1 = 0.f, best = -INFINITY;
   int arg = 0x7fffffff;
-#pragma unroll 4
-  for (int j = threadIdx.x; j < nts; j += blockDim.x) {
-    const TcStat t = ts[(size_t)i * nts + j];
-    Z += t.Z;
-    S1 += t.S1;
-    if (better(t.best, t.arg, best, arg)) { best = t.best; arg = t.arg; }
+  if (row_ok) {
+    const float4* ts4 = reinterpret_cast<const float4*>(ts + (size_t)i * nts);
+#pragma unroll 8
+    for (int j = tid; j < nts; j += kMergeThreadsPerRow) {
+      const float4 t = ts4[j];                 // {Z, S1, best, arg}
+      const int ta = __float_as_int(t.w);
+      Z += t.x;
+      S1 += t.y;
+      if (better(t.z, ta, best, arg)) { best = t.z; arg = ta; }
+    }
   }
   for (int o = 16; o; o >>= 1) {
     Z += __shfl_xor_sync(0xffffffffu, Z, o);
@@ -866,58 +894,72 @@ __global__ void __launch_bounds__(256) k_merge_tc(DevState* st, const TcStat* ts
     const int oa = __shfl_xor_sync(0xffffffffu, arg, o);
     if (better(ob, oa, best, arg)) { best = ob; arg = oa; }
   }
-  __shared__ float sZ[8], sS[8], sB[8];
-  __shared__ int sA[8];
-  __shared__ float sh_inv, sh_best;
-  __shared__ int sh_redo;
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  if (l == 0) { sZ[w] = Z; sS[w] = S1; sB[w] = best; sA[w] = arg; }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    Z = sZ[0]; S1 = sS[0]; best = sB[0]; arg = sA[0];
-    for (int j = 1; j < (int)(blockDim.x >> 5); ++j) {
-      Z += sZ[j];
-      S1 += sS[j];
-      if (better(sB[j], sA[j], best, arg)) { best = sB[j]; arg = sA[j]; }
-    }
-    H[i] = fmaxf(logf(Z) - S1 / Z, 0.f);
-    argmax[i] = arg;
-    RowStat rs;
-    rs.m = mref[i]; rs.Z = Z; rs.pad[0] = best; rs.pad[1] = 0.f;
-    rowstat[i] = rs;
-    const float gap = best - mref[i];
-    const int redo = !(gap <= redo_gap) || !(Z > 0.f) || !(Z < INFINITY);
-    if (redo) atomicAdd(&st->redo, 1);
-    sh_redo = redo;
-    sh_inv = 1.0f / Z;
-    sh_best = best;
-  }
-  __syncthreads();
-  if (!sh_redo) {
-    const float inv = sh_inv;
-    const size_t pstride = (size_t)C * d;
-#pragma unroll 2
-    for (int k = threadIdx.x; k < d; k += blockDim.x) {
-      float acc = 0.f;
-#pragma unroll 4
-      for (int g = 0; g < nO; ++g) acc += Opart[g * pstride + (size_t)i * d + k];
-      sc[(size_t)i * d + k] = acc * inv;
-    }
-  } else {
-    merge_recompute(i, V, d, h, E, scale_tab, S, st, sh_best, H, sc, sacc);
-  }
-  // The last row to finish runs the sampler for the whole canvas (its H and
-  // argmax inputs are final once every row has passed this point).
+  constexpr int WPR = kMergeThreadsPerRow / 32;   // warps per row
+  __shared__ float sZ[kMergeRows][WPR], sS[kMergeRows][WPR], sB[kMergeRows][WPR];
+  __shared__ int sA[kMergeRows][WPR];
+  __shared__ float sh_inv[kMergeRows], sh_best[kMergeRows];
+  __shared__ int sh_redo[kMergeRows];
   __shared__ unsigned sh_ticket;
+  const int w = tid >> 5, l = tid & 31;
+  if (l == 0) { sZ[r][w] = Z; sS[r][w] = S1; sB[r][w] = best; sA[r][w] = arg; }
   __syncthreads();
+  if (tid == 0) {
+    int redo = 0;
+    if (row_ok) {
+      Z = sZ[r][0]; S1 = sS[r][0]; best = sB[r][0]; arg = sA[r][0];
+      for (int j = 1; j < WPR; ++j) {
+        Z += sZ[r][j];
+        S1 += sS[r][j];
+        if (better(sB[r][j], sA[r][j], best, arg)) { best = sB[r][j]; arg = sA[r][j]; }
+      }
+      H[i] = fmaxf(logf(Z) - S1 / Z, 0.f);
+      argmax[i] = arg;
+      RowStat rs;
+      rs.m = mref_i; rs.Z = Z; rs.pad[0] = best; rs.pad[1] = 0.f;
+      rowstat[i] = rs;
+      const float gap = best - mref_i;
+      redo = !(gap <= redo_gap) || !(Z > 0.f) || !(Z < INFINITY);
+      if (redo) atomicAdd(&st->redo, 1);
+    }
+    sh_redo[r] = redo;
+    sh_inv[r] = 1.0f / Z;
+    sh_best[r] = best;
+  }
+  __syncthreads();
+  // A row whose reference was too low gets its exact H (and sc) before it
+  // counts as finished.
+  for (int q = 0; q < kMergeRows; ++q)
+    if (sh_redo[q]) merge_recompute(i0 + q, V, d, h, E, scale_tab, S, st, sh_best[q], H, sc, sacc);
+  // The sampler needs every row's H and argmax, not sc: the last CTA to post
+  // them runs it for the whole canvas while the other CTAs still sum sc.
   if (threadIdx.x == 0) {
     __threadfence();
     sh_ticket = atomicAdd(ticket, 1u);
   }
   __syncthreads();
-  if (sh_ticket != (unsigned)(C - 1)) return;
-  __threadfence();
-  sample_and_stop(sa, sm);
+  if (sh_ticket == gridDim.x - 1) {
+    __threadfence();
+    sample_and_stop(sa, sm);
+  }
+  // sc of the rows that were not recomputed: four columns per thread and
+  // pass, the partials added in g order.
+  const size_t pstride = (size_t)C * d;
+  const int d4 = d / 4;
+  for (int x = threadIdx.x; x < kMergeRows * d4; x += blockDim.x) {
+    const int q = x / d4, k = (x % d4) * 4;
+    const int row = i0 + q;
+    if (row >= C || sh_redo[q]) continue;
+    const float* orow = Opart + (size_t)row * d + k;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int g = 0; g < nO; ++g) {
+      const float4 o = *reinterpret_cast<const float4*>(orow + g * pstride);
+      acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
+    }
+    const float inv = sh_inv[q];
+    *reinterpret_cast<float4*>(sc + (size_t)row * d + k) =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  }
 }
 
 
@@ -1033,18 +1075,23 @@ cudaError_t launch_kernel(cudaStream_t s, int units, const CUtensorMap* maps, co
   cfg.blockDim = dim3(tc::THREADS);
   cfg.dynamicSmemBytes = tc::Pipe<CG>::SMEM;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
+  cfg.attrs = attr;
   if (CG == 2) {
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // May start (barrier set-up, TMEM allocation) while the prologue finishes;
+    // every CTA of the prologue has started by then, so the grid still fits.
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.numAttrs = 2;
   } else {
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
+    cfg.numAttrs = 1;
   }
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, tc::k_vocab_attention<CG>, maps[0], maps[1], maps[2], maps[3], prm);
 }
 
@@ -1155,12 +1202,21 @@ cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& pl, DevState* st, cons
   TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
   const float* Opart = reinterpret_cast<const float*>(static_cast<const char*>(pl.ws) + L.Opart);
   (void)redo_rows;
-  tc::k_merge_tc<<<pl.C, 256, sizeof(float) * pl.d, s>>>(
-      st, reinterpret_cast<const TcStat*>(tstats), 2 * L.n_vt, mref, Opart, L.G, pl.C, pl.V, pl.d,
-      rowstat, H, argmax, sc, redo_gap, static_cast<const __nv_bfloat16*>(h),
-      static_cast<const __nv_bfloat16*>(E), scale_tab, S,
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((pl.C + tc::kMergeRows - 1) / tc::kMergeRows);
+  cfg.blockDim = dim3(tc::kMergeRows * tc::kMergeThreadsPerRow);
+  cfg.dynamicSmemBytes = sizeof(float) * pl.d;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(
+      &cfg, tc::k_merge_tc, st, reinterpret_cast<const TcStat*>(tstats), 2 * L.n_vt, mref, Opart,
+      L.G, pl.C, pl.V, pl.d, rowstat, H, argmax, sc, redo_gap,
+      static_cast<const __nv_bfloat16*>(h), static_cast<const __nv_bfloat16*>(E), scale_tab, S,
       reinterpret_cast<unsigned*>(static_cast<char*>(pl.ws) + L.counters) + 2 * L.n_vt + 2, sa);
-  return cudaGetLastError();
 }
 
 void tc_partials(const TcPlan& pl, const float** Opart, int* nO) {
