@@ -395,7 +395,7 @@ __global__ void __launch_bounds__(1024) k_sampler(SamplerArgs a) {
     if (a.use_cond && threadIdx.x == 0) cudaGraphSetConditional(a.cond, 0);
     return;
   }
-  sample_and_stop(a, sm);
+  sample_and_stop(a, sm, blockDim.x);
 }
 
 // ---------------------------------------------------------------------------

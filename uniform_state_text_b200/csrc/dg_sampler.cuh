@@ -1,19 +1,41 @@
 // Entropy-bounded sampler and adaptive stop ("A Visual Guide to DiffusionGemma",
 // 5.3 adaptive stop, 5.4 token acceptance and re-noising), as a device function
-// run by one CTA with blockDim >= C. Used by k_sampler (CUDA-core path) and by
-// the last CTA of the tensor-core merge.
+// run by the first nthreads >= C threads of one CTA. Used by k_sampler
+// (CUDA-core path) and by the last CTA of the tensor-core merge.
 #pragma once
 #include "dg_common.cuh"
 #include "dg_kernels.h"
 
 namespace dg {
 
+// Barrier 1 over the first n threads of the CTA (n a multiple of 32): the
+// sampler synchronises only the threads that run it, so the rest of the CTA
+// may do other work meanwhile.
+__device__ __forceinline__ void sampler_bar(int n) {
+  asm volatile("bar.sync 1, %0;" ::"r"(n) : "memory");
+}
+__device__ __forceinline__ int sampler_bar_count(int n, bool pred) {
+  int c;
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.popc.u32 %0, 1, %2, p;\n\t}"
+               : "=r"(c) : "r"((unsigned)pred), "r"(n) : "memory");
+  return c;
+}
+__device__ __forceinline__ bool sampler_bar_and(int n, bool pred) {
+  unsigned r;
+  asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, %2, p;"
+               "\n\tselp.u32 %0, 1, 0, q;\n\t}"
+               : "=r"(r) : "r"((unsigned)pred), "r"(n) : "memory");
+  return r != 0;
+}
+
 // ---------------------------------------------------------------------------
-// Entropy-bounded sampler and adaptive stop, run by one CTA (blockDim >= C):
+// Entropy-bounded sampler and adaptive stop, run by threads [0, nthreads) of
+// one CTA (nthreads >= C, a multiple of 32; they synchronise on barrier 1):
 // the body of k_sampler, also run by the last CTA of the tensor-core merge.
 // The caller has checked that the block is not done.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void sample_and_stop(const SamplerArgs& a, SamplerSmem& sm) {
+__device__ __forceinline__ void sample_and_stop(const SamplerArgs& a, SamplerSmem& sm,
+                                                int nthreads) {
   DevState* st = a.st;
   const int C = a.C, V = a.V, accept_rule = a.accept_rule, stop_rule = a.stop_rule;
   const float tau = a.tau;
@@ -40,7 +62,7 @@ __device__ __forceinline__ void sample_and_stop(const SamplerArgs& a, SamplerSme
   const int C2 = (C + 1) & ~1;
   if (valid) sm.key[i] = key;
   else if (i < C2) sm.key[i] = ~0ull;    // padding never ranks below a real entry
-  __syncthreads();
+  sampler_bar(nthreads);
   int rank = 0;
   if (valid) {
     const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(sm.key);
@@ -52,7 +74,7 @@ __device__ __forceinline__ void sample_and_stop(const SamplerArgs& a, SamplerSme
     sm.order[rank] = i;
     sm.sorted[rank] = Hi;
   }
-  __syncthreads();
+  sampler_bar(nthreads);
   // Running entropy sums in sorted order, added one at a time in fp32 (a fixed
   // summation order) by one thread.
   if (i == 0) {
@@ -63,7 +85,7 @@ __device__ __forceinline__ void sample_and_stop(const SamplerArgs& a, SamplerSme
       sm.prefix[j] = run;
     }
   }
-  __syncthreads();
+  sampler_bar(nthreads);
   // Running sums of non-negative terms never decrease, so the accepted
   // positions are a prefix of the sorted order: count them.
   bool take = false;
@@ -74,7 +96,7 @@ __device__ __forceinline__ void sample_and_stop(const SamplerArgs& a, SamplerSme
     const float before = i ? sm.prefix[i - 1] : 0.f;
     take = accept_rule == 0 ? (pj <= tau) : (before <= tau);
   }
-  const int k = __syncthreads_count(take);
+  const int k = sampler_bar_count(nthreads, take);
   int32_t nw = 0;
   bool acc = false;
   if (valid) {
@@ -83,10 +105,10 @@ __device__ __forceinline__ void sample_and_stop(const SamplerArgs& a, SamplerSme
     const int32_t noise = (int32_t)(sm64(pre ^ (uint64_t)i) & (uint64_t)(V - 1));
     nw = acc ? am : noise;
   }
-  const int all_conf = __syncthreads_and(!valid || Hi < a.stop_entropy);
+  const int all_conf = sampler_bar_and(nthreads, !valid || Hi < a.stop_entropy);
   int same;
-  if (stop_rule == 0) same = __syncthreads_and(!valid || nw == old);
-  else same = __syncthreads_and(!valid || am == am_prev) && has_prev;
+  if (stop_rule == 0) same = sampler_bar_and(nthreads, !valid || nw == old);
+  else same = sampler_bar_and(nthreads, !valid || am == am_prev) && has_prev;
   if (valid) {
     a.canvas[i] = nw;
     a.accept[i] = acc ? 1 : 0;

@@ -931,21 +931,33 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
   for (int q = 0; q < kMergeRows; ++q)
     if (sh_redo[q]) merge_recompute(i0 + q, V, d, h, E, scale_tab, S, st, sh_best[q], H, sc, sacc);
   // The sampler needs every row's H and argmax, not sc: the last CTA to post
-  // them runs it for the whole canvas while the other CTAs still sum sc.
+  // them runs it for the whole canvas while the other CTAs still sum sc. The
+  // ticket is an acquire-release add: this CTA's H and argmax are visible
+  // before it counts, and the last CTA sees every other CTA's.
   if (threadIdx.x == 0) {
-    __threadfence();
-    sh_ticket = atomicAdd(ticket, 1u);
+    unsigned old;
+    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(old) : "l"(ticket) : "memory");
+    sh_ticket = old;
   }
   __syncthreads();
-  if (sh_ticket == gridDim.x - 1) {
-    __threadfence();
-    sample_and_stop(sa, sm);
+  // In the last CTA the first nsamp threads run the sampler and the others
+  // sum sc; elsewhere every thread sums sc.
+  const bool last = sh_ticket == gridDim.x - 1;
+  const int nsamp = (C + 31) / 32 * 32;
+  int x0 = threadIdx.x, xstep = blockDim.x;
+  if (last) {
+    if (threadIdx.x < nsamp) {
+      sample_and_stop(sa, sm, nsamp);
+      return;
+    }
+    x0 = threadIdx.x - nsamp;
+    xstep = blockDim.x - nsamp;
   }
   // sc of the rows that were not recomputed: four columns per thread and
   // pass, the partials added in g order.
   const size_t pstride = (size_t)C * d;
   const int d4 = d / 4;
-  for (int x = threadIdx.x; x < kMergeRows * d4; x += blockDim.x) {
+  for (int x = x0; x < kMergeRows * d4; x += xstep) {
     const int q = x / d4, k = (x % d4) * 4;
     const int row = i0 + q;
     if (row >= C || sh_redo[q]) continue;
@@ -1202,6 +1214,8 @@ cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& pl, DevState* st, cons
   TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
   const float* Opart = reinterpret_cast<const float*>(static_cast<const char*>(pl.ws) + L.Opart);
   (void)redo_rows;
+  // the sampler runs on one row's threads of the last CTA
+  if (pl.C > tc::kMergeThreadsPerRow) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((pl.C + tc::kMergeRows - 1) / tc::kMergeRows);
   cfg.blockDim = dim3(tc::kMergeRows * tc::kMergeThreadsPerRow);
