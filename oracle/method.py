@@ -29,7 +29,12 @@ Readings where the pages are silent or garbled (each also listed in the design doc):
     maximum so far is the current entry, so a position is accepted when the sum
     of the entries before it is <= tau (always accepts at least one).
   * Tokens are chosen by argmax (the most likely token per position, [VG] 3.2);
-    ties go to the lowest vocabulary index.
+    ties go to the lowest vocabulary index. token_rule 1 instead draws each
+    position's token from its softmax distribution ([VG] 3.2 names the
+    multinomial draw): the Gumbel-max form, argmax_v (z_v + G_v) with one
+    keyed standard Gumbel variate G_v per (position, entry) (rng.gumbel, step
+    field TAG_GUMBEL + t, index position * V + v). Entropy, sc, the stop test
+    and the emitted prediction still use the distribution and its argmax.
   * Logits temperature: T_t = T_end + (T_start - T_end) * (1 + cos(pi t/(S-1)))/2,
     t = 0..S-1 (the cosine schedule of [WS]; lower temperature at later steps,
     [VG] 5.3); S = 1 gives T_start.
@@ -134,16 +139,42 @@ class Attention:
     sc: np.ndarray          # fp64 [rows, d]; sum_v p_v E_v
     zmax: np.ndarray        # fp64 [rows]; largest logit
     margin: np.ndarray      # fp64 [rows]; gap between the two largest logits
+    sampled: np.ndarray | None = None   # int64 [rows]; Gumbel-max draw (token_rule 1)
+    smargin: np.ndarray | None = None   # fp64 [rows]; gap between the two best z + G
 
 
-def vocab_attention(h: np.ndarray, E: np.ndarray, scale: float) -> Attention:
+def gumbel_max(z: np.ndarray, seed: int, block: int, t: int, rows0: int = 0):
+    """Draw one token per row from softmax(z) as argmax_v (z_v + G_v).
+
+    G_v are independent standard Gumbel variates keyed on (seed, block,
+    TAG_GUMBEL + t, row * V + v); row numbers start at rows0. Returns the tokens
+    (first index on exact ties) and the gap between the two best scores.
+    """
+    rows, V = z.shape
+    tok = np.empty(rows, dtype=np.int64)
+    gap = np.empty(rows)
+    for i in range(rows):
+        idx = np.uint64((rows0 + i) * V) + np.arange(V, dtype=np.uint64)
+        score = z[i] + rng.gumbel(seed, block, rng.TAG_GUMBEL + t, idx)
+        tok[i] = int(np.argmax(score))
+        if V > 1:
+            top2 = np.partition(score, -2)[-2:]
+            gap[i] = abs(top2[1] - top2[0])
+        else:
+            gap[i] = np.inf
+    return tok, gap
+
+
+def vocab_attention(h: np.ndarray, E: np.ndarray, scale: float,
+                    gumbel_key: tuple[int, int, int] | None = None) -> Attention:
     """Per position: softmax of the tempered logits, its entropy, argmax and p.E.
 
     The probability of each vocabulary token is the softmax of the logits
     divided by the temperature ([VG] 5.3 logits scheduler); confidence is the
     entropy of that distribution ([VG] 5.3 adaptive stop, 5.4 acceptance); the
     self-conditioning vector is the probability row times the embedding table
-    ([VG] 5.1, [EX] self-conditioning).
+    ([VG] 5.1, [EX] self-conditioning). With gumbel_key = (seed, block, t) it
+    also draws one token per position from that distribution (gumbel_max).
     """
     z = logits(h, E, scale)
     rows = z.shape[0]
@@ -168,7 +199,11 @@ def vocab_attention(h: np.ndarray, E: np.ndarray, scale: float) -> Attention:
     for v0 in range(0, E.shape[0], _VOCAB_CHUNK):
         Ec = E[v0:v0 + _VOCAB_CHUNK].astype(np.float64)
         sc += p[:, v0:v0 + Ec.shape[0]] @ Ec
-    return Attention(argmax=argmax, H=H, sc=sc, zmax=zmax, margin=margin)
+    sampled = smargin = None
+    if gumbel_key is not None:
+        sampled, smargin = gumbel_max(z, *gumbel_key)
+    return Attention(argmax=argmax, H=H, sc=sc, zmax=zmax, margin=margin,
+                     sampled=sampled, smargin=smargin)
 
 
 # ----------------------------------------------------------------------------
@@ -213,7 +248,8 @@ def entropy_bounded_accept(H32: np.ndarray, tau: float, rule: int) -> Acceptance
 
 
 def renoise(w, accepted, argmax, block: int, t: int) -> np.ndarray:
-    """Accepted positions take the argmax; every rejected one a fresh uniform token."""
+    """Accepted positions take the chosen token (argmax, or the draw under
+    token_rule 1); every rejected one a fresh uniform token."""
     noise = rng.tokens(w.seed, block, t, np.arange(w.C, dtype=np.uint64), w.V)
     return np.where(accepted, argmax, noise).astype(np.int64)
 
@@ -261,11 +297,16 @@ def step(w, E: np.ndarray, st: State, h: np.ndarray | None = None) -> StepRecord
     T = temperature(t, w.max_steps, w.T_start, w.T_end)
     if h is None:
         h = standin_hidden(w, E, st.target, st.canvas, st.sc, st.block, t)
-    att = vocab_attention(h, E, w.logit_scale / T)
+    multinomial = getattr(w, "token_rule", 0) == 1
+    if multinomial:
+        att = vocab_attention(h, E, w.logit_scale / T, gumbel_key=(w.seed, st.block, t))
+    else:
+        att = vocab_attention(h, E, w.logit_scale / T)
     H32 = att.H.astype(np.float32)
     acc = entropy_bounded_accept(H32, w.tau, w.accept_rule)
     noise = rng.tokens(w.seed, st.block, t, np.arange(w.C, dtype=np.uint64), w.V)
-    canvas_out = np.where(acc.accepted, att.argmax, noise).astype(np.int64)
+    chosen = att.sampled if multinomial else att.argmax
+    canvas_out = np.where(acc.accepted, chosen, noise).astype(np.int64)
     all_conf = bool(np.all(H32 < np.float32(w.stop_entropy)))
     if w.stop_rule == 0:
         same = bool(np.array_equal(canvas_out, st.canvas))

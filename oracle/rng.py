@@ -20,6 +20,13 @@ Token draws take key & (V - 1) (V is a power of two, so this is exact and
 unbiased). Gaussian draws use Box-Muller on two 24-bit uniforms cut from one
 key: u1 = ((k >> 40) + 1) / 2**24 in (0, 1], u2 = ((k >> 16) & 0xFFFFFF) / 2**24
 in [0, 1), g = sqrt(-2 ln u1) * cos(2 pi u2).
+
+The multinomial token choice (A Visual Guide to DiffusionGemma, 3.2: tokens
+are drawn from the predicted distribution) uses one Gumbel variate per
+(position, vocabulary entry). Standard Gumbel draws come from one key each:
+W = (2 (k >> 41) + 1) / 2**24, an odd multiple of 2**-24 in (0, 1) that fp32
+holds exactly; X = -ln(1 - W) is then a unit exponential and G = -ln X a
+standard Gumbel variate (P(G <= x) = exp(-exp(-x))).
 """
 from __future__ import annotations
 
@@ -34,6 +41,7 @@ _MASK = (1 << 64) - 1
 TAG_INIT_CANVAS = (1 << 63) + 1
 TAG_TARGET = (1 << 63) + 2
 TAG_NOISE = 1 << 62          # + step index
+TAG_GUMBEL = 1 << 61         # + step index; index = position * V + vocabulary entry
 
 
 def _u64(x) -> np.ndarray:
@@ -78,3 +86,14 @@ def gaussian(seed: int, block: int, step: int, index) -> np.ndarray:
     u1 = ((k >> np.uint64(40)).astype(np.float64) + 1.0) * 2.0 ** -24
     u2 = ((k >> np.uint64(16)) & np.uint64(0xFFFFFF)).astype(np.float64) * 2.0 ** -24
     return np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)
+
+
+def gumbel_uniform(k) -> np.ndarray:
+    """W = (2 (k >> 41) + 1) / 2**24 in (0, 1), fp64 (exact in fp32 as well)."""
+    return ((k >> np.uint64(41)).astype(np.float64) * 2.0 + 1.0) * 2.0 ** -24
+
+
+def gumbel(seed: int, block: int, step: int, index) -> np.ndarray:
+    """Standard Gumbel draws (fp64): G = -ln(-ln(1 - W)) from one key per index."""
+    W = gumbel_uniform(key(seed, block, step, index))
+    return -np.log(-np.log1p(-W))

@@ -66,6 +66,7 @@ class Workload:
     stop_unchanged: int = 3
     stop_rule: int = 0      # 0: canvas unchanged, 1: argmax unchanged
     accept_rule: int = 0    # 0: cumulative sum, 1: cumulative sum minus max
+    token_rule: int = 0     # 0: argmax, 1: multinomial draw (Gumbel-max)
     fixed_steps: int = 0    # 1: run exactly max_steps (timing mode)
     seed: int = 0
     blocks: int = 1

@@ -107,3 +107,42 @@ def test_dropped_noise_term_is_caught(monkeypatch):
     real = rng.gaussian
     monkeypatch.setattr(rng, "gaussian", lambda *a: 0.0 * real(*a))
     assert _fails(T_std.test_standin_noise_statistics_and_sc_term)
+
+
+# --- multinomial draw (Gumbel-max) -------------------------------------------
+import test_oracle_gumbel as T_gum
+
+
+def test_gumbel_sign_flip_is_caught(monkeypatch):
+    def bad(seed, block, step, index):
+        W = rng.gumbel_uniform(rng.key(seed, block, step, index))
+        return np.log(-np.log1p(-W))
+    monkeypatch.setattr(rng, "gumbel", bad)
+    assert _fails(T_gum.test_gumbel_cdf_mean_variance)
+
+
+def test_gumbel_draw_at_wrong_temperature_is_caught(monkeypatch):
+    real = M.gumbel_max
+    monkeypatch.setattr(M, "gumbel_max", lambda z, *a, **k: real(2.0 * z, *a, **k))
+    assert _fails(T_gum.test_draw_follows_softmax, [0.0, 1.0, 2.0, -1.0])
+
+
+def test_gumbel_key_without_row_is_caught(monkeypatch):
+    real = rng.gumbel
+
+    def bad(seed, block, step, index):
+        return real(seed, block, step, np.asarray(index, dtype=np.uint64) % np.uint64(4))
+    monkeypatch.setattr(rng, "gumbel", bad)
+    assert _fails(T_gum.test_draw_follows_softmax, [0.0, 1.0, 2.0, -1.0])
+
+
+def test_multinomial_step_taking_the_argmax_is_caught(monkeypatch):
+    real = M.vocab_attention
+
+    def bad(h, E, scale, gumbel_key=None):
+        a = real(h, E, scale, gumbel_key=gumbel_key)
+        if a.sampled is not None:
+            a.sampled = a.argmax.copy()
+        return a
+    monkeypatch.setattr(M, "vocab_attention", bad)
+    assert _fails(T_gum.test_step_accepts_the_draw_and_keeps_the_distribution)
