@@ -64,6 +64,12 @@ extern "C" {
 #define DG_ACCEPT_CUMSUM    0  /* inclusive running entropy sum <= tau         */
 #define DG_ACCEPT_MINUS_MAX 1  /* running sum minus the largest so far <= tau  */
 
+/* Token chosen at an accepted position ([VG] 3.2). */
+#define DG_TOKEN_ARGMAX       0  /* the most likely token (lowest index on ties) */
+#define DG_TOKEN_MULTINOMIAL  1  /* a draw from the position's softmax: the      */
+                                 /* Gumbel-max argmax_v (z_v + G_v), G_v keyed on */
+                                 /* (seed, block, 2^61 + step, pos * V + v)       */
+
 /* Kernel family for the vocabulary-attention step. */
 #define DG_IMPL_AUTO  0      /* tensor-core path when the shape allows it     */
 #define DG_IMPL_SIMT  1      /* CUDA-core kernels (any shape, f32 or bf16)    */
@@ -87,7 +93,7 @@ typedef struct dg_config {
   int32_t  accept_rule;     /* DG_ACCEPT_*                                     */
   int32_t  fixed_steps;     /* 1: ignore adaptive stop, run exactly S steps    */
   int32_t  impl;            /* DG_IMPL_*                                       */
-  int32_t  reserved0;
+  int32_t  token_rule;      /* DG_TOKEN_*                                      */
   uint64_t seed;            /* keys every draw: key(seed, block, step, index)  */
 } dg_config;
 
@@ -105,6 +111,8 @@ typedef struct dg_ctx dg_ctx;
 #define DG_PREFIX    8   /* float [C]   fp32 running entropy sums, sorted order */
 #define DG_STATE     9   /* int32 [16]  see DG_ST_* below                       */
 #define DG_MREF     10   /* float [C]   tensor-core path: per-row logit reference */
+#define DG_SAMPLED  11   /* int32 [C]   multinomial draw of the last step       */
+                         /*             (DG_TOKEN_MULTINOMIAL only; read-only) */
 
 /* Indices into the DG_STATE array. */
 #define DG_ST_T          0  /* next step index within the block               */

@@ -29,6 +29,7 @@ class Tally:
     worst_H: float = 0.0
     worst_sc: float = 0.0
     steps: int = 0
+    draws_off_mode: int = 0     # multinomial draws that differ from the argmax
 
     def check_budget(self):
         assert self.tie_mismatch <= TIE_BUDGET * max(self.positions, 1), (
@@ -76,12 +77,30 @@ def compare_attention(tally: Tally, att, H_gpu, argmax_gpu, sc_gpu, flags, rows=
     assert r.max() <= SC_RTOL, f"sc relative error {r.max()} at row {int(r.argmax())}"
 
 
-def check_sampler_exact(w, block, t, H_gpu, argmax_gpu, canvas_in, out):
-    """The sampler given the GPU's own entropies and argmax must agree bit for bit."""
+def compare_draw(tally: Tally, att, sampled_gpu):
+    """Multinomial draws of the GPU against the oracle's Gumbel-max for the same h.
+
+    A mismatch is allowed only where the oracle's two best z + G are within TIE
+    (the GPU's logits and fast-log Gumbel variates carry errors well below it);
+    such positions count toward the near-tie budget.
+    """
+    mism = np.flatnonzero(np.asarray(sampled_gpu) != att.sampled)
+    bad = [int(i) for i in mism if not att.smargin[i] < TIE]
+    assert not bad, f"draw mismatch off a near-tie at rows {bad[:8]} (gaps {att.smargin[bad[:8]]})"
+    tally.tie_mismatch += len(mism)
+
+
+def check_sampler_exact(w, block, t, H_gpu, argmax_gpu, canvas_in, out, chosen_gpu=None):
+    """The sampler given the GPU's own entropies and tokens must agree bit for bit.
+
+    chosen_gpu: the tokens accepted positions take (the GPU's draws under the
+    multinomial rule); the argmax when None.
+    """
     H32 = np.asarray(H_gpu, np.float32)
     acc = M.entropy_bounded_accept(H32, w.tau, w.accept_rule)
     noise = rng.tokens(w.seed, block, t, np.arange(w.C, dtype=np.uint64), w.V)
-    want_canvas = np.where(acc.accepted, np.asarray(argmax_gpu), noise)
+    tok = np.asarray(argmax_gpu if chosen_gpu is None else chosen_gpu)
+    want_canvas = np.where(acc.accepted, tok, noise)
     assert np.array_equal(out["order"], acc.order), "sort order differs"
     assert np.array_equal(out["prefix"], acc.prefix), "prefix sums differ"
     assert np.array_equal(out["accept"].astype(bool), acc.accepted), "accept mask differs"

@@ -14,7 +14,7 @@ import torch
 import synthetic
 import uniform_state_text_b200 as dg
 from oracle import method as M
-from parity import (Tally, check_sampler_exact, compare_attention, h_agreement,
+from parity import (Tally, check_sampler_exact, compare_attention, compare_draw, h_agreement,
                     near_tie_flags)
 
 pytestmark = pytest.mark.gpu
@@ -73,6 +73,8 @@ def step_and_compare(den, w, E32, tally: Tally, prev_amax=None):
     sc = _np(den.read(dg.DG_SC)).astype(np.float64)
     out = dict(accept=_np(den.read(dg.DG_ACCEPT)), canvas=_np(den.read(dg.DG_CANVAS)),
                order=_np(den.read(dg.DG_ORDER)), prefix=_np(den.read(dg.DG_PREFIX)))
+    multinomial = w.token_rule == dg.DG_TOKEN_MULTINOMIAL
+    sampled = _np(den.read(dg.DG_SAMPLED)).astype(np.int64) if multinomial else None
     st1 = den.state()
     out["state"] = st1
     assert st1["status"] == 0
@@ -80,11 +82,17 @@ def step_and_compare(den, w, E32, tally: Tally, prev_amax=None):
     h_orc = M.standin_hidden(w, E32, target, canvas_in, sc_in, b, t)
     assert h_agreement(w, h, h_orc) < 2e-3
     T = M.temperature(t, w.max_steps, w.T_start, w.T_end)
-    att = M.vocab_attention(h, E32, w.logit_scale / T)
+    if multinomial:
+        att = M.vocab_attention(h, E32, w.logit_scale / T, gumbel_key=(w.seed, b, t))
+    else:
+        att = M.vocab_attention(h, E32, w.logit_scale / T)
     acc_orc = M.entropy_bounded_accept(att.H.astype(np.float32), w.tau, w.accept_rule)
     flags = near_tie_flags(att, acc_orc, w.tau, w.accept_rule)
     compare_attention(tally, att, H, amax, sc, flags)
-    check_sampler_exact(w, b, t, H, amax, canvas_in, out)
+    if multinomial:
+        compare_draw(tally, att, sampled)
+        tally.draws_off_mode += int(np.sum(sampled != amax))
+    check_sampler_exact(w, b, t, H, amax, canvas_in, out, chosen_gpu=sampled)
     mism = np.flatnonzero(acc_orc.accepted != out["accept"].astype(bool))
     bad = [int(i) for i in mism if not flags[i]]
     assert not bad, f"accept mismatch off a near-tie at {bad[:8]}"
@@ -162,17 +170,40 @@ def test_tiny_block_trajectory(impl):
 
 
 @pytest.mark.parametrize("impl", IMPLS)
-@pytest.mark.parametrize("variant", ["fixed", "stress", "minus_max", "argmax_stop", "tau0"])
+@pytest.mark.parametrize("variant", ["fixed", "stress", "minus_max", "argmax_stop", "tau0",
+                                     "multinomial"])
 def test_tiny_teacher_forced(impl, variant):
     base = synthetic.TINY.replace(coef_target=0.5, coef_canvas=0.5, logit_scale=1.5, tau=2.0)
     w = {"fixed": base.replace(fixed_steps=1),
          "stress": base,
          "minus_max": base.replace(accept_rule=1, fixed_steps=1),
          "argmax_stop": base.replace(stop_rule=1),
-         "tau0": base.replace(tau=0.0, max_steps=4)}[variant]
+         "tau0": base.replace(tau=0.0, max_steps=4),
+         "multinomial": base.replace(token_rule=1, fixed_steps=1)}[variant]
     den, E32 = make(w, impl)
     tally = run_teacher_forced(den, w, E32)
     assert tally.steps >= 1
+    if variant == "multinomial":
+        assert tally.draws_off_mode > 0      # a soft distribution does not always give its mode
+    den.close()
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_small_multinomial_teacher_forced(impl):
+    """Multinomial draws (Gumbel-max) on the partial-acceptance stress set, 4 steps."""
+    w = synthetic.STRESS_PARTIAL.replace(token_rule=1, max_steps=4, fixed_steps=1)
+    den, E32 = make(w, impl)
+    tally = run_teacher_forced(den, w, E32)
+    assert tally.steps == 4 and tally.draws_off_mode > 0
+    den.close()
+
+
+def test_full_size_multinomial_step():
+    """One headline-size step under the multinomial rule, every row's draw compared."""
+    w = synthetic.HEADLINE.replace(token_rule=1, fixed_steps=1)
+    den, E32 = make(w, dg.DG_IMPL_TC)
+    tally = run_teacher_forced(den, w, E32, max_steps=1)
+    assert tally.steps == 1
     den.close()
 
 

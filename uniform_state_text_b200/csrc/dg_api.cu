@@ -34,7 +34,7 @@ struct Layout {
   int nsplit = 0;      // CUDA-core path: vocabulary splits of sc
   size_t state = 0, scale = 0, target = 0, canvas = 0, argmax = 0, argmax_prev = 0, accept = 0,
          order = 0, prefix = 0, H = 0, mref = 0, rowstat = 0, redo_rows = 0, h = 0, sc = 0,
-         tstats = 0, zbuf = 0, partial = 0, O = 0, tc = 0, total = 0;
+         tstats = 0, zbuf = 0, partial = 0, O = 0, tc = 0, sampled = 0, tsamp = 0, total = 0;
   size_t tc_bytes = 0;
 };
 
@@ -63,6 +63,7 @@ int check_config(const dg_config* c, char* why, size_t n) {
   if (c->stop_rule != DG_STOP_CANVAS && c->stop_rule != DG_STOP_ARGMAX) { snprintf(why, n, "bad stop_rule"); return DG_EINVAL; }
   if (c->accept_rule != DG_ACCEPT_CUMSUM && c->accept_rule != DG_ACCEPT_MINUS_MAX) { snprintf(why, n, "bad accept_rule"); return DG_EINVAL; }
   if (c->impl < DG_IMPL_AUTO || c->impl > DG_IMPL_TC) { snprintf(why, n, "bad impl"); return DG_EINVAL; }
+  if (c->token_rule != DG_TOKEN_ARGMAX && c->token_rule != DG_TOKEN_MULTINOMIAL) { snprintf(why, n, "bad token_rule"); return DG_EINVAL; }
   return DG_OK;
 }
 
@@ -104,6 +105,7 @@ int make_layout(const dg_config* c, Layout* L, char* why, size_t n) {
   L->redo_rows = take(4 * C);
   L->h = take(esz * C * d);
   L->sc = take(4 * C * d);
+  L->sampled = take(4 * C);
   if (impl == DG_IMPL_SIMT) {
     L->ntiles = (int)(V / 64);
     const size_t rt = (C + 63) / 64, dt = (d + 63) / 64;
@@ -118,6 +120,7 @@ int make_layout(const dg_config* c, Layout* L, char* why, size_t n) {
     L->tstats = take(sizeof(TileStat) * C * L->ntiles);
     L->tc_bytes = tc_workspace_bytes(c->C, c->V, c->d);
     L->tc = take(L->tc_bytes);
+    if (c->token_rule == DG_TOKEN_MULTINOMIAL) L->tsamp = take(tc_draw_bytes(c->C, c->V, c->d));
   }
   L->total = off;
   return DG_OK;
@@ -145,6 +148,7 @@ struct dg_ctx {
         *partial = nullptr, *O = nullptr;
   RowStat* rowstat = nullptr;
   TileStat* tstats = nullptr;
+  DrawArgs draw;            // multinomial draw (sampled == nullptr under the argmax rule)
   void* h = nullptr;
   void* tc = nullptr;
   TcPlan tc_plan;
@@ -210,24 +214,22 @@ int launch_step(dg_ctx* ctx, bool standin, bool use_cond) {
   const SamplerArgs sa = make_sampler_args(
       ctx->st, ctx->H, ctx->argmax, ctx->canvas, ctx->argmax_prev, ctx->accept, ctx->order,
       ctx->prefix, c.C, c.V, c.seed, c.tau, c.stop_entropy, c.stop_unchanged, c.stop_rule,
-      c.accept_rule, c.fixed_steps, c.max_steps, ctx->cond, use_cond ? 1 : 0);
+      c.accept_rule, c.fixed_steps, c.max_steps, ctx->cond, use_cond ? 1 : 0, ctx->draw.sampled);
   if (tc) {
     DG_CK(launch_tc_attention(s, ctx->tc_plan, ctx->st, ctx->h, ctx->E, ctx->mref, ctx->scale_tab,
-                              c.max_steps, ctx->tstats, ctx->O, ctx->tc));
+                              c.max_steps, ctx->tstats, ctx->O, ctx->tc, ctx->draw));
     if (e1) DG_CK(cudaEventRecord(e1, s));
     // merge, then (inside the same kernel) the sampler and stop test
     DG_CK(launch_tc_merge(s, ctx->tc_plan, ctx->st, ctx->tstats, ctx->mref, ctx->rowstat, ctx->H,
                           ctx->argmax, ctx->sc, ctx->redo_rows, kRedoGap, ctx->h, ctx->E,
-                          ctx->scale_tab, c.max_steps, sa));
+                          ctx->scale_tab, c.max_steps, sa, ctx->draw));
   } else {
     DG_CK(launch_simt_attention(s, c.dtype, ctx->st, ctx->h, ctx->E, ctx->zbuf, ctx->tstats,
                                 ctx->rowstat, ctx->partial, ctx->H, ctx->argmax, ctx->sc, c.C,
-                                c.V, c.d, ctx->L.nsplit, ctx->scale_tab, c.max_steps));
+                                c.V, c.d, ctx->L.nsplit, ctx->scale_tab, c.max_steps,
+                                ctx->draw));
     if (e1) DG_CK(cudaEventRecord(e1, s));
-    DG_CK(launch_sampler(s, ctx->st, ctx->H, ctx->argmax, ctx->canvas, ctx->argmax_prev,
-                         ctx->accept, ctx->order, ctx->prefix, c.C, c.V, c.seed, c.tau,
-                         c.stop_entropy, c.stop_unchanged, c.stop_rule, c.accept_rule,
-                         c.fixed_steps, c.max_steps, ctx->cond, use_cond ? 1 : 0));
+    DG_CK(launch_sampler(s, sa));
   }
   return DG_OK;
 }
@@ -322,6 +324,11 @@ int dg_init(const dg_config* cfg, const void* E, void* workspace, size_t ws_byte
   ctx->h = at<void>(ctx, L.h);
   ctx->sc = at<float>(ctx, L.sc);
   ctx->tstats = at<TileStat>(ctx, L.tstats);
+  if (cfg->token_rule == DG_TOKEN_MULTINOMIAL) {
+    ctx->draw.sampled = at<int32_t>(ctx, L.sampled);
+    ctx->draw.tsamp = L.impl == DG_IMPL_TC ? at<void>(ctx, L.tsamp) : nullptr;
+    ctx->draw.seed = cfg->seed;
+  }
   if (L.impl == DG_IMPL_SIMT) {
     ctx->zbuf = at<float>(ctx, L.zbuf);
     ctx->partial = at<float>(ctx, L.partial);
@@ -446,6 +453,7 @@ int dg_read(dg_ctx* ctx, int32_t what, void* dst) {
     case DG_PREFIX: src = ctx->prefix; bytes = 4 * C; break;
     case DG_STATE: src = ctx->st; bytes = 64; break;
     case DG_MREF: src = ctx->mref; bytes = 4 * C; break;
+    case DG_SAMPLED: src = at<int32_t>(ctx, ctx->L.sampled); bytes = 4 * C; break;
     default: return fail(ctx, DG_EINVAL, "unknown item %d", what);
   }
   DG_CK(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, ctx->stream));

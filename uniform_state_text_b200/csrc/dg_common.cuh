@@ -31,6 +31,7 @@ struct DevState {
 constexpr uint64_t kTagInitCanvas = (1ull << 63) + 1;
 constexpr uint64_t kTagTarget = (1ull << 63) + 2;
 constexpr uint64_t kTagNoise = 1ull << 62;  // + step
+constexpr uint64_t kTagGumbel = 1ull << 61; // + step; index = position * V + entry
 
 __host__ __device__ __forceinline__ uint64_t sm64(uint64_t x) {
   uint64_t z = x + 0x9E3779B97F4A7C15ull;
@@ -52,6 +53,22 @@ __device__ __forceinline__ float gauss_from_key(uint64_t k) {
   return sqrtf(-2.0f * logf(u1)) * cospif(2.0f * u2);
 }
 
+// Standard Gumbel variate from one key, for the multinomial token draw
+// ("A Visual Guide to DiffusionGemma", 3.2: each position's token drawn from
+// its distribution, taken as argmax_v (z_v + G_v)). W = (2 (k >> 41) + 1) 2^-24
+// is exact in fp32 and lies in (0, 1); X = -ln(1 - W) is a unit exponential,
+// G = -ln X. Below W = 2^-8, 1 - W keeps too few digits for the fast log2, so
+// X takes the series W + W^2/2 + W^3/3 (relative truncation < 2e-8); above it
+// |log2(1 - W)| >= 0.0056, so the fast log2's absolute error (about 2^-22)
+// leaves X within a relative 5e-5 and G within an absolute 5e-5.
+__device__ __forceinline__ float gumbel_from_key(uint64_t k) {
+  const float W = (float)(2u * (uint32_t)(k >> 41) + 1u) * 5.9604644775390625e-8f;
+  const float x_series = W * fmaf(W, fmaf(W, 0.333333343f, 0.5f), 1.0f);
+  const float x_log = -0.693147182f * __log2f(1.0f - W);
+  const float X = W < 0.00390625f ? x_series : x_log;
+  return -0.693147182f * __log2f(X);
+}
+
 template <typename T> __device__ __forceinline__ float to_f32(T x);
 template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
@@ -65,7 +82,9 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 
 // Per-(row, vocabulary tile) partial softmax statistics, relative to the
 // tile's own maximum m: Z = sum e^(z-m), S1 = sum e^(z-m) (z-m), and the
-// tile's best logit with its vocabulary index (lowest index on ties).
+// tile's best logit with its vocabulary index (lowest index on ties). For the
+// multinomial draw, pad[0] holds the bits of the tile's best z + G and pad[1]
+// its index.
 struct TileStat {
   float m, Z, S1, best;
   int32_t arg;
@@ -77,6 +96,13 @@ struct TileStat {
 // (z - m_ref), and the best logit with its vocabulary index.
 struct TcStat {
   float Z, S1, best;
+  int32_t arg;
+};
+
+// Tensor-core path, multinomial draw: per-(row, half tile) best z + G and
+// its vocabulary index.
+struct TcSamp {
+  float score;
   int32_t arg;
 };
 

@@ -199,7 +199,8 @@ constexpr int SK = 32;   // k chunk
 
 template <typename T>
 __global__ void __launch_bounds__(256) k_simt_logits(const DevState* st, const T* h, const T* E,
-    float* zbuf, TileStat* tstats, int C, int V, int d, const float* scale_tab, int S) {
+    float* zbuf, TileStat* tstats, int C, int V, int d, const float* scale_tab, int S,
+    uint64_t seed, int draw) {
   if (st->done) return;
   __shared__ __align__(16) float hs[SK][ST + 4];
   __shared__ __align__(16) float es[SK][ST + 4];
@@ -229,6 +230,9 @@ __global__ void __launch_bounds__(256) k_simt_logits(const DevState* st, const T
   }
   const float scale = scale_tab[min(max(st->t, 0), S - 1)];
   const int ntiles = V / ST;
+  // multinomial draw: key prefix of this step's Gumbel variates
+  const uint64_t gpre =
+      draw ? key_prefix(seed, (uint64_t)(uint32_t)st->block, kTagGumbel + (uint64_t)st->t) : 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int row = r0 + ty * 4 + i;
@@ -250,13 +254,31 @@ __global__ void __launch_bounds__(256) k_simt_logits(const DevState* st, const T
       s.S1 += e * dz;
     }
     for (int o = 8; o; o >>= 1) s = stat_combine(s, stat_shfl_xor(s, o));
+    // best z + G of the row's 64 entries (uniform branch)
+    float gbest = -INFINITY;
+    int garg = 0x7fffffff;
+    if (draw) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int v = v0 + tx * 4 + j;
+        const float g = z[j] + gumbel_from_key(sm64(gpre ^ ((uint64_t)row * (uint64_t)V + (uint64_t)v)));
+        if (better(g, v, gbest, garg)) { gbest = g; garg = v; }
+      }
+      for (int o = 8; o; o >>= 1) {
+        const float ob = __shfl_xor_sync(0xffffffffu, gbest, o);
+        const int oa = __shfl_xor_sync(0xffffffffu, garg, o);
+        if (better(ob, oa, gbest, garg)) { gbest = ob; garg = oa; }
+      }
+    }
     if (row < C) {
       *reinterpret_cast<float4*>(&zbuf[(size_t)row * V + v0 + tx * 4]) =
           make_float4(z[0], z[1], z[2], z[3]);
       if (tx == 0) {
         TileStat ts;
         ts.m = s.m; ts.Z = s.Z; ts.S1 = s.S1; ts.best = s.best; ts.arg = s.arg;
-        ts.pad[0] = ts.pad[1] = ts.pad[2] = 0;
+        ts.pad[0] = __float_as_int(gbest);
+        ts.pad[1] = garg;
+        ts.pad[2] = 0;
         tstats[(size_t)row * ntiles + blockIdx.x] = ts;
       }
     }
@@ -271,26 +293,46 @@ __global__ void __launch_bounds__(256) k_simt_logits(const DevState* st, const T
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_merge(DevState* st, const TileStat* tstats, int ntiles,
     RowStat* rowstat, float* H, int32_t* argmax, int C, const float* O, int nO,
-    const float* mref, float* sc, int d, int32_t* redo_rows, float redo_gap) {
+    const float* mref, float* sc, int d, int32_t* redo_rows, float redo_gap, int32_t* sampled) {
   if (st->done) return;
   const int i = blockIdx.x;
   Stat s;
   s.m = -INFINITY; s.Z = 0.f; s.S1 = 0.f; s.best = -INFINITY; s.arg = 0x7fffffff;
+  float gbest = -INFINITY;          // multinomial draw: best z + G and its index
+  int garg = 0x7fffffff;
   for (int j = threadIdx.x; j < ntiles; j += blockDim.x) {
     const TileStat ts = tstats[(size_t)i * ntiles + j];
     Stat b; b.m = ts.m; b.Z = ts.Z; b.S1 = ts.S1; b.best = ts.best; b.arg = ts.arg;
     s = stat_combine(s, b);
+    if (sampled && better(__int_as_float(ts.pad[0]), ts.pad[1], gbest, garg)) {
+      gbest = __int_as_float(ts.pad[0]);
+      garg = ts.pad[1];
+    }
   }
-  for (int o = 16; o; o >>= 1) s = stat_combine(s, stat_shfl_xor(s, o));
+  for (int o = 16; o; o >>= 1) {
+    s = stat_combine(s, stat_shfl_xor(s, o));
+    const float ob = __shfl_xor_sync(0xffffffffu, gbest, o);
+    const int oa = __shfl_xor_sync(0xffffffffu, garg, o);
+    if (better(ob, oa, gbest, garg)) { gbest = ob; garg = oa; }
+  }
   __shared__ Stat part[8];
+  __shared__ float gpart[8];
+  __shared__ int gapart[8];
   __shared__ float sh_scale;
   __shared__ int sh_redo;
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  if (l == 0) part[w] = s;
+  if (l == 0) { part[w] = s; gpart[w] = gbest; gapart[w] = garg; }
   __syncthreads();
   if (threadIdx.x == 0) {
     Stat r = part[0];
     for (int j = 1; j < (int)(blockDim.x >> 5); ++j) r = stat_combine(r, part[j]);
+    if (sampled) {
+      float gb = gpart[0];
+      int ga = gapart[0];
+      for (int j = 1; j < (int)(blockDim.x >> 5); ++j)
+        if (better(gpart[j], gapart[j], gb, ga)) { gb = gpart[j]; ga = gapart[j]; }
+      sampled[i] = ga;
+    }
     const float Hv = logf(r.Z) - r.S1 / r.Z;
     H[i] = fmaxf(Hv, 0.f);
     argmax[i] = r.arg;
@@ -437,19 +479,21 @@ cudaError_t launch_prologue(cudaStream_t s, int dtype, const DevState* st, const
 cudaError_t launch_simt_attention(cudaStream_t s, int dtype, DevState* st, const void* h,
                                   const void* E, float* zbuf, TileStat* tstats, RowStat* rowstat,
                                   float* partial, float* H, int32_t* argmax, float* sc, int C,
-                                  int V, int d, int nsplit, const float* scale_tab, int S) {
+                                  int V, int d, int nsplit, const float* scale_tab, int S,
+                                  const DrawArgs& draw) {
   dim3 g1(V / ST, (C + ST - 1) / ST);
+  const int drawing = draw.sampled != nullptr;
   if (dtype == 0)
     k_simt_logits<float><<<g1, 256, 0, s>>>(st, (const float*)h, (const float*)E, zbuf, tstats,
-                                            C, V, d, scale_tab, S);
+                                            C, V, d, scale_tab, S, draw.seed, drawing);
   else
     k_simt_logits<__nv_bfloat16><<<g1, 256, 0, s>>>(st, (const __nv_bfloat16*)h,
                                                      (const __nv_bfloat16*)E, zbuf, tstats, C, V,
-                                                     d, scale_tab, S);
+                                                     d, scale_tab, S, draw.seed, drawing);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   k_merge<<<C, 256, 0, s>>>(st, tstats, V / ST, rowstat, H, argmax, C, nullptr, 0, nullptr,
-                            nullptr, d, nullptr, 0.f);
+                            nullptr, d, nullptr, 0.f, draw.sampled);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   dim3 g2((d + ST - 1) / ST, (C + ST - 1) / ST, nsplit);
   if (dtype == 0)
@@ -466,25 +510,9 @@ cudaError_t launch_simt_attention(cudaStream_t s, int dtype, DevState* st, const
   return cudaGetLastError();
 }
 
-cudaError_t launch_merge(cudaStream_t s, DevState* st, const TileStat* tstats, int ntiles,
-                         RowStat* rowstat, float* H, int32_t* argmax, int C, const float* O,
-                         int nO, const float* mref, float* sc, int d, int32_t* redo_rows,
-                         float redo_gap) {
-  k_merge<<<C, 256, 0, s>>>(st, tstats, ntiles, rowstat, H, argmax, C, O, nO, mref, sc, d,
-                            redo_rows, redo_gap);
-  return cudaGetLastError();
-}
 
-cudaError_t launch_sampler(cudaStream_t s, DevState* st, const float* H, const int32_t* argmax,
-                           int32_t* canvas, int32_t* argmax_prev, int32_t* accept,
-                           int32_t* order, float* prefix, int C, int V, uint64_t seed, float tau,
-                           float stop_entropy, int stop_unchanged, int stop_rule,
-                           int accept_rule, int fixed_steps, int S,
-                           cudaGraphConditionalHandle cond, int use_cond) {
-  const int threads = ((C + 31) / 32) * 32;
-  SamplerArgs a = make_sampler_args(st, H, argmax, canvas, argmax_prev, accept, order, prefix, C, V,
-                                    seed, tau, stop_entropy, stop_unchanged, stop_rule,
-                                    accept_rule, fixed_steps, S, cond, use_cond);
+cudaError_t launch_sampler(cudaStream_t s, const SamplerArgs& a) {
+  const int threads = ((a.C + 31) / 32) * 32;
   k_sampler<<<1, threads, 0, s>>>(a);
   return cudaGetLastError();
 }

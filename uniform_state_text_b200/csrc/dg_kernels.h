@@ -19,6 +19,7 @@ struct SamplerArgs {
   int stop_unchanged, stop_rule, accept_rule, fixed_steps, S;
   cudaGraphConditionalHandle cond;
   int use_cond;
+  const int32_t* sampled;   // [C] multinomial draws to accept; nullptr: accept the argmax
 };
 struct SamplerSmem {
   unsigned long long key[1024];   // (entropy bits, position); padded with ~0
@@ -31,15 +32,24 @@ inline SamplerArgs make_sampler_args(DevState* st, const float* H, const int32_t
                                      int32_t* order, float* prefix, int C, int V, uint64_t seed,
                                      float tau, float stop_entropy, int stop_unchanged,
                                      int stop_rule, int accept_rule, int fixed_steps, int S,
-                                     cudaGraphConditionalHandle cond, int use_cond) {
+                                     cudaGraphConditionalHandle cond, int use_cond,
+                                     const int32_t* sampled = nullptr) {
   SamplerArgs a;
   a.st = st; a.H = H; a.argmax = argmax; a.canvas = canvas; a.argmax_prev = argmax_prev;
   a.accept = accept; a.order = order; a.prefix = prefix; a.C = C; a.V = V; a.seed = seed;
   a.tau = tau; a.stop_entropy = stop_entropy; a.stop_unchanged = stop_unchanged;
   a.stop_rule = stop_rule; a.accept_rule = accept_rule; a.fixed_steps = fixed_steps; a.S = S;
-  a.cond = cond; a.use_cond = use_cond;
+  a.cond = cond; a.use_cond = use_cond; a.sampled = sampled;
   return a;
 }
+
+// Multinomial token draw (DG_TOKEN_MULTINOMIAL): where the per-row draws go.
+// sampled == nullptr selects the argmax rule and nothing is drawn.
+struct DrawArgs {
+  int32_t* sampled = nullptr;   // [C]
+  void* tsamp = nullptr;        // tensor-core path: [C][2 * V/256] TcSamp
+  uint64_t seed = 0;
+};
 
 cudaError_t launch_begin_block(cudaStream_t s, DevState* st, int32_t* target, int32_t* canvas,
                                float* sc, int C, int d, int V, uint64_t seed, int block);
@@ -54,18 +64,9 @@ cudaError_t launch_prologue(cudaStream_t s, int dtype, const DevState* st, const
 cudaError_t launch_simt_attention(cudaStream_t s, int dtype, DevState* st, const void* h,
                                   const void* E, float* zbuf, TileStat* tstats, RowStat* rowstat,
                                   float* partial, float* H, int32_t* argmax, float* sc, int C,
-                                  int V, int d, int nsplit, const float* scale_tab, int S);
+                                  int V, int d, int nsplit, const float* scale_tab, int S,
+                                  const DrawArgs& draw = DrawArgs());
 
-cudaError_t launch_merge(cudaStream_t s, DevState* st, const TileStat* tstats, int ntiles,
-                         RowStat* rowstat, float* H, int32_t* argmax, int C, const float* O,
-                         int nO, const float* mref, float* sc, int d, int32_t* redo_rows,
-                         float redo_gap);
-
-cudaError_t launch_sampler(cudaStream_t s, DevState* st, const float* H, const int32_t* argmax,
-                           int32_t* canvas, int32_t* argmax_prev, int32_t* accept,
-                           int32_t* order, float* prefix, int C, int V, uint64_t seed, float tau,
-                           float stop_entropy, int stop_unchanged, int stop_rule,
-                           int accept_rule, int fixed_steps, int S,
-                           cudaGraphConditionalHandle cond, int use_cond);
+cudaError_t launch_sampler(cudaStream_t s, const SamplerArgs& a);
 
 }  // namespace dg

@@ -42,18 +42,19 @@ __device__ __forceinline__ void sample_and_stop(const SamplerArgs& a, SamplerSme
   const int i = threadIdx.x;
   const bool valid = i < C;
   // Every global input is read up front (one round trip): the loop state and
-  // this position's entropy, argmax, canvas token and previous argmax.
+  // this position's entropy, argmax, canvas token, previous argmax and draw.
   const int t = st->t;
   const int blk = st->block;
   const int has_prev = st->has_prev;
   const int unchanged_before = st->unchanged;
   float Hi = 0.f;
-  int32_t am = 0, old = 0, am_prev = 0;
+  int32_t am = 0, old = 0, am_prev = 0, chosen = 0;
   if (valid) {
     Hi = a.H[i];
     am = a.argmax[i];
     old = a.canvas[i];
     am_prev = a.argmax_prev[i];
+    chosen = a.sampled ? a.sampled[i] : am;   // the token an accepted position takes
   }
   // Stable rank by (entropy, position) as one 64-bit key: entropies are >= 0,
   // so their bit patterns order like their values (-0 is taken as +0).
@@ -103,7 +104,7 @@ __device__ __forceinline__ void sample_and_stop(const SamplerArgs& a, SamplerSme
     acc = rank < k;
     const uint64_t pre = key_prefix(a.seed, (uint64_t)(uint32_t)blk, (uint64_t)t);
     const int32_t noise = (int32_t)(sm64(pre ^ (uint64_t)i) & (uint64_t)(V - 1));
-    nw = acc ? am : noise;
+    nw = acc ? chosen : noise;
   }
   const int all_conf = sampler_bar_and(nthreads, !valid || Hi < a.stop_entropy);
   int same;

@@ -49,7 +49,7 @@ constexpr int BK = 64;         // K per pipeline stage (one 128-byte swizzle row
 constexpr int KV2 = 256;       // vocabulary entries per range (unit of G2 ownership): one tile,
                                // so range group g owns tiles g, g+G, ... and all groups
                                // advance through the ring together
-constexpr int RING = 96;       // P tiles (256 vocabulary entries each) resident at once
+constexpr int RING = 64;       // P tiles (256 vocabulary entries each) resident at once
 constexpr int THREADS = 320;    // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr int EPI_WARPS = 8;
 constexpr int QN = 8;          // G1 item queue depth (tile indices handed to the CTA's warps)
@@ -81,6 +81,8 @@ struct Params {
   DevState* st;
   unsigned long long* trace;   // [grid][32] wait-time counters (DG_TC_TRACE builds only)
   TcStat* tstats2;             // [C][2 * n_vt] half-tile statistics
+  TcSamp* tsamp;               // [C][2 * n_vt] best z + G (multinomial draw), or nullptr
+  uint64_t seed;               // keys the draw's Gumbel variates
 };
 
 // Per-CTA wait-time tracing, compiled in only with -DDG_TC_TRACE (measurement
@@ -398,7 +400,9 @@ __device__ __forceinline__ bool is_g1_unit(const Params& p, int CG) {
   return (int)(blockIdx.x / CG) < p.n1;
 }
 
-template <int CG>
+// DRAW: the multinomial rule's Gumbel-max draw in the G1 epilogue (a separate
+// instantiation, so the argmax kernel keeps its register budget).
+template <int CG, bool DRAW>
 __global__ void __launch_bounds__(THREADS, 1)
     k_vocab_attention(const __grid_constant__ CUtensorMap tm_h,
                       const __grid_constant__ CUtensorMap tm_ek,
@@ -669,6 +673,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (is_g1) {
       const float scale = p.scale_tab[min(max(p.st->t, 0), p.S - 1)];
       const float k1 = scale * 1.4426950408889634f;           // logit scale in log2 units
+      // multinomial draw: key prefix of this step's Gumbel variates
+      const uint64_t gpre = DRAW ? key_prefix(p.seed, (uint64_t)(uint32_t)p.st->block,
+                                              kTagGumbel + (uint64_t)p.st->t)
+                                 : 0;
       int n = 0;
       for (;; ++n) {
         int it = 0;
@@ -693,6 +701,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         // P = 2^(k1 v + k0) = e^(z - mref); Z = sum P; S2 = sum P (z - mref) log2(e).
         float Z = 0.f, S2 = 0.f, vbest = -INFINITY;
         int arg = 0x7fffffff;
+        float gbest = -INFINITY;    // multinomial draw: best z + G, first index on ties
+        int garg = 0x7fffffff;
         __nv_bfloat16* prow = p.P + ((size_t)((vt % RING) * p.C + row)) * BN + c0;
 #pragma unroll 1
         for (int c = 0; c < HALF / 32; ++c) {
@@ -719,6 +729,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             vbest = cm;
             arg = vt * BN + c0 + c * 32 + jj;
           }
+          if constexpr (DRAW) {
+            const int col0 = vt * BN + c0 + c * 32;
+            const uint64_t rbase = (uint64_t)row * (uint64_t)p.V + (uint64_t)col0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float g = v[j] * scale + gumbel_from_key(sm64(gpre ^ (rbase + (uint64_t)j)));
+              if (g > gbest) { gbest = g; garg = col0 + j; }
+            }
+          }
           uint32_t pk[16];
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
@@ -744,6 +763,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         ts.best = vbest * scale;
         ts.arg = arg;
         p.tstats2[(size_t)row * (2 * p.n_vt) + 2 * vt + half] = ts;
+        if constexpr (DRAW) {
+          TcSamp sp;
+          sp.score = gbest;
+          sp.arg = garg;
+          p.tsamp[(size_t)row * (2 * p.n_vt) + 2 * vt + half] = sp;
+        }
         // Publish this warp's part of the P tile: generic-proxy stores, read later
         // by TMA on other SMs. Each epilogue warp counts once per tile.
         {
@@ -857,7 +882,7 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
     const TcStat* ts, int nts, const float* mref, const float* Opart, int nO, int C, int V, int d,
     RowStat* rowstat, float* H, int32_t* argmax, float* sc, float redo_gap,
     const __nv_bfloat16* h, const __nv_bfloat16* E, const float* scale_tab, int S,
-    unsigned* ticket, const SamplerArgs sa) {
+    unsigned* ticket, const TcSamp* tsamp, int32_t* sampled, const SamplerArgs sa) {
   // Programmatic dependent launch: wait for the attention kernel's results,
   // then let the next step's prologue be scheduled (it waits for this grid).
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -876,6 +901,8 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
   const float mref_i = row_ok ? mref[i] : 0.f;
   float Z = 0.f, S1 = 0.f, best = -INFINITY;
   int arg = 0x7fffffff;
+  float gbest = -INFINITY;          // multinomial draw: best z + G and its index
+  int garg = 0x7fffffff;
   if (row_ok) {
     const float4* ts4 = reinterpret_cast<const float4*>(ts + (size_t)i * nts);
 #pragma unroll 8
@@ -886,6 +913,15 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
       S1 += t.y;
       if (better(t.z, ta, best, arg)) { best = t.z; arg = ta; }
     }
+    if (tsamp) {
+      const float2* sp2 = reinterpret_cast<const float2*>(tsamp + (size_t)i * nts);
+#pragma unroll 8
+      for (int j = tid; j < nts; j += kMergeThreadsPerRow) {
+        const float2 q = sp2[j];               // {score, arg}
+        const int qa = __float_as_int(q.y);
+        if (better(q.x, qa, gbest, garg)) { gbest = q.x; garg = qa; }
+      }
+    }
   }
   for (int o = 16; o; o >>= 1) {
     Z += __shfl_xor_sync(0xffffffffu, Z, o);
@@ -893,15 +929,23 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
     const float ob = __shfl_xor_sync(0xffffffffu, best, o);
     const int oa = __shfl_xor_sync(0xffffffffu, arg, o);
     if (better(ob, oa, best, arg)) { best = ob; arg = oa; }
+    const float gb = __shfl_xor_sync(0xffffffffu, gbest, o);
+    const int ga = __shfl_xor_sync(0xffffffffu, garg, o);
+    if (better(gb, ga, gbest, garg)) { gbest = gb; garg = ga; }
   }
   constexpr int WPR = kMergeThreadsPerRow / 32;   // warps per row
   __shared__ float sZ[kMergeRows][WPR], sS[kMergeRows][WPR], sB[kMergeRows][WPR];
   __shared__ int sA[kMergeRows][WPR];
+  __shared__ float sG[kMergeRows][WPR];
+  __shared__ int sGA[kMergeRows][WPR];
   __shared__ float sh_inv[kMergeRows], sh_best[kMergeRows];
   __shared__ int sh_redo[kMergeRows];
   __shared__ unsigned sh_ticket;
   const int w = tid >> 5, l = tid & 31;
-  if (l == 0) { sZ[r][w] = Z; sS[r][w] = S1; sB[r][w] = best; sA[r][w] = arg; }
+  if (l == 0) {
+    sZ[r][w] = Z; sS[r][w] = S1; sB[r][w] = best; sA[r][w] = arg;
+    sG[r][w] = gbest; sGA[r][w] = garg;
+  }
   __syncthreads();
   if (tid == 0) {
     int redo = 0;
@@ -914,6 +958,13 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
       }
       H[i] = fmaxf(logf(Z) - S1 / Z, 0.f);
       argmax[i] = arg;
+      if (sampled) {
+        float gb = sG[r][0];
+        int ga = sGA[r][0];
+        for (int j = 1; j < WPR; ++j)
+          if (better(sG[r][j], sGA[r][j], gb, ga)) { gb = sG[r][j]; ga = sGA[r][j]; }
+        sampled[i] = ga;
+      }
       RowStat rs;
       rs.m = mref_i; rs.Z = Z; rs.pad[0] = best; rs.pad[1] = 0.f;
       rowstat[i] = rs;
@@ -1078,9 +1129,11 @@ int tc_stat_tiles(int, int V, int) { return V / tc::BN; }
 
 size_t tc_workspace_bytes(int C, int V, int d) { return tc_layout(C, V, d, device_sms()).total; }
 
+size_t tc_draw_bytes(int C, int V, int) { return sizeof(TcSamp) * (size_t)C * 2 * (V / tc::BN); }
+
 int tc_launches(const TcPlan&) { return 1; }
 
-template <int CG>
+template <int CG, bool DRAW>
 cudaError_t launch_kernel(cudaStream_t s, int units, const CUtensorMap* maps, const tc::Params& prm) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(units * CG);
@@ -1104,13 +1157,14 @@ cudaError_t launch_kernel(cudaStream_t s, int units, const CUtensorMap* maps, co
     attr[0].val.cooperative = 1;
     cfg.numAttrs = 1;
   }
-  return cudaLaunchKernelEx(&cfg, tc::k_vocab_attention<CG>, maps[0], maps[1], maps[2], maps[3], prm);
+  return cudaLaunchKernelEx(&cfg, tc::k_vocab_attention<CG, DRAW>, maps[0], maps[1], maps[2],
+                            maps[3], prm);
 }
 
 // Every unit of the persistent grid must be resident at once (they wait on one another).
-template <int CG>
+template <int CG, bool DRAW>
 int check_residency(int units, int sms, char* err, size_t errn) {
-  cudaError_t e = cudaFuncSetAttribute(tc::k_vocab_attention<CG>,
+  cudaError_t e = cudaFuncSetAttribute(tc::k_vocab_attention<CG, DRAW>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)tc::Pipe<CG>::SMEM);
   if (e != cudaSuccess) {
@@ -1130,10 +1184,10 @@ int check_residency(int units, int sms, char* err, size_t errn) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaOccupancyMaxActiveClusters(&fit, tc::k_vocab_attention<CG>, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&fit, tc::k_vocab_attention<CG, DRAW>, &cfg);
   } else {
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tc::k_vocab_attention<CG>,
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tc::k_vocab_attention<CG, DRAW>,
                                                       tc::THREADS, tc::Pipe<CG>::SMEM);
     fit = per_sm * sms;
   }
@@ -1165,8 +1219,12 @@ int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, float* 
     snprintf(err, errn, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
     return -3;
   }
-  const int rc = L.CG == 2 ? check_residency<2>(p->grid, p->num_sms, err, errn)
-                           : check_residency<1>(p->grid, p->num_sms, err, errn);
+  // both instantiations (argmax rule, multinomial draw) must fit
+  int rc = L.CG == 2 ? check_residency<2, false>(p->grid, p->num_sms, err, errn)
+                     : check_residency<1, false>(p->grid, p->num_sms, err, errn);
+  if (!rc)
+    rc = L.CG == 2 ? check_residency<2, true>(p->grid, p->num_sms, err, errn)
+                   : check_residency<1, true>(p->grid, p->num_sms, err, errn);
   if (rc) return rc;
   p->ready = true;
   return 0;
@@ -1182,7 +1240,8 @@ void tc_counters(const TcPlan& p, unsigned** ptr, int* count) {
 
 cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, const void* h,
                                 const void* E, const float* mref, const float* scale_tab,
-                                int S, TileStat* tstats, float* O, void* ws) {
+                                int S, TileStat* tstats, float* O, void* ws,
+                                const DrawArgs& draw) {
   (void)h; (void)E; (void)O;
   TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
   char* base = static_cast<char*>(ws);
@@ -1201,16 +1260,22 @@ cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, 
   prm.g1_next = ctr + 2 * L.n_vt + 1;
   prm.st = st;
   prm.trace = reinterpret_cast<unsigned long long*>(base + L.trace);
+  prm.tsamp = draw.sampled ? static_cast<TcSamp*>(draw.tsamp) : nullptr;
+  prm.seed = draw.seed;
   const CUtensorMap* maps = reinterpret_cast<const CUtensorMap*>(pl.maps);
-  return L.CG == 2 ? launch_kernel<2>(s, L.n1 + L.n2, maps, prm)
-                   : launch_kernel<1>(s, L.n1 + L.n2, maps, prm);
+  const int units = L.n1 + L.n2;
+  if (prm.tsamp)
+    return L.CG == 2 ? launch_kernel<2, true>(s, units, maps, prm)
+                     : launch_kernel<1, true>(s, units, maps, prm);
+  return L.CG == 2 ? launch_kernel<2, false>(s, units, maps, prm)
+                   : launch_kernel<1, false>(s, units, maps, prm);
 }
 
 cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& pl, DevState* st, const TileStat* tstats,
                             const float* mref, RowStat* rowstat, float* H, int32_t* argmax,
                             float* sc, int32_t* redo_rows, float redo_gap, const void* h,
                             const void* E, const float* scale_tab, int S,
-                            const SamplerArgs& sa) {
+                            const SamplerArgs& sa, const DrawArgs& draw) {
   TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
   const float* Opart = reinterpret_cast<const float*>(static_cast<const char*>(pl.ws) + L.Opart);
   (void)redo_rows;
@@ -1230,7 +1295,8 @@ cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& pl, DevState* st, cons
       &cfg, tc::k_merge_tc, st, reinterpret_cast<const TcStat*>(tstats), 2 * L.n_vt, mref, Opart,
       L.G, pl.C, pl.V, pl.d, rowstat, H, argmax, sc, redo_gap,
       static_cast<const __nv_bfloat16*>(h), static_cast<const __nv_bfloat16*>(E), scale_tab, S,
-      reinterpret_cast<unsigned*>(static_cast<char*>(pl.ws) + L.counters) + 2 * L.n_vt + 2, sa);
+      reinterpret_cast<unsigned*>(static_cast<char*>(pl.ws) + L.counters) + 2 * L.n_vt + 2,
+      draw.sampled ? static_cast<const TcSamp*>(draw.tsamp) : nullptr, draw.sampled, sa);
 }
 
 void tc_partials(const TcPlan& pl, const float** Opart, int* nO) {

@@ -27,14 +27,18 @@ void tc_plan_free(TcPlan* p);
 int tc_launches(const TcPlan& p);   // kernels per launch_tc_attention call
 cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& p, DevState* st, const void* h,
                                 const void* E, const float* mref, const float* scale_tab,
-                                int S, TileStat* tstats, float* O, void* ws);
+                                int S, TileStat* tstats, float* O, void* ws,
+                                const DrawArgs& draw);
 // Per-row merge of the kernel's statistics and partials into sc, H and argmax
 // (rows whose maximum overshot the reference are recomputed exactly); the last
 // row's CTA then runs the sampler and stop test for the whole canvas.
 cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& p, DevState* st, const TileStat* tstats,
                             const float* mref, RowStat* rowstat, float* H, int32_t* argmax,
                             float* sc, int32_t* redo_rows, float redo_gap, const void* h,
-                            const void* E, const float* scale_tab, int S, const SamplerArgs& sa);
+                            const void* E, const float* scale_tab, int S, const SamplerArgs& sa,
+                            const DrawArgs& draw);
+// Bytes of the per-half-tile draw statistics (DrawArgs::tsamp) of the multinomial rule.
+size_t tc_draw_bytes(int C, int V, int d);
 // Hand-off counters the prologue zeroes before every step.
 void tc_counters(const TcPlan& p, unsigned** ptr, int* count);
 // Per-range-group partials of O = P E that the merge sums.
