@@ -49,7 +49,7 @@ constexpr int BK = 64;         // K per pipeline stage (one 128-byte swizzle row
 constexpr int KV2 = 256;       // vocabulary entries per range (unit of G2 ownership): one tile,
                                // so range group g owns tiles g, g+G, ... and all groups
                                // advance through the ring together
-constexpr int RING = 64;       // P tiles (256 vocabulary entries each) resident at once
+constexpr int RING = 72;       // P tiles (256 vocabulary entries each) resident at once
 constexpr int THREADS = 320;    // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr int EPI_WARPS = 8;
 constexpr int QN = 8;          // G1 item queue depth (tile indices handed to the CTA's warps)
@@ -729,13 +729,19 @@ __global__ void __launch_bounds__(THREADS, 1)
             vbest = cm;
             arg = vt * BN + c0 + c * 32 + jj;
           }
+          // Gumbel variates lie in [-2.82, 16.64], so the winning z + G is at least
+          // (row max) - 2.82 >= mref - 2.82, and an entry with z < mref - 19.46
+          // cannot win: such chunks are skipped (1.0 of slack covers the
+          // rounding differences between mref and these logits).
           if constexpr (DRAW) {
-            const int col0 = vt * BN + c0 + c * 32;
-            const uint64_t rbase = (uint64_t)row * (uint64_t)p.V + (uint64_t)col0;
+            if (cm * scale >= mref - 20.5f) {
+              const int col0 = vt * BN + c0 + c * 32;
+              const uint64_t rbase = (uint64_t)row * (uint64_t)p.V + (uint64_t)col0;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float g = v[j] * scale + gumbel_from_key(sm64(gpre ^ (rbase + (uint64_t)j)));
-              if (g > gbest) { gbest = g; garg = col0 + j; }
+              for (int j = 0; j < 32; ++j) {
+                const float g = v[j] * scale + gumbel_from_key(sm64(gpre ^ (rbase + (uint64_t)j)));
+                if (g > gbest) { gbest = g; garg = col0 + j; }
+              }
             }
           }
           uint32_t pk[16];
