@@ -183,6 +183,16 @@ def run_reference(args, w):
     return 0
 
 
+# DRAM bytes (read + write) per launch of the tensor-core kernel, from the ncu
+# capture summarised under profiles/ (taken on the V=65536 profiling shape and
+# scaled by the vocabulary, since E and the P ring both grow with V).
+DRAM_TRAFFIC = {
+    synthetic.HEADLINE.name: (4 * (289.856512e6 + 8.805888e6),
+                              "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at "
+                              "C=256, V=65536, d=2048, scaled by 4 to V=262144"),
+}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -314,8 +324,11 @@ def main():
     attn_s = (attn_ms / 1e3) / max(attn_steps, 1)
     achieved_tflops = flops / attn_s / 1e12
     peak = pk["tflops_sustained"]
+    traffic = DRAM_TRAFFIC.get(w.name) if den.impl == dg.DG_IMPL_TC else None
     roof = {"bound": "tensor", "achieved": achieved_tflops, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved_tflops / peak, "traffic": None,
+            "frac": achieved_tflops / peak,
+            "traffic": traffic[0] if traffic else None,
+            "traffic_src": traffic[1] if traffic else None,
             "kernel": "vocabulary attention (" + ("tcgen05" if den.impl == dg.DG_IMPL_TC else "CUDA-core") + ")",
             "kernel_ms_per_step": attn_s * 1e3,
             "peak_src": f"{pk['src']} bf16 sustained (kernel timed inside a long step loop)",
