@@ -34,7 +34,8 @@ struct Layout {
   int nsplit = 0;      // CUDA-core path: vocabulary splits of sc
   size_t state = 0, scale = 0, target = 0, canvas = 0, argmax = 0, argmax_prev = 0, accept = 0,
          order = 0, prefix = 0, H = 0, mref = 0, rowstat = 0, redo_rows = 0, h = 0, sc = 0,
-         tstats = 0, zbuf = 0, partial = 0, O = 0, tc = 0, sampled = 0, tsamp = 0, total = 0;
+         tstats = 0, zbuf = 0, partial = 0, O = 0, tc = 0, sampled = 0, tsamp = 0, h_last = 0,
+         mref_last = 0, total = 0;
   size_t tc_bytes = 0;
 };
 
@@ -120,6 +121,8 @@ int make_layout(const dg_config* c, Layout* L, char* why, size_t n) {
     L->tstats = take(sizeof(TileStat) * C * L->ntiles);
     L->tc_bytes = tc_workspace_bytes(c->C, c->V, c->d);
     L->tc = take(L->tc_bytes);
+    L->h_last = take(esz * C * d);
+    L->mref_last = take(4 * C);
     if (c->token_rule == DG_TOKEN_MULTINOMIAL) L->tsamp = take(tc_draw_bytes(c->C, c->V, c->d));
   }
   L->total = off;
@@ -158,6 +161,7 @@ struct dg_ctx {
   cudaGraphExec_t graph_exec = nullptr;
   cudaGraphConditionalHandle cond = 0;
   // profiling
+  bool h_ready = false;      // host mirror of DevState::h_ready for stepwise calls
   bool prof = false;
   std::vector<cudaEvent_t> ev;
   size_t ev_used = 0;
@@ -193,10 +197,15 @@ int launch_step(dg_ctx* ctx, bool standin, bool use_cond) {
   unsigned* zero = nullptr;
   int nzero = 0;
   if (tc) tc_counters(ctx->tc_plan, &zero, &nzero);
-  DG_CK(launch_prologue(s, c.dtype, ctx->st, ctx->E, ctx->target, ctx->canvas, ctx->sc, ctx->h,
-                        c.C, c.V, c.d, c.seed, c.coef_target, c.coef_canvas, sigma, standin ? 1 : 0,
-                        ctx->scale_tab, c.max_steps, ctx->argmax_prev, tc ? ctx->mref : nullptr,
-                        zero, nzero));
+  // After a tensor-core step the merge kernel has already written this step's
+  // stand-in h and m_ref (DevState::h_ready); a stepwise call then skips the
+  // prologue launch. A captured loop keeps it: it checks h_ready on the device.
+  const bool skip_prologue = tc && standin && !use_cond && ctx->h_ready;
+  if (!skip_prologue)
+    DG_CK(launch_prologue(s, c.dtype, ctx->st, ctx->E, ctx->target, ctx->canvas, ctx->sc, ctx->h,
+                          c.C, c.V, c.d, c.seed, c.coef_target, c.coef_canvas, sigma,
+                          standin ? 1 : 0, ctx->scale_tab, c.max_steps, ctx->argmax_prev,
+                          tc ? ctx->mref : nullptr, zero, nzero));
   cudaEvent_t e0 = nullptr, e1 = nullptr;
   if (ctx->prof && !use_cond) {
     if (ctx->ev_used + 2 > ctx->ev.size()) {
@@ -210,7 +219,7 @@ int launch_step(dg_ctx* ctx, bool standin, bool use_cond) {
     e1 = ctx->ev[ctx->ev_used++];
     DG_CK(cudaEventRecord(e0, s));
   }
-  ctx->launches += tc ? 2 + tc_launches(ctx->tc_plan) : 6;
+  ctx->launches += tc ? (skip_prologue ? 1 : 2) + tc_launches(ctx->tc_plan) : 6;
   const SamplerArgs sa = make_sampler_args(
       ctx->st, ctx->H, ctx->argmax, ctx->canvas, ctx->argmax_prev, ctx->accept, ctx->order,
       ctx->prefix, c.C, c.V, c.seed, c.tau, c.stop_entropy, c.stop_unchanged, c.stop_rule,
@@ -220,9 +229,22 @@ int launch_step(dg_ctx* ctx, bool standin, bool use_cond) {
                               c.max_steps, ctx->tstats, ctx->O, ctx->tc, ctx->draw));
     if (e1) DG_CK(cudaEventRecord(e1, s));
     // merge, then (inside the same kernel) the sampler and stop test
+    NextStandin nx;
+    nx.target = ctx->target;
+    nx.seed = c.seed;
+    nx.A = c.coef_target;
+    nx.B = c.coef_canvas;
+    nx.sigma = sigma;
+    nx.zero = zero;
+    nx.nzero = nzero;
+    nx.h_last = at<void>(ctx, ctx->L.h_last);
+    nx.mref_last = at<float>(ctx, ctx->L.mref_last);
     DG_CK(launch_tc_merge(s, ctx->tc_plan, ctx->st, ctx->tstats, ctx->mref, ctx->rowstat, ctx->H,
                           ctx->argmax, ctx->sc, ctx->redo_rows, kRedoGap, ctx->h, ctx->E,
-                          ctx->scale_tab, c.max_steps, sa, ctx->draw));
+                          ctx->scale_tab, c.max_steps, sa, ctx->draw, nx));
+    // the merge prepares the next step's h unless the block stopped, and then
+    // nothing more runs until dg_begin_block
+    ctx->h_ready = true;
   } else {
     DG_CK(launch_simt_attention(s, c.dtype, ctx->st, ctx->h, ctx->E, ctx->zbuf, ctx->tstats,
                                 ctx->rowstat, ctx->partial, ctx->H, ctx->argmax, ctx->sc, c.C,
@@ -377,6 +399,7 @@ int dg_begin_block(dg_ctx* ctx, int32_t block) {
   DG_CK(launch_begin_block(ctx->stream, ctx->st, ctx->target, ctx->canvas, ctx->sc, c.C, c.d, c.V,
                            c.seed, block));
   ctx->launches += 1;
+  ctx->h_ready = false;
   return DG_OK;
 }
 
@@ -447,16 +470,27 @@ int dg_read(dg_ctx* ctx, int32_t what, void* dst) {
     case DG_ENTROPY: src = ctx->H; bytes = 4 * C; break;
     case DG_ACCEPT: src = ctx->accept; bytes = 4 * C; break;
     case DG_SC: src = ctx->sc; bytes = 4 * Cd; break;
-    case DG_HIDDEN: src = ctx->h; bytes = Cd * (c.dtype == DG_F32 ? 4 : 2); break;
+    // the tensor-core merge overwrites h and m_ref with the next step's; it
+    // keeps copies of the last step's
+    case DG_HIDDEN:
+      src = ctx->L.impl == DG_IMPL_TC ? at<void>(ctx, ctx->L.h_last) : ctx->h;
+      bytes = Cd * (c.dtype == DG_F32 ? 4 : 2);
+      break;
     case DG_TARGET: src = ctx->target; bytes = 4 * C; break;
     case DG_ORDER: src = ctx->order; bytes = 4 * C; break;
     case DG_PREFIX: src = ctx->prefix; bytes = 4 * C; break;
     case DG_STATE: src = ctx->st; bytes = 64; break;
-    case DG_MREF: src = ctx->mref; bytes = 4 * C; break;
+    case DG_MREF:
+      src = ctx->L.impl == DG_IMPL_TC ? at<float>(ctx, ctx->L.mref_last) : ctx->mref;
+      bytes = 4 * C;
+      break;
     case DG_SAMPLED: src = at<int32_t>(ctx, ctx->L.sampled); bytes = 4 * C; break;
     default: return fail(ctx, DG_EINVAL, "unknown item %d", what);
   }
   DG_CK(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, ctx->stream));
+  // the stand-in h prepared by the last merge may depend on what was written
+  ctx->h_ready = false;
+  DG_CK(cudaMemsetAsync(&ctx->st->h_ready, 0, sizeof(int32_t), ctx->stream));
   return DG_OK;
 }
 
@@ -477,6 +511,9 @@ int dg_write(dg_ctx* ctx, int32_t what, const void* src) {
     default: return fail(ctx, DG_EINVAL, "item %d is not writable", what);
   }
   DG_CK(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, ctx->stream));
+  // the stand-in h prepared by the last merge may depend on what was written
+  ctx->h_ready = false;
+  DG_CK(cudaMemsetAsync(&ctx->st->h_ready, 0, sizeof(int32_t), ctx->stream));
   return DG_OK;
 }
 

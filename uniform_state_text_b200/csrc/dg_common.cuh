@@ -24,7 +24,9 @@ struct DevState {
   int32_t status;     // 0 or a negative error code raised on the device
   int32_t has_prev;   // an argmax of a previous step exists
   int32_t redo;       // rows re-evaluated because the logit reference was low
-  int32_t pad[7];
+  int32_t epoch;      // tensor-core merge: bumped once per step after the sampler ran
+  int32_t h_ready;    // 1: h and m_ref already hold the stand-in state for step t
+  int32_t pad[5];
 };
 
 // Domain tags carried in the step field of the key.

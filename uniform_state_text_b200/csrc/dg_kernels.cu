@@ -18,6 +18,7 @@
 #include "dg_common.cuh"
 #include "dg_kernels.h"
 #include "dg_sampler.cuh"
+#include "dg_standin.cuh"
 
 namespace dg {
 
@@ -48,6 +49,7 @@ __global__ void k_begin_block(DevState* st, int32_t* target, int32_t* canvas, fl
     st->status = 0;
     st->has_prev = 0;
     st->redo = 0;
+    st->h_ready = 0;
   }
 }
 
@@ -55,34 +57,6 @@ __global__ void k_begin_block(DevState* st, int32_t* target, int32_t* canvas, fl
 // Stand-in hidden state and per-row logit reference.
 // One CTA per canvas row.
 // ---------------------------------------------------------------------------
-// Eight consecutive elements of E, sc or h (16-byte aligned for bf16, 32 for fp32).
-__device__ __forceinline__ void load8(const float* p, float v[8]) {
-  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float v[8]) {
-  const uint4 u = *reinterpret_cast<const uint4*>(p);
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    v[2 * j] = __uint_as_float(w[j] << 16);
-    v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-  }
-}
-__device__ __forceinline__ void store8(float* p, const float v[8]) {
-  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
-  *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
-}
-__device__ __forceinline__ void store8(__nv_bfloat16* p, const float v[8]) {
-  uint32_t w[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
-    w[j] = *reinterpret_cast<const uint32_t*>(&b2);
-  }
-  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
-}
-
 template <typename T>
 __global__ void __launch_bounds__(256) k_prologue(const DevState* st, const T* E,
     const int32_t* target, const int32_t* canvas, const float* sc, T* h, int C, int V, int d,
@@ -99,50 +73,18 @@ __global__ void __launch_bounds__(256) k_prologue(const DevState* st, const T* E
   const int tgt = target[i] & (V - 1), can = canvas[i] & (V - 1);
   const int prev_raw = argmax_prev[i] & (V - 1);
   if (st->done) return;
+  // The tensor-core merge of the previous step already wrote this step's
+  // stand-in h, m_ref and zeroed counters.
+  if (standin && st->h_ready) return;
   if (zero && blockIdx.x == 0)
     for (int j = threadIdx.x; j < nzero; j += blockDim.x) zero[j] = 0u;
   const int t = st->t;
   const int ts = min(max(t, 0), S - 1);
   const int prev = st->has_prev ? prev_raw : can;
   const uint64_t pre = key_prefix(seed, (uint64_t)(uint32_t)st->block, kTagNoise + (uint64_t)t);
-  const T* Et = E + (size_t)tgt * d;
-  const T* Ec = E + (size_t)can * d;
-  const T* Ep = E + (size_t)prev * d;
-  T* hrow = h + (size_t)i * d;
-  const float* scrow = sc + (size_t)i * d;
   float dc = 0.f, dp = 0.f;
-  for (int k0 = threadIdx.x * 8; k0 < d; k0 += blockDim.x * 8) {
-    float ec[8], hv[8];
-    load8(Ec + k0, ec);
-    if (standin) {
-      float et[8], s8[8];
-      load8(Et + k0, et);
-      load8(scrow + k0, s8);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint64_t idx = (uint64_t)i * (uint64_t)d + (uint64_t)(k0 + j);
-        float v = A * et[j] + B * ec[j];
-        v = v + s8[j];
-        v = v + sigma * gauss_from_key(sm64(pre ^ idx));
-        hv[j] = v;
-      }
-      store8(hrow + k0, hv);
-      // what the contraction reads is the stored (rounded) value
-#pragma unroll
-      for (int j = 0; j < 8; ++j) hv[j] = to_f32(from_f32<T>(hv[j]));
-    } else {
-      load8(hrow + k0, hv);
-    }
-    if (mref) {
-      float ep[8];
-      load8(Ep + k0, ep);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        dc = fmaf(hv[j], ec[j], dc);
-        dp = fmaf(hv[j], ep[j], dp);
-      }
-    }
-  }
+  standin_row_part<T>(i, threadIdx.x, blockDim.x, E, tgt, can, prev, sc + (size_t)i * d,
+                      h + (size_t)i * d, d, pre, A, B, sigma, standin, mref != nullptr, &dc, &dp);
   if (!mref) return;
   __shared__ float red[2][32];
   for (int o = 16; o; o >>= 1) {

@@ -43,6 +43,18 @@ inline SamplerArgs make_sampler_args(DevState* st, const float* H, const int32_t
   return a;
 }
 
+// What the tensor-core merge needs to prepare the next step's stand-in hidden
+// state (the prologue's work) and to reset the attention kernel's counters.
+struct NextStandin {
+  const int32_t* target = nullptr;
+  uint64_t seed = 0;
+  float A = 0.f, B = 0.f, sigma = 0.f;   // h = A E[target] + B E[canvas] + sc + sigma g
+  unsigned* zero = nullptr;               // counters to zero for the next step
+  int nzero = 0;
+  void* h_last = nullptr;                 // [C][d] bf16: copy of the step's own h
+  float* mref_last = nullptr;             // [C]: copy of the step's own m_ref
+};
+
 // Multinomial token draw (DG_TOKEN_MULTINOMIAL): where the per-row draws go.
 // sampled == nullptr selects the argmax rule and nothing is drawn.
 struct DrawArgs {

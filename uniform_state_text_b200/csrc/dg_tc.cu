@@ -39,6 +39,7 @@
 
 #include "dg_tc.h"
 #include "dg_sampler.cuh"
+#include "dg_standin.cuh"
 
 namespace dg {
 namespace tc {
@@ -885,20 +886,23 @@ __device__ __noinline__ void merge_recompute(int i, int V, int d, const __nv_bfl
 }
 
 __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(DevState* st,
-    const TcStat* ts, int nts, const float* mref, const float* Opart, int nO, int C, int V, int d,
+    const TcStat* ts, int nts, float* mref, const float* Opart, int nO, int C, int V, int d,
     RowStat* rowstat, float* H, int32_t* argmax, float* sc, float redo_gap,
-    const __nv_bfloat16* h, const __nv_bfloat16* E, const float* scale_tab, int S,
-    unsigned* ticket, const TcSamp* tsamp, int32_t* sampled, const SamplerArgs sa) {
-  // Programmatic dependent launch: wait for the attention kernel's results,
-  // then let the next step's prologue be scheduled (it waits for this grid).
+    __nv_bfloat16* h, const __nv_bfloat16* E, const float* scale_tab, int S,
+    unsigned* ticket, const TcSamp* tsamp, int32_t* sampled, const NextStandin nx,
+    const SamplerArgs sa) {
+  // Programmatic dependent launch: wait for the attention kernel's results.
+  // No early trigger: the next kernel is usually the next step's attention
+  // kernel, and its CTAs waiting beside this grid slowed it (measured).
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;");
   if (st->done) {
     if (sa.use_cond && blockIdx.x == 0 && threadIdx.x == 0) cudaGraphSetConditional(sa.cond, 0);
     return;
   }
   __shared__ SamplerSmem sm;
   extern __shared__ float sacc[];   // [d], exact recomputation only
+  __shared__ int sh_epoch0;
+  if (threadIdx.x == 0) sh_epoch0 = *(volatile int*)&st->epoch;   // before this CTA's ticket
   const int r = threadIdx.x / kMergeThreadsPerRow;      // row of this CTA
   const int tid = threadIdx.x % kMergeThreadsPerRow;
   const int i0 = blockIdx.x * kMergeRows;
@@ -974,6 +978,7 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
       RowStat rs;
       rs.m = mref_i; rs.Z = Z; rs.pad[0] = best; rs.pad[1] = 0.f;
       rowstat[i] = rs;
+      nx.mref_last[i] = mref_i;
       const float gap = best - mref_i;
       redo = !(gap <= redo_gap) || !(Z > 0.f) || !(Z < INFINITY);
       if (redo) atomicAdd(&st->redo, 1);
@@ -1002,19 +1007,27 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
   const bool last = sh_ticket == gridDim.x - 1;
   const int nsamp = (C + 31) / 32 * 32;
   int x0 = threadIdx.x, xstep = blockDim.x;
+  bool sum_sc = true;
   if (last) {
     if (threadIdx.x < nsamp) {
       sample_and_stop(sa, sm, nsamp);
-      return;
+      sum_sc = false;
     }
     x0 = threadIdx.x - nsamp;
     xstep = blockDim.x - nsamp;
+  }
+  // Keep this step's h rows (the next step's overwrite them below).
+  {
+    const uint4* hs = reinterpret_cast<const uint4*>(h + (size_t)i0 * d);
+    uint4* hd = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(nx.h_last) + (size_t)i0 * d);
+    const int n16 = min(kMergeRows, C - i0) * d / 8;
+    for (int x = x0; sum_sc && x < n16; x += xstep) hd[x] = hs[x];
   }
   // sc of the rows that were not recomputed: four columns per thread and
   // pass, the partials added in g order.
   const size_t pstride = (size_t)C * d;
   const int d4 = d / 4;
-  for (int x = x0; x < kMergeRows * d4; x += xstep) {
+  for (int x = x0; sum_sc && x < kMergeRows * d4; x += xstep) {
     const int q = x / d4, k = (x % d4) * 4;
     const int row = i0 + q;
     if (row >= C || sh_redo[q]) continue;
@@ -1028,6 +1041,63 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
     const float inv = sh_inv[q];
     *reinterpret_cast<float4*>(sc + (size_t)row * d + k) =
         make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  }
+
+  // Next step's stand-in hidden state and logit reference for this CTA's rows
+  // (the work of the prologue kernel, which the next step then skips). It
+  // needs the sampler's canvas: the last CTA publishes it by bumping the epoch
+  // (release); the others wait for that (acquire, bounded).
+  __shared__ int sh_go;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int go = 1;
+    if (last) {
+      asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(&st->epoch) : "memory");
+    } else {
+      const uint64_t t0 = gtimer();
+      for (uint32_t n = 0;; ++n) {
+        int e;
+        asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(e) : "l"(&st->epoch) : "memory");
+        if (e != sh_epoch0) break;
+        __nanosleep(128);
+        if ((n & 15) == 15 && gtimer() - t0 > TIMEOUT_NS) {
+          atomicCAS(&st->status, 0, -4 /* DG_ETIMEOUT */);
+          go = 0;
+          break;
+        }
+      }
+    }
+    sh_go = go && !*(volatile int*)&st->done;
+  }
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    // every CTA took its ticket before the epoch moved: the hand-off counters
+    // and the ticket start the next step at zero
+    for (int j = threadIdx.x; j < nx.nzero; j += blockDim.x) nx.zero[j] = 0u;
+    if (threadIdx.x == 0) st->h_ready = sh_go;
+  }
+  if (!sh_go) return;
+  const int t1 = *(volatile int*)&st->t;                 // the next step (the sampler advanced it)
+  const uint64_t pre = key_prefix(nx.seed, (uint64_t)(uint32_t)*(volatile int*)&st->block,
+                                  kTagNoise + (uint64_t)t1);
+  float dc = 0.f, dp = 0.f;
+  const int tgt = row_ok ? nx.target[i] & (V - 1) : 0;
+  const int can = row_ok ? sa.canvas[i] & (V - 1) : 0;
+  const int prev = row_ok ? argmax[i] & (V - 1) : 0;
+  if (row_ok)
+    standin_row_part<__nv_bfloat16>(i, tid, kMergeThreadsPerRow, E, tgt, can, prev,
+                                    sc + (size_t)i * d, h + (size_t)i * d, d, pre, nx.A, nx.B,
+                                    nx.sigma, 1, true, &dc, &dp);
+  for (int o = 16; o; o >>= 1) {
+    dc += __shfl_xor_sync(0xffffffffu, dc, o);
+    dp += __shfl_xor_sync(0xffffffffu, dp, o);
+  }
+  if (l == 0) { sZ[r][w] = dc; sS[r][w] = dp; }
+  __syncthreads();
+  if (tid == 0 && row_ok) {
+    float a = 0.f, b = 0.f;
+    for (int j = 0; j < WPR; ++j) { a += sZ[r][j]; b += sS[r][j]; }
+    mref[i] = scale_tab[min(max(t1, 0), S - 1)] * fmaxf(a, b);
   }
 }
 
@@ -1281,7 +1351,7 @@ cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& pl, DevState* st, cons
                             const float* mref, RowStat* rowstat, float* H, int32_t* argmax,
                             float* sc, int32_t* redo_rows, float redo_gap, const void* h,
                             const void* E, const float* scale_tab, int S,
-                            const SamplerArgs& sa, const DrawArgs& draw) {
+                            const SamplerArgs& sa, const DrawArgs& draw, const NextStandin& nx) {
   TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
   const float* Opart = reinterpret_cast<const float*>(static_cast<const char*>(pl.ws) + L.Opart);
   (void)redo_rows;
@@ -1298,11 +1368,12 @@ cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& pl, DevState* st, cons
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(
-      &cfg, tc::k_merge_tc, st, reinterpret_cast<const TcStat*>(tstats), 2 * L.n_vt, mref, Opart,
-      L.G, pl.C, pl.V, pl.d, rowstat, H, argmax, sc, redo_gap,
-      static_cast<const __nv_bfloat16*>(h), static_cast<const __nv_bfloat16*>(E), scale_tab, S,
+      &cfg, tc::k_merge_tc, st, reinterpret_cast<const TcStat*>(tstats), 2 * L.n_vt,
+      const_cast<float*>(mref), Opart, L.G, pl.C, pl.V, pl.d, rowstat, H, argmax, sc, redo_gap,
+      static_cast<__nv_bfloat16*>(const_cast<void*>(h)), static_cast<const __nv_bfloat16*>(E),
+      scale_tab, S,
       reinterpret_cast<unsigned*>(static_cast<char*>(pl.ws) + L.counters) + 2 * L.n_vt + 2,
-      draw.sampled ? static_cast<const TcSamp*>(draw.tsamp) : nullptr, draw.sampled, sa);
+      draw.sampled ? static_cast<const TcSamp*>(draw.tsamp) : nullptr, draw.sampled, nx, sa);
 }
 
 void tc_partials(const TcPlan& pl, const float** Opart, int* nO) {

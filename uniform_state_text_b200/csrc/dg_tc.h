@@ -31,12 +31,14 @@ cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& p, DevState* st, c
                                 const DrawArgs& draw);
 // Per-row merge of the kernel's statistics and partials into sc, H and argmax
 // (rows whose maximum overshot the reference are recomputed exactly); the last
-// row's CTA then runs the sampler and stop test for the whole canvas.
+// CTA then runs the sampler and stop test for the whole canvas, after which
+// every CTA writes the next step's stand-in h and m_ref for its rows and the
+// counters are reset (DevState::h_ready = 1: the next prologue has no work).
 cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& p, DevState* st, const TileStat* tstats,
                             const float* mref, RowStat* rowstat, float* H, int32_t* argmax,
                             float* sc, int32_t* redo_rows, float redo_gap, const void* h,
                             const void* E, const float* scale_tab, int S, const SamplerArgs& sa,
-                            const DrawArgs& draw);
+                            const DrawArgs& draw, const NextStandin& nx);
 // Bytes of the per-half-tile draw statistics (DrawArgs::tsamp) of the multinomial rule.
 size_t tc_draw_bytes(int C, int V, int d);
 // Hand-off counters the prologue zeroes before every step.
