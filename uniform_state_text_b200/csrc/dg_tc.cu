@@ -471,11 +471,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   if constexpr (CG == 2) cluster_sync();   // peer barriers initialised before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_base_slot;
-  // Programmatic dependent launch: the set-up above overlapped the prologue;
-  // its outputs (h, m_ref, zeroed counters, loop state) are visible after the
-  // wait. The merge kernel may then start its own set-up.
+  // Programmatic dependent launch: the set-up above overlapped the previous
+  // kernel; its outputs (h, m_ref, zeroed counters, loop state) are visible
+  // after the wait. No early trigger: merge CTAs waiting beside this kernel
+  // for its whole duration cost more than their launch saves (measured).
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;");
   const bool skip = p.st->done != 0;                     // uniform over the grid
 
   // Work description. RBI: row blocks iterated by G1 items (1 for pairs, which
