@@ -226,7 +226,8 @@ int launch_step(dg_ctx* ctx, bool standin, bool use_cond) {
       c.accept_rule, c.fixed_steps, c.max_steps, ctx->cond, use_cond ? 1 : 0, ctx->draw.sampled);
   if (tc) {
     DG_CK(launch_tc_attention(s, ctx->tc_plan, ctx->st, ctx->h, ctx->E, ctx->mref, ctx->scale_tab,
-                              c.max_steps, ctx->tstats, ctx->O, ctx->tc, ctx->draw));
+                              c.max_steps, ctx->tstats, ctx->O, ctx->tc, ctx->draw, ctx->H,
+                              ctx->argmax, ctx->rowstat, kRedoGap, sa));
     if (e1) DG_CK(cudaEventRecord(e1, s));
     // merge, then (inside the same kernel) the sampler and stop test
     NextStandin nx;

@@ -26,7 +26,8 @@ struct DevState {
   int32_t redo;       // rows re-evaluated because the logit reference was low
   int32_t epoch;      // tensor-core merge: bumped once per step after the sampler ran
   int32_t h_ready;    // 1: h and m_ref already hold the stand-in state for step t
-  int32_t pad[5];
+  int32_t tc_sampled; // 1: the attention kernel's G1 CTAs merged the rows and ran the sampler
+  int32_t pad[4];
 };
 
 // Domain tags carried in the step field of the key.

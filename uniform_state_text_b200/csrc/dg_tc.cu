@@ -84,6 +84,17 @@ struct Params {
   TcStat* tstats2;             // [C][2 * n_vt] half-tile statistics
   TcSamp* tsamp;               // [C][2 * n_vt] best z + G (multinomial draw), or nullptr
   uint64_t seed;               // keys the draw's Gumbel variates
+  // Row merge and sampler, run by the G1 CTAs once every G1 item is done
+  // (while the G2 CTAs finish): per-row outputs, counters, sampler arguments.
+  float* H;
+  int32_t* argmax;
+  RowStat* rowstat;
+  int32_t* sampled;            // multinomial draws, or nullptr
+  float redo_gap;
+  unsigned* g1_done;           // G1 CTAs whose statistics are all written
+  unsigned* g1_ticket;         // G1 CTAs whose rows are merged
+  int* redo_flag;              // a row needs the exact recomputation
+  SamplerArgs sa;
 };
 
 // Per-CTA wait-time tracing, compiled in only with -DDG_TC_TRACE (measurement
@@ -401,6 +412,103 @@ __device__ __forceinline__ bool is_g1_unit(const Params& p, int CG) {
   return (int)(blockIdx.x / CG) < p.n1;
 }
 
+// After its last item each G1 CTA publishes that its statistics are written;
+// once all G1 CTAs have, they merge the rows' statistics (G1 CTA k takes rows
+// k, k + ng1, ...; fixed order) into H, argmax, the draw and the row
+// statistics, and the last one to finish runs the sampler and stop test for
+// the whole canvas -- all while the G2 CTAs are still finishing. A row whose
+// reference was too low leaves the rows' merge and the sampler to the merge
+// kernel (redo_flag), which then recomputes it exactly.
+template <bool DRAW>
+__device__ __noinline__ void g1_finish(const Params& p, int ng1, unsigned char* smem) {
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  const int nw = nthr >> 5, w = tid >> 5, l = tid & 31;
+  int* flag = reinterpret_cast<int*>(smem);                     // [2]
+  float* wZ = reinterpret_cast<float*>(smem + 64);              // [nw] each
+  float* wS = wZ + 32;
+  float* wB = wS + 32;
+  int* wA = reinterpret_cast<int*>(wB + 32);
+  float* wG = reinterpret_cast<float*>(wA + 32);
+  int* wGA = reinterpret_cast<int*>(wG + 32);
+  if (tid == 0) {
+    red_release_add(p.g1_done, 1u);
+    flag[0] = counter_wait(p.g1_done, (unsigned)ng1, p) ? 1 : 0;
+  }
+  __syncthreads();
+  if (!flag[0]) return;
+  const int nts = 2 * p.n_vt;
+  for (int i = blockIdx.x; i < p.C; i += ng1) {
+    float Z = 0.f, S1 = 0.f, best = -INFINITY, gbest = -INFINITY;
+    int arg = 0x7fffffff, garg = 0x7fffffff;
+    const float4* ts4 = reinterpret_cast<const float4*>(p.tstats2 + (size_t)i * nts);
+#pragma unroll 4
+    for (int j = tid; j < nts; j += nthr) {
+      const float4 t = ts4[j];                 // {Z, S1, best, arg}
+      const int ta = __float_as_int(t.w);
+      Z += t.x;
+      S1 += t.y;
+      if (better(t.z, ta, best, arg)) { best = t.z; arg = ta; }
+    }
+    if constexpr (DRAW) {
+      const float2* sp2 = reinterpret_cast<const float2*>(p.tsamp + (size_t)i * nts);
+#pragma unroll 4
+      for (int j = tid; j < nts; j += nthr) {
+        const float2 q = sp2[j];               // {score, arg}
+        const int qa = __float_as_int(q.y);
+        if (better(q.x, qa, gbest, garg)) { gbest = q.x; garg = qa; }
+      }
+    }
+    for (int o = 16; o; o >>= 1) {
+      Z += __shfl_xor_sync(0xffffffffu, Z, o);
+      S1 += __shfl_xor_sync(0xffffffffu, S1, o);
+      const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oa = __shfl_xor_sync(0xffffffffu, arg, o);
+      if (better(ob, oa, best, arg)) { best = ob; arg = oa; }
+      if constexpr (DRAW) {
+        const float gb = __shfl_xor_sync(0xffffffffu, gbest, o);
+        const int ga = __shfl_xor_sync(0xffffffffu, garg, o);
+        if (better(gb, ga, gbest, garg)) { gbest = gb; garg = ga; }
+      }
+    }
+    if (l == 0) { wZ[w] = Z; wS[w] = S1; wB[w] = best; wA[w] = arg; wG[w] = gbest; wGA[w] = garg; }
+    __syncthreads();
+    if (tid == 0) {
+      Z = wZ[0]; S1 = wS[0]; best = wB[0]; arg = wA[0]; gbest = wG[0]; garg = wGA[0];
+      for (int j = 1; j < nw; ++j) {
+        Z += wZ[j];
+        S1 += wS[j];
+        if (better(wB[j], wA[j], best, arg)) { best = wB[j]; arg = wA[j]; }
+        if (better(wG[j], wGA[j], gbest, garg)) { gbest = wG[j]; garg = wGA[j]; }
+      }
+      const float mref_i = p.mref[i];
+      p.H[i] = fmaxf(logf(Z) - S1 / Z, 0.f);
+      p.argmax[i] = arg;
+      if constexpr (DRAW) p.sampled[i] = garg;
+      RowStat rs;
+      rs.m = mref_i; rs.Z = Z; rs.pad[0] = best; rs.pad[1] = 0.f;
+      p.rowstat[i] = rs;
+      const float gap = best - mref_i;
+      if (!(gap <= p.redo_gap) || !(Z > 0.f) || !(Z < INFINITY)) atomicOr(p.redo_flag, 1);
+    }
+    __syncthreads();
+  }
+  // Acquire-release ticket: this CTA's rows are visible before it counts, and
+  // the last CTA sees every row and every redo flag.
+  if (tid == 0) {
+    unsigned old;
+    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(old) : "l"(p.g1_ticket) : "memory");
+    flag[1] = (old == (unsigned)(ng1 - 1)) && !*(volatile int*)p.redo_flag;
+  }
+  __syncthreads();
+  if (!flag[1]) return;
+  SamplerSmem& sm = *reinterpret_cast<SamplerSmem*>(smem + 1024);
+  const int nsamp = (p.C + 31) / 32 * 32;
+  if (tid < nsamp) {
+    sample_and_stop(p.sa, sm, nsamp);
+    if (tid == 0) p.st->tc_sampled = 1;
+  }
+}
+
 // DRAW: the multinomial rule's Gumbel-max draw in the G1 epilogue (a separate
 // instantiation, so the argmax kernel keeps its register budget).
 template <int CG, bool DRAW>
@@ -408,7 +516,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     k_vocab_attention(const __grid_constant__ CUtensorMap tm_h,
                       const __grid_constant__ CUtensorMap tm_ek,
                       const __grid_constant__ CUtensorMap tm_emn,
-                      const __grid_constant__ CUtensorMap tm_p, const Params p) {
+                      const __grid_constant__ CUtensorMap tm_p,
+                      const __grid_constant__ Params p) {
   constexpr int NSTAGE_MAX = Pipe<CG>::STAGES;         // barrier array size
   constexpr int NB_ROWS = BN / CG;                      // B rows (G1) / columns (G2) per CTA
   // G1 CTAs and single-accumulator G2 CTAs: Pipe::STAGES stages of A + B/CG;
@@ -477,6 +586,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   // for its whole duration cost more than their launch saves (measured).
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const bool skip = p.st->done != 0;                     // uniform over the grid
+  // CTA 0 is a G1 CTA: this reset precedes its g1_done release, so it is
+  // ordered before the sampler sets the flag again at the end of G1. A skipped
+  // step (block already stopped) leaves it 0 too.
+  if (blockIdx.x == 0 && threadIdx.x == 0) p.st->tc_sampled = 0;
 
   // Work description. RBI: row blocks iterated by G1 items (1 for pairs, which
   // cover both row blocks with M = 256).
@@ -830,6 +943,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
                    : "memory");
   }
+  // Every copy into this CTA's stage buffers has landed (the producers drained
+  // before the barriers above), so they serve as scratch now.
+  if (is_g1 && !skip) g1_finish<DRAW>(p, CG * p.n1, smem);
 }
 
 // ---------------------------------------------------------------------------
@@ -895,20 +1011,43 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
   // No early trigger: the next kernel is usually the next step's attention
   // kernel, and its CTAs waiting beside this grid slowed it (measured).
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (st->done) {
+  // The attention kernel's G1 CTAs normally merged the rows and ran the
+  // sampler already (tc_sampled); then only sc, the copies of this step's h
+  // and the next step's h remain -- sc even when that sampler stopped the
+  // block. Without it, a stopped block means the step was skipped.
+  const bool fast = *(volatile int*)&st->tc_sampled != 0;
+  if (!fast && st->done) {
     if (sa.use_cond && blockIdx.x == 0 && threadIdx.x == 0) cudaGraphSetConditional(sa.cond, 0);
     return;
   }
   __shared__ SamplerSmem sm;
   extern __shared__ float sacc[];   // [d], exact recomputation only
+  constexpr int WPR = kMergeThreadsPerRow / 32;   // warps per row
+  __shared__ float sZ[kMergeRows][WPR], sS[kMergeRows][WPR], sB[kMergeRows][WPR];
+  __shared__ int sA[kMergeRows][WPR];
+  __shared__ float sG[kMergeRows][WPR];
+  __shared__ int sGA[kMergeRows][WPR];
+  __shared__ float sh_inv[kMergeRows], sh_best[kMergeRows];
+  __shared__ int sh_redo[kMergeRows];
+  __shared__ unsigned sh_ticket;
   __shared__ int sh_epoch0;
-  if (threadIdx.x == 0) sh_epoch0 = *(volatile int*)&st->epoch;   // before this CTA's ticket
   const int r = threadIdx.x / kMergeThreadsPerRow;      // row of this CTA
   const int tid = threadIdx.x % kMergeThreadsPerRow;
+  const int w = tid >> 5, l = tid & 31;
   const int i0 = blockIdx.x * kMergeRows;
   const int i = i0 + r;
   const bool row_ok = i < C;
   const float mref_i = row_ok ? mref[i] : 0.f;
+  if (fast) {
+    if (tid == 0) {
+      sh_redo[r] = 0;
+      sh_inv[r] = row_ok ? 1.0f / rowstat[i].Z : 0.f;
+      if (row_ok) nx.mref_last[i] = mref_i;
+    }
+    if (threadIdx.x == 0) sh_ticket = 0;
+    __syncthreads();
+  } else {
+  if (threadIdx.x == 0) sh_epoch0 = *(volatile int*)&st->epoch;   // before this CTA's ticket
   float Z = 0.f, S1 = 0.f, best = -INFINITY;
   int arg = 0x7fffffff;
   float gbest = -INFINITY;          // multinomial draw: best z + G and its index
@@ -943,15 +1082,6 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
     const int ga = __shfl_xor_sync(0xffffffffu, garg, o);
     if (better(gb, ga, gbest, garg)) { gbest = gb; garg = ga; }
   }
-  constexpr int WPR = kMergeThreadsPerRow / 32;   // warps per row
-  __shared__ float sZ[kMergeRows][WPR], sS[kMergeRows][WPR], sB[kMergeRows][WPR];
-  __shared__ int sA[kMergeRows][WPR];
-  __shared__ float sG[kMergeRows][WPR];
-  __shared__ int sGA[kMergeRows][WPR];
-  __shared__ float sh_inv[kMergeRows], sh_best[kMergeRows];
-  __shared__ int sh_redo[kMergeRows];
-  __shared__ unsigned sh_ticket;
-  const int w = tid >> 5, l = tid & 31;
   if (l == 0) {
     sZ[r][w] = Z; sS[r][w] = S1; sB[r][w] = best; sA[r][w] = arg;
     sG[r][w] = gbest; sGA[r][w] = garg;
@@ -1002,9 +1132,10 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
     sh_ticket = old;
   }
   __syncthreads();
+  }
   // In the last CTA the first nsamp threads run the sampler and the others
   // sum sc; elsewhere every thread sums sc.
-  const bool last = sh_ticket == gridDim.x - 1;
+  const bool last = !fast && sh_ticket == gridDim.x - 1;
   const int nsamp = (C + 31) / 32 * 32;
   int x0 = threadIdx.x, xstep = blockDim.x;
   bool sum_sc = true;
@@ -1051,7 +1182,9 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
   __syncthreads();
   if (threadIdx.x == 0) {
     int go = 1;
-    if (last) {
+    if (fast) {
+      // the sampler ran in the attention kernel, which has completed
+    } else if (last) {
       asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(&st->epoch) : "memory");
     } else {
       const uint64_t t0 = gtimer();
@@ -1317,7 +1450,8 @@ void tc_counters(const TcPlan& p, unsigned** ptr, int* count) {
 cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, const void* h,
                                 const void* E, const float* mref, const float* scale_tab,
                                 int S, TileStat* tstats, float* O, void* ws,
-                                const DrawArgs& draw) {
+                                const DrawArgs& draw, float* H, int32_t* argmax,
+                                RowStat* rowstat, float redo_gap, const SamplerArgs& sa) {
   (void)h; (void)E; (void)O;
   TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
   char* base = static_cast<char*>(ws);
@@ -1338,6 +1472,15 @@ cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, 
   prm.trace = reinterpret_cast<unsigned long long*>(base + L.trace);
   prm.tsamp = draw.sampled ? static_cast<TcSamp*>(draw.tsamp) : nullptr;
   prm.seed = draw.seed;
+  prm.H = H;
+  prm.argmax = argmax;
+  prm.rowstat = rowstat;
+  prm.sampled = draw.sampled;
+  prm.redo_gap = redo_gap;
+  prm.g1_done = ctr + 2 * L.n_vt + 3;
+  prm.g1_ticket = ctr + 2 * L.n_vt + 4;
+  prm.redo_flag = reinterpret_cast<int*>(ctr + 2 * L.n_vt + 5);
+  prm.sa = sa;
   const CUtensorMap* maps = reinterpret_cast<const CUtensorMap*>(pl.maps);
   const int units = L.n1 + L.n2;
   if (prm.tsamp)

@@ -25,10 +25,14 @@ int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, float* 
                  TileStat* tstats, void* ws, char* err, size_t errn);
 void tc_plan_free(TcPlan* p);
 int tc_launches(const TcPlan& p);   // kernels per launch_tc_attention call
+// The attention kernel; its G1 CTAs also merge the rows' statistics into H,
+// argmax and rowstat and run the sampler, unless a row needs the exact
+// recomputation (then the merge kernel does both).
 cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& p, DevState* st, const void* h,
                                 const void* E, const float* mref, const float* scale_tab,
                                 int S, TileStat* tstats, float* O, void* ws,
-                                const DrawArgs& draw);
+                                const DrawArgs& draw, float* H, int32_t* argmax,
+                                RowStat* rowstat, float redo_gap, const SamplerArgs& sa);
 // Per-row merge of the kernel's statistics and partials into sc, H and argmax
 // (rows whose maximum overshot the reference are recomputed exactly); the last
 // CTA then runs the sampler and stop test for the whole canvas, after which
