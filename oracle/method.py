@@ -44,6 +44,14 @@ Readings where the pages are silent or garbled (each also listed in the design doc):
     OR all entropies < stop_entropy, OR the step budget reached. stop_rule 1
     compares the argmax predictions of consecutive steps instead.
   * A finished block emits the final step's argmax at every position.
+  * Batched canvases (canvases = B > 1): B independent canvases of C/B
+    positions share each step's vocabulary attention (the rows are
+    independent). Entropy sort, acceptance (tau per canvas), re-noise and the
+    adaptive stop apply to each canvas on its own; a canvas that has stopped is
+    frozen (its tokens and emitted prediction no longer change) while the
+    others go on, and the block ends when every canvas has stopped. Keys stay
+    those of the combined row index, so canvas c is rows [c C/B, (c+1) C/B)
+    of a C-row canvas.
   * Self-conditioning feeds sc = softmax(z) E of the tempered logits straight
     into the next step's stand-in hidden state (the small FFNN of [VG] 5.1
     needs trained weights and is left out).
@@ -247,6 +255,33 @@ def entropy_bounded_accept(H32: np.ndarray, tau: float, rule: int) -> Acceptance
     return Acceptance(order=order, accepted=accepted, k=k, prefix=prefix)
 
 
+def accept_canvases(H32: np.ndarray, tau: float, rule: int, B: int, frozen=None):
+    """The entropy-bounded sampler on each of B canvases of len(H32)/B positions.
+
+    Canvas c is positions [c C/B, (c+1) C/B); it is sorted and accepted on its
+    own with its own budget tau. Frozen canvases (frozen[c] true) accept
+    nothing and keep the identity order. Returns (accepted bool [C], order
+    int64 [C] of global positions, per-canvas fp32 prefix sums [C], k per canvas).
+    """
+    H32 = np.asarray(H32, dtype=np.float32)
+    C = H32.shape[0]
+    Cc = C // B
+    accepted = np.zeros(C, dtype=bool)
+    order = np.arange(C, dtype=np.int64)
+    prefix = np.zeros(C, dtype=np.float32)
+    k = np.zeros(B, dtype=np.int64)
+    for c in range(B):
+        if frozen is not None and frozen[c]:
+            continue
+        seg = slice(c * Cc, (c + 1) * Cc)
+        a = entropy_bounded_accept(H32[seg], tau, rule)
+        accepted[seg] = a.accepted
+        order[seg] = a.order + c * Cc
+        prefix[seg] = a.prefix
+        k[c] = a.k
+    return accepted, order, prefix, k
+
+
 def renoise(w, accepted, argmax, block: int, t: int) -> np.ndarray:
     """Accepted positions take the chosen token (argmax, or the draw under
     token_rule 1); every rejected one a fresh uniform token."""
@@ -268,6 +303,11 @@ class State:
     argmax_prev: np.ndarray | None = None
     done: bool = False
     steps_done: int = 0
+    # batched canvases: per-canvas stop state and the emitted predictions
+    unchanged_c: np.ndarray | None = None
+    done_c: np.ndarray | None = None
+    steps_c: np.ndarray | None = None
+    emit: np.ndarray | None = None
 
 
 @dataclasses.dataclass
@@ -285,10 +325,17 @@ class StepRecord:
     done: bool
 
 
+def canvases(w) -> int:
+    return int(getattr(w, "canvases", 1))
+
+
 def begin_block(w, block: int) -> State:
     target, canvas = init_block(w, block)
+    B = canvases(w)
     return State(block=block, t=0, target=target, canvas=canvas,
-                 sc=np.zeros((w.C, w.d), dtype=np.float64))
+                 sc=np.zeros((w.C, w.d), dtype=np.float64),
+                 unchanged_c=np.zeros(B, dtype=np.int64), done_c=np.zeros(B, dtype=bool),
+                 steps_c=np.zeros(B, dtype=np.int64), emit=np.zeros(w.C, dtype=np.int64))
 
 
 def step(w, E: np.ndarray, st: State, h: np.ndarray | None = None) -> StepRecord:
@@ -303,21 +350,41 @@ def step(w, E: np.ndarray, st: State, h: np.ndarray | None = None) -> StepRecord
     else:
         att = vocab_attention(h, E, w.logit_scale / T)
     H32 = att.H.astype(np.float32)
-    acc = entropy_bounded_accept(H32, w.tau, w.accept_rule)
     noise = rng.tokens(w.seed, st.block, t, np.arange(w.C, dtype=np.uint64), w.V)
     chosen = att.sampled if multinomial else att.argmax
-    canvas_out = np.where(acc.accepted, chosen, noise).astype(np.int64)
-    all_conf = bool(np.all(H32 < np.float32(w.stop_entropy)))
-    if w.stop_rule == 0:
-        same = bool(np.array_equal(canvas_out, st.canvas))
-    else:
-        same = st.argmax_prev is not None and bool(np.array_equal(att.argmax, st.argmax_prev))
-    unchanged = st.unchanged + 1 if same else 0
+    B = canvases(w)
+    Cc = w.C // B
     last = (t + 1 >= w.max_steps)
-    if w.fixed_steps:
-        done = last
+    canvas_out = st.canvas.copy()
+    accepted, order, prefix, k_c = accept_canvases(H32, w.tau, w.accept_rule, B, st.done_c)
+    conf_c = np.zeros(B, dtype=bool)
+    for c in range(B):
+        seg = slice(c * Cc, (c + 1) * Cc)
+        if st.done_c[c]:
+            continue                      # a stopped canvas is frozen
+        canvas_out[seg] = np.where(accepted[seg], chosen[seg], noise[seg])
+        conf_c[c] = bool(np.all(H32[seg] < np.float32(w.stop_entropy)))
+        if w.stop_rule == 0:
+            same = bool(np.array_equal(canvas_out[seg], st.canvas[seg]))
+        else:
+            same = st.argmax_prev is not None and bool(
+                np.array_equal(att.argmax[seg], st.argmax_prev[seg]))
+        st.unchanged_c[c] = st.unchanged_c[c] + 1 if same else 0
+        if w.fixed_steps:
+            stop = last
+        else:
+            stop = last or conf_c[c] or st.unchanged_c[c] >= w.stop_unchanged
+        if stop:
+            st.done_c[c] = True
+            st.steps_c[c] = t + 1
+            st.emit[seg] = att.argmax[seg]
+    if B == 1:
+        acc = entropy_bounded_accept(H32, w.tau, w.accept_rule)
     else:
-        done = last or all_conf or unchanged >= w.stop_unchanged
+        acc = Acceptance(order=order, accepted=accepted, k=int(k_c.sum()), prefix=prefix)
+    done = bool(np.all(st.done_c))
+    unchanged = int(st.unchanged_c[0])
+    all_conf = bool(np.all(conf_c))
     rec = StepRecord(t=t, temperature=T, h=h, att=att, acc=acc, canvas_in=st.canvas.copy(),
                      canvas_out=canvas_out, noise=noise, unchanged=unchanged,
                      all_confident=all_conf, done=done)
@@ -332,12 +399,16 @@ def step(w, E: np.ndarray, st: State, h: np.ndarray | None = None) -> StepRecord
 
 
 def denoise_block(w, E: np.ndarray, block: int):
-    """Run one canvas to its stop; returns (final argmax, steps, per-step records)."""
+    """Run the block's canvases to their stops.
+
+    Returns (emitted tokens -- each canvas's argmax at its own final step --,
+    steps the block ran, per-step records).
+    """
     st = begin_block(w, block)
     records = []
     while not st.done:
         records.append(step(w, E, st))
-    return records[-1].att.argmax.copy(), st.steps_done, records
+    return st.emit.copy(), st.steps_done, records
 
 
 def generate(w, E: np.ndarray):

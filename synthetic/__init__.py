@@ -67,6 +67,7 @@ class Workload:
     stop_rule: int = 0      # 0: canvas unchanged, 1: argmax unchanged
     accept_rule: int = 0    # 0: cumulative sum, 1: cumulative sum minus max
     token_rule: int = 0     # 0: argmax, 1: multinomial draw (Gumbel-max)
+    canvases: int = 1       # independent canvases of C / canvases positions per step
     fixed_steps: int = 0    # 1: run exactly max_steps (timing mode)
     seed: int = 0
     blocks: int = 1

@@ -146,3 +146,29 @@ def test_multinomial_step_taking_the_argmax_is_caught(monkeypatch):
         return a
     monkeypatch.setattr(M, "vocab_attention", bad)
     assert _fails(T_gum.test_step_accepts_the_draw_and_keeps_the_distribution)
+
+
+# --- batched canvases ----------------------------------------------------------
+import test_oracle_batched as T_bat
+
+
+def test_sort_across_canvases_is_caught(monkeypatch):
+    def bad(H32, tau, rule, B, frozen=None):
+        a = M.entropy_bounded_accept(H32, tau, rule)
+        return a.accepted, a.order, a.prefix, np.array([a.k] + [0] * (B - 1))
+    monkeypatch.setattr(M, "accept_canvases", bad)
+    assert _fails(T_bat.test_two_canvas_example)
+
+
+def test_budget_shared_between_canvases_is_caught(monkeypatch):
+    real = M.accept_canvases
+    monkeypatch.setattr(M, "accept_canvases",
+                        lambda H32, tau, rule, B, frozen=None: real(H32, tau / B, rule, B, frozen))
+    assert _fails(T_bat.test_two_canvas_example)
+
+
+def test_stopped_canvas_not_frozen_is_caught(monkeypatch):
+    real = M.accept_canvases
+    monkeypatch.setattr(M, "accept_canvases",
+                        lambda H32, tau, rule, B, frozen=None: real(H32, tau, rule, B, None))
+    assert _fails(T_bat.test_block_invariants_and_freezing)
