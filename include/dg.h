@@ -94,6 +94,8 @@ typedef struct dg_config {
   int32_t  fixed_steps;     /* 1: ignore adaptive stop, run exactly S steps    */
   int32_t  impl;            /* DG_IMPL_*                                       */
   int32_t  token_rule;      /* DG_TOKEN_*                                      */
+  int32_t  canvases;        /* independent canvases per step, 0 or 1 = one;    */
+                            /* C % canvases == 0, at most 64 ([VG] 5.2)        */
   uint64_t seed;            /* keys every draw: key(seed, block, step, index)  */
 } dg_config;
 
@@ -113,6 +115,10 @@ typedef struct dg_ctx dg_ctx;
 #define DG_MREF     10   /* float [C]   tensor-core path: per-row logit reference */
 #define DG_SAMPLED  11   /* int32 [C]   multinomial draw of the last step       */
                          /*             (DG_TOKEN_MULTINOMIAL only; read-only) */
+#define DG_EMIT     12   /* int32 [C]   each canvas's prediction at its own     */
+                         /*             stop (read-only)                       */
+#define DG_CANVAS_STATE 13 /* int32 [3*canvases]: unchanged steps, stopped   */
+                           /* (0/1), steps run, per canvas (read-only)       */
 
 /* Indices into the DG_STATE array. */
 #define DG_ST_T          0  /* next step index within the block               */

@@ -109,8 +109,14 @@ STRESS_TIES = SMALL.replace(name="stress_ties_c256_v32768_d1024_bf16",
 # L2): small enough for a multi-pass profiler capture of one step.
 PROFILE = HEADLINE.replace(name="profile_c256_v65536_d2048_bf16", V=65536)
 
+# Batched canvases: two independent 128-token canvases per step at the headline
+# vocabulary and width, and one 128-token canvas alone for comparison.
+BATCHED = HEADLINE.replace(name="batched2x128_v262144_d2048_bf16", canvases=2,
+                           tau=_tau(128, 0.5))
+SINGLE128 = HEADLINE.replace(name="canvas_c128_v262144_d2048_bf16", C=128, tau=_tau(128, 0.5))
+
 WORKLOADS = {w.name: w for w in (TINY, SMALL, HEADLINE, LATENCY, BLOCKS,
-                                 STRESS_PARTIAL, STRESS_TIES, PROFILE)}
+                                 STRESS_PARTIAL, STRESS_TIES, PROFILE, BATCHED, SINGLE128)}
 
 
 def _chunk(args):

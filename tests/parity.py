@@ -90,23 +90,31 @@ def compare_draw(tally: Tally, att, sampled_gpu):
     tally.tie_mismatch += len(mism)
 
 
-def check_sampler_exact(w, block, t, H_gpu, argmax_gpu, canvas_in, out, chosen_gpu=None):
+def check_sampler_exact(w, block, t, H_gpu, argmax_gpu, canvas_in, out, chosen_gpu=None,
+                        frozen=None):
     """The sampler given the GPU's own entropies and tokens must agree bit for bit.
 
     chosen_gpu: the tokens accepted positions take (the GPU's draws under the
-    multinomial rule); the argmax when None.
+    multinomial rule); the argmax when None. frozen: per canvas, stopped
+    before this step (batched canvases).
     """
     H32 = np.asarray(H_gpu, np.float32)
-    acc = M.entropy_bounded_accept(H32, w.tau, w.accept_rule)
+    B = M.canvases(w)
+    accepted, order, prefix, k = M.accept_canvases(H32, w.tau, w.accept_rule, B, frozen)
     noise = rng.tokens(w.seed, block, t, np.arange(w.C, dtype=np.uint64), w.V)
     tok = np.asarray(argmax_gpu if chosen_gpu is None else chosen_gpu)
-    want_canvas = np.where(acc.accepted, tok, noise)
-    assert np.array_equal(out["order"], acc.order), "sort order differs"
-    assert np.array_equal(out["prefix"], acc.prefix), "prefix sums differ"
-    assert np.array_equal(out["accept"].astype(bool), acc.accepted), "accept mask differs"
+    want_canvas = np.where(accepted, tok, noise)
+    if frozen is not None:
+        Cc = w.C // B
+        for c in range(B):
+            if frozen[c]:
+                want_canvas[c * Cc:(c + 1) * Cc] = canvas_in[c * Cc:(c + 1) * Cc]
+    assert np.array_equal(out["order"], order), "sort order differs"
+    assert np.array_equal(out["prefix"], prefix), "prefix sums differ"
+    assert np.array_equal(out["accept"].astype(bool), accepted), "accept mask differs"
     assert np.array_equal(out["canvas"], want_canvas), "canvas update differs"
-    assert out["state"]["k"] == acc.k
-    return acc
+    assert out["state"]["k"] == int(k.sum())
+    return accepted
 
 
 def h_agreement(w, h_gpu, h_orc) -> float:

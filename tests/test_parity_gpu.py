@@ -63,6 +63,9 @@ def step_and_compare(den, w, E32, tally: Tally, prev_amax=None):
     st0 = den.state()
     if st0["done"]:
         return False
+    B = M.canvases(w)
+    cst0 = _np(den.read(dg.DG_CANVAS_STATE)).astype(np.int64).reshape(3, B)
+    frozen = cst0[1] != 0
     canvas_in = _np(den.read(dg.DG_CANVAS)).astype(np.int64)
     sc_in = _np(den.read(dg.DG_SC)).astype(np.float64)
     target = _np(den.read(dg.DG_TARGET)).astype(np.int64)
@@ -86,27 +89,47 @@ def step_and_compare(den, w, E32, tally: Tally, prev_amax=None):
         att = M.vocab_attention(h, E32, w.logit_scale / T, gumbel_key=(w.seed, b, t))
     else:
         att = M.vocab_attention(h, E32, w.logit_scale / T)
-    acc_orc = M.entropy_bounded_accept(att.H.astype(np.float32), w.tau, w.accept_rule)
-    flags = near_tie_flags(att, acc_orc, w.tau, w.accept_rule)
+    Cc = w.C // B
+    flags = att.margin < 1e-3          # argmax near-ties (frozen canvases included)
+    acc_orc = np.zeros(w.C, dtype=bool)
+    for c in range(B):
+        seg = slice(c * Cc, (c + 1) * Cc)
+        if frozen[c]:
+            continue
+        a_c = M.entropy_bounded_accept(att.H[seg].astype(np.float32), w.tau, w.accept_rule)
+        acc_orc[seg] = a_c.accepted
+        sub = M.Attention(argmax=att.argmax[seg], H=att.H[seg], sc=att.sc[seg],
+                          zmax=att.zmax[seg], margin=att.margin[seg])
+        flags[seg] |= near_tie_flags(sub, a_c, w.tau, w.accept_rule)
     compare_attention(tally, att, H, amax, sc, flags)
     if multinomial:
         compare_draw(tally, att, sampled)
         tally.draws_off_mode += int(np.sum(sampled != amax))
-    check_sampler_exact(w, b, t, H, amax, canvas_in, out, chosen_gpu=sampled)
-    mism = np.flatnonzero(acc_orc.accepted != out["accept"].astype(bool))
+    check_sampler_exact(w, b, t, H, amax, canvas_in, out, chosen_gpu=sampled, frozen=frozen)
+    mism = np.flatnonzero(acc_orc != out["accept"].astype(bool))
     bad = [int(i) for i in mism if not flags[i]]
     assert not bad, f"accept mismatch off a near-tie at {bad[:8]}"
     tally.tie_mismatch += len(mism)
     tally.positions += w.C
     tally.steps += 1
-    # adaptive stop from the same outputs
-    same = np.array_equal(out["canvas"], canvas_in) if w.stop_rule == 0 else \
-        (st0["has_prev"] == 1 and np.array_equal(amax, prev_amax))
-    unchanged = st0["unchanged"] + 1 if same else 0
-    conf = bool(np.all(H.astype(np.float32) < np.float32(w.stop_entropy)))
+    # adaptive stop of each running canvas from the same outputs
+    cst1 = _np(den.read(dg.DG_CANVAS_STATE)).astype(np.int64).reshape(3, B)
     last = t + 1 >= w.max_steps
-    done = last if w.fixed_steps else (last or conf or unchanged >= w.stop_unchanged)
-    assert st1["unchanged"] == unchanged and st1["done"] == int(done) and st1["t"] == t + 1
+    for c in range(B):
+        seg = slice(c * Cc, (c + 1) * Cc)
+        if frozen[c]:
+            assert np.array_equal(cst1[:, c], cst0[:, c])
+            continue
+        same = np.array_equal(out["canvas"][seg], canvas_in[seg]) if w.stop_rule == 0 else \
+            (st0["has_prev"] == 1 and np.array_equal(amax[seg], prev_amax[seg]))
+        unchanged = cst0[0, c] + 1 if same else 0
+        conf = bool(np.all(H[seg].astype(np.float32) < np.float32(w.stop_entropy)))
+        stop = last if w.fixed_steps else (last or conf or unchanged >= w.stop_unchanged)
+        assert cst1[0, c] == unchanged and cst1[1, c] == int(stop)
+        if stop:
+            assert cst1[2, c] == t + 1
+    assert st1["unchanged"] == cst1[0, 0] and st1["t"] == t + 1
+    assert st1["done"] == int(bool(np.all(cst1[1] != 0)))
     return True
 
 
@@ -185,6 +208,41 @@ def test_tiny_teacher_forced(impl, variant):
     assert tally.steps >= 1
     if variant == "multinomial":
         assert tally.draws_off_mode > 0      # a soft distribution does not always give its mode
+    den.close()
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("canvases", [2, 4])
+def test_batched_canvases_teacher_forced(impl, canvases):
+    """Canvases sharing a step: per-canvas sort, acceptance, re-noise and stop."""
+    if impl == dg.DG_IMPL_TC:
+        base = synthetic.STRESS_PARTIAL.replace(C=256, max_steps=6)
+    else:
+        base = synthetic.TINY.replace(coef_target=0.5, coef_canvas=0.5, logit_scale=1.5)
+    Cc = base.C // canvases
+    w = base.replace(canvases=canvases, tau=0.5 * Cc * np.log(2))
+    den, E32 = make(w, impl)
+    tally = run_teacher_forced(den, w, E32)
+    assert tally.steps >= 1
+    den.close()
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_batched_canvases_block(impl):
+    """Whole blocks of batched canvases through the graph loop: each canvas's
+    prediction at its own stop, and the block's step count, match the oracle."""
+    if impl == dg.DG_IMPL_TC:
+        w = synthetic.SMALL.replace(canvases=2, tau=0.5 * 128 * np.log(2), max_steps=24)
+    else:
+        w = synthetic.TINY.replace(canvases=4, tau=0.5 * 4 * np.log(2))
+    den, E32 = make(w, impl)
+    for b in range(2):
+        out, steps = den.block(b)
+        want, want_steps, _ = M.denoise_block(w, E32, b)
+        assert steps == want_steps
+        assert np.array_equal(_np(out), want)
+        cst = _np(den.read(dg.DG_CANVAS_STATE)).reshape(3, w.canvases)
+        assert np.all(cst[1] == 1)
     den.close()
 
 

@@ -25,7 +25,7 @@ DG_ACCEPT_CUMSUM, DG_ACCEPT_MINUS_MAX = 0, 1
 DG_IMPL_AUTO, DG_IMPL_SIMT, DG_IMPL_TC = 0, 1, 2
 DG_TOKEN_ARGMAX, DG_TOKEN_MULTINOMIAL = 0, 1
 (DG_CANVAS, DG_ARGMAX, DG_ENTROPY, DG_ACCEPT, DG_SC, DG_HIDDEN, DG_TARGET, DG_ORDER, DG_PREFIX,
- DG_STATE, DG_MREF, DG_SAMPLED) = range(12)
+ DG_STATE, DG_MREF, DG_SAMPLED, DG_EMIT, DG_CANVAS_STATE) = range(14)
 DG_ST_T, DG_ST_BLOCK, DG_ST_UNCHANGED, DG_ST_DONE, DG_ST_STEPS, DG_ST_K, DG_ST_STATUS, \
     DG_ST_HASPREV, DG_ST_REDO = range(9)
 
@@ -40,6 +40,7 @@ class dg_config(ctypes.Structure):
         ("stop_entropy", ctypes.c_float), ("stop_unchanged", ctypes.c_int32),
         ("stop_rule", ctypes.c_int32), ("accept_rule", ctypes.c_int32),
         ("fixed_steps", ctypes.c_int32), ("impl", ctypes.c_int32), ("token_rule", ctypes.c_int32),
+        ("canvases", ctypes.c_int32),
         ("seed", ctypes.c_uint64),
     ]
 
@@ -105,7 +106,8 @@ def make_config(w, impl: int = DG_IMPL_AUTO) -> dg_config:
                      stop_entropy=w.stop_entropy, stop_unchanged=w.stop_unchanged,
                      stop_rule=w.stop_rule, accept_rule=w.accept_rule,
                      fixed_steps=w.fixed_steps, impl=impl,
-                     token_rule=getattr(w, "token_rule", 0), seed=w.seed)
+                     token_rule=getattr(w, "token_rule", 0),
+                     canvases=getattr(w, "canvases", 1), seed=w.seed)
 
 
 # ----------------------------------------------------------------------------
@@ -229,7 +231,9 @@ class Denoiser:
                 DG_SC: ((C, d), torch.float32), DG_HIDDEN: ((C, d), self._dtype),
                 DG_TARGET: ((C,), torch.int32), DG_ORDER: ((C,), torch.int32),
                 DG_PREFIX: ((C,), torch.float32), DG_STATE: ((16,), torch.int32),
-                DG_MREF: ((C,), torch.float32), DG_SAMPLED: ((C,), torch.int32)}[what]
+                DG_MREF: ((C,), torch.float32), DG_SAMPLED: ((C,), torch.int32),
+                DG_EMIT: ((C,), torch.int32),
+                DG_CANVAS_STATE: ((3 * getattr(self.w, "canvases", 1),), torch.int32)}[what]
 
     def read(self, what):
         import torch

@@ -35,7 +35,8 @@ struct Layout {
   size_t state = 0, scale = 0, target = 0, canvas = 0, argmax = 0, argmax_prev = 0, accept = 0,
          order = 0, prefix = 0, H = 0, mref = 0, rowstat = 0, redo_rows = 0, h = 0, sc = 0,
          tstats = 0, zbuf = 0, partial = 0, O = 0, tc = 0, sampled = 0, tsamp = 0, h_last = 0,
-         mref_last = 0, total = 0;
+         mref_last = 0, cstate = 0, emit = 0, total = 0;
+  int canvases = 1;
   size_t tc_bytes = 0;
 };
 
@@ -65,6 +66,11 @@ int check_config(const dg_config* c, char* why, size_t n) {
   if (c->accept_rule != DG_ACCEPT_CUMSUM && c->accept_rule != DG_ACCEPT_MINUS_MAX) { snprintf(why, n, "bad accept_rule"); return DG_EINVAL; }
   if (c->impl < DG_IMPL_AUTO || c->impl > DG_IMPL_TC) { snprintf(why, n, "bad impl"); return DG_EINVAL; }
   if (c->token_rule != DG_TOKEN_ARGMAX && c->token_rule != DG_TOKEN_MULTINOMIAL) { snprintf(why, n, "bad token_rule"); return DG_EINVAL; }
+  const int B = c->canvases == 0 ? 1 : c->canvases;
+  if (B < 1 || B > kMaxCanvases || c->C % B) {
+    snprintf(why, n, "canvases=%d must divide C=%d and be at most %d", c->canvases, c->C, kMaxCanvases);
+    return DG_EINVAL;
+  }
   return DG_OK;
 }
 
@@ -107,6 +113,9 @@ int make_layout(const dg_config* c, Layout* L, char* why, size_t n) {
   L->h = take(esz * C * d);
   L->sc = take(4 * C * d);
   L->sampled = take(4 * C);
+  L->canvases = c->canvases == 0 ? 1 : c->canvases;
+  L->cstate = take(4 * 3 * (size_t)L->canvases);
+  L->emit = take(4 * C);
   if (impl == DG_IMPL_SIMT) {
     L->ntiles = (int)(V / 64);
     const size_t rt = (C + 63) / 64, dt = (d + 63) / 64;
@@ -223,7 +232,8 @@ int launch_step(dg_ctx* ctx, bool standin, bool use_cond) {
   const SamplerArgs sa = make_sampler_args(
       ctx->st, ctx->H, ctx->argmax, ctx->canvas, ctx->argmax_prev, ctx->accept, ctx->order,
       ctx->prefix, c.C, c.V, c.seed, c.tau, c.stop_entropy, c.stop_unchanged, c.stop_rule,
-      c.accept_rule, c.fixed_steps, c.max_steps, ctx->cond, use_cond ? 1 : 0, ctx->draw.sampled);
+      c.accept_rule, c.fixed_steps, c.max_steps, ctx->cond, use_cond ? 1 : 0, ctx->draw.sampled,
+      ctx->L.canvases, at<int32_t>(ctx, ctx->L.cstate), at<int32_t>(ctx, ctx->L.emit));
   if (tc) {
     DG_CK(launch_tc_attention(s, ctx->tc_plan, ctx->st, ctx->h, ctx->E, ctx->mref, ctx->scale_tab,
                               c.max_steps, ctx->tstats, ctx->O, ctx->tc, ctx->draw, ctx->H,
@@ -398,7 +408,7 @@ int dg_begin_block(dg_ctx* ctx, int32_t block) {
   if (block < 0) return fail(ctx, DG_EINVAL, "block must be >= 0");
   const dg_config& c = ctx->cfg;
   DG_CK(launch_begin_block(ctx->stream, ctx->st, ctx->target, ctx->canvas, ctx->sc, c.C, c.d, c.V,
-                           c.seed, block));
+                           c.seed, block, at<int32_t>(ctx, ctx->L.cstate), 3 * ctx->L.canvases));
   ctx->launches += 1;
   ctx->h_ready = false;
   return DG_OK;
@@ -447,7 +457,8 @@ int dg_denoise_block(dg_ctx* ctx, int32_t block, int32_t* out_dev, int32_t* step
   if (rc) return rc;
   if (!ctx->graph_ready && (rc = build_graph(ctx))) return rc;
   DG_CK(cudaGraphLaunch(ctx->graph_exec, ctx->stream));
-  DG_CK(cudaMemcpyAsync(out_dev, ctx->argmax, sizeof(int32_t) * ctx->cfg.C,
+  // each canvas's argmax at its own stop (one canvas: the final step's argmax)
+  DG_CK(cudaMemcpyAsync(out_dev, at<int32_t>(ctx, ctx->L.emit), sizeof(int32_t) * ctx->cfg.C,
                         cudaMemcpyDeviceToDevice, ctx->stream));
   if (steps_host) {
     DevState hs;
@@ -486,6 +497,11 @@ int dg_read(dg_ctx* ctx, int32_t what, void* dst) {
       bytes = 4 * C;
       break;
     case DG_SAMPLED: src = at<int32_t>(ctx, ctx->L.sampled); bytes = 4 * C; break;
+    case DG_EMIT: src = at<int32_t>(ctx, ctx->L.emit); bytes = 4 * C; break;
+    case DG_CANVAS_STATE:
+      src = at<int32_t>(ctx, ctx->L.cstate);
+      bytes = 4 * 3 * (size_t)ctx->L.canvases;
+      break;
     default: return fail(ctx, DG_EINVAL, "unknown item %d", what);
   }
   DG_CK(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, ctx->stream));

@@ -26,7 +26,8 @@ namespace dg {
 // Canvas initialisation.
 // ---------------------------------------------------------------------------
 __global__ void k_begin_block(DevState* st, int32_t* target, int32_t* canvas, float* sc,
-                              int C, int d, int V, uint64_t seed, int block) {
+                              int C, int d, int V, uint64_t seed, int block, int32_t* cstate,
+                              int ncstate) {
   const uint64_t sb = seed + (uint64_t)(uint32_t)block;
   const uint64_t pt = key_prefix(sb, 0, kTagTarget);
   const uint64_t pc = key_prefix(sb, 0, kTagInitCanvas);
@@ -51,6 +52,9 @@ __global__ void k_begin_block(DevState* st, int32_t* target, int32_t* canvas, fl
     st->redo = 0;
     st->h_ready = 0;
   }
+  // per-canvas stop state (unchanged, done, steps)
+  if (blockIdx.x == 0)
+    for (int j = threadIdx.x; j < ncstate; j += blockDim.x) cstate[j] = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -386,12 +390,14 @@ __global__ void __launch_bounds__(1024) k_sampler(SamplerArgs a) {
 // Host launchers.
 // ---------------------------------------------------------------------------
 cudaError_t launch_begin_block(cudaStream_t s, DevState* st, int32_t* target, int32_t* canvas,
-                               float* sc, int C, int d, int V, uint64_t seed, int block) {
+                               float* sc, int C, int d, int V, uint64_t seed, int block,
+                               int32_t* cstate, int ncstate) {
   const size_t n = (size_t)C * d;
   int grid = (int)((n + 255) / 256);
   if (grid > 4096) grid = 4096;
   if (grid < 1) grid = 1;
-  k_begin_block<<<grid, 256, 0, s>>>(st, target, canvas, sc, C, d, V, seed, block);
+  k_begin_block<<<grid, 256, 0, s>>>(st, target, canvas, sc, C, d, V, seed, block, cstate,
+                                     ncstate);
   return cudaGetLastError();
 }
 

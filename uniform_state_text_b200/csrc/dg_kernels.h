@@ -20,12 +20,21 @@ struct SamplerArgs {
   cudaGraphConditionalHandle cond;
   int use_cond;
   const int32_t* sampled;   // [C] multinomial draws to accept; nullptr: accept the argmax
+  // Batched canvases: canvases of C / canvases positions each, with their own
+  // stop state ([canvases] each) and emitted predictions ([C]).
+  int canvases;
+  int32_t *cunchanged, *cdone, *csteps, *emit;
 };
+constexpr int kMaxCanvases = 64;
 struct SamplerSmem {
-  unsigned long long key[1024];   // (entropy bits, position); padded with ~0
-  float sorted[1024];             // entropies in rank order
+  __align__(16) unsigned long long key[1024];   // (entropy bits, position)
+  float sorted[1024];             // entropies in rank order within each canvas
   float prefix[1024];             // their running sums
-  int32_t order[1024];            // positions in rank order
+  int32_t order[1024];            // positions in rank order within each canvas
+  int ck[kMaxCanvases];           // accepted per canvas
+  int cconf[kMaxCanvases];        // every entropy below the stop threshold
+  int csame[kMaxCanvases];        // canvas (or argmax) unchanged
+  int cstop[kMaxCanvases];        // the canvas stops at this step
 };
 inline SamplerArgs make_sampler_args(DevState* st, const float* H, const int32_t* argmax,
                                      int32_t* canvas, int32_t* argmax_prev, int32_t* accept,
@@ -33,13 +42,19 @@ inline SamplerArgs make_sampler_args(DevState* st, const float* H, const int32_t
                                      float tau, float stop_entropy, int stop_unchanged,
                                      int stop_rule, int accept_rule, int fixed_steps, int S,
                                      cudaGraphConditionalHandle cond, int use_cond,
-                                     const int32_t* sampled = nullptr) {
+                                     const int32_t* sampled, int canvases, int32_t* cstate,
+                                     int32_t* emit) {
   SamplerArgs a;
   a.st = st; a.H = H; a.argmax = argmax; a.canvas = canvas; a.argmax_prev = argmax_prev;
   a.accept = accept; a.order = order; a.prefix = prefix; a.C = C; a.V = V; a.seed = seed;
   a.tau = tau; a.stop_entropy = stop_entropy; a.stop_unchanged = stop_unchanged;
   a.stop_rule = stop_rule; a.accept_rule = accept_rule; a.fixed_steps = fixed_steps; a.S = S;
   a.cond = cond; a.use_cond = use_cond; a.sampled = sampled;
+  a.canvases = canvases;
+  a.cunchanged = cstate;
+  a.cdone = cstate + canvases;
+  a.csteps = cstate + 2 * canvases;
+  a.emit = emit;
   return a;
 }
 
@@ -64,7 +79,8 @@ struct DrawArgs {
 };
 
 cudaError_t launch_begin_block(cudaStream_t s, DevState* st, int32_t* target, int32_t* canvas,
-                               float* sc, int C, int d, int V, uint64_t seed, int block);
+                               float* sc, int C, int d, int V, uint64_t seed, int block,
+                               int32_t* cstate, int ncstate);
 
 cudaError_t launch_prologue(cudaStream_t s, int dtype, const DevState* st, const void* E,
                             const int32_t* target, const int32_t* canvas, const float* sc,

@@ -31,96 +31,139 @@ __device__ __forceinline__ bool sampler_bar_and(int n, bool pred) {
 // ---------------------------------------------------------------------------
 // Entropy-bounded sampler and adaptive stop, run by threads [0, nthreads) of
 // one CTA (nthreads >= C, a multiple of 32; they synchronise on barrier 1):
-// the body of k_sampler, also run by the last CTA of the tensor-core merge.
-// The caller has checked that the block is not done.
+// the body of k_sampler, also run by the tensor-core path. With batched
+// canvases each canvas of C / canvases positions is sorted, accepted,
+// re-noised and stopped on its own; a stopped canvas is frozen and the block
+// is done when every canvas is. The caller has checked that the block is not
+// done.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void sample_and_stop(const SamplerArgs& a, SamplerSmem& sm,
                                                 int nthreads) {
   DevState* st = a.st;
   const int C = a.C, V = a.V, accept_rule = a.accept_rule, stop_rule = a.stop_rule;
   const float tau = a.tau;
+  const int B = a.canvases, Cc = C / B;   // canvases and positions per canvas
   const int i = threadIdx.x;
   const bool valid = i < C;
-  // Every global input is read up front (one round trip): the loop state and
-  // this position's entropy, argmax, canvas token, previous argmax and draw.
+  const int c = valid ? i / Cc : 0;        // this position's canvas
+  const int seg0 = c * Cc;
+  // Every global input is read up front (one round trip): the loop state, the
+  // canvas's stop flag and this position's entropy, argmax, canvas token,
+  // previous argmax and draw.
   const int t = st->t;
   const int blk = st->block;
   const int has_prev = st->has_prev;
-  const int unchanged_before = st->unchanged;
   float Hi = 0.f;
   int32_t am = 0, old = 0, am_prev = 0, chosen = 0;
+  bool frozen = false;                     // the canvas stopped at an earlier step
   if (valid) {
     Hi = a.H[i];
     am = a.argmax[i];
     old = a.canvas[i];
     am_prev = a.argmax_prev[i];
     chosen = a.sampled ? a.sampled[i] : am;   // the token an accepted position takes
+    frozen = a.cdone[c] != 0;
   }
-  // Stable rank by (entropy, position) as one 64-bit key: entropies are >= 0,
-  // so their bit patterns order like their values (-0 is taken as +0).
+  if (i < B) { sm.ck[i] = 0; sm.cconf[i] = 1; sm.csame[i] = 1; }
+  // Stable rank within the canvas by (entropy, position) as one 64-bit key:
+  // entropies are >= 0, so their bit patterns order like their values (-0 is
+  // taken as +0).
   const unsigned long long key =
       ((unsigned long long)(Hi == 0.f ? 0u : __float_as_uint(Hi)) << 32) | (unsigned)i;
-  const int C2 = (C + 1) & ~1;
   if (valid) sm.key[i] = key;
-  else if (i < C2) sm.key[i] = ~0ull;    // padding never ranks below a real entry
   sampler_bar(nthreads);
   int rank = 0;
-  if (valid) {
-    const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(sm.key);
+  if (valid && !frozen) {
+    if ((Cc & 1) == 0) {
+      const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(sm.key + seg0);
 #pragma unroll 8
-    for (int j2 = 0; j2 < C2 / 2; ++j2) {
-      const ulonglong2 q = k2[j2];
-      rank += (q.x < key) + (q.y < key);
+      for (int j2 = 0; j2 < Cc / 2; ++j2) {
+        const ulonglong2 q = k2[j2];
+        rank += (q.x < key) + (q.y < key);
+      }
+    } else {
+      for (int j = 0; j < Cc; ++j) rank += sm.key[seg0 + j] < key;
     }
-    sm.order[rank] = i;
-    sm.sorted[rank] = Hi;
+    sm.order[seg0 + rank] = i;
+    sm.sorted[seg0 + rank] = Hi;
+  } else if (valid) {
+    sm.order[i] = i;                       // a frozen canvas keeps the identity order
   }
   sampler_bar(nthreads);
-  // Running entropy sums in sorted order, added one at a time in fp32 (a fixed
-  // summation order) by one thread.
-  if (i == 0) {
-    float run = 0.f;
+  // Running entropy sums of each canvas in its sorted order, added one at a
+  // time in fp32 (a fixed summation order): thread b runs canvas b.
+  if (i < B) {
+    const int s0 = i * Cc;
+    if (a.cdone[i] == 0) {
+      float run = 0.f;
 #pragma unroll 16
-    for (int j = 0; j < C; ++j) {
-      run = __fadd_rn(run, sm.sorted[j]);
-      sm.prefix[j] = run;
+      for (int j = 0; j < Cc; ++j) {
+        run = __fadd_rn(run, sm.sorted[s0 + j]);
+        sm.prefix[s0 + j] = run;
+      }
+    } else {
+      for (int j = 0; j < Cc; ++j) sm.prefix[s0 + j] = 0.f;
     }
   }
   sampler_bar(nthreads);
-  // Running sums of non-negative terms never decrease, so the accepted
-  // positions are a prefix of the sorted order: count them.
-  bool take = false;
+  // Running sums of non-negative terms never decrease, so each canvas's
+  // accepted positions are a prefix of its sorted order: count them.
   if (valid) {
     const float pj = sm.prefix[i];
     a.prefix[i] = pj;
     a.order[i] = sm.order[i];
-    const float before = i ? sm.prefix[i - 1] : 0.f;
-    take = accept_rule == 0 ? (pj <= tau) : (before <= tau);
+    if (!frozen) {
+      const float before = i > seg0 ? sm.prefix[i - 1] : 0.f;
+      const bool take = accept_rule == 0 ? (pj <= tau) : (before <= tau);
+      if (take) atomicAdd(&sm.ck[c], 1);
+    }
   }
-  const int k = sampler_bar_count(nthreads, take);
-  int32_t nw = 0;
+  sampler_bar(nthreads);
+  int32_t nw = old;
   bool acc = false;
-  if (valid) {
-    acc = rank < k;
+  if (valid && !frozen) {
+    acc = rank < sm.ck[c];
     const uint64_t pre = key_prefix(a.seed, (uint64_t)(uint32_t)blk, (uint64_t)t);
     const int32_t noise = (int32_t)(sm64(pre ^ (uint64_t)i) & (uint64_t)(V - 1));
     nw = acc ? chosen : noise;
+    if (!(Hi < a.stop_entropy)) atomicAnd(&sm.cconf[c], 0);
+    const bool same_i = stop_rule == 0 ? nw == old : am == am_prev;
+    if (!same_i) atomicAnd(&sm.csame[c], 0);
   }
-  const int all_conf = sampler_bar_and(nthreads, !valid || Hi < a.stop_entropy);
-  int same;
-  if (stop_rule == 0) same = sampler_bar_and(nthreads, !valid || nw == old);
-  else same = sampler_bar_and(nthreads, !valid || am == am_prev) && has_prev;
   if (valid) {
     a.canvas[i] = nw;
     a.accept[i] = acc ? 1 : 0;
     a.argmax_prev[i] = am;
   }
+  sampler_bar(nthreads);
+  // Adaptive stop of each running canvas (thread b for canvas b).
+  const bool last = t + 1 >= a.S;
+  if (i < B) {
+    int stop = 0;
+    if (a.cdone[i] == 0) {
+      const bool same = sm.csame[i] && (stop_rule == 0 || has_prev);
+      const int unchanged = same ? a.cunchanged[i] + 1 : 0;
+      a.cunchanged[i] = unchanged;
+      stop = a.fixed_steps ? last : (last || sm.cconf[i] || unchanged >= a.stop_unchanged);
+      if (stop) {
+        a.cdone[i] = 1;
+        a.csteps[i] = t + 1;
+      }
+    }
+    sm.cstop[i] = stop;
+  }
+  sampler_bar(nthreads);
+  // A canvas that stops now emits this step's argmax as its prediction.
+  if (valid && sm.cstop[c]) a.emit[i] = am;
   if (i == 0) {
-    const int unchanged = same ? unchanged_before + 1 : 0;
-    const bool last = t + 1 >= a.S;
-    const bool done = a.fixed_steps ? last : (last || all_conf || unchanged >= a.stop_unchanged);
-    st->unchanged = unchanged;
-    st->k = k;
+    int ndone = 0, ktot = 0;
+    for (int b = 0; b < B; ++b) {
+      ndone += a.cdone[b] != 0;
+      ktot += sm.ck[b];
+    }
+    const bool done = ndone == B;
+    st->unchanged = a.cunchanged[0];
+    st->k = ktot;
     st->t = t + 1;
     st->steps = t + 1;
     st->has_prev = 1;
