@@ -97,6 +97,9 @@ typedef struct dg_config {
   int32_t  canvases;        /* independent canvases per step, 0 or 1 = one;    */
                             /* C % canvases == 0, at most 64 ([VG] 5.2)        */
   uint64_t seed;            /* keys every draw: key(seed, block, step, index)  */
+  int32_t  shard_v0;        /* vocabulary-parallel step: this context's share  */
+  int32_t  shard_nv;        /* is entries [shard_v0, shard_v0 + shard_nv) of E */
+                            /* (both multiples of 256; shard_nv = 0: all V)    */
 } dg_config;
 
 typedef struct dg_ctx dg_ctx;
@@ -182,6 +185,33 @@ int dg_denoise_step(dg_ctx* ctx, int32_t* done_host);
  */
 int dg_denoise_step_h(dg_ctx* ctx, const void* h_src, int32_t h_on_host,
                       int32_t* canvas_host, int32_t* done_host);
+
+/*
+ * Vocabulary-parallel step (the split of the vocabulary over ranks with one
+ * exchange; no page describes it -- it shards the vocabulary attention of
+ * [VG] 5.1/5.3 by vocabulary rows). Every rank holds the whole E and the same
+ * canvas state, so the stand-in h and the logit reference m_ref are computed
+ * identically everywhere; each rank's context (cfg.shard_v0, shard_nv) covers
+ * its share of the vocabulary. Tensor-core path only (DG_EUNSUPPORTED else).
+ *   dg_partials_bytes  bytes of one partials buffer (device, caller-owned,
+ *                      8-byte aligned).
+ *   dg_denoise_step_partial  the step up to the rows' partial results over
+ *                      the shard, written to `partials`:
+ *                        float zs[C][2]  Z and S1 against m_ref   -> sum over ranks
+ *                        float O[C][d]   sum of e^(z - m_ref) E_v -> sum over ranks
+ *                        uint64 keys[C][2] order-preserving keys of (best logit,
+ *                                        index) and (best z + G, index)
+ *                                                                 -> max over ranks
+ *                      (the first 2C + C*d floats are one sum-reduction, the
+ *                      2C uint64 after them one max-reduction).
+ *   dg_denoise_step_finish  after the caller reduced the buffers over all
+ *                      ranks (e.g. NCCL all-reduce): H, argmax, draw, sc,
+ *                      sampler and stop test, identically on every rank.
+ * Asynchronous on the context's stream; errors as dg_denoise_step.
+ */
+size_t dg_partials_bytes(const dg_config* cfg);
+int dg_denoise_step_partial(dg_ctx* ctx, void* partials);
+int dg_denoise_step_finish(dg_ctx* ctx, const void* partials);
 
 /*
  * A whole block ([VG] 5.2): dg_begin_block, then denoise steps until the

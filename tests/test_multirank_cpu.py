@@ -56,3 +56,68 @@ def test_single_process_needs_no_group():
     import bench
     assert bench.max_over_ranks(3.5) == 3.5
     assert bench.whole_job_rate(10, 1, 20.0) == pytest.approx(500.0)
+
+
+# --- vocabulary-parallel exchange: one sum and one max all-reduce ------------------
+C_X, D_X = 4, 8
+
+
+def _partials(rank):
+    import torch
+
+    import uniform_state_text_b200 as dg
+    buf = torch.zeros((4 * (2 * C_X + C_X * D_X) + 16 * C_X) // 8, dtype=torch.int64)
+    f, k = dg.partials_views(buf, C_X, D_X)
+    f.copy_(torch.arange(f.numel(), dtype=torch.float32) * (rank + 1) + 0.25 * rank)
+    # unsigned keys, some with the top bit set; rank 1 wins rows 0 and 3
+    vals = [[0x8000000000000005, 7], [0x7FFFFFFF00000000, 9], [3, 0xC000000000000000], [1, 2]]
+    if rank == 1:
+        vals = [[0x8000000000000006, 6], [0x7FFFFFFE00000000, 1], [2, 0xBFFFFFFFFFFFFFFF], [5, 2]]
+    flat = [v for row in vals for v in row]
+    k.copy_(torch.tensor([v - (1 << 64) if v >= 1 << 63 else v for v in flat], dtype=torch.int64))
+    return buf
+
+
+def _exchange_rank(rank, world, port, q):
+    import datetime
+
+    import torch.distributed as dist
+
+    import uniform_state_text_b200 as dg
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        buf = _partials(rank)
+        dg.allreduce_partials(buf, C_X, D_X)
+        q.put((rank, buf.tolist()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_vocab_parallel_exchange_two_gloo_ranks():
+    import torch
+
+    import uniform_state_text_b200 as dg
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_exchange_rank, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = dict(q.get(timeout=10) for _ in range(world))
+    assert res[0] == res[1]                       # every rank holds the same result
+    got = torch.tensor(res[0], dtype=torch.int64)
+    f, k = dg.partials_views(got, C_X, D_X)
+    f0, _ = dg.partials_views(_partials(0), C_X, D_X)
+    f1, _ = dg.partials_views(_partials(1), C_X, D_X)
+    assert torch.equal(f, f0 + f1)
+    want = [0x8000000000000006, 7, 0x7FFFFFFF00000000, 9, 3, 0xC000000000000000, 5, 2]
+    assert [v % (1 << 64) for v in k.tolist()] == want
+    # the single-process helper gives the same buffers
+    a, b = _partials(0), _partials(1)
+    dg.reduce_partials_local([a, b], C_X, D_X)
+    assert torch.equal(a, got) and torch.equal(b, got)

@@ -408,3 +408,54 @@ def test_block_loop_needs_a_stream():
         den.block(0)
     assert e.value.code == dg.DG_EINVAL
     den.close()
+
+
+@pytest.mark.parametrize("token_rule", [0, 1])
+def test_vocab_parallel_shards(token_rule):
+    """Two vocabulary shards, run one after the other on this GPU and reduced
+    in-process (the exchange a multi-GPU run does with NCCL), give the step of
+    the whole vocabulary: every shard ends in the same state, matching the
+    oracle within the usual tolerances (only summation order differs)."""
+    w = synthetic.STRESS_PARTIAL.replace(max_steps=4, fixed_steps=1, token_rule=token_rule)
+    Eg, E32 = embedding(w)
+    half = w.V // 2
+    shards = [dg.Denoiser(w, Eg, impl=dg.DG_IMPL_TC, shard=(0, half)),
+              dg.Denoiser(w, Eg, impl=dg.DG_IMPL_TC, shard=(half, half))]
+    with pytest.raises(dg.DgError):
+        shards[0].step()                          # a shard alone cannot run a whole step
+    bufs = [s.partials() for s in shards]
+    tally = Tally()
+    for _ in range(w.max_steps):
+        st0 = shards[0].state()
+        canvas_in = _np(shards[0].read(dg.DG_CANVAS)).astype(np.int64)
+        for s, b in zip(shards, bufs):
+            s.step_partial(b)
+            s.stream.synchronize()
+        dg.reduce_partials_local(bufs, w.C, w.d)
+        torch.cuda.synchronize()
+        for s, b in zip(shards, bufs):
+            s.step_finish(b)
+            s.stream.synchronize()
+        outs = []
+        for s in shards:
+            outs.append({k: _np(s.read(k)) for k in (dg.DG_HIDDEN, dg.DG_ENTROPY, dg.DG_ARGMAX,
+                                                     dg.DG_SC, dg.DG_CANVAS, dg.DG_ACCEPT)})
+            assert s.state()["status"] == 0
+        for k in outs[0]:
+            assert np.array_equal(outs[0][k], outs[1][k]), k
+        t, b = st0["t"], st0["block"]
+        h = outs[0][dg.DG_HIDDEN].astype(np.float64)
+        T = M.temperature(t, w.max_steps, w.T_start, w.T_end)
+        att = M.vocab_attention(h, E32, w.logit_scale / T,
+                                gumbel_key=(w.seed, b, t) if token_rule else None)
+        acc = M.entropy_bounded_accept(att.H.astype(np.float32), w.tau, w.accept_rule)
+        flags = near_tie_flags(att, acc, w.tau, w.accept_rule)
+        compare_attention(tally, att, outs[0][dg.DG_ENTROPY], outs[0][dg.DG_ARGMAX].astype(np.int64),
+                          outs[0][dg.DG_SC].astype(np.float64), flags)
+        if token_rule:
+            compare_draw(tally, att, _np(shards[0].read(dg.DG_SAMPLED)).astype(np.int64))
+        tally.positions += w.C
+    tally.check_budget()
+    assert shards[0].state()["done"] == 1
+    for s in shards:
+        s.close()

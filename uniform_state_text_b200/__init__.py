@@ -42,6 +42,7 @@ class dg_config(ctypes.Structure):
         ("fixed_steps", ctypes.c_int32), ("impl", ctypes.c_int32), ("token_rule", ctypes.c_int32),
         ("canvases", ctypes.c_int32),
         ("seed", ctypes.c_uint64),
+        ("shard_v0", ctypes.c_int32), ("shard_nv", ctypes.c_int32),
     ]
 
 
@@ -80,12 +81,17 @@ def lib():
                                   ctypes.POINTER(ctypes.c_int64)]
     L.dg_impl.argtypes = [_P]
     L.dg_vocab_attention_static.argtypes = [_I, _I, _I, _I, ctypes.c_float, _P, _P, _P, _P, _P, _P]
+    L.dg_partials_bytes.argtypes = [cfgp]
+    L.dg_partials_bytes.restype = ctypes.c_size_t
+    L.dg_denoise_step_partial.argtypes = [_P, _P]
+    L.dg_denoise_step_finish.argtypes = [_P, _P]
     L.dg_free.argtypes = [_P]
     L.dg_last_error.argtypes = [_P]
     L.dg_last_error.restype = ctypes.c_char_p
     for name in ("dg_init", "dg_begin_block", "dg_denoise_step", "dg_denoise_step_h",
                  "dg_denoise_block", "dg_read", "dg_write", "dg_profile", "dg_profile_read",
-                 "dg_impl", "dg_free", "dg_vocab_attention_static"):
+                 "dg_impl", "dg_free", "dg_vocab_attention_static", "dg_denoise_step_partial",
+                 "dg_denoise_step_finish"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -97,8 +103,13 @@ def _check(rc: int, ctx) -> int:
     return rc
 
 
-def make_config(w, impl: int = DG_IMPL_AUTO) -> dg_config:
-    """dg_config from a synthetic.Workload-like object (same field names)."""
+def make_config(w, impl: int = DG_IMPL_AUTO, shard=None) -> dg_config:
+    """dg_config from a synthetic.Workload-like object (same field names).
+
+    shard = (v0, nv): a context for vocabulary entries [v0, v0 + nv) of a
+    vocabulary-parallel step.
+    """
+    v0, nv = shard if shard is not None else (0, 0)
     return dg_config(C=w.C, V=w.V, d=w.d, dtype=DG_BF16 if w.dtype == "bf16" else DG_F32,
                      max_steps=w.max_steps, T_start=w.T_start, T_end=w.T_end, tau=w.tau,
                      logit_scale=w.logit_scale, coef_target=w.coef_target,
@@ -107,7 +118,8 @@ def make_config(w, impl: int = DG_IMPL_AUTO) -> dg_config:
                      stop_rule=w.stop_rule, accept_rule=w.accept_rule,
                      fixed_steps=w.fixed_steps, impl=impl,
                      token_rule=getattr(w, "token_rule", 0),
-                     canvases=getattr(w, "canvases", 1), seed=w.seed)
+                     canvases=getattr(w, "canvases", 1), seed=w.seed,
+                     shard_v0=v0, shard_nv=nv)
 
 
 # ----------------------------------------------------------------------------
@@ -183,6 +195,18 @@ def dg_vocab_attention_static(C: int, V: int, d: int, dtype: int, scale: float, 
                                            _P(argmax_ptr), _P(sc_ptr), _P(stream_ptr)), None)
 
 
+def dg_partials_bytes(cfg: dg_config) -> int:
+    return int(lib().dg_partials_bytes(ctypes.byref(cfg)))
+
+
+def dg_denoise_step_partial(ctx, partials_ptr: int) -> None:
+    _check(lib().dg_denoise_step_partial(ctx, _P(partials_ptr)), ctx)
+
+
+def dg_denoise_step_finish(ctx, partials_ptr: int) -> None:
+    _check(lib().dg_denoise_step_finish(ctx, _P(partials_ptr)), ctx)
+
+
 def dg_impl(ctx) -> int:
     return _check(lib().dg_impl(ctx), ctx)
 
@@ -202,11 +226,11 @@ def dg_last_error(ctx) -> str:
 class Denoiser:
     """One context with its workspace; E must be a CUDA tensor [V, d] of the workload dtype."""
 
-    def __init__(self, w, E, stream=None, impl: int = DG_IMPL_AUTO):
+    def __init__(self, w, E, stream=None, impl: int = DG_IMPL_AUTO, shard=None):
         import torch
 
         self.w = w
-        self.cfg = make_config(w, impl)
+        self.cfg = make_config(w, impl, shard)
         if not E.is_cuda or not E.is_contiguous():
             raise ValueError("E must be a contiguous CUDA tensor")
         self.E = E
@@ -279,6 +303,22 @@ class Denoiser:
         steps = dg_denoise_block(self.ctx, block, out.data_ptr())
         return out, steps
 
+    # vocabulary-parallel step --------------------------------------------------
+    def partials(self):
+        """A partials buffer for step_partial / step_finish (see dg_partials_bytes)."""
+        import torch
+
+        n = dg_partials_bytes(self.cfg)
+        if n == 0:
+            raise DgError(DG_EUNSUPPORTED, "no vocabulary-parallel step for this configuration")
+        return torch.zeros(n // 8, dtype=torch.int64, device=self.device)
+
+    def step_partial(self, buf) -> None:
+        dg_denoise_step_partial(self.ctx, buf.data_ptr())
+
+    def step_finish(self, buf) -> None:
+        dg_denoise_step_finish(self.ctx, buf.data_ptr())
+
     def close(self) -> None:
         if getattr(self, "ctx", None) is not None:
             self.stream.synchronize()
@@ -290,3 +330,45 @@ class Denoiser:
             self.close()
         except Exception:
             pass
+
+
+# ----------------------------------------------------------------------------
+# Cross-shard reduction of the partials (torch only as plumbing: views and
+# collectives on the caller's buffers).
+# ----------------------------------------------------------------------------
+def partials_views(buf, C: int, d: int):
+    """(float view summed over shards, int64 view max-reduced over shards)."""
+    import torch
+
+    nf = 2 * C + C * d
+    b = buf.view(torch.uint8)
+    fsum = b[:4 * nf].view(torch.float32)
+    keys = b[4 * nf:4 * nf + 16 * C].view(torch.int64)
+    return fsum, keys
+
+
+def allreduce_partials(buf, C: int, d: int, group=None) -> None:
+    """Reduce one rank's partials with every other rank's (torch.distributed)."""
+    import torch.distributed as dist
+
+    fsum, keys = partials_views(buf, C, d)
+    dist.all_reduce(fsum, op=dist.ReduceOp.SUM, group=group)
+    # the keys are unsigned; flipping the top bit makes signed order agree
+    keys.bitwise_xor_(-(1 << 63))
+    dist.all_reduce(keys, op=dist.ReduceOp.MAX, group=group)
+    keys.bitwise_xor_(-(1 << 63))
+
+
+def reduce_partials_local(bufs, C: int, d: int) -> None:
+    """The same reduction over buffers of one process (every buffer gets the result)."""
+    import torch
+
+    views = [partials_views(b, C, d) for b in bufs]
+    fs = views[0][0].clone()
+    for f, _ in views[1:]:
+        fs += f
+    ks = torch.stack([k.bitwise_xor(-(1 << 63)) for _, k in views]).amax(dim=0)
+    ks.bitwise_xor_(-(1 << 63))
+    for f, k in views:
+        f.copy_(fs)
+        k.copy_(ks)

@@ -71,11 +71,30 @@ int check_config(const dg_config* c, char* why, size_t n) {
     snprintf(why, n, "canvases=%d must divide C=%d and be at most %d", c->canvases, c->C, kMaxCanvases);
     return DG_EINVAL;
   }
+  if (c->shard_nv != 0 || c->shard_v0 != 0) {
+    if (c->shard_v0 < 0 || c->shard_nv <= 0 || c->shard_v0 % 256 || c->shard_nv % 256 ||
+        (long long)c->shard_v0 + c->shard_nv > c->V) {
+      snprintf(why, n, "vocabulary shard [%d, %d + %d) must lie in [0, V) on 256-entry bounds",
+               c->shard_v0, c->shard_v0, c->shard_nv);
+      return DG_EINVAL;
+    }
+  }
   return DG_OK;
 }
 
+bool sharded(const dg_config* c) { return c->shard_nv != 0; }
+int shard_nv(const dg_config* c) { return sharded(c) ? c->shard_nv : c->V; }
+
 int resolve_impl(const dg_config* c, char* why, size_t n) {
-  const bool tc_ok = c->dtype == DG_BF16 && tc_supported(c->C, c->V, c->d);
+  const bool tc_ok = c->dtype == DG_BF16 && tc_supported(c->C, shard_nv(c), c->d);
+  if (sharded(c)) {
+    if (!tc_ok || c->impl == DG_IMPL_SIMT) {
+      snprintf(why, n, "a vocabulary shard needs the tensor-core path (bf16, C in {128, 256}, "
+               "d %% 256 == 0)");
+      return -1;
+    }
+    return DG_IMPL_TC;
+  }
   if (c->impl == DG_IMPL_TC) {
     if (!tc_ok) {
       snprintf(why, n, "tensor-core path needs bf16, C in {128, 256}, d %% 256 == 0, V %% 256 == 0");
@@ -126,13 +145,14 @@ int make_layout(const dg_config* c, Layout* L, char* why, size_t n) {
     L->zbuf = take(4 * C * V);
     L->partial = take(4 * ns * C * d);
   } else {
-    L->ntiles = tc_stat_tiles(c->C, c->V, c->d);
+    const int nv = shard_nv(c);             // the vocabulary this context's kernels cover
+    L->ntiles = tc_stat_tiles(c->C, nv, c->d);
     L->tstats = take(sizeof(TileStat) * C * L->ntiles);
-    L->tc_bytes = tc_workspace_bytes(c->C, c->V, c->d);
+    L->tc_bytes = tc_workspace_bytes(c->C, nv, c->d);
     L->tc = take(L->tc_bytes);
     L->h_last = take(esz * C * d);
     L->mref_last = take(4 * C);
-    if (c->token_rule == DG_TOKEN_MULTINOMIAL) L->tsamp = take(tc_draw_bytes(c->C, c->V, c->d));
+    if (c->token_rule == DG_TOKEN_MULTINOMIAL) L->tsamp = take(tc_draw_bytes(c->C, nv, c->d));
   }
   L->total = off;
   return DG_OK;
@@ -198,10 +218,37 @@ int fail(dg_ctx* ctx, int code, const char* fmt, ...) {
 
 template <typename T> T* at(dg_ctx* c, size_t off) { return reinterpret_cast<T*>(c->ws + off); }
 
-int launch_step(dg_ctx* ctx, bool standin, bool use_cond) {
+SamplerArgs sampler_args(dg_ctx* ctx, bool use_cond) {
   const dg_config& c = ctx->cfg;
-  cudaStream_t s = ctx->stream;
-  const float sigma = (float)std::sqrt((double)c.noise_var_d / (double)c.d);
+  return make_sampler_args(
+      ctx->st, ctx->H, ctx->argmax, ctx->canvas, ctx->argmax_prev, ctx->accept, ctx->order,
+      ctx->prefix, c.C, c.V, c.seed, c.tau, c.stop_entropy, c.stop_unchanged, c.stop_rule,
+      c.accept_rule, c.fixed_steps, c.max_steps, ctx->cond, use_cond ? 1 : 0, ctx->draw.sampled,
+      ctx->L.canvases, at<int32_t>(ctx, ctx->L.cstate), at<int32_t>(ctx, ctx->L.emit));
+}
+
+float standin_sigma(const dg_config& c) {
+  return (float)std::sqrt((double)c.noise_var_d / (double)c.d);
+}
+
+NextStandin next_standin(dg_ctx* ctx) {
+  const dg_config& c = ctx->cfg;
+  NextStandin nx;
+  nx.target = ctx->target;
+  nx.seed = c.seed;
+  nx.A = c.coef_target;
+  nx.B = c.coef_canvas;
+  nx.sigma = standin_sigma(c);
+  tc_counters(ctx->tc_plan, &nx.zero, &nx.nzero);
+  nx.h_last = at<void>(ctx, ctx->L.h_last);
+  nx.mref_last = at<float>(ctx, ctx->L.mref_last);
+  return nx;
+}
+
+// The stand-in (or, for an external h, only m_ref) unless the last merge
+// already wrote it. Returns whether a kernel was launched, or a negative error.
+int prologue_if_needed(dg_ctx* ctx, bool standin, bool use_cond) {
+  const dg_config& c = ctx->cfg;
   const bool tc = ctx->L.impl == DG_IMPL_TC;
   unsigned* zero = nullptr;
   int nzero = 0;
@@ -209,12 +256,20 @@ int launch_step(dg_ctx* ctx, bool standin, bool use_cond) {
   // After a tensor-core step the merge kernel has already written this step's
   // stand-in h and m_ref (DevState::h_ready); a stepwise call then skips the
   // prologue launch. A captured loop keeps it: it checks h_ready on the device.
-  const bool skip_prologue = tc && standin && !use_cond && ctx->h_ready;
-  if (!skip_prologue)
-    DG_CK(launch_prologue(s, c.dtype, ctx->st, ctx->E, ctx->target, ctx->canvas, ctx->sc, ctx->h,
-                          c.C, c.V, c.d, c.seed, c.coef_target, c.coef_canvas, sigma,
-                          standin ? 1 : 0, ctx->scale_tab, c.max_steps, ctx->argmax_prev,
-                          tc ? ctx->mref : nullptr, zero, nzero));
+  if (tc && standin && !use_cond && ctx->h_ready) return 0;
+  DG_CK(launch_prologue(ctx->stream, c.dtype, ctx->st, ctx->E, ctx->target, ctx->canvas, ctx->sc,
+                        ctx->h, c.C, c.V, c.d, c.seed, c.coef_target, c.coef_canvas,
+                        standin_sigma(c), standin ? 1 : 0, ctx->scale_tab, c.max_steps,
+                        ctx->argmax_prev, tc ? ctx->mref : nullptr, zero, nzero));
+  return 1;
+}
+
+int launch_step(dg_ctx* ctx, bool standin, bool use_cond) {
+  const dg_config& c = ctx->cfg;
+  cudaStream_t s = ctx->stream;
+  const bool tc = ctx->L.impl == DG_IMPL_TC;
+  const int pro = prologue_if_needed(ctx, standin, use_cond);
+  if (pro < 0) return pro;
   cudaEvent_t e0 = nullptr, e1 = nullptr;
   if (ctx->prof && !use_cond) {
     if (ctx->ev_used + 2 > ctx->ev.size()) {
@@ -228,31 +283,18 @@ int launch_step(dg_ctx* ctx, bool standin, bool use_cond) {
     e1 = ctx->ev[ctx->ev_used++];
     DG_CK(cudaEventRecord(e0, s));
   }
-  ctx->launches += tc ? (skip_prologue ? 1 : 2) + tc_launches(ctx->tc_plan) : 6;
-  const SamplerArgs sa = make_sampler_args(
-      ctx->st, ctx->H, ctx->argmax, ctx->canvas, ctx->argmax_prev, ctx->accept, ctx->order,
-      ctx->prefix, c.C, c.V, c.seed, c.tau, c.stop_entropy, c.stop_unchanged, c.stop_rule,
-      c.accept_rule, c.fixed_steps, c.max_steps, ctx->cond, use_cond ? 1 : 0, ctx->draw.sampled,
-      ctx->L.canvases, at<int32_t>(ctx, ctx->L.cstate), at<int32_t>(ctx, ctx->L.emit));
+  ctx->launches += tc ? pro + 1 + tc_launches(ctx->tc_plan) : 6;
+  const SamplerArgs sa = sampler_args(ctx, use_cond);
   if (tc) {
     DG_CK(launch_tc_attention(s, ctx->tc_plan, ctx->st, ctx->h, ctx->E, ctx->mref, ctx->scale_tab,
                               c.max_steps, ctx->tstats, ctx->O, ctx->tc, ctx->draw, ctx->H,
                               ctx->argmax, ctx->rowstat, kRedoGap, sa));
     if (e1) DG_CK(cudaEventRecord(e1, s));
-    // merge, then (inside the same kernel) the sampler and stop test
-    NextStandin nx;
-    nx.target = ctx->target;
-    nx.seed = c.seed;
-    nx.A = c.coef_target;
-    nx.B = c.coef_canvas;
-    nx.sigma = sigma;
-    nx.zero = zero;
-    nx.nzero = nzero;
-    nx.h_last = at<void>(ctx, ctx->L.h_last);
-    nx.mref_last = at<float>(ctx, ctx->L.mref_last);
+    // sc, the next step's h (and, if a row needs the exact recomputation, the
+    // rows' merge and the sampler)
     DG_CK(launch_tc_merge(s, ctx->tc_plan, ctx->st, ctx->tstats, ctx->mref, ctx->rowstat, ctx->H,
                           ctx->argmax, ctx->sc, ctx->redo_rows, kRedoGap, ctx->h, ctx->E,
-                          ctx->scale_tab, c.max_steps, sa, ctx->draw, nx));
+                          ctx->scale_tab, c.max_steps, sa, ctx->draw, next_standin(ctx)));
     // the merge prepares the next step's h unless the block stopped, and then
     // nothing more runs until dg_begin_block
     ctx->h_ready = true;
@@ -368,8 +410,9 @@ int dg_init(const dg_config* cfg, const void* E, void* workspace, size_t ws_byte
   } else {
     ctx->O = at<float>(ctx, L.O);
     ctx->tc = at<void>(ctx, L.tc);
-    rc = tc_plan_init(&ctx->tc_plan, cfg->C, cfg->V, cfg->d, E, ctx->h, ctx->O, ctx->tstats,
-                      ctx->tc, ctx->err, sizeof(ctx->err));
+    rc = tc_plan_init(&ctx->tc_plan, cfg->C, shard_nv(cfg), cfg->d, E, ctx->h, ctx->O,
+                      ctx->tstats, ctx->tc, ctx->err, sizeof(ctx->err),
+                      sharded(cfg) ? cfg->shard_v0 : 0, cfg->V);
     if (rc) {
       snprintf(g_init_err, sizeof(g_init_err), "%s", ctx->err);
       delete ctx;
@@ -416,6 +459,8 @@ int dg_begin_block(dg_ctx* ctx, int32_t block) {
 
 int dg_denoise_step(dg_ctx* ctx, int32_t* done_host) {
   if (!ctx) return fail(nullptr, DG_EINVAL, "ctx is NULL");
+  if (sharded(&ctx->cfg))
+    return fail(ctx, DG_EUNSUPPORTED, "a vocabulary shard steps with dg_denoise_step_partial/_finish");
   int rc = launch_step(ctx, true, false);
   if (rc) return rc;
   if (done_host) {
@@ -431,6 +476,8 @@ int dg_denoise_step_h(dg_ctx* ctx, const void* h_src, int32_t h_on_host, int32_t
                       int32_t* done_host) {
   if (!ctx) return fail(nullptr, DG_EINVAL, "ctx is NULL");
   if (!h_src) return fail(ctx, DG_EINVAL, "h_src is NULL");
+  if (sharded(&ctx->cfg))
+    return fail(ctx, DG_EUNSUPPORTED, "a vocabulary shard steps with dg_denoise_step_partial/_finish");
   const dg_config& c = ctx->cfg;
   const size_t bytes = (size_t)c.C * c.d * (c.dtype == DG_F32 ? 4 : 2);
   DG_CK(cudaMemcpyAsync(ctx->h, h_src, bytes,
@@ -452,6 +499,8 @@ int dg_denoise_step_h(dg_ctx* ctx, const void* h_src, int32_t h_on_host, int32_t
 
 int dg_denoise_block(dg_ctx* ctx, int32_t block, int32_t* out_dev, int32_t* steps_host) {
   if (!ctx) return fail(nullptr, DG_EINVAL, "ctx is NULL");
+  if (sharded(&ctx->cfg))
+    return fail(ctx, DG_EUNSUPPORTED, "a vocabulary shard steps with dg_denoise_step_partial/_finish");
   if (!out_dev) return fail(ctx, DG_EINVAL, "out_dev is NULL");
   int rc = dg_begin_block(ctx, block);
   if (rc) return rc;
@@ -466,6 +515,40 @@ int dg_denoise_block(dg_ctx* ctx, int32_t block, int32_t* out_dev, int32_t* step
     if (rc) return rc;
     *steps_host = hs.steps;
   }
+  return DG_OK;
+}
+
+size_t dg_partials_bytes(const dg_config* cfg) {
+  Layout L;
+  char why[256];
+  if (make_layout(cfg, &L, why, sizeof(why)) != DG_OK || L.impl != DG_IMPL_TC) return 0;
+  return tc_partials_bytes(cfg->C, cfg->d);
+}
+
+int dg_denoise_step_partial(dg_ctx* ctx, void* partials) {
+  if (!ctx) return fail(nullptr, DG_EINVAL, "ctx is NULL");
+  if (!partials || ((uintptr_t)partials) % 16) return fail(ctx, DG_EINVAL, "partials must be a 16-byte aligned device buffer");
+  if (ctx->L.impl != DG_IMPL_TC) return fail(ctx, DG_EUNSUPPORTED, "the vocabulary-parallel step needs the tensor-core path");
+  const dg_config& c = ctx->cfg;
+  const int pro = prologue_if_needed(ctx, true, false);
+  if (pro < 0) return pro;
+  ctx->launches += pro + 2;
+  DG_CK(launch_tc_partial(ctx->stream, ctx->tc_plan, ctx->st, ctx->h, ctx->E, ctx->mref,
+                          ctx->scale_tab, c.max_steps, ctx->tstats, ctx->tc, ctx->draw, partials));
+  return DG_OK;
+}
+
+int dg_denoise_step_finish(dg_ctx* ctx, const void* partials) {
+  if (!ctx) return fail(nullptr, DG_EINVAL, "ctx is NULL");
+  if (!partials || ((uintptr_t)partials) % 16) return fail(ctx, DG_EINVAL, "partials must be a 16-byte aligned device buffer");
+  if (ctx->L.impl != DG_IMPL_TC) return fail(ctx, DG_EUNSUPPORTED, "the vocabulary-parallel step needs the tensor-core path");
+  const dg_config& c = ctx->cfg;
+  ctx->launches += 2;
+  DG_CK(launch_tc_finish(ctx->stream, ctx->tc_plan, ctx->st, partials, ctx->tstats, ctx->draw,
+                         ctx->mref, ctx->rowstat, ctx->H, ctx->argmax, ctx->sc, kRedoGap, ctx->h,
+                         ctx->E, ctx->scale_tab, c.max_steps, sampler_args(ctx, false),
+                         next_standin(ctx)));
+  ctx->h_ready = true;
   return DG_OK;
 }
 

@@ -95,7 +95,28 @@ struct Params {
   unsigned* g1_ticket;         // G1 CTAs whose rows are merged
   int* redo_flag;              // a row needs the exact recomputation
   SamplerArgs sa;
+  // Vocabulary shard: this launch covers entries [v0, v0 + n_vt * BN) of a
+  // vocabulary of V; with `partial` the G1 CTAs write partial row results
+  // (pzs, pkeys) for a cross-shard reduction instead of merging the rows.
+  int v0;
+  int partial;
+  float2* pzs;                 // [C] (Z, S1)
+  unsigned long long* pkeys;   // [C][2] max keys of (best, arg) and (best z + G, arg)
 };
+
+// Order-preserving 64-bit key of (value, index): a larger value, then a lower
+// index, gives a larger key, so a max-reduction over shards picks the argmax
+// with the lowest index on ties.
+__device__ __forceinline__ unsigned long long max_key(float v, int idx) {
+  const uint32_t u = __float_as_uint(v);
+  const uint32_t k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((unsigned long long)k << 32) | (0xFFFFFFFFu - (uint32_t)idx);
+}
+__device__ __forceinline__ void max_key_decode(unsigned long long key, float* v, int* idx) {
+  const uint32_t k = (uint32_t)(key >> 32);
+  *v = __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+  *idx = (int)(0xFFFFFFFFu - (uint32_t)key);
+}
 
 // Per-CTA wait-time tracing, compiled in only with -DDG_TC_TRACE (measurement
 // builds). Each role accumulates in registers and stores once at its end.
@@ -480,18 +501,25 @@ __device__ __noinline__ void g1_finish(const Params& p, int ng1, unsigned char* 
         if (better(wB[j], wA[j], best, arg)) { best = wB[j]; arg = wA[j]; }
         if (better(wG[j], wGA[j], gbest, garg)) { gbest = wG[j]; garg = wGA[j]; }
       }
-      const float mref_i = p.mref[i];
-      p.H[i] = fmaxf(logf(Z) - S1 / Z, 0.f);
-      p.argmax[i] = arg;
-      if constexpr (DRAW) p.sampled[i] = garg;
-      RowStat rs;
-      rs.m = mref_i; rs.Z = Z; rs.pad[0] = best; rs.pad[1] = 0.f;
-      p.rowstat[i] = rs;
-      const float gap = best - mref_i;
-      if (!(gap <= p.redo_gap) || !(Z > 0.f) || !(Z < INFINITY)) atomicOr(p.redo_flag, 1);
+      if (p.partial) {
+        p.pzs[i] = make_float2(Z, S1);
+        p.pkeys[2 * i] = max_key(best, arg);
+        p.pkeys[2 * i + 1] = DRAW ? max_key(gbest, garg) : 0ull;
+      } else {
+        const float mref_i = p.mref[i];
+        p.H[i] = fmaxf(logf(Z) - S1 / Z, 0.f);
+        p.argmax[i] = arg;
+        if constexpr (DRAW) p.sampled[i] = garg;
+        RowStat rs;
+        rs.m = mref_i; rs.Z = Z; rs.pad[0] = best; rs.pad[1] = 0.f;
+        p.rowstat[i] = rs;
+        const float gap = best - mref_i;
+        if (!(gap <= p.redo_gap) || !(Z > 0.f) || !(Z < INFINITY)) atomicOr(p.redo_flag, 1);
+      }
     }
     __syncthreads();
   }
+  if (p.partial) return;     // the rows are merged after the cross-shard reduction
   // Acquire-release ticket: this CTA's rows are visible before it counts, and
   // the last CTA sees every row and every redo flag.
   if (tid == 0) {
@@ -841,7 +869,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int j = 31; j >= 0; --j) jj = (v[j] == cm) ? j : jj;
             vbest = cm;
-            arg = vt * BN + c0 + c * 32 + jj;
+            arg = p.v0 + vt * BN + c0 + c * 32 + jj;
           }
           // Gumbel variates lie in [-2.82, 16.64], so the winning z + G is at least
           // (row max) - 2.82 >= mref - 2.82, and an entry with z < mref - 19.46
@@ -849,7 +877,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           // rounding differences between mref and these logits).
           if constexpr (DRAW) {
             if (cm * scale >= mref - 20.5f) {
-              const int col0 = vt * BN + c0 + c * 32;
+              const int col0 = p.v0 + vt * BN + c0 + c * 32;
               const uint64_t rbase = (uint64_t)row * (uint64_t)p.V + (uint64_t)col0;
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
@@ -1409,10 +1437,13 @@ int check_residency(int units, int sms, char* err, size_t errn) {
 }
 
 int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, float* O,
-                 TileStat* tstats, void* ws, char* err, size_t errn) {
+                 TileStat* tstats, void* ws, char* err, size_t errn, int v0, int Vg) {
   (void)O;
   (void)tstats;
   p->C = C; p->V = V; p->d = d;
+  p->v0 = v0; p->Vg = Vg;
+  // the kernels' E tensor maps start at the shard's first row
+  E = static_cast<const __nv_bfloat16*>(E) + (size_t)v0 * d;
   p->num_sms = device_sms();
   TcLayout L = tc_layout(C, V, d, p->num_sms);
   p->grid = L.n1 + L.n2;
@@ -1447,16 +1478,13 @@ void tc_counters(const TcPlan& p, unsigned** ptr, int* count) {
   *count = 2 * L.n_vt + 64;
 }
 
-cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, const void* h,
-                                const void* E, const float* mref, const float* scale_tab,
-                                int S, TileStat* tstats, float* O, void* ws,
-                                const DrawArgs& draw, float* H, int32_t* argmax,
-                                RowStat* rowstat, float redo_gap, const SamplerArgs& sa) {
-  (void)h; (void)E; (void)O;
-  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
+tc::Params base_params(const TcPlan& pl, const TcLayout& L, DevState* st, const float* mref,
+                       const float* scale_tab, int S, TileStat* tstats, void* ws,
+                       const DrawArgs& draw, float* H, int32_t* argmax, RowStat* rowstat,
+                       float redo_gap, const SamplerArgs& sa) {
   char* base = static_cast<char*>(ws);
   tc::Params prm;
-  prm.C = pl.C; prm.V = pl.V; prm.d = pl.d; prm.RB = L.RB; prm.n_vt = L.n_vt;
+  prm.C = pl.C; prm.V = pl.Vg; prm.d = pl.d; prm.RB = L.RB; prm.n_vt = L.n_vt;
   prm.n_ranges = L.n_ranges; prm.n_dt = L.n_dt; prm.G = L.G; prm.n1 = L.n1; prm.W2 = L.W2;
   prm.tiles_per_range = tc::KV2 / tc::BN; prm.S = S;
   prm.mref = mref; prm.scale_tab = scale_tab;
@@ -1481,6 +1509,15 @@ cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, 
   prm.g1_ticket = ctr + 2 * L.n_vt + 4;
   prm.redo_flag = reinterpret_cast<int*>(ctr + 2 * L.n_vt + 5);
   prm.sa = sa;
+  prm.v0 = pl.v0;
+  prm.partial = 0;
+  prm.pzs = nullptr;
+  prm.pkeys = nullptr;
+  return prm;
+}
+
+cudaError_t launch_params(cudaStream_t s, const TcPlan& pl, const TcLayout& L,
+                          const tc::Params& prm) {
   const CUtensorMap* maps = reinterpret_cast<const CUtensorMap*>(pl.maps);
   const int units = L.n1 + L.n2;
   if (prm.tsamp)
@@ -1490,6 +1527,87 @@ cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, 
                    : launch_kernel<1, false>(s, units, maps, prm);
 }
 
+cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, const void* h,
+                                const void* E, const float* mref, const float* scale_tab,
+                                int S, TileStat* tstats, float* O, void* ws,
+                                const DrawArgs& draw, float* H, int32_t* argmax,
+                                RowStat* rowstat, float redo_gap, const SamplerArgs& sa) {
+  (void)h; (void)E; (void)O;
+  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
+  const tc::Params prm = base_params(pl, L, st, mref, scale_tab, S, tstats, ws, draw, H, argmax,
+                                     rowstat, redo_gap, sa);
+  return launch_params(s, pl, L, prm);
+}
+
+size_t tc_partials_bytes(int C, int d) {
+  return sizeof(float) * ((size_t)2 * C + (size_t)C * d) + sizeof(unsigned long long) * 2 * (size_t)C;
+}
+
+namespace tc {
+// O[i] = sum over the range groups of the shard's partials (no normalisation).
+__global__ void k_partial_o(const DevState* st, const float* Opart, int nO, size_t n4,
+                            float* O) {
+  if (st->done) return;
+  const size_t stride = n4 * 4;
+  for (size_t x = blockIdx.x * (size_t)blockDim.x + threadIdx.x; x < n4;
+       x += (size_t)gridDim.x * blockDim.x) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int g = 0; g < nO; ++g) {
+      const float4 o = reinterpret_cast<const float4*>(Opart + g * stride)[x];
+      acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
+    }
+    reinterpret_cast<float4*>(O)[x] = acc;
+  }
+}
+
+// Per-row statistics from the reduced partials: one TcStat (and TcSamp) per
+// row, which the merge kernel then treats as a row of a single tile.
+__global__ void k_partials_to_stats(const DevState* st, int C, const float2* zs,
+                                    const unsigned long long* keys, TcStat* ts, TcSamp* tsamp) {
+  if (st->done) return;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= C) return;
+  TcStat t;
+  t.Z = zs[i].x;
+  t.S1 = zs[i].y;
+  max_key_decode(keys[2 * i], &t.best, &t.arg);
+  ts[i] = t;
+  if (tsamp) {
+    TcSamp q;
+    max_key_decode(keys[2 * i + 1], &q.score, &q.arg);
+    tsamp[i] = q;
+  }
+}
+}  // namespace tc
+
+cudaError_t launch_tc_partial(cudaStream_t s, const TcPlan& pl, DevState* st, const void* h,
+                              const void* E, const float* mref, const float* scale_tab, int S,
+                              TileStat* tstats, void* ws, const DrawArgs& draw, void* partials) {
+  (void)h; (void)E;
+  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
+  SamplerArgs none = {};
+  tc::Params prm = base_params(pl, L, st, mref, scale_tab, S, tstats, ws, draw, nullptr, nullptr,
+                               nullptr, 0.f, none);
+  float* zs = static_cast<float*>(partials);
+  float* O = zs + 2 * (size_t)pl.C;
+  prm.partial = 1;
+  prm.pzs = reinterpret_cast<float2*>(zs);
+  prm.pkeys = reinterpret_cast<unsigned long long*>(O + (size_t)pl.C * pl.d);
+  cudaError_t e = launch_params(s, pl, L, prm);
+  if (e != cudaSuccess) return e;
+  const size_t n4 = (size_t)pl.C * pl.d / 4;
+  tc::k_partial_o<<<2 * device_sms(), 256, 0, s>>>(
+      st, reinterpret_cast<const float*>(static_cast<const char*>(ws) + L.Opart), L.G, n4, O);
+  return cudaGetLastError();
+}
+
+cudaError_t merge_launch(cudaStream_t s, const TcPlan& pl, DevState* st, const TcStat* ts,
+                         int nts, const float* Opart, int nO, const TcSamp* tsamp,
+                         const float* mref, RowStat* rowstat, float* H, int32_t* argmax,
+                         float* sc, float redo_gap, const void* h, const void* E,
+                         const float* scale_tab, int S, const SamplerArgs& sa,
+                         const DrawArgs& draw, const NextStandin& nx);
+
 cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& pl, DevState* st, const TileStat* tstats,
                             const float* mref, RowStat* rowstat, float* H, int32_t* argmax,
                             float* sc, int32_t* redo_rows, float redo_gap, const void* h,
@@ -1498,6 +1616,38 @@ cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& pl, DevState* st, cons
   TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
   const float* Opart = reinterpret_cast<const float*>(static_cast<const char*>(pl.ws) + L.Opart);
   (void)redo_rows;
+  return merge_launch(s, pl, st, reinterpret_cast<const TcStat*>(tstats), 2 * L.n_vt, Opart, L.G,
+                      draw.sampled ? static_cast<const TcSamp*>(draw.tsamp) : nullptr, mref,
+                      rowstat, H, argmax, sc, redo_gap, h, E, scale_tab, S, sa, draw, nx);
+}
+
+cudaError_t launch_tc_finish(cudaStream_t s, const TcPlan& pl, DevState* st,
+                             const void* partials, TileStat* tstats, const DrawArgs& draw,
+                             const float* mref, RowStat* rowstat, float* H, int32_t* argmax,
+                             float* sc, float redo_gap, const void* h, const void* E,
+                             const float* scale_tab, int S, const SamplerArgs& sa,
+                             const NextStandin& nx) {
+  const float* zs = static_cast<const float*>(partials);
+  const float* O = zs + 2 * (size_t)pl.C;
+  const unsigned long long* keys =
+      reinterpret_cast<const unsigned long long*>(O + (size_t)pl.C * pl.d);
+  TcStat* ts = reinterpret_cast<TcStat*>(tstats);
+  TcSamp* tsamp = draw.sampled ? static_cast<TcSamp*>(draw.tsamp) : nullptr;
+  tc::k_partials_to_stats<<<(pl.C + 127) / 128, 128, 0, s>>>(
+      st, pl.C, reinterpret_cast<const float2*>(zs), keys, ts, tsamp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return merge_launch(s, pl, st, ts, 1, O, 1, tsamp, mref, rowstat, H, argmax, sc,
+                      redo_gap, h, E, scale_tab, S, sa, draw, nx);
+}
+
+cudaError_t merge_launch(cudaStream_t s, const TcPlan& pl, DevState* st, const TcStat* ts,
+                         int nts, const float* Opart, int nO, const TcSamp* tsamp,
+                         const float* mref, RowStat* rowstat, float* H, int32_t* argmax,
+                         float* sc, float redo_gap, const void* h, const void* E,
+                         const float* scale_tab, int S, const SamplerArgs& sa,
+                         const DrawArgs& draw, const NextStandin& nx) {
+  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
   // the sampler runs on one row's threads of the last CTA
   if (pl.C > tc::kMergeThreadsPerRow) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
@@ -1511,12 +1661,11 @@ cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& pl, DevState* st, cons
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(
-      &cfg, tc::k_merge_tc, st, reinterpret_cast<const TcStat*>(tstats), 2 * L.n_vt,
-      const_cast<float*>(mref), Opart, L.G, pl.C, pl.V, pl.d, rowstat, H, argmax, sc, redo_gap,
-      static_cast<__nv_bfloat16*>(const_cast<void*>(h)), static_cast<const __nv_bfloat16*>(E),
-      scale_tab, S,
+      &cfg, tc::k_merge_tc, st, ts, nts, const_cast<float*>(mref), Opart, nO, pl.C, pl.Vg, pl.d,
+      rowstat, H, argmax, sc, redo_gap, static_cast<__nv_bfloat16*>(const_cast<void*>(h)),
+      static_cast<const __nv_bfloat16*>(E), scale_tab, S,
       reinterpret_cast<unsigned*>(static_cast<char*>(pl.ws) + L.counters) + 2 * L.n_vt + 2,
-      draw.sampled ? static_cast<const TcSamp*>(draw.tsamp) : nullptr, draw.sampled, nx, sa);
+      tsamp, draw.sampled, nx, sa);
 }
 
 void tc_partials(const TcPlan& pl, const float** Opart, int* nO) {

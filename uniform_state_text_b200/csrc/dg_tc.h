@@ -10,7 +10,8 @@ namespace dg {
 
 // Plan of the tensor-core kernels for one context (tensor maps, tile counts).
 struct TcPlan {
-  int C = 0, V = 0, d = 0;
+  int C = 0, V = 0, d = 0;   // V: the vocabulary this context's kernels cover (a shard or all)
+  int v0 = 0, Vg = 0;        // first vocabulary entry of the shard; the whole vocabulary
   bool ready = false;
   alignas(64) unsigned char maps[8][128];   // CUtensorMap objects
   int num_sms = 0;
@@ -21,8 +22,9 @@ struct TcPlan {
 bool tc_supported(int C, int V, int d);
 int tc_stat_tiles(int C, int V, int d);
 size_t tc_workspace_bytes(int C, int V, int d);
+// E: the whole [Vg][d] table; the kernels cover entries [v0, v0 + V).
 int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, float* O,
-                 TileStat* tstats, void* ws, char* err, size_t errn);
+                 TileStat* tstats, void* ws, char* err, size_t errn, int v0, int Vg);
 void tc_plan_free(TcPlan* p);
 int tc_launches(const TcPlan& p);   // kernels per launch_tc_attention call
 // The attention kernel; its G1 CTAs also merge the rows' statistics into H,
@@ -45,6 +47,27 @@ cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& p, DevState* st, const
                             const DrawArgs& draw, const NextStandin& nx);
 // Bytes of the per-half-tile draw statistics (DrawArgs::tsamp) of the multinomial rule.
 size_t tc_draw_bytes(int C, int V, int d);
+
+// Vocabulary-parallel step, first half: the attention over this context's
+// vocabulary shard, ending in partial row results instead of H, sc and the
+// sampler. Layout of `partials` (device, tc_partials_bytes):
+//   float zs[C][2]   Z and S1 against the shared reference m_ref     (sum over shards)
+//   float O[C][d]    sum over the shard of e^(z - m_ref) E_v         (sum over shards)
+//   u64 keys[C][2]   (best logit, index) and (best z + G, index) as
+//                    order-preserving keys                           (max over shards)
+cudaError_t launch_tc_partial(cudaStream_t s, const TcPlan& p, DevState* st, const void* h,
+                              const void* E, const float* mref, const float* scale_tab, int S,
+                              TileStat* tstats, void* ws, const DrawArgs& draw, void* partials);
+size_t tc_partials_bytes(int C, int d);
+// Second half, after the partials were reduced over all shards: per-row
+// statistics from them, then the merge kernel (sc, exact recomputation of a
+// row if needed, sampler, stop test, next step's h) as for a whole vocabulary.
+cudaError_t launch_tc_finish(cudaStream_t s, const TcPlan& p, DevState* st,
+                             const void* partials, TileStat* tstats, const DrawArgs& draw,
+                             const float* mref, RowStat* rowstat, float* H, int32_t* argmax,
+                             float* sc, float redo_gap, const void* h, const void* E,
+                             const float* scale_tab, int S, const SamplerArgs& sa,
+                             const NextStandin& nx);
 // Hand-off counters the prologue zeroes before every step.
 void tc_counters(const TcPlan& p, unsigned** ptr, int* count);
 // Per-range-group partials of O = P E that the merge sums.
