@@ -11,8 +11,9 @@ HBM every step, so no L2 flush is needed between steps.
   value  device-timed throughput with inputs resident (CUDA events around K
          steps on the context's stream, max over ranks).
   e2e    the same metric through dg_denoise_step_h: every step copies that
-         step's hidden state from pinned host memory and reads the updated
-         canvas and loop state back to the host.
+         step's hidden state from pinned host memory and the updated canvas
+         back to pinned host memory; CUDA events on the context's stream
+         bracket all of it (one synchronisation after the last step).
   roofline  the vocabulary-attention kernels (the dominant kernel) against the
          tensor roofline: 4*C*d*V flops per step over their event-timed duration.
   cpu_baseline  the CPU oracle (fp64 numpy) on a bounded sample of rows.
@@ -296,25 +297,33 @@ def main():
         den.begin_block(0)
         n_e2e = max(8, args.steps // 2)
         for _ in range(3):
-            den.step_h(h_host, canvas_host=canvas_host, want_done=True)
+            den.step_h(h_host, canvas_host=canvas_host)
+        torch.cuda.synchronize()
         den.begin_block(0)
         if dist:
             dist.barrier()
         torch.cuda.synchronize()
-        t0 = time.perf_counter()
+        # Device-timed on the library's stream: the events bracket every copy
+        # and kernel, and any gap the host leaves between steps. Each step
+        # copies h in from pinned memory and the canvas back out (the canvas
+        # read-back is asynchronous; the stream is synchronised once, after).
+        e2e0 = torch.cuda.Event(enable_timing=True)
+        e2e1 = torch.cuda.Event(enable_timing=True)
+        e2e0.record(stream)
         done_steps = 0
         for i in range(n_e2e):
             if done_steps == S:
                 den.begin_block(0)
                 done_steps = 0
-            den.step_h(h_host, canvas_host=canvas_host, want_done=True)
+            den.step_h(h_host, canvas_host=canvas_host)
             done_steps += 1
+        e2e1.record(stream)
         torch.cuda.synchronize()
-        el = time.perf_counter() - t0
+        el = e2e0.elapsed_time(e2e1) / 1e3
         el = max_over_ranks(el, dist, "cuda")
         e2e = {"value": n_e2e * world / el, "unit": "steps/s",
                "h2d_bytes_per_step": int(h_host.numel() * h_host.element_size()),
-               "d2h_bytes_per_step": int(w.C * 4 + 64),
+               "d2h_bytes_per_step": int(w.C * 4),
                "tok_per_s": w.C * n_e2e * world / el,
                "path": "dg_denoise_step_h, hidden state from pinned host memory"}
 

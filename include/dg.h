@@ -180,8 +180,10 @@ int dg_denoise_step(dg_ctx* ctx, int32_t* done_host);
  * The same step with the hidden state supplied by the caller instead of the
  * stand-in backbone: h_src holds [C][d] of cfg->dtype, in host memory when
  * h_on_host != 0 (pinned memory keeps the copy asynchronous) or device memory
- * otherwise. canvas_host (nullable) receives the updated canvas, int32 [C];
- * done_host (nullable) the done flag. A non-NULL host output synchronises.
+ * otherwise. canvas_host (nullable, pinned) receives the updated canvas,
+ * int32 [C], asynchronously: it is valid once the stream has reached it.
+ * done_host (nullable) receives the done flag; a non-NULL done_host
+ * synchronises.
  */
 int dg_denoise_step_h(dg_ctx* ctx, const void* h_src, int32_t h_on_host,
                       int32_t* canvas_host, int32_t* done_host);

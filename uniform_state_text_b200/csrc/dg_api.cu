@@ -33,8 +33,8 @@ struct Layout {
   int ntiles = 0;      // vocabulary tiles carrying per-row statistics
   int nsplit = 0;      // CUDA-core path: vocabulary splits of sc
   size_t state = 0, scale = 0, target = 0, canvas = 0, argmax = 0, argmax_prev = 0, accept = 0,
-         order = 0, prefix = 0, H = 0, mref = 0, rowstat = 0, redo_rows = 0, h = 0, sc = 0,
-         tstats = 0, zbuf = 0, partial = 0, O = 0, tc = 0, sampled = 0, tsamp = 0, h_last = 0,
+         order = 0, prefix = 0, H = 0, mref = 0, rowstat = 0, h = 0, sc = 0,
+         tstats = 0, zbuf = 0, partial = 0, tc = 0, sampled = 0, tsamp = 0, h_last = 0,
          mref_last = 0, cstate = 0, emit = 0, total = 0;
   int canvases = 1;
   size_t tc_bytes = 0;
@@ -128,7 +128,6 @@ int make_layout(const dg_config* c, Layout* L, char* why, size_t n) {
   L->H = take(4 * C);
   L->mref = take(4 * C);
   L->rowstat = take(sizeof(RowStat) * C);
-  L->redo_rows = take(4 * C);
   L->h = take(esz * C * d);
   L->sc = take(4 * C * d);
   L->sampled = take(4 * C);
@@ -175,9 +174,9 @@ struct dg_ctx {
   DevState* st = nullptr;
   float* scale_tab = nullptr;
   int32_t *target = nullptr, *canvas = nullptr, *argmax = nullptr, *argmax_prev = nullptr,
-          *accept = nullptr, *order = nullptr, *redo_rows = nullptr;
+          *accept = nullptr, *order = nullptr;
   float *prefix = nullptr, *H = nullptr, *mref = nullptr, *sc = nullptr, *zbuf = nullptr,
-        *partial = nullptr, *O = nullptr;
+        *partial = nullptr;
   RowStat* rowstat = nullptr;
   TileStat* tstats = nullptr;
   DrawArgs draw;            // multinomial draw (sampled == nullptr under the argmax rule)
@@ -287,13 +286,13 @@ int launch_step(dg_ctx* ctx, bool standin, bool use_cond) {
   const SamplerArgs sa = sampler_args(ctx, use_cond);
   if (tc) {
     DG_CK(launch_tc_attention(s, ctx->tc_plan, ctx->st, ctx->h, ctx->E, ctx->mref, ctx->scale_tab,
-                              c.max_steps, ctx->tstats, ctx->O, ctx->tc, ctx->draw, ctx->H,
+                              c.max_steps, ctx->tstats, ctx->tc, ctx->draw, ctx->H,
                               ctx->argmax, ctx->rowstat, kRedoGap, sa));
     if (e1) DG_CK(cudaEventRecord(e1, s));
     // sc, the next step's h (and, if a row needs the exact recomputation, the
     // rows' merge and the sampler)
     DG_CK(launch_tc_merge(s, ctx->tc_plan, ctx->st, ctx->tstats, ctx->mref, ctx->rowstat, ctx->H,
-                          ctx->argmax, ctx->sc, ctx->redo_rows, kRedoGap, ctx->h, ctx->E,
+                          ctx->argmax, ctx->sc, kRedoGap, ctx->h, ctx->E,
                           ctx->scale_tab, c.max_steps, sa, ctx->draw, next_standin(ctx)));
     // the merge prepares the next step's h unless the block stopped, and then
     // nothing more runs until dg_begin_block
@@ -395,7 +394,6 @@ int dg_init(const dg_config* cfg, const void* E, void* workspace, size_t ws_byte
   ctx->H = at<float>(ctx, L.H);
   ctx->mref = at<float>(ctx, L.mref);
   ctx->rowstat = at<RowStat>(ctx, L.rowstat);
-  ctx->redo_rows = at<int32_t>(ctx, L.redo_rows);
   ctx->h = at<void>(ctx, L.h);
   ctx->sc = at<float>(ctx, L.sc);
   ctx->tstats = at<TileStat>(ctx, L.tstats);
@@ -408,10 +406,9 @@ int dg_init(const dg_config* cfg, const void* E, void* workspace, size_t ws_byte
     ctx->zbuf = at<float>(ctx, L.zbuf);
     ctx->partial = at<float>(ctx, L.partial);
   } else {
-    ctx->O = at<float>(ctx, L.O);
     ctx->tc = at<void>(ctx, L.tc);
-    rc = tc_plan_init(&ctx->tc_plan, cfg->C, shard_nv(cfg), cfg->d, E, ctx->h, ctx->O,
-                      ctx->tstats, ctx->tc, ctx->err, sizeof(ctx->err),
+    rc = tc_plan_init(&ctx->tc_plan, cfg->C, shard_nv(cfg), cfg->d, E, ctx->h, ctx->tc,
+                      ctx->err, sizeof(ctx->err),
                       sharded(cfg) ? cfg->shard_v0 : 0, cfg->V);
     if (rc) {
       snprintf(g_init_err, sizeof(g_init_err), "%s", ctx->err);
@@ -488,11 +485,11 @@ int dg_denoise_step_h(dg_ctx* ctx, const void* h_src, int32_t h_on_host, int32_t
   if (canvas_host)
     DG_CK(cudaMemcpyAsync(canvas_host, ctx->canvas, sizeof(int32_t) * c.C, cudaMemcpyDeviceToHost,
                           ctx->stream));
-  if (canvas_host || done_host) {
+  if (done_host) {
     DevState hs;
     rc = read_state(ctx, &hs);
     if (rc) return rc;
-    if (done_host) *done_host = hs.done;
+    *done_host = hs.done;
   }
   return DG_OK;
 }

@@ -11,7 +11,7 @@
 //   k_simt_logits   z = (L/T_t) h E^T on CUDA cores, 64x64 tiles, plus the
 //                   per-tile softmax statistics.
 //   k_merge         per row: max, partition sum, entropy H = log Z - S1/Z,
-//                   argmax; optionally normalises the tensor-core path's sc.
+//                   argmax (and the multinomial draw).
 //   k_simt_pe       sc = softmax(z) E on CUDA cores (split over the vocabulary).
 //   k_simt_reduce   fixed-order sum of the vocabulary splits.
 //   k_sampler       entropy sort, acceptance, re-noise, adaptive stop.
@@ -234,12 +234,10 @@ __global__ void __launch_bounds__(256) k_simt_logits(const DevState* st, const T
 // ---------------------------------------------------------------------------
 // Merge per-tile statistics into per-row max, Z, entropy and argmax. One CTA
 // (256 threads) per row; fixed combination order, so results are
-// deterministic. With O != nullptr (tensor-core path) it also writes
-// sc = O e^(mref - m) / Z and flags rows whose logit reference was too low.
+// deterministic. Also the row's multinomial draw when `sampled` is set.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_merge(DevState* st, const TileStat* tstats, int ntiles,
-    RowStat* rowstat, float* H, int32_t* argmax, int C, const float* O, int nO,
-    const float* mref, float* sc, int d, int32_t* redo_rows, float redo_gap, int32_t* sampled) {
+    RowStat* rowstat, float* H, int32_t* argmax, int32_t* sampled) {
   if (st->done) return;
   const int i = blockIdx.x;
   Stat s;
@@ -264,8 +262,6 @@ __global__ void __launch_bounds__(256) k_merge(DevState* st, const TileStat* tst
   __shared__ Stat part[8];
   __shared__ float gpart[8];
   __shared__ int gapart[8];
-  __shared__ float sh_scale;
-  __shared__ int sh_redo;
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
   if (l == 0) { part[w] = s; gpart[w] = gbest; gapart[w] = garg; }
   __syncthreads();
@@ -284,24 +280,6 @@ __global__ void __launch_bounds__(256) k_merge(DevState* st, const TileStat* tst
     argmax[i] = r.arg;
     RowStat rs; rs.m = r.m; rs.Z = r.Z; rs.pad[0] = r.best; rs.pad[1] = 0.f;
     rowstat[i] = rs;
-    int redo = 0;
-    if (O) {
-      const float gap = r.best - mref[i];
-      redo = !(gap <= redo_gap);   // also catches NaN
-      sh_scale = __expf(mref[i] - r.m) / r.Z;
-      if (redo) { redo_rows[atomicAdd(&st->redo, 1)] = i; }
-    }
-    sh_redo = redo;
-  }
-  if (!O) return;
-  __syncthreads();
-  if (sh_redo) return;
-  const float f = sh_scale;
-  const size_t pstride = (size_t)C * d;
-  for (int k = threadIdx.x; k < d; k += blockDim.x) {
-    float acc = 0.f;
-    for (int g = 0; g < nO; ++g) acc += O[g * pstride + (size_t)i * d + k];
-    sc[(size_t)i * d + k] = acc * f;
   }
 }
 
@@ -440,8 +418,7 @@ cudaError_t launch_simt_attention(cudaStream_t s, int dtype, DevState* st, const
                                                      d, scale_tab, S, draw.seed, drawing);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_merge<<<C, 256, 0, s>>>(st, tstats, V / ST, rowstat, H, argmax, C, nullptr, 0, nullptr,
-                            nullptr, d, nullptr, 0.f, draw.sampled);
+  k_merge<<<C, 256, 0, s>>>(st, tstats, V / ST, rowstat, H, argmax, draw.sampled);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   dim3 g2((d + ST - 1) / ST, (C + ST - 1) / ST, nsplit);
   if (dtype == 0)

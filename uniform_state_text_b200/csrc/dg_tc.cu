@@ -1436,10 +1436,8 @@ int check_residency(int units, int sms, char* err, size_t errn) {
   return 0;
 }
 
-int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, float* O,
-                 TileStat* tstats, void* ws, char* err, size_t errn, int v0, int Vg) {
-  (void)O;
-  (void)tstats;
+int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, void* ws, char* err,
+                 size_t errn, int v0, int Vg) {
   p->C = C; p->V = V; p->d = d;
   p->v0 = v0; p->Vg = Vg;
   // the kernels' E tensor maps start at the shard's first row
@@ -1529,10 +1527,10 @@ cudaError_t launch_params(cudaStream_t s, const TcPlan& pl, const TcLayout& L,
 
 cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, const void* h,
                                 const void* E, const float* mref, const float* scale_tab,
-                                int S, TileStat* tstats, float* O, void* ws,
+                                int S, TileStat* tstats, void* ws,
                                 const DrawArgs& draw, float* H, int32_t* argmax,
                                 RowStat* rowstat, float redo_gap, const SamplerArgs& sa) {
-  (void)h; (void)E; (void)O;
+  (void)h; (void)E;
   TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
   const tc::Params prm = base_params(pl, L, st, mref, scale_tab, S, tstats, ws, draw, H, argmax,
                                      rowstat, redo_gap, sa);
@@ -1610,12 +1608,11 @@ cudaError_t merge_launch(cudaStream_t s, const TcPlan& pl, DevState* st, const T
 
 cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& pl, DevState* st, const TileStat* tstats,
                             const float* mref, RowStat* rowstat, float* H, int32_t* argmax,
-                            float* sc, int32_t* redo_rows, float redo_gap, const void* h,
+                            float* sc, float redo_gap, const void* h,
                             const void* E, const float* scale_tab, int S,
                             const SamplerArgs& sa, const DrawArgs& draw, const NextStandin& nx) {
   TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
   const float* Opart = reinterpret_cast<const float*>(static_cast<const char*>(pl.ws) + L.Opart);
-  (void)redo_rows;
   return merge_launch(s, pl, st, reinterpret_cast<const TcStat*>(tstats), 2 * L.n_vt, Opart, L.G,
                       draw.sampled ? static_cast<const TcSamp*>(draw.tsamp) : nullptr, mref,
                       rowstat, H, argmax, sc, redo_gap, h, E, scale_tab, S, sa, draw, nx);

@@ -23,8 +23,8 @@ bool tc_supported(int C, int V, int d);
 int tc_stat_tiles(int C, int V, int d);
 size_t tc_workspace_bytes(int C, int V, int d);
 // E: the whole [Vg][d] table; the kernels cover entries [v0, v0 + V).
-int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, float* O,
-                 TileStat* tstats, void* ws, char* err, size_t errn, int v0, int Vg);
+int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, void* ws, char* err,
+                 size_t errn, int v0, int Vg);
 void tc_plan_free(TcPlan* p);
 int tc_launches(const TcPlan& p);   // kernels per launch_tc_attention call
 // The attention kernel; its G1 CTAs also merge the rows' statistics into H,
@@ -32,7 +32,7 @@ int tc_launches(const TcPlan& p);   // kernels per launch_tc_attention call
 // recomputation (then the merge kernel does both).
 cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& p, DevState* st, const void* h,
                                 const void* E, const float* mref, const float* scale_tab,
-                                int S, TileStat* tstats, float* O, void* ws,
+                                int S, TileStat* tstats, void* ws,
                                 const DrawArgs& draw, float* H, int32_t* argmax,
                                 RowStat* rowstat, float redo_gap, const SamplerArgs& sa);
 // Per-row merge of the kernel's statistics and partials into sc, H and argmax
@@ -42,7 +42,7 @@ cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& p, DevState* st, c
 // counters are reset (DevState::h_ready = 1: the next prologue has no work).
 cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& p, DevState* st, const TileStat* tstats,
                             const float* mref, RowStat* rowstat, float* H, int32_t* argmax,
-                            float* sc, int32_t* redo_rows, float redo_gap, const void* h,
+                            float* sc, float redo_gap, const void* h,
                             const void* E, const float* scale_tab, int S, const SamplerArgs& sa,
                             const DrawArgs& draw, const NextStandin& nx);
 // Bytes of the per-half-tile draw statistics (DrawArgs::tsamp) of the multinomial rule.
