@@ -1029,6 +1029,99 @@ __device__ __noinline__ void merge_recompute(int i, int V, int d, const __nv_bfl
   __syncthreads();
 }
 
+// The merge after the attention kernel already ran the sampler: one pass per
+// element over the CTA's rows does sc = (sum of the G2 partials) / Z, keeps the
+// step's h, writes the next step's stand-in h (the prologue's arithmetic, in
+// the same order) and accumulates the two dot products of the next m_ref.
+__device__ __forceinline__ void merge_fast_tail(DevState* st, const float* Opart, int nO, int C,
+    int V, int d, float* sc, __nv_bfloat16* h, const __nv_bfloat16* E, const float* scale_tab,
+    int S, const int32_t* argmax, const int32_t* canvas, float* mref, const float* inv_row,
+    const NextStandin& nx, int i0) {
+  __shared__ float red[kMergeRows * kMergeThreadsPerRow / 32][2 * kMergeRows];
+  const bool prep = *(volatile int*)&st->done == 0;
+  const int t1 = *(volatile int*)&st->t;                 // the next step (the sampler advanced it)
+  const uint64_t pre = key_prefix(nx.seed, (uint64_t)(uint32_t)*(volatile int*)&st->block,
+                                  kTagNoise + (uint64_t)t1);
+  const int nrows = min(kMergeRows, C - i0);
+  static_assert(kMergeRows == 2, "two rows per CTA");
+  const int r1 = min(i0 + 1, C - 1);
+  const int tgt0 = nx.target[i0] & (V - 1), tgt1 = nx.target[r1] & (V - 1);
+  const int can0 = canvas[i0] & (V - 1), can1 = canvas[r1] & (V - 1);
+  const int prev0 = argmax[i0] & (V - 1), prev1 = argmax[r1] & (V - 1);   // next step's previous argmax
+  float dc0 = 0.f, dp0 = 0.f, dc1 = 0.f, dp1 = 0.f;
+  const size_t pstride = (size_t)C * d;
+  const int d4 = d / 4;
+  __nv_bfloat16* hl = static_cast<__nv_bfloat16*>(nx.h_last);
+  for (int x = threadIdx.x; x < nrows * d4; x += blockDim.x) {
+    const int q = x / d4, k = (x % d4) * 4;
+    const size_t off = (size_t)(i0 + q) * d + k;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int g = 0; g < nO; ++g) {
+      const float4 o = *reinterpret_cast<const float4*>(Opart + g * pstride + off);
+      acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
+    }
+    const float inv = inv_row[q];
+    const float s4[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+    *reinterpret_cast<float4*>(sc + off) = make_float4(s4[0], s4[1], s4[2], s4[3]);
+    const uint2 hold = *reinterpret_cast<const uint2*>(h + off);
+    *reinterpret_cast<uint2*>(hl + off) = hold;
+    if (!prep) continue;
+    const uint2 ut = *reinterpret_cast<const uint2*>(E + (size_t)(q ? tgt1 : tgt0) * d + k);
+    const uint2 uc = *reinterpret_cast<const uint2*>(E + (size_t)(q ? can1 : can0) * d + k);
+    const uint2 up = *reinterpret_cast<const uint2*>(E + (size_t)(q ? prev1 : prev0) * d + k);
+    float pc = 0.f, pp = 0.f;
+    const uint32_t wt[2] = {ut.x, ut.y}, wc[2] = {uc.x, uc.y}, wp[2] = {up.x, up.y};
+    uint32_t hw[2];
+#pragma unroll
+    for (int j2 = 0; j2 < 2; ++j2) {
+      float hv[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float et = __uint_as_float(e ? (wt[j2] & 0xFFFF0000u) : (wt[j2] << 16));
+        const float ec = __uint_as_float(e ? (wc[j2] & 0xFFFF0000u) : (wc[j2] << 16));
+        const uint64_t idx = (uint64_t)(i0 + q) * (uint64_t)d + (uint64_t)(k + 2 * j2 + e);
+        float v = nx.A * et + nx.B * ec;
+        v = v + s4[2 * j2 + e];
+        v = v + nx.sigma * gauss_from_key(sm64(pre ^ idx));
+        hv[e] = v;
+      }
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(hv[0], hv[1]);
+      hw[j2] = *reinterpret_cast<const uint32_t*>(&b2);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float hr = __uint_as_float(e ? (hw[j2] & 0xFFFF0000u) : (hw[j2] << 16));
+        const float ec = __uint_as_float(e ? (wc[j2] & 0xFFFF0000u) : (wc[j2] << 16));
+        const float ep = __uint_as_float(e ? (wp[j2] & 0xFFFF0000u) : (wp[j2] << 16));
+        pc = fmaf(hr, ec, pc);
+        pp = fmaf(hr, ep, pp);
+      }
+    }
+    *reinterpret_cast<uint2*>(h + off) = make_uint2(hw[0], hw[1]);
+    if (q) { dc1 += pc; dp1 += pp; } else { dc0 += pc; dp0 += pp; }
+  }
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  for (int o = 16; o; o >>= 1) {
+    dc0 += __shfl_xor_sync(0xffffffffu, dc0, o);
+    dp0 += __shfl_xor_sync(0xffffffffu, dp0, o);
+    dc1 += __shfl_xor_sync(0xffffffffu, dc1, o);
+    dp1 += __shfl_xor_sync(0xffffffffu, dp1, o);
+  }
+  if (l == 0) { red[w][0] = dc0; red[w][1] = dp0; red[w][2] = dc1; red[w][3] = dp1; }
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    // the attention kernel has completed: its counters start the next step at zero
+    for (int j = threadIdx.x; j < nx.nzero; j += blockDim.x) nx.zero[j] = 0u;
+    if (threadIdx.x == 0) st->h_ready = prep ? 1 : 0;
+  }
+  if (threadIdx.x < nrows && prep) {
+    const int q = threadIdx.x;
+    float a = 0.f, b = 0.f;
+    for (int j = 0; j < (int)(blockDim.x >> 5); ++j) { a += red[j][2 * q]; b += red[j][2 * q + 1]; }
+    mref[i0 + q] = scale_tab[min(max(t1, 0), S - 1)] * fmaxf(a, b);
+  }
+}
+
 __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(DevState* st,
     const TcStat* ts, int nts, float* mref, const float* Opart, int nO, int C, int V, int d,
     RowStat* rowstat, float* H, int32_t* argmax, float* sc, float redo_gap,
@@ -1068,12 +1161,13 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
   const float mref_i = row_ok ? mref[i] : 0.f;
   if (fast) {
     if (tid == 0) {
-      sh_redo[r] = 0;
       sh_inv[r] = row_ok ? 1.0f / rowstat[i].Z : 0.f;
       if (row_ok) nx.mref_last[i] = mref_i;
     }
-    if (threadIdx.x == 0) sh_ticket = 0;
     __syncthreads();
+    merge_fast_tail(st, Opart, nO, C, V, d, sc, h, E, scale_tab, S, argmax, sa.canvas, mref,
+                    sh_inv, nx, i0);
+    return;
   } else {
   if (threadIdx.x == 0) sh_epoch0 = *(volatile int*)&st->epoch;   // before this CTA's ticket
   float Z = 0.f, S1 = 0.f, best = -INFINITY;
@@ -1163,7 +1257,7 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
   }
   // In the last CTA the first nsamp threads run the sampler and the others
   // sum sc; elsewhere every thread sums sc.
-  const bool last = !fast && sh_ticket == gridDim.x - 1;
+  const bool last = sh_ticket == gridDim.x - 1;
   const int nsamp = (C + 31) / 32 * 32;
   int x0 = threadIdx.x, xstep = blockDim.x;
   bool sum_sc = true;
@@ -1210,9 +1304,7 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
   __syncthreads();
   if (threadIdx.x == 0) {
     int go = 1;
-    if (fast) {
-      // the sampler ran in the attention kernel, which has completed
-    } else if (last) {
+    if (last) {
       asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(&st->epoch) : "memory");
     } else {
       const uint64_t t0 = gtimer();
