@@ -188,7 +188,7 @@ def run_reference(args, w):
 # capture summarised under profiles/ (taken on the V=65536 profiling shape and
 # scaled by the vocabulary, since E and the P ring both grow with V).
 DRAM_TRAFFIC = {
-    synthetic.HEADLINE.name: (4 * (292.882688e6 + 8.840192e6),
+    synthetic.HEADLINE.name: (4 * (286.7264e6 + 6.975744e6),
                               "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at "
                               "C=256, V=65536, d=2048, scaled by 4 to V=262144"),
 }
