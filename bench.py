@@ -118,8 +118,9 @@ def cpu_baseline(w, E32, rows: int, seed_steps: int = 1):
     h = M.standin_hidden(w, E32, st.target, st.canvas, st.sc, 0, 0)
     T = M.temperature(0, w.max_steps, w.T_start, w.T_end)
     t0 = time.perf_counter()
+    key = (w.seed, 0, 0) if getattr(w, "token_rule", 0) == 1 else None
     for _ in range(seed_steps):
-        att = M.vocab_attention(h[:rows], E32, w.logit_scale / T)
+        att = M.vocab_attention(h[:rows], E32, w.logit_scale / T, gumbel_key=key)
         M.entropy_bounded_accept(att.H.astype(np.float32), w.tau, w.accept_rule)
     dt = (time.perf_counter() - t0) / seed_steps
     step_s = dt * w.C / rows
@@ -175,7 +176,10 @@ def run_reference(args, w):
             "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "tok_per_s": w.C * val,
-            "config": {"workload": w.name, "C": w.C, "V": w.V, "d": w.d, "mode": "fixed_steps"},
+            "config": {"workload": w.name, "C": w.C, "V": w.V, "d": w.d,
+                       "canvases": w.canvases,
+                       "token_rule": "multinomial" if w.token_rule == 1 else "argmax",
+                       "mode": "fixed_steps"},
             "cpu_baseline": {"value": val, "unit": "steps/s", "cores": cb["cores"],
                              "kind": "oracle", "sample": cb["sample"]},
             "e2e": {"value": val, "unit": "steps/s", "h2d_bytes_per_step": 0,
@@ -202,6 +206,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=synthetic.HEADLINE.name, choices=sorted(synthetic.WORKLOADS))
     ap.add_argument("--kernels", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--token-rule", default="argmax", choices=["argmax", "multinomial"],
+                    help="token an accepted position takes")
+    ap.add_argument("--canvases", type=int, default=0,
+                    help="split the workload's C positions into this many independent "
+                         "canvases (tau scaled per canvas); 0 keeps the workload's own")
     ap.add_argument("--cpu-rows", type=int, default=32, help="rows of the oracle baseline sample")
     ap.add_argument("--ref-rows", type=int, default=16, help="rows per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -210,6 +219,10 @@ def main():
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     w = synthetic.WORKLOADS[args.workload].replace(fixed_steps=1)
+    if args.token_rule == "multinomial":
+        w = w.replace(token_rule=1)
+    if args.canvases > 0:
+        w = w.replace(canvases=args.canvases, tau=w.tau * w.canvases / args.canvases)
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -361,6 +374,8 @@ def main():
                 "tok_per_s": w.C * value,
                 "roofline_pct": roof["step_roofline_pct"],
                 "config": {"workload": w.name, "C": w.C, "V": w.V, "d": w.d,
+                           "canvases": w.canvases,
+                           "token_rule": "multinomial" if w.token_rule == 1 else "argmax",
                            "max_steps": S, "mode": "fixed_steps (adaptive stop off)",
                            "kernels": "tc" if den.impl == dg.DG_IMPL_TC else "simt",
                            "l2": "no flush: E (%.2f GB) exceeds the 126 MB L2 and is streamed every step" % (w.e_bytes / 1e9),

@@ -73,9 +73,35 @@ def test_workspace_bytes_valid_configs(lib):
 @pytest.mark.parametrize("kw", [dict(V=1000), dict(V=32), dict(C=0), dict(C=2048), dict(d=12),
                                 dict(max_steps=0), dict(T_start=0.0), dict(tau=-1.0),
                                 dict(stop_unchanged=0), dict(stop_rule=5), dict(accept_rule=2),
-                                dict(tau=float("inf")), dict(T_end=float("nan"))])
+                                dict(tau=float("inf")), dict(T_end=float("nan")),
+                                dict(token_rule=2), dict(canvases=3), dict(canvases=-1),
+                                dict(canvases=128, C=128)])
 def test_workspace_bytes_rejects_invalid(lib, kw):
     assert dg.dg_workspace_bytes(_cfg(**kw)) == 0
+
+
+def test_canvases_and_draw_options_are_accepted(lib):
+    for kw in (dict(canvases=1), dict(canvases=4), dict(canvases=16), dict(token_rule=1)):
+        assert dg.dg_workspace_bytes(_cfg(**kw)) > 0
+
+
+@pytest.mark.parametrize("shard", [(0, 1024), (512, 4096), (300, 512), (0, 0 + 1)])
+def test_vocabulary_shard_bounds(lib, shard):
+    w = synthetic.SMALL.replace(C=128, V=4096, d=256)
+    cfg = dg.make_config(w, dg.DG_IMPL_AUTO, shard=shard)
+    v0, nv = shard
+    ok = v0 % 256 == 0 and nv % 256 == 0 and nv > 0 and v0 + nv <= w.V
+    assert (dg.dg_workspace_bytes(cfg) > 0) == ok
+    # a shard needs the tensor-core kernels; the partials buffer exists only then
+    assert (dg.dg_partials_bytes(cfg) > 0) == ok
+    if ok:
+        assert dg.dg_partials_bytes(cfg) == 4 * (2 * w.C + w.C * w.d) + 16 * w.C
+
+
+def test_vocabulary_shard_needs_tensor_cores(lib):
+    w = synthetic.SMALL.replace(C=128, V=4096, d=256)
+    assert dg.dg_workspace_bytes(dg.make_config(w, dg.DG_IMPL_SIMT, shard=(0, 1024))) == 0
+    assert dg.dg_partials_bytes(dg.make_config(w, dg.DG_IMPL_SIMT)) == 0
 
 
 def test_tensor_core_request_on_unsupported_shape(lib):
