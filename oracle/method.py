@@ -21,7 +21,7 @@ Sources (page title, section):
         gemma.gh.miniasp.com): self-conditioning multiplies the probability
         matrix by the token embedding table; 256-token canvases, block by block.
 
-Readings where the pages are silent or garbled (each also listed in the design doc):
+Readings where the pages are silent or garbled:
   * The acceptance formula is lost in extraction ([VG] 5.4 ends "based on the
     following formula:"). Default rule (accept_rule 0): accept the sorted
     prefix whose inclusive running entropy sum is <= tau ([WS]). Rule 1 reads

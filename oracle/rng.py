@@ -5,7 +5,7 @@ TEST INFRASTRUCTURE (see the package docstring).
 The pages draw three kinds of random values: the uniform random initial canvas
 (A Visual Guide to DiffusionGemma, 5.4 "canvas initialisation": tokens drawn
 uniformly from the vocabulary), the fresh uniform token given to every rejected
-position (5.4 "token re-noising"), and, in this build's stand-in backbone, a
+position (5.4 "token re-noising"), and, in the synthetic stand-in backbone, a
 Gaussian perturbation of the hidden state. All are keyed, not sequential, so
 that a position's draw depends only on (seed, block, step, index).
 

@@ -1,8 +1,9 @@
 """Pins of the oracle's batched canvases (independent canvases sharing a step).
 
-SURVEY's next rows name batched canvases (B users x C positions): the rows of
-the vocabulary attention are independent, so B canvases can share one step,
-while the sampler and the stop test act on each canvas alone. Pinned here: a
+Batched canvases (B users x C positions; A Visual Guide to DiffusionGemma, 5.2
+multi-canvas sampling): the rows of the vocabulary attention are independent,
+so B canvases can share one step, while the sampler and the stop test act on
+each canvas alone. Pinned here: a
 hand-worked two-canvas acceptance example (exact in binary) that a sort across
 canvases would get wrong, the reduction to the single-canvas sampler, the
 independence of one canvas's decisions from another's hidden state, and the
