@@ -8,28 +8,37 @@
 // without ever storing the C x V logits.
 //
 // Design (B200):
-//   * Both contractions run on tcgen05 (bf16 in, fp32 accumulate in TMEM).
+//   * Both contractions run on tcgen05 (bf16 in, fp32 accumulate in TMEM). For
+//     C = 256 the CTAs work in pairs (cta_group::2, M = 256); for C = 128 alone.
 //   * A fixed per-row logit reference m_ref (the larger of the logits of the
-//     row's current canvas token and of its previous argmax, computed by the
-//     prologue) replaces the running maximum: probabilities are
+//     row's current canvas token and of its previous argmax, computed with the
+//     stand-in h) replaces the running maximum: probabilities are
 //     P = exp(z - m_ref). With no running maximum there is nothing to agree on
 //     between CTAs, so the P.E contraction can run on other SMs than the h.E^T
 //     contraction. The exact maximum is tracked alongside; a row whose maximum
 //     exceeds m_ref by more than 64 (P could overflow) is recomputed exactly by
-//     the fix-up kernels below. Entropy and argmax never depend on m_ref.
-//   * One persistent cooperative kernel, two CTA roles:
-//       G1 CTAs: S = h E_tile^T for 128 rows x 256 vocabulary entries (K = d)
-//                into a double-buffered TMEM accumulator; the epilogue warps
-//                turn S into per-tile statistics and bf16 P, written into an
-//                L2-resident ring of P tiles.
-//       G2 CTAs: each owns (row block, 256-column slice of d, range group) and
-//                accumulates O = P E over its ranges in TMEM, then writes one
-//                partial; the merge kernel sums the partials in fixed order.
+//     the merge kernel below. Entropy and argmax never depend on m_ref.
+//   * One persistent kernel per step, two CTA roles:
+//       G1 units: S = h E_tile^T for all rows x 256 vocabulary entries (K = d),
+//                taken from a dynamic tile queue, into a double-buffered TMEM
+//                accumulator; the epilogue warps turn S into per-half-tile
+//                statistics (and the multinomial draw) and bf16 P, written
+//                into an L2-resident ring of P tiles. When every G1 item is
+//                done, the G1 CTAs merge the rows' statistics and the last one
+//                runs the sampler and stop test (g1_finish).
+//       G2 units: each owns (512-column slice of d, range group) and
+//                accumulates O = P E over its ranges in two TMEM accumulators,
+//                then writes one partial.
 //     Hand-off: per-tile "ready" and "consumed" counters in global memory
 //     (release/acquire); every wait is bounded by %globaltimer and aborts the
 //     whole kernel through a flag, after draining its in-flight copies.
-//   * Warp roles per CTA (192 threads): warp 0 TMA producer, warp 1 TMEM
-//     allocator + MMA issuer, warps 2-5 epilogue (one TMEM lane per thread).
+//   * The merge kernel sums the partials into sc in fixed order and writes the
+//     next step's stand-in h and m_ref (so the next step needs no prologue).
+//   * Warp roles per CTA (320 threads): warp 0 TMA producer, warp 1 TMEM
+//     allocator + MMA issuer, warps 2-9 epilogue (two warps per TMEM lane
+//     quarter, each half of the accumulator's columns).
+//   * A vocabulary-parallel step runs the same kernel over a shard of the
+//     vocabulary and ends in partial row results for a cross-rank reduction.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
