@@ -111,16 +111,21 @@ class Clocks:
 
 
 def cpu_baseline(w, E32, rows: int, seed_steps: int = 1):
-    """The oracle, as it stands, on `rows` canvas rows of one step; scaled to steps/s."""
+    """The oracle, as it stands, on `rows` canvas rows of one step; scaled to steps/s.
+
+    The sample is the first `rows` rows: their stand-in hidden state, the
+    vocabulary attention (and draw) and the acceptance over them.
+    """
     from oracle import method as M
 
     st = M.begin_block(w, 0)
-    h = M.standin_hidden(w, E32, st.target, st.canvas, st.sc, 0, 0)
+    wr = w.replace(C=rows, canvases=1)
     T = M.temperature(0, w.max_steps, w.T_start, w.T_end)
-    t0 = time.perf_counter()
     key = (w.seed, 0, 0) if getattr(w, "token_rule", 0) == 1 else None
+    t0 = time.perf_counter()
     for _ in range(seed_steps):
-        att = M.vocab_attention(h[:rows], E32, w.logit_scale / T, gumbel_key=key)
+        h = M.standin_hidden(wr, E32, st.target[:rows], st.canvas[:rows], st.sc[:rows], 0, 0)
+        att = M.vocab_attention(h, E32, w.logit_scale / T, gumbel_key=key)
         M.entropy_bounded_accept(att.H.astype(np.float32), w.tau, w.accept_rule)
     dt = (time.perf_counter() - t0) / seed_steps
     step_s = dt * w.C / rows
@@ -162,14 +167,22 @@ def run_reference(args, w):
     if w.dtype == "bf16":
         import torch
         E32 = torch.from_numpy(E32).to(torch.bfloat16).float().numpy()
+    # Each timed step is a sample of --ref-rows rows (enough to amortise the
+    # oracle's fixed per-call cost: it widens all of E to fp64 in chunks). At
+    # most as many samples as fit in about two minutes are timed, so a large
+    # --steps still ends in bounded time; "steps" reports how many ran.
     rows = max(1, min(w.C, args.ref_rows))
+    first = cpu_baseline(w, E32, rows)                       # warm-up and calibration
+    sample_s = rows / (w.C * first["value"])        # seconds per sample
+    n = int(max(1, min(args.steps, 120.0 // max(sample_s, 1e-9))))
     times = []
-    if args.warmup > 0:
+    for _ in range(max(0, min(args.warmup, n) - 1)):
         cpu_baseline(w, E32, rows)
-    for _ in range(args.steps):
+    for _ in range(n):
         times.append(1.0 / cpu_baseline(w, E32, rows)["value"])
     step_s = float(np.mean(times))
     cb = cpu_baseline(w, E32, rows)
+    args.steps = n
     val = 1.0 / step_s
     line = {"metric": METRIC, "value": val, "unit": "steps/s", "impl": "reference",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
