@@ -227,6 +227,42 @@ def test_batched_canvases_teacher_forced(impl, canvases):
     den.close()
 
 
+def test_batched_canvases_with_draw_and_shards():
+    """Two canvases per step under the multinomial rule, stepped as two
+    vocabulary shards: the options compose (per-canvas sampler after the
+    cross-shard reduction), against the oracle."""
+    w = synthetic.STRESS_PARTIAL.replace(canvases=2, tau=0.5 * 128 * np.log(2), token_rule=1,
+                                         max_steps=4, fixed_steps=1)
+    Eg, E32 = embedding(w)
+    half = w.V // 2
+    shards = [dg.Denoiser(w, Eg, impl=dg.DG_IMPL_TC, shard=(0, half)),
+              dg.Denoiser(w, Eg, impl=dg.DG_IMPL_TC, shard=(half, half))]
+    bufs = [s.partials() for s in shards]
+    st = M.begin_block(w, 0)
+    for _ in range(w.max_steps):
+        for s, b in zip(shards, bufs):
+            s.step_partial(b)
+            s.stream.synchronize()
+        dg.reduce_partials_local(bufs, w.C, w.d)
+        torch.cuda.synchronize()
+        for s, b in zip(shards, bufs):
+            s.step_finish(b)
+            s.stream.synchronize()
+        h = _np(shards[0].read(dg.DG_HIDDEN)).astype(np.float64)
+        rec = M.step(w, E32, st, h=h)
+        canvas = _np(shards[0].read(dg.DG_CANVAS)).astype(np.int64)
+        assert np.array_equal(canvas, _np(shards[1].read(dg.DG_CANVAS)))
+        # the trajectory is teacher-forced through h; tokens agree except on near-ties
+        ties = (rec.att.smargin < 1e-3) | (rec.att.margin < 1e-3)
+        bad = np.flatnonzero((canvas != rec.canvas_out) & ~ties)
+        assert bad.size <= max(1, w.C // 1000), bad[:8]
+        st.canvas = canvas
+        cst = _np(shards[0].read(dg.DG_CANVAS_STATE)).reshape(3, 2)
+        assert np.array_equal(cst[1] != 0, st.done_c)
+    for s in shards:
+        s.close()
+
+
 @pytest.mark.parametrize("impl", IMPLS)
 def test_batched_canvases_block(impl):
     """Whole blocks of batched canvases through the graph loop: each canvas's
