@@ -173,6 +173,8 @@ int dg_begin_block(dg_ctx* ctx, int32_t block);
  * self-conditioning vector, entropy sort, acceptance, re-noise, stop test.
  * No-op once the block is done. done_host: NULL = stay asynchronous;
  * otherwise the stream is synchronised and *done_host receives the done flag.
+ * A vocabulary-shard context returns DG_EUNSUPPORTED (it steps with
+ * dg_denoise_step_partial / dg_denoise_step_finish).
  */
 int dg_denoise_step(dg_ctx* ctx, int32_t* done_host);
 
@@ -196,7 +198,8 @@ int dg_denoise_step_h(dg_ctx* ctx, const void* h_src, int32_t h_on_host,
  * identically everywhere; each rank's context (cfg.shard_v0, shard_nv) covers
  * its share of the vocabulary. Tensor-core path only (DG_EUNSUPPORTED else).
  *   dg_partials_bytes  bytes of one partials buffer (device, caller-owned,
- *                      8-byte aligned).
+ *                      16-byte aligned); 0 if the configuration has no
+ *                      vocabulary-parallel step.
  *   dg_denoise_step_partial  the step up to the rows' partial results over
  *                      the shard, written to `partials`:
  *                        float zs[C][2]  Z and S1 against m_ref   -> sum over ranks
@@ -218,8 +221,10 @@ int dg_denoise_step_finish(dg_ctx* ctx, const void* partials);
 /*
  * A whole block ([VG] 5.2): dg_begin_block, then denoise steps until the
  * adaptive stop or the step budget (one CUDA graph launch with a device-side
- * loop), then the final step's argmax is written to out_dev (device, int32 [C]).
+ * loop), then each canvas's argmax at its own final step (the final step's
+ * argmax for one canvas) is written to out_dev (device, int32 [C]).
  * steps_host (nullable) receives the number of steps run (synchronises).
+ * Needs a non-default stream; not for a vocabulary-shard context.
  */
 int dg_denoise_block(dg_ctx* ctx, int32_t block, int32_t* out_dev, int32_t* steps_host);
 
