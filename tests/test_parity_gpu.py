@@ -148,7 +148,8 @@ def run_teacher_forced(den, w, E32, max_steps=None):
 
 
 # ----------------------------------------------------------------------------
-@pytest.mark.parametrize("shape", [(128, 4096, 256), (256, 8192, 512), (128, 16384, 768)])
+@pytest.mark.parametrize("shape", [(128, 256, 256), (256, 512, 256), (128, 4096, 256),
+                                   (256, 8192, 512), (128, 16384, 768)])
 def test_tc_small_shapes(shape):
     """The tensor-core kernel on small shapes (one range group up to several), 3 steps."""
     C, V, d = shape
