@@ -413,6 +413,22 @@ def test_ragged_shapes_simt(shape):
     den.close()
 
 
+@pytest.mark.parametrize("C,canvases", [(1024, 1), (1024, 64), (64, 64)])
+def test_largest_and_single_position_canvases_simt(C, canvases):
+    """The most positions a context takes (C = 1024) as one canvas and as the most
+    canvases per step (64 of 16 positions), and canvases of one position each:
+    sort, acceptance, re-noise and stop over up to 1024 keys."""
+    Cc = C // canvases
+    w = synthetic.TINY.replace(C=C, V=2048, d=64, canvases=canvases, tau=0.5 * Cc * np.log(2),
+                               coef_target=1.0, coef_canvas=0.5, logit_scale=2.0, max_steps=4,
+                               fixed_steps=1)
+    assert supported(w, dg.DG_IMPL_SIMT)
+    den, E32 = make(w, dg.DG_IMPL_SIMT)
+    tally = run_teacher_forced(den, w, E32)
+    assert tally.steps == w.max_steps
+    den.close()
+
+
 def test_workspace_too_small_is_rejected():
     w = synthetic.TINY
     Eg, _ = embedding(w)

@@ -254,8 +254,9 @@ int prologue_if_needed(dg_ctx* ctx, bool standin, bool use_cond) {
   if (tc) tc_counters(ctx->tc_plan, &zero, &nzero);
   // After a tensor-core step the merge kernel has already written this step's
   // stand-in h and m_ref (DevState::h_ready); a stepwise call then skips the
-  // prologue launch. A captured loop keeps it: it checks h_ready on the device.
-  if (tc && standin && !use_cond && ctx->h_ready) return 0;
+  // prologue launch. The captured block loop has none: dg_denoise_block runs
+  // it once before the loop, and every later step's h comes from the merge.
+  if (tc && standin && (use_cond || ctx->h_ready)) return 0;
   DG_CK(launch_prologue(ctx->stream, c.dtype, ctx->st, ctx->E, ctx->target, ctx->canvas, ctx->sc,
                         ctx->h, c.C, c.V, c.d, c.seed, c.coef_target, c.coef_canvas,
                         standin_sigma(c), standin ? 1 : 0, ctx->scale_tab, c.max_steps,
@@ -501,6 +502,13 @@ int dg_denoise_block(dg_ctx* ctx, int32_t block, int32_t* out_dev, int32_t* step
   if (!out_dev) return fail(ctx, DG_EINVAL, "out_dev is NULL");
   int rc = dg_begin_block(ctx, block);
   if (rc) return rc;
+  // The tensor-core loop's first step needs the stand-in h and m_ref; the
+  // merge of each step prepares the next one's.
+  if (ctx->L.impl == DG_IMPL_TC) {
+    rc = prologue_if_needed(ctx, true, false);
+    if (rc < 0) return rc;
+    ctx->launches += rc;
+  }
   if (!ctx->graph_ready && (rc = build_graph(ctx))) return rc;
   DG_CK(cudaGraphLaunch(ctx->graph_exec, ctx->stream));
   // each canvas's argmax at its own stop (one canvas: the final step's argmax)
