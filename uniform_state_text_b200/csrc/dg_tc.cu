@@ -131,7 +131,10 @@ __device__ __forceinline__ void max_key_decode(unsigned long long key, float* v,
 // builds). Each role accumulates in registers and stores once at its end.
 // Slots: 0 start, 1 end, 2 producer waits on free stages, 3 producer waits on
 // counters, 4 MMA waits on full stages, 5 MMA waits on free accumulators,
-// 6 epilogue waits on full accumulators, 7 items, 8 epilogue busy.
+// 6 epilogue waits on full accumulators, 7 items, 8 epilogue busy, and within
+// it 9 TMEM loads, 10 softmax arithmetic, 11 P stores, 12 publishing the tile.
+// The block of [grid][32] int64 lies in the tensor-core workspace after the
+// counters, the P ring and the O partials.
 #ifdef DG_TC_TRACE
 #define TR_DECL(v) unsigned long long v = 0
 #define TR_T0() const unsigned long long tr_t0_ = gtimer()
