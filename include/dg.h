@@ -249,6 +249,31 @@ int dg_profile_read(dg_ctx* ctx, double* ms_total, int32_t* steps, int64_t* laun
 int dg_impl(const dg_ctx* ctx);
 
 /*
+ * The tensor-core kernel's work split for a shape, as dg_init plans it on a
+ * GPU with `sms` streaming multiprocessors. Host only: no device, context or
+ * CUDA call is involved, so tools and tests can check the schedule of any
+ * shape. The kernel is one persistent grid of n1 + n2 units (CTA pairs or
+ * single CTAs) with two roles:
+ *   - units 0 .. n1-1 (G1) compute S = h.E^T for one 256-entry vocabulary tile
+ *     at a time, taken from a shared queue in tile order, and write
+ *     P = e^(z - m_ref) into a ring of resident tiles;
+ *   - unit n1 + o (G2 unit o) accumulates O = P.E over the 256-entry ranges
+ *     g, g + G, g + 2G, ... with g = o / (RBI * n_dt), for the column slice
+ *     o % n_dt of W2 * 256 columns of d and, for single CTAs, the row block
+ *     (o % (RBI * n_dt)) / n_dt (RBI = 1 for pairs, which cover all rows, and
+ *     RB otherwise).
+ * Writes to out (host, n >= 11 values):
+ *   [0] CG: CTAs per MMA group (2: CTA pairs, M = 256)   [1] W2
+ *   [2] RB: 128-row blocks   [3] n_vt: 256-entry tiles   [4] n_ranges
+ *   [5] n_dt: slices of d    [6] G: range groups         [7] n1: G1 units
+ *   [8] n2: G2 units         [9] ring: P tiles resident  [10] CTAs launched
+ * Returns 11, DG_EUNSUPPORTED if the tensor-core kernels do not cover the
+ * shape, or DG_EINVAL (NULL out, n < 11, sms < 2); dg_last_error(NULL) gives
+ * the message.
+ */
+int dg_tc_schedule(int32_t C, int32_t V, int32_t d, int32_t sms, int32_t* out, int32_t n);
+
+/*
  * Vocabulary attention without any allocation. The pages have no counterpart:
  * this entry point exists for callers that cannot call cudaMalloc (code inside
  * a host callback, a plugin whose host framework owns every device allocation,

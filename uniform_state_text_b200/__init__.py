@@ -85,13 +85,14 @@ def lib():
     L.dg_partials_bytes.restype = ctypes.c_size_t
     L.dg_denoise_step_partial.argtypes = [_P, _P]
     L.dg_denoise_step_finish.argtypes = [_P, _P]
+    L.dg_tc_schedule.argtypes = [_I, _I, _I, _I, _P, _I]
     L.dg_free.argtypes = [_P]
     L.dg_last_error.argtypes = [_P]
     L.dg_last_error.restype = ctypes.c_char_p
     for name in ("dg_init", "dg_begin_block", "dg_denoise_step", "dg_denoise_step_h",
                  "dg_denoise_block", "dg_read", "dg_write", "dg_profile", "dg_profile_read",
                  "dg_impl", "dg_free", "dg_vocab_attention_static", "dg_denoise_step_partial",
-                 "dg_denoise_step_finish"):
+                 "dg_denoise_step_finish", "dg_tc_schedule"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -209,6 +210,18 @@ def dg_denoise_step_finish(ctx, partials_ptr: int) -> None:
 
 def dg_impl(ctx) -> int:
     return _check(lib().dg_impl(ctx), ctx)
+
+
+TC_SCHEDULE_FIELDS = ("CG", "W2", "RB", "n_vt", "n_ranges", "n_dt", "G", "n1", "n2", "ring",
+                      "ctas")
+
+
+def dg_tc_schedule(C: int, V: int, d: int, sms: int = 148) -> dict:
+    """The tensor-core kernel's work split for a shape (host only; see include/dg.h)."""
+    out = (ctypes.c_int32 * len(TC_SCHEDULE_FIELDS))()
+    n = _check(lib().dg_tc_schedule(C, V, d, sms, ctypes.cast(out, ctypes.c_void_p),
+                                    len(TC_SCHEDULE_FIELDS)), None)
+    return dict(zip(TC_SCHEDULE_FIELDS, list(out)[:n]))
 
 
 def dg_free(ctx) -> None:

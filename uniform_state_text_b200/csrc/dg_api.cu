@@ -523,6 +523,14 @@ int dg_denoise_block(dg_ctx* ctx, int32_t block, int32_t* out_dev, int32_t* step
   return DG_OK;
 }
 
+int dg_tc_schedule(int32_t C, int32_t V, int32_t d, int32_t sms, int32_t* out, int32_t n) {
+  if (!out || n < kTcScheduleValues || sms < 2)
+    return fail(nullptr, DG_EINVAL, "out must hold %d values and sms be at least 2", kTcScheduleValues);
+  if (!tc_schedule_info(C, V, d, sms, out))
+    return fail(nullptr, DG_EUNSUPPORTED, "the tensor-core kernels do not cover C=%d V=%d d=%d", C, V, d);
+  return kTcScheduleValues;
+}
+
 size_t dg_partials_bytes(const dg_config* cfg) {
   Layout L;
   char why[256];

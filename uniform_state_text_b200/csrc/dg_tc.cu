@@ -1468,6 +1468,16 @@ bool tc_supported(int C, int V, int d) {
 
 int tc_stat_tiles(int, int V, int) { return V / tc::BN; }
 
+bool tc_schedule_info(int C, int V, int d, int sms, int32_t* out) {
+  if (!tc_supported(C, V, d) || sms < 2) return false;
+  const TcLayout L = tc_layout(C, V, d, sms);
+  if (L.G < 1 || L.n1 < 1) return false;
+  const int32_t v[kTcScheduleValues] = {L.CG, L.W2, L.RB, L.n_vt, L.n_ranges, L.n_dt, L.G,
+                                        L.n1, L.n2, tc::RING, L.CG * (L.n1 + L.n2)};
+  for (int i = 0; i < kTcScheduleValues; ++i) out[i] = v[i];
+  return true;
+}
+
 size_t tc_workspace_bytes(int C, int V, int d) { return tc_layout(C, V, d, device_sms()).total; }
 
 size_t tc_draw_bytes(int C, int V, int) { return sizeof(TcSamp) * (size_t)C * 2 * (V / tc::BN); }

@@ -20,6 +20,10 @@ struct TcPlan {
 };
 
 bool tc_supported(int C, int V, int d);
+// The work split tc_layout picks on a GPU with `sms` SMs, in the order
+// dg_tc_schedule documents; false if the kernels do not cover the shape.
+constexpr int kTcScheduleValues = 11;
+bool tc_schedule_info(int C, int V, int d, int sms, int32_t* out);
 int tc_stat_tiles(int C, int V, int d);
 size_t tc_workspace_bytes(int C, int V, int d);
 // E: the whole [Vg][d] table; the kernels cover entries [v0, v0 + V).
