@@ -53,8 +53,11 @@ Readings where the pages are silent or garbled:
     those of the combined row index, so canvas c is rows [c C/B, (c+1) C/B)
     of a C-row canvas.
   * Self-conditioning feeds sc = softmax(z) E of the tempered logits straight
-    into the next step's stand-in hidden state (the small FFNN of [VG] 5.1
-    needs trained weights and is left out).
+    into the next step's stand-in hidden state. The small feed-forward network
+    that [VG] 5.1 puts between sc and the next step's token embeddings is
+    self_condition_ffnn (for a caller's backbone and weights): the pages give
+    no shape, so the reading is two linear layers with a GELU between them
+    (the tanh form), y = W2 gelu(W1 sc + b1) + b2, weights [out][in].
 
 Precision: fp64 throughout. Decisions that turn floats into integers are taken
 in fp32, the precision the CUDA kernels take them in: argmax over fp32-rounded
@@ -215,6 +218,38 @@ def vocab_attention(h: np.ndarray, E: np.ndarray, scale: float,
 
 
 # ----------------------------------------------------------------------------
+# Self-conditioning feed-forward network ([VG] 5.1: the probability-weighted
+# embeddings "are passed to a small FFNN and added to the next step's token
+# embeddings"; [EX] self-conditioning).
+# ----------------------------------------------------------------------------
+def gelu_tanh(a: np.ndarray) -> np.ndarray:
+    """GELU in its tanh form: a/2 (1 + tanh(sqrt(2/pi) (a + 0.044715 a^3)))."""
+    a = np.asarray(a, dtype=np.float64)
+    return 0.5 * a * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (a + 0.044715 * a ** 3)))
+
+
+def self_condition_ffnn(sc, W1, b1, W2, b2) -> np.ndarray:
+    """y = W2 gelu(W1 sc + b1) + b2 for every canvas row of sc [C][d].
+
+    W1 [d_ff][d] and W2 [d][d_ff] (each row: one output unit's weights), b1
+    [d_ff], b2 [d]. The tensor-core kernels take sc and the hidden activations
+    as bf16 operands, so both are rounded to bf16 (round to nearest even) before
+    the products, as there; everything else is fp64.
+    """
+    x = bf16_round(np.asarray(sc, np.float64))
+    a = x @ np.asarray(W1, np.float64).T + np.asarray(b1, np.float64)[None, :]
+    g = bf16_round(gelu_tanh(a))
+    return g @ np.asarray(W2, np.float64).T + np.asarray(b2, np.float64)[None, :]
+
+
+def add_to_embeddings(emb, y, dtype: str) -> np.ndarray:
+    """The next step's token embeddings plus the network's output, in emb's type
+    (bf16 embeddings: the sum rounded to bf16)."""
+    s = np.asarray(emb, np.float64) + np.asarray(y, np.float64)
+    return bf16_round(s) if dtype == "bf16" else s
+
+
+# ----------------------------------------------------------------------------
 # Entropy-bounded sampler ([VG] 5.4, [WS] entropy-constrained sampler).
 # ----------------------------------------------------------------------------
 @dataclasses.dataclass
@@ -282,11 +317,14 @@ def accept_canvases(H32: np.ndarray, tau: float, rule: int, B: int, frozen=None)
     return accepted, order, prefix, k
 
 
-def renoise(w, accepted, argmax, block: int, t: int) -> np.ndarray:
-    """Accepted positions take the chosen token (argmax, or the draw under
-    token_rule 1); every rejected one a fresh uniform token."""
+def renoise(w, accepted, chosen, block: int, t: int):
+    """Token re-noising ([VG] 5.4): accepted positions take the chosen token
+    (argmax, or the draw under token_rule 1); every rejected one a fresh
+    uniform token key(seed, block, t, position) & (V - 1) ([VG] 3.2: the noise
+    of uniform-state diffusion is a uniformly random vocabulary token).
+    Returns (proposed canvas, the noise tokens)."""
     noise = rng.tokens(w.seed, block, t, np.arange(w.C, dtype=np.uint64), w.V)
-    return np.where(accepted, argmax, noise).astype(np.int64)
+    return np.where(accepted, chosen, noise).astype(np.int64), noise
 
 
 # ----------------------------------------------------------------------------
@@ -350,19 +388,19 @@ def step(w, E: np.ndarray, st: State, h: np.ndarray | None = None) -> StepRecord
     else:
         att = vocab_attention(h, E, w.logit_scale / T)
     H32 = att.H.astype(np.float32)
-    noise = rng.tokens(w.seed, st.block, t, np.arange(w.C, dtype=np.uint64), w.V)
     chosen = att.sampled if multinomial else att.argmax
     B = canvases(w)
     Cc = w.C // B
     last = (t + 1 >= w.max_steps)
     canvas_out = st.canvas.copy()
     accepted, order, prefix, k_c = accept_canvases(H32, w.tau, w.accept_rule, B, st.done_c)
+    proposed, noise = renoise(w, accepted, chosen, st.block, t)
     conf_c = np.zeros(B, dtype=bool)
     for c in range(B):
         seg = slice(c * Cc, (c + 1) * Cc)
         if st.done_c[c]:
             continue                      # a stopped canvas is frozen
-        canvas_out[seg] = np.where(accepted[seg], chosen[seg], noise[seg])
+        canvas_out[seg] = proposed[seg]
         conf_c[c] = bool(np.all(H32[seg] < np.float32(w.stop_entropy)))
         if w.stop_rule == 0:
             same = bool(np.array_equal(canvas_out[seg], st.canvas[seg]))
