@@ -132,7 +132,8 @@ typedef struct dg_ctx dg_ctx;
 #define DG_ST_K          5  /* positions accepted in the last step             */
 #define DG_ST_STATUS     6  /* 0, or a DG_E* code raised on the device         */
 #define DG_ST_HASPREV    7  /* 1 once an argmax of a previous step exists      */
-#define DG_ST_REDO       8  /* rows recomputed because the reference was low   */
+#define DG_ST_REDO       8  /* rows whose logit reference was raised to their */
+                            /* exact maximum (the step's tensor-core redo pass) */
 
 /*
  * Bytes of device workspace the configuration needs (0 if it is invalid).
@@ -182,10 +183,14 @@ int dg_denoise_step(dg_ctx* ctx, int32_t* done_host);
  * The same step with the hidden state supplied by the caller instead of the
  * stand-in backbone: h_src holds [C][d] of cfg->dtype, in host memory when
  * h_on_host != 0 (pinned memory keeps the copy asynchronous) or device memory
- * otherwise. canvas_host (nullable, pinned) receives the updated canvas,
- * int32 [C], asynchronously: it is valid once the stream has reached it.
- * done_host (nullable) receives the done flag; a non-NULL done_host
- * synchronises.
+ * otherwise. A host h_src is copied on a stream the context creates at its
+ * first such call (released by dg_free) into one of two staging slots of the
+ * workspace, so that the copy of one step overlaps the kernels of the step
+ * before; the step itself waits for its copy on the context's stream. The
+ * caller keeps h_src unchanged until the context's stream has passed this
+ * step. canvas_host (nullable, pinned) receives the updated canvas, int32 [C],
+ * asynchronously: it is valid once the stream has reached it. done_host
+ * (nullable) receives the done flag; a non-NULL done_host synchronises.
  */
 int dg_denoise_step_h(dg_ctx* ctx, const void* h_src, int32_t h_on_host,
                       int32_t* canvas_host, int32_t* done_host);
@@ -228,6 +233,35 @@ int dg_denoise_step_finish(dg_ctx* ctx, const void* partials);
  */
 int dg_denoise_block(dg_ctx* ctx, int32_t block, int32_t* out_dev, int32_t* steps_host);
 
+/*
+ * Self-conditioning network ([VG] 5.1: the probability-weighted embeddings are
+ * "passed to a small feed-forward network and added to the next step's token
+ * embeddings"; [EX] self-conditioning). For a caller whose own backbone makes
+ * the hidden state: after a step, this adds the network's output for the
+ * context's current sc to the caller's next-step token embeddings, on the
+ * tensor cores. The pages give no shape; the network is two linear layers
+ * with a GELU (tanh form) between them:
+ *   emb[i] += W2 gelu(W1 sc[i] + b1) + b2          for i in 0..C-1
+ *   d_ff     hidden width, a multiple of 128 (<= 65536); cfg->d must be a
+ *            multiple of 128 too.
+ *   W1       device, bf16 [d_ff][d] (row u: the weights of hidden unit u),
+ *            16-byte aligned; b1 device, float [d_ff].
+ *   W2       device, bf16 [d][d_ff], 16-byte aligned; b2 device, float [d].
+ *   emb      device, [C][d] of emb_dtype (DG_F32 or DG_BF16), 16-byte
+ *            aligned; read and written (bf16: the sum is rounded to bf16).
+ *   scratch  device, >= dg_self_condition_scratch_bytes(cfg, d_ff) bytes,
+ *            256-byte aligned, caller-owned (sc as bf16 and the hidden
+ *            activations, bf16).
+ * sc enters as bf16 and the hidden activations are rounded to bf16 (the
+ * tensor cores' operand type); accumulation is fp32. All buffers are
+ * caller-owned; asynchronous on the context's stream. Errors: DG_EINVAL,
+ * DG_EUNSUPPORTED (d or d_ff not a multiple of 128), DG_ECUDA; a device wait
+ * that runs out raises DG_ETIMEOUT in the status word.
+ */
+size_t dg_self_condition_scratch_bytes(const dg_config* cfg, int32_t d_ff);
+int dg_self_condition(dg_ctx* ctx, int32_t d_ff, const void* W1, const float* b1, const void* W2,
+                      const float* b2, void* emb, int32_t emb_dtype, void* scratch);
+
 /* Copy one piece of state to / from a caller device buffer (see DG_CANVAS...). */
 int dg_read(dg_ctx* ctx, int32_t what, void* dst_dev);
 int dg_write(dg_ctx* ctx, int32_t what, const void* src_dev);
@@ -247,6 +281,23 @@ int dg_profile_read(dg_ctx* ctx, double* ms_total, int32_t* steps, int64_t* laun
 
 /* Which kernel family the context runs (DG_IMPL_SIMT or DG_IMPL_TC). */
 int dg_impl(const dg_ctx* ctx);
+
+/*
+ * Failure-path testing of the tensor-core kernels' bounded waits (no page
+ * describes it). Every wait of the attention kernel (on a copy landing, on a
+ * pipeline stage, on the other CTA role's hand-off counters) gives up after a
+ * time limit; the kernel then raises DG_ETIMEOUT in the device status word,
+ * every CTA drains its own copies in flight and returns, and the next
+ * synchronising call reports DG_ETIMEOUT. dg_begin_block clears the status.
+ *   wait_limit_ns  the limit of every wait in later steps (0: the default, 2 s).
+ *   stall          0 for normal operation; > 0 adds that much to the hand-off
+ *                  target the P.E CTAs wait for, which no step reaches, so the
+ *                  next step's waits run out after wait_limit_ns.
+ * Host only; takes effect at the next launch (a captured block loop is
+ * rebuilt). Errors: DG_EINVAL (limit outside [0, 60 s], stall < 0),
+ * DG_EUNSUPPORTED (a CUDA-core context, which has no waits).
+ */
+int dg_inject_stall(dg_ctx* ctx, int64_t wait_limit_ns, int32_t stall);
 
 /*
  * The tensor-core kernel's work split for a shape, as dg_init plans it on a
@@ -291,9 +342,12 @@ int dg_tc_schedule(int32_t C, int32_t V, int32_t d, int32_t sms, int32_t* out, i
  * The array is held by every GPU that loads the library until the process
  * exits. All calls share it and it keeps the last call's contents (this call
  * writes every scratch word before reading it); calls whose kernels overlap on
- * the GPU race on it, so serialise them. The first call on each device looks
- * up the array's address (cudaGetSymbolAddress, that device current); make it
- * before capturing a stream into a graph. No cudaMalloc or cudaFree is called.
+ * the GPU race on it, so serialise them. Each call looks up the array's address
+ * (cudaGetSymbolAddress, the calling device current), so it follows the module
+ * if a device reset loads it again; a call made while its stream is being
+ * captured into a graph uses the address of the last call outside capture, so
+ * make the first call on each device before any capture (DG_EINVAL otherwise).
+ * No cudaMalloc or cudaFree is called.
  * Errors: DG_EINVAL (bad shape, dtype or NULL pointer), DG_EUNSUPPORTED (the
  * shape needs more than DG_STATIC_SCRATCH_BYTES of scratch, about
  * 4.5*C*V + 4*C*d bytes), DG_ECUDA; dg_last_error(NULL) gives the message.

@@ -80,6 +80,10 @@ def lib():
     L.dg_profile_read.argtypes = [_P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I),
                                   ctypes.POINTER(ctypes.c_int64)]
     L.dg_impl.argtypes = [_P]
+    L.dg_inject_stall.argtypes = [_P, ctypes.c_int64, _I]
+    L.dg_self_condition_scratch_bytes.argtypes = [cfgp, _I]
+    L.dg_self_condition_scratch_bytes.restype = ctypes.c_size_t
+    L.dg_self_condition.argtypes = [_P, _I, _P, _P, _P, _P, _P, _I, _P]
     L.dg_vocab_attention_static.argtypes = [_I, _I, _I, _I, ctypes.c_float, _P, _P, _P, _P, _P, _P]
     L.dg_partials_bytes.argtypes = [cfgp]
     L.dg_partials_bytes.restype = ctypes.c_size_t
@@ -92,7 +96,8 @@ def lib():
     for name in ("dg_init", "dg_begin_block", "dg_denoise_step", "dg_denoise_step_h",
                  "dg_denoise_block", "dg_read", "dg_write", "dg_profile", "dg_profile_read",
                  "dg_impl", "dg_free", "dg_vocab_attention_static", "dg_denoise_step_partial",
-                 "dg_denoise_step_finish", "dg_tc_schedule"):
+                 "dg_denoise_step_finish", "dg_tc_schedule", "dg_inject_stall",
+                 "dg_self_condition"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -210,6 +215,22 @@ def dg_denoise_step_finish(ctx, partials_ptr: int) -> None:
 
 def dg_impl(ctx) -> int:
     return _check(lib().dg_impl(ctx), ctx)
+
+
+def dg_self_condition_scratch_bytes(cfg: dg_config, d_ff: int) -> int:
+    return int(lib().dg_self_condition_scratch_bytes(ctypes.byref(cfg), d_ff))
+
+
+def dg_self_condition(ctx, d_ff: int, W1_ptr: int, b1_ptr: int, W2_ptr: int, b2_ptr: int,
+                      emb_ptr: int, emb_dtype: int, scratch_ptr: int) -> None:
+    """emb += W2 gelu(W1 sc + b1) + b2 on the context's stream (see include/dg.h)."""
+    _check(lib().dg_self_condition(ctx, d_ff, _P(W1_ptr), _P(b1_ptr), _P(W2_ptr), _P(b2_ptr),
+                                   _P(emb_ptr), emb_dtype, _P(scratch_ptr)), ctx)
+
+
+def dg_inject_stall(ctx, wait_limit_ns: int, stall: int) -> None:
+    """Failure-path testing: limit every bounded wait and make the hand-off unreachable."""
+    _check(lib().dg_inject_stall(ctx, int(wait_limit_ns), int(stall)), ctx)
 
 
 TC_SCHEDULE_FIELDS = ("CG", "W2", "RB", "n_vt", "n_ranges", "n_dt", "G", "n1", "n2", "ring",
@@ -331,6 +352,26 @@ class Denoiser:
 
     def step_finish(self, buf) -> None:
         dg_denoise_step_finish(self.ctx, buf.data_ptr())
+
+    # self-conditioning network ----------------------------------------------
+    def self_condition(self, W1, b1, W2, b2, emb):
+        """emb += W2 gelu(W1 sc + b1) + b2 with this context's sc (in place on emb).
+
+        W1 [d_ff, d] and W2 [d, d_ff] bf16, b1 [d_ff] and b2 [d] fp32, emb [C, d]
+        fp32 or bf16, all contiguous CUDA tensors; scratch is allocated here.
+        """
+        import torch
+
+        d_ff = W1.shape[0]
+        n = dg_self_condition_scratch_bytes(self.cfg, d_ff)
+        if n == 0:
+            raise DgError(DG_EUNSUPPORTED, "d and d_ff must be multiples of 128")
+        scratch = torch.empty(n, dtype=torch.uint8, device=self.device)
+        dg_self_condition(self.ctx, d_ff, W1.data_ptr(), b1.data_ptr(), W2.data_ptr(),
+                          b2.data_ptr(), emb.data_ptr(),
+                          DG_BF16 if emb.dtype == torch.bfloat16 else DG_F32, scratch.data_ptr())
+        self.stream.synchronize()
+        return emb
 
     def close(self) -> None:
         if getattr(self, "ctx", None) is not None:

@@ -35,7 +35,7 @@ struct Layout {
   size_t state = 0, scale = 0, target = 0, canvas = 0, argmax = 0, argmax_prev = 0, accept = 0,
          order = 0, prefix = 0, H = 0, mref = 0, rowstat = 0, h = 0, sc = 0,
          tstats = 0, zbuf = 0, partial = 0, tc = 0, sampled = 0, tsamp = 0, h_last = 0,
-         mref_last = 0, cstate = 0, emit = 0, total = 0;
+         mref_last = 0, cstate = 0, emit = 0, stage[2] = {0, 0}, total = 0;
   int canvases = 1;
   size_t tc_bytes = 0;
 };
@@ -103,7 +103,7 @@ int resolve_impl(const dg_config* c, char* why, size_t n) {
     return DG_IMPL_TC;
   }
   if (c->impl == DG_IMPL_SIMT) return DG_IMPL_SIMT;
-  return tc_ok ? DG_IMPL_TC : DG_IMPL_SIMT;
+  return tc_ok && tc_fits_device(c->C, shard_nv(c), c->d) ? DG_IMPL_TC : DG_IMPL_SIMT;
 }
 
 int make_layout(const dg_config* c, Layout* L, char* why, size_t n) {
@@ -134,6 +134,10 @@ int make_layout(const dg_config* c, Layout* L, char* why, size_t n) {
   L->canvases = c->canvases == 0 ? 1 : c->canvases;
   L->cstate = take(4 * 3 * (size_t)L->canvases);
   L->emit = take(4 * C);
+  // two staging slots for hidden states copied in from the host (the copy of
+  // step t+1 overlaps step t)
+  L->stage[0] = take(esz * C * d);
+  L->stage[1] = take(esz * C * d);
   if (impl == DG_IMPL_SIMT) {
     L->ntiles = (int)(V / 64);
     const size_t rt = (C + 63) / 64, dt = (d + 63) / 64;
@@ -188,6 +192,11 @@ struct dg_ctx {
   cudaGraph_t graph = nullptr;
   cudaGraphExec_t graph_exec = nullptr;
   cudaGraphConditionalHandle cond = 0;
+  // host-to-device copies of external hidden states: a copy stream, and per
+  // staging slot an event when its copy landed and one when its last reader ran
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t ev_copied[2] = {nullptr, nullptr}, ev_free[2] = {nullptr, nullptr};
+  int stage_slot = 0;
   // profiling
   bool h_ready = false;      // host mirror of DevState::h_ready for stepwise calls
   bool prof = false;
@@ -246,7 +255,7 @@ NextStandin next_standin(dg_ctx* ctx) {
 
 // The stand-in (or, for an external h, only m_ref) unless the last merge
 // already wrote it. Returns whether a kernel was launched, or a negative error.
-int prologue_if_needed(dg_ctx* ctx, bool standin, bool use_cond) {
+int prologue_if_needed(dg_ctx* ctx, bool standin, bool use_cond, const void* hsrc = nullptr) {
   const dg_config& c = ctx->cfg;
   const bool tc = ctx->L.impl == DG_IMPL_TC;
   unsigned* zero = nullptr;
@@ -260,15 +269,15 @@ int prologue_if_needed(dg_ctx* ctx, bool standin, bool use_cond) {
   DG_CK(launch_prologue(ctx->stream, c.dtype, ctx->st, ctx->E, ctx->target, ctx->canvas, ctx->sc,
                         ctx->h, c.C, c.V, c.d, c.seed, c.coef_target, c.coef_canvas,
                         standin_sigma(c), standin ? 1 : 0, ctx->scale_tab, c.max_steps,
-                        ctx->argmax_prev, tc ? ctx->mref : nullptr, zero, nzero));
+                        ctx->argmax_prev, tc ? ctx->mref : nullptr, zero, nzero, hsrc));
   return 1;
 }
 
-int launch_step(dg_ctx* ctx, bool standin, bool use_cond) {
+int launch_step(dg_ctx* ctx, bool standin, bool use_cond, const void* hsrc = nullptr) {
   const dg_config& c = ctx->cfg;
   cudaStream_t s = ctx->stream;
   const bool tc = ctx->L.impl == DG_IMPL_TC;
-  const int pro = prologue_if_needed(ctx, standin, use_cond);
+  const int pro = prologue_if_needed(ctx, standin, use_cond, hsrc);
   if (pro < 0) return pro;
   cudaEvent_t e0 = nullptr, e1 = nullptr;
   if (ctx->prof && !use_cond) {
@@ -478,11 +487,35 @@ int dg_denoise_step_h(dg_ctx* ctx, const void* h_src, int32_t h_on_host, int32_t
     return fail(ctx, DG_EUNSUPPORTED, "a vocabulary shard steps with dg_denoise_step_partial/_finish");
   const dg_config& c = ctx->cfg;
   const size_t bytes = (size_t)c.C * c.d * (c.dtype == DG_F32 ? 4 : 2);
-  DG_CK(cudaMemcpyAsync(ctx->h, h_src, bytes,
-                        h_on_host ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice,
-                        ctx->stream));
-  int rc = launch_step(ctx, false, false);
-  if (rc) return rc;
+  int rc;
+  if (h_on_host) {
+    // The copy runs on the context's copy stream into a staging slot, so that
+    // it overlaps the previous step's kernels; the step waits for it, and the
+    // prologue moves the slot into h. A slot is refilled only after the step
+    // that read it (two slots: step t+1's copy never waits for step t).
+    if (!ctx->copy_stream) {
+      DG_CK(cudaStreamCreateWithFlags(&ctx->copy_stream, cudaStreamNonBlocking));
+      for (int j = 0; j < 2; ++j) {
+        DG_CK(cudaEventCreateWithFlags(&ctx->ev_copied[j], cudaEventDisableTiming));
+        DG_CK(cudaEventCreateWithFlags(&ctx->ev_free[j], cudaEventDisableTiming));
+        DG_CK(cudaEventRecord(ctx->ev_free[j], ctx->stream));
+      }
+    }
+    const int slot = ctx->stage_slot;
+    ctx->stage_slot ^= 1;
+    void* stage = at<void>(ctx, ctx->L.stage[slot]);
+    DG_CK(cudaStreamWaitEvent(ctx->copy_stream, ctx->ev_free[slot], 0));
+    DG_CK(cudaMemcpyAsync(stage, h_src, bytes, cudaMemcpyHostToDevice, ctx->copy_stream));
+    DG_CK(cudaEventRecord(ctx->ev_copied[slot], ctx->copy_stream));
+    DG_CK(cudaStreamWaitEvent(ctx->stream, ctx->ev_copied[slot], 0));
+    rc = launch_step(ctx, false, false, stage);
+    if (rc) return rc;
+    DG_CK(cudaEventRecord(ctx->ev_free[slot], ctx->stream));
+  } else {
+    DG_CK(cudaMemcpyAsync(ctx->h, h_src, bytes, cudaMemcpyDeviceToDevice, ctx->stream));
+    rc = launch_step(ctx, false, false);
+    if (rc) return rc;
+  }
   if (canvas_host)
     DG_CK(cudaMemcpyAsync(canvas_host, ctx->canvas, sizeof(int32_t) * c.C, cudaMemcpyDeviceToHost,
                           ctx->stream));
@@ -520,6 +553,31 @@ int dg_denoise_block(dg_ctx* ctx, int32_t block, int32_t* out_dev, int32_t* step
     if (rc) return rc;
     *steps_host = hs.steps;
   }
+  return DG_OK;
+}
+
+size_t dg_self_condition_scratch_bytes(const dg_config* cfg, int32_t d_ff) {
+  Layout L;
+  char why[256];
+  if (make_layout(cfg, &L, why, sizeof(why)) != DG_OK) return 0;
+  if (cfg->d % 128 || d_ff < 128 || d_ff % 128 || d_ff > 65536) return 0;
+  return ffn_scratch_bytes(cfg->C, cfg->d, d_ff);
+}
+
+int dg_self_condition(dg_ctx* ctx, int32_t d_ff, const void* W1, const float* b1, const void* W2,
+                      const float* b2, void* emb, int32_t emb_dtype, void* scratch) {
+  if (!ctx) return fail(nullptr, DG_EINVAL, "ctx is NULL");
+  const dg_config& c = ctx->cfg;
+  if (c.d % 128 || d_ff < 128 || d_ff % 128 || d_ff > 65536)
+    return fail(ctx, DG_EUNSUPPORTED, "the network needs d and d_ff multiples of 128 (d_ff <= 65536)");
+  if (emb_dtype != DG_F32 && emb_dtype != DG_BF16) return fail(ctx, DG_EINVAL, "bad emb_dtype");
+  if (!W1 || !b1 || !W2 || !b2 || !emb || !scratch)
+    return fail(ctx, DG_EINVAL, "NULL weight, bias, embedding or scratch pointer");
+  if ((((uintptr_t)W1) | ((uintptr_t)W2) | ((uintptr_t)emb)) % 16 || ((uintptr_t)scratch) % kAlign)
+    return fail(ctx, DG_EINVAL, "W1, W2 and emb must be 16-byte aligned, scratch 256-byte aligned");
+  DG_CK(launch_self_condition(ctx->stream, c.C, c.d, d_ff, ctx->sc, W1, b1, W2, b2, emb,
+                              emb_dtype == DG_BF16 ? 1 : 0, scratch, &ctx->st->status));
+  ctx->launches += 3;
   return DG_OK;
 }
 
@@ -655,11 +713,39 @@ int dg_profile_read(dg_ctx* ctx, double* ms_total, int32_t* steps, int64_t* laun
 
 int dg_impl(const dg_ctx* ctx) { return ctx ? ctx->L.impl : DG_EINVAL; }
 
+int dg_inject_stall(dg_ctx* ctx, int64_t wait_limit_ns, int32_t stall) {
+  if (!ctx) return fail(nullptr, DG_EINVAL, "ctx is NULL");
+  if (ctx->L.impl != DG_IMPL_TC)
+    return fail(ctx, DG_EUNSUPPORTED, "only the tensor-core kernels have bounded waits");
+  if (wait_limit_ns < 0 || wait_limit_ns > 60ll * 1000000000ll || stall < 0)
+    return fail(ctx, DG_EINVAL, "wait limit must lie in [0, 60 s] and stall be >= 0");
+  ctx->tc_plan.timeout_ns = (unsigned long long)wait_limit_ns;
+  ctx->tc_plan.stall = (unsigned)stall;
+  // a graph captured with the old values would keep them
+  if (ctx->graph_ready) {
+    DG_CK(cudaStreamSynchronize(ctx->stream));
+    cudaGraphExecDestroy(ctx->graph_exec);
+    cudaGraphDestroy(ctx->graph);
+    ctx->graph_exec = nullptr;
+    ctx->graph = nullptr;
+    ctx->graph_ready = false;
+  }
+  return DG_OK;
+}
+
 int dg_free(dg_ctx* ctx) {
   if (!ctx) return DG_OK;
   if (ctx->graph_exec) cudaGraphExecDestroy(ctx->graph_exec);
   if (ctx->graph) cudaGraphDestroy(ctx->graph);
   for (cudaEvent_t e : ctx->ev) cudaEventDestroy(e);
+  if (ctx->copy_stream) {
+    cudaStreamSynchronize(ctx->copy_stream);
+    cudaStreamDestroy(ctx->copy_stream);
+    for (int j = 0; j < 2; ++j) {
+      if (ctx->ev_copied[j]) cudaEventDestroy(ctx->ev_copied[j]);
+      if (ctx->ev_free[j]) cudaEventDestroy(ctx->ev_free[j]);
+    }
+  }
   tc_plan_free(&ctx->tc_plan);
   delete ctx;
   return DG_OK;

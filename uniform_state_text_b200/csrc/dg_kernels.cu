@@ -65,7 +65,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) k_prologue(const DevState* st, const T* E,
     const int32_t* target, const int32_t* canvas, const float* sc, T* h, int C, int V, int d,
     uint64_t seed, float A, float B, float sigma, int standin, const float* scale_tab, int S,
-    const int32_t* argmax_prev, float* mref, unsigned* zero, int nzero) {
+    const int32_t* argmax_prev, float* mref, unsigned* zero, int nzero, const T* hsrc) {
   // Programmatic dependent launch: the previous step's kernels are complete
   // after this wait; the attention kernel may start its set-up meanwhile.
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -88,7 +88,8 @@ __global__ void __launch_bounds__(256) k_prologue(const DevState* st, const T* E
   const uint64_t pre = key_prefix(seed, (uint64_t)(uint32_t)st->block, kTagNoise + (uint64_t)t);
   float dc = 0.f, dp = 0.f;
   standin_row_part<T>(i, threadIdx.x, blockDim.x, E, tgt, can, prev, sc + (size_t)i * d,
-                      h + (size_t)i * d, d, pre, A, B, sigma, standin, mref != nullptr, &dc, &dp);
+                      h + (size_t)i * d, d, pre, A, B, sigma, standin, mref != nullptr, &dc, &dp,
+                      hsrc ? hsrc + (size_t)i * d : nullptr);
   if (!mref) return;
   __shared__ float red[2][32];
   for (int o = 16; o; o >>= 1) {
@@ -383,7 +384,8 @@ cudaError_t launch_prologue(cudaStream_t s, int dtype, const DevState* st, const
                             const int32_t* target, const int32_t* canvas, const float* sc,
                             void* h, int C, int V, int d, uint64_t seed, float A, float B, float sigma,
                             int standin, const float* scale_tab, int S,
-                            const int32_t* argmax_prev, float* mref, unsigned* zero, int nzero) {
+                            const int32_t* argmax_prev, float* mref, unsigned* zero, int nzero,
+                            const void* hsrc) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C);
   cfg.blockDim = dim3(256);
@@ -396,10 +398,11 @@ cudaError_t launch_prologue(cudaStream_t s, int dtype, const DevState* st, const
   if (dtype == 0)
     return cudaLaunchKernelEx(&cfg, k_prologue<float>, st, (const float*)E, target, canvas, sc,
                               (float*)h, C, V, d, seed, A, B, sigma, standin, scale_tab, S,
-                              argmax_prev, mref, zero, nzero);
+                              argmax_prev, mref, zero, nzero, (const float*)hsrc);
   return cudaLaunchKernelEx(&cfg, k_prologue<__nv_bfloat16>, st, (const __nv_bfloat16*)E, target,
                             canvas, sc, (__nv_bfloat16*)h, C, V, d, seed, A, B, sigma, standin,
-                            scale_tab, S, argmax_prev, mref, zero, nzero);
+                            scale_tab, S, argmax_prev, mref, zero, nzero,
+                            (const __nv_bfloat16*)hsrc);
 }
 
 cudaError_t launch_simt_attention(cudaStream_t s, int dtype, DevState* st, const void* h,

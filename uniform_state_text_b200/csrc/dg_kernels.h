@@ -87,7 +87,7 @@ cudaError_t launch_prologue(cudaStream_t s, int dtype, const DevState* st, const
                             void* h, int C, int V, int d, uint64_t seed, float A, float B, float sigma,
                             int standin, const float* scale_tab, int S,
                             const int32_t* argmax_prev, float* mref, unsigned* zero = nullptr,
-                            int nzero = 0);
+                            int nzero = 0, const void* hsrc = nullptr);
 
 cudaError_t launch_simt_attention(cudaStream_t s, int dtype, DevState* st, const void* h,
                                   const void* E, float* zbuf, TileStat* tstats, RowStat* rowstat,

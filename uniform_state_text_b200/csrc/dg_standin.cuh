@@ -38,8 +38,9 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float v[8]) {
 }
 
 // Threads tid, tid + nthr, ... of a row each take 8 consecutive elements of
-// h_i (d a multiple of 8). standin = 0 leaves h as written by the caller and
-// only forms the dot products. On return *dc and *dp hold this thread's
+// h_i (d a multiple of 8). standin = 0 takes h as the caller supplied it: from
+// hsrc when that is given (a staging copy, written through to h) or as already
+// stored in h, and only forms the dot products. On return *dc and *dp hold this thread's
 // partial sums of h_i . E[canvas_i] and h_i . E[prev_i] over the stored
 // (rounded) h (with_dots = false skips them).
 template <typename T>
@@ -47,7 +48,7 @@ __device__ __forceinline__ void standin_row_part(int i, int tid, int nthr, const
                                                  int can, int prev, const float* scrow, T* hrow,
                                                  int d, uint64_t pre, float A, float B,
                                                  float sigma, int standin, bool with_dots,
-                                                 float* dc, float* dp) {
+                                                 float* dc, float* dp, const T* hsrc = nullptr) {
   const T* Et = E + (size_t)tgt * d;
   const T* Ec = E + (size_t)can * d;
   const T* Ep = E + (size_t)prev * d;
@@ -71,6 +72,9 @@ __device__ __forceinline__ void standin_row_part(int i, int tid, int nthr, const
       // what the contraction reads is the stored (rounded) value
 #pragma unroll
       for (int j = 0; j < 8; ++j) hv[j] = to_f32(from_f32<T>(hv[j]));
+    } else if (hsrc) {
+      load8(hsrc + k0, hv);
+      store8(hrow + k0, hv);
     } else {
       load8(hrow + k0, hv);
     }

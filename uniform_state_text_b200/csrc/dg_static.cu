@@ -15,9 +15,14 @@
 // has to be cleared. Calls whose kernels overlap on the GPU (for example, on
 // two streams) race on the array: serialise them.
 //
-// Set-up: the first call on each device looks up the array's device address
-// with cudaGetSymbolAddress (with that device current) and caches it. Make
-// that first call before capturing any stream into a CUDA graph.
+// Set-up: every call looks up the array's device address with
+// cudaGetSymbolAddress (a host-side lookup, with the calling device current),
+// so a module that was loaded again -- after cudaDeviceReset, or after the
+// primary context was torn down and created again -- is found at its new
+// address. While the stream is being captured into a CUDA graph the lookup is
+// skipped and the address cached by the last call outside capture is used, so
+// the first call on each device must come before any stream capture (and a
+// device reset invalidates graphs captured earlier, as it does every graph).
 #include <cstdio>
 #include <mutex>
 
@@ -43,14 +48,19 @@ int fail(int code, const char* msg) {
   return code;
 }
 
-// Device address of the scratch array on the current device (looked up once).
-int scratch_address(void** out) {
+// Device address of the scratch array on the current device: looked up on
+// every call outside stream capture; during capture, the address the last
+// uncaptured call found.
+int scratch_address(cudaStream_t s, void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(DG_ECUDA, cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices) return fail(DG_EUNSUPPORTED, "device index too large");
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(s, &cap);
+  if (e != cudaSuccess) return fail(DG_ECUDA, cudaGetErrorString(e));
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_dg_scratch);
     if (e != cudaSuccess || p == nullptr) {
@@ -58,12 +68,20 @@ int scratch_address(void** out) {
       return fail(DG_ECUDA, "cudaGetSymbolAddress of the scratch array failed");
     }
     g_scratch_ptr[dev] = p;
+  } else if (!g_scratch_ptr[dev]) {
+    return fail(DG_EINVAL, "the first call on a device must come before any stream capture");
   }
   *out = g_scratch_ptr[dev];
   return DG_OK;
 }
 
-size_t al(size_t x) { return (x + 255) / 256 * 256; }
+// Every piece carved from the array starts on a kPiece boundary of the
+// 256-byte aligned array; the CUDA-core kernels' vector accesses to their
+// scratch (float4 logits, 16-byte statistics records) need 16 bytes.
+constexpr size_t kPiece = 256;
+size_t al(size_t x) { return (x + kPiece - 1) / kPiece * kPiece; }
+static_assert(kPiece % 16 == 0, "pieces must stay 16-byte aligned for vector accesses");
+static_assert(DG_STATIC_SCRATCH_BYTES % kPiece == 0, "the array holds whole pieces");
 
 // Per-call loop state the shared kernels read: step 0, not done, scale table
 // of one entry.
@@ -106,7 +124,7 @@ extern "C" int dg_vocab_attention_static(int32_t C, int32_t V, int32_t d, int32_
     return fail(DG_EUNSUPPORTED, msg);
   }
   void* base = nullptr;
-  int rc = scratch_address(&base);
+  int rc = scratch_address(static_cast<cudaStream_t>(stream), &base);
   if (rc) return rc;
   char* p = static_cast<char*>(base);
   size_t off = 0;

@@ -15,9 +15,12 @@
 //     stand-in h) replaces the running maximum: probabilities are
 //     P = exp(z - m_ref). With no running maximum there is nothing to agree on
 //     between CTAs, so the P.E contraction can run on other SMs than the h.E^T
-//     contraction. The exact maximum is tracked alongside; a row whose maximum
-//     exceeds m_ref by more than 64 (P could overflow) is recomputed exactly by
-//     the merge kernel below. Entropy and argmax never depend on m_ref.
+//     contraction. The exact maximum is tracked alongside; if a row's maximum
+//     exceeds m_ref by more than 64 (P could overflow), the first pass replaces
+//     that row's m_ref by its exact maximum and a second launch of the same
+//     kernel (the redo pass, which returns at once when no row needs it) runs
+//     the step again on the tensor cores. Entropy and argmax never depend on
+//     m_ref.
 //   * One persistent kernel per step, two CTA roles:
 //       G1 units: S = h E_tile^T for all rows x 256 vocabulary entries (K = d),
 //                taken from a dynamic tile queue, into a double-buffered TMEM
@@ -47,6 +50,7 @@
 #include <cstring>
 
 #include "dg_tc.h"
+#include "dg_tcgen05.cuh"
 #include "dg_sampler.cuh"
 #include "dg_standin.cuh"
 
@@ -75,12 +79,12 @@ template <int CG> struct Pipe {
   static constexpr uint32_t STAGE_W2 = A_BYTES + 2 * (B_BYTES / CG);
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 512;
 };
-constexpr unsigned long long TIMEOUT_NS = 2000000000ull;   // 2 s
+constexpr unsigned long long TIMEOUT_NS = 2000000000ull;   // 2 s: the default wait limit
 
 struct Params {
   int C, V, d, RB, n_vt, n_ranges, n_dt, G, n1, tiles_per_range, S;
   int W2;                    // G2 accumulators per CTA: a G2 unit owns W2*256 columns of d
-  const float* mref;
+  float* mref;                 // per-row logit reference; the first pass raises a low one
   const float* scale_tab;
   float* Opart;              // [G][C][d]
   __nv_bfloat16* P;          // [RING][C][BN]: ring of P tiles
@@ -90,6 +94,15 @@ struct Params {
   unsigned* g1_next;         // next G1 item to hand out (dynamic schedule)
   DevState* st;
   unsigned long long* trace;   // [grid][32] wait-time counters (DG_TC_TRACE builds only)
+  // Failure-path testing (dg_inject_stall): the limit of every bounded wait,
+  // and an amount added to the hand-off target the G2 producers wait for
+  // (non-zero: a target nothing reaches, so that wait runs out).
+  unsigned long long timeout_ns;
+  unsigned stall;
+  // 0: the step's first pass; 1: the redo pass, which runs only if the first
+  // pass raised its redo flag (redo_in) and then uses its own counter set.
+  int pass;
+  const int* redo_in;
   TcStat* tstats2;             // [C][2 * n_vt] half-tile statistics
   TcSamp* tsamp;               // [C][2 * n_vt] best z + G (multinomial draw), or nullptr
   uint64_t seed;               // keys the draw's Gumbel variates
@@ -147,39 +160,6 @@ __device__ __forceinline__ void max_key_decode(unsigned long long key, float* v,
 #define TR_STORE(slot, v) ((void)0)
 #endif
 
-// ---------------------------------------------------------------------------
-// PTX wrappers.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ uint64_t gtimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 __device__ __forceinline__ void raise_abort(const Params& p) {
   atomicExch(p.abort_flag, 1);
   atomicCAS(&p.st->status, 0, -4 /* DG_ETIMEOUT */);
@@ -196,26 +176,9 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Par
     if (mbar_try(bar, parity)) return true;
     if ((n & 63) == 0) {
       if (check_abort && *(volatile int*)p.abort_flag) return false;
-      if (gtimer() - t0 > TIMEOUT_NS) { raise_abort(p); return false; }
+      if (gtimer() - t0 > p.timeout_ns) { raise_abort(p); return false; }
     }
   }
-}
-
-__device__ __forceinline__ unsigned ld_acquire(const unsigned* ptr) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
-  return v;
-}
-__device__ __forceinline__ void red_release_add(unsigned* ptr, unsigned v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
-}
-// Relaxed add: for counters whose only meaning is "my reads of this data have
-// completed" (the reads finished before the add is issued), no release needed.
-__device__ __forceinline__ void red_relaxed_add(unsigned* ptr, unsigned v) {
-  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // Bounded wait until a global counter reaches target.
@@ -227,169 +190,8 @@ __device__ __noinline__ bool counter_wait(const unsigned* ptr, unsigned target, 
     __nanosleep(64);
     if ((n & 15) == 0) {
       if (*(volatile int*)p.abort_flag) return false;
-      if (gtimer() - t0 > TIMEOUT_NS) { raise_abort(p); return false; }
+      if (gtimer() - t0 > p.timeout_ns) { raise_abort(p); return false; }
     }
-  }
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
-      : "memory");
-}
-
-// L2 eviction policies for TMA loads: G1 marks the E tiles (and h) it reads as
-// evict_last so that they are still in L2 when the G2 CTAs read the same
-// tiles; G2 reads them evict_first (they are dead afterwards).
-__device__ __forceinline__ uint64_t policy_evict_last() {
-  uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
-__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                                 int x, int y, uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(pol)
-      : "memory");
-}
-
-// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
-__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
-}
-// Instruction descriptor: bf16 x bf16 -> f32, A K-major, B K- or MN-major.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn_major << 16) |
-         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::
-                   "r"(smem_u32(bar))
-               : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// 32 lanes x 32 columns of fp32 from TMEM: thread t of the warp gets its lane's columns.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
-// ---------------------------------------------------------------------------
-// CTA-pair helpers (CG = 2: two CTAs of a cluster share one MMA of M = 256).
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
-                   "memory");
-}
-// Address of the same shared variable in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
-// Relaxed arrive: signals only that this warp's TMEM reads are done (ordered by
-// tcgen05.fence::before_thread_sync), without waiting for its global stores.
-__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-// TMA load whose completion is counted on the pair leader's barrier.
-__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                                 int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar) & 0xFEFFFFFFu), "r"(x), "r"(y)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_2d_pair_hint(void* dst, const CUtensorMap* map,
-                                                      uint64_t* bar, int x, int y, uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar) & 0xFEFFFFFFu), "r"(x), "r"(y),
-      "l"(pol)
-      : "memory");
-}
-template <int CG>
-__device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
-                                         int y, uint64_t pol) {
-  if constexpr (CG == 2) tma_load_2d_pair_hint(dst, map, bar, x, y, pol);
-  else tma_load_2d_hint(dst, map, bar, x, y, pol);
-}
-template <int CG>
-__device__ __forceinline__ void mma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                    uint32_t accumulate) {
-  if constexpr (CG == 2) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-        : "memory");
-  } else {
-    mma_bf16(d_tmem, a, b, idesc, accumulate);
-  }
-}
-// Arrive on `bar` in every CTA of the group once this thread's MMAs complete.
-template <int CG>
-__device__ __forceinline__ void commit(uint64_t* bar) {
-  if constexpr (CG == 2) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-        " [%0], %1;" ::"r"(smem_u32(bar)), "h"((uint16_t)3)
-        : "memory");
-  } else {
-    mma_commit(bar);
   }
 }
 
@@ -398,11 +200,6 @@ __device__ __forceinline__ void commit(uint64_t* bar) {
 // CG = 2: CTA pairs, M = 256 rows (both row blocks), each CTA stages its own
 // 128 rows of A and half of B; the pair leader (rank 0) issues the MMAs.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 // G1 items are handed out dynamically: the producer of the pair leader (or of
 // the single CTA) takes the next item from a global counter and publishes it
@@ -526,7 +323,16 @@ __device__ __noinline__ void g1_finish(const Params& p, int ng1, unsigned char* 
         rs.m = mref_i; rs.Z = Z; rs.pad[0] = best; rs.pad[1] = 0.f;
         p.rowstat[i] = rs;
         const float gap = best - mref_i;
-        if (!(gap <= p.redo_gap) || !(Z > 0.f) || !(Z < INFINITY)) atomicOr(p.redo_flag, 1);
+        if (!(gap <= p.redo_gap) || !(Z > 0.f) || !(Z < INFINITY)) {
+          // P of this row could overflow (or its sums are not finite): the
+          // redo pass takes the row's exact maximum as its reference. Every G1
+          // item is done, so no epilogue reads m_ref any more in this pass.
+          atomicOr(p.redo_flag, 1);
+          if (p.pass == 0) {
+            p.mref[i] = best;
+            atomicAdd(&p.st->redo, 1);
+          }
+        }
       }
     }
     __syncthreads();
@@ -566,6 +372,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int STAGES = w2 ? Pipe<CG>::STAGES_W2 : Pipe<CG>::STAGES;
   const uint32_t STAGE_BYTES = w2 ? Pipe<CG>::STAGE_W2 : Pipe<CG>::STAGE;
   const int HALF = (is_g1_unit(p, CG) ? BN : BN * p.W2) / 2;   // columns per epilogue warp
+  if (p.pass == 1) {
+    // The redo pass: after the first pass has completed, every thread reads
+    // its redo flag; with no row to redo the whole grid returns before any
+    // set-up, and lets the next kernel launch at once.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (*(volatile const int*)p.redo_in == 0) {
+      asm volatile("griddepcontrol.launch_dependents;");
+      return;
+    }
+  }
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -697,7 +513,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int vt = r * p.tiles_per_range + kc / (BN / BK);
             if (kc % (BN / BK) == 0) {
               TR_T0();
-              if (!counter_wait(&p.ready[vt], ready_target, p)) { ok = false; break; }
+              if (!counter_wait(&p.ready[vt], ready_target + p.stall, p)) { ok = false; break; }
               TR_ADD(w_ctr);
               fence_proxy_async_global();
             }
@@ -844,7 +660,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int buf = n & 1;
         {
           TR_T0();
-          if (!mbar_wait(&acc_full[buf], (n >> 1) & 1, p)) break;
+          // every lane waits; the warp goes on only if all of them saw the
+          // accumulator (an abort seen by some lanes stops the whole warp
+          // before its warp-wide TMEM loads)
+          const bool got = mbar_wait(&acc_full[buf], (n >> 1) & 1, p);
+          if (!__all_sync(0xffffffffu, got)) break;
           TR_ADD(w_acc);
         }
         TR_T0();
@@ -950,7 +770,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       float* orow = p.Opart + ((size_t)g * p.C + row) * p.d + (size_t)dt * BN * p.W2 + c0;
       bool ok = true;
       if (has_work) {
-        ok = mbar_wait(&acc_full[0], 0, p);
+        ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[0], 0, p));   // warp-uniform, as in G1
         tc_fence_after();
       }
       if (ok) {
@@ -1422,7 +1242,8 @@ TcLayout tc_layout(int C, int V, int d, int sms) {
     if (t < best) { best = t; L.G = G; L.n1 = n1; L.n2 = n2; }
   }
   size_t off = 0;
-  L.counters = off; off = al(off + sizeof(unsigned) * (2 * (size_t)L.n_vt + 64));
+  // two sets of hand-off counters: the first pass's and the redo pass's
+  L.counters = off; off = al(off + sizeof(unsigned) * 2 * (2 * (size_t)L.n_vt + 64));
   L.P = off; off = al(off + (size_t)tc::RING * C * tc::BN * 2);
   L.Opart = off; off = al(off + (size_t)(L.G > 0 ? L.G : 1) * C * d * 4);
   L.trace = off; off = al(off + (size_t)256 * 32 * 8);
@@ -1461,12 +1282,23 @@ bool encode(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, ui
 
 }  // namespace
 
+bool tc_encode_2d_bf16(void* map, const void* base, uint64_t inner, uint64_t outer,
+                       uint32_t box_inner, uint32_t box_outer) {
+  return encode(static_cast<CUtensorMap*>(map), base, inner, outer, box_inner, box_outer);
+}
+
 bool tc_supported(int C, int V, int d) {
   return (C == 128 || C == 256) && d % 256 == 0 && d >= 256 && d <= 8192 && V % tc::KV2 == 0 &&
          V >= tc::KV2 && V <= (1 << 24);
 }
 
 int tc_stat_tiles(int, int V, int) { return V / tc::BN; }
+
+bool tc_fits_device(int C, int V, int d) {
+  if (!tc_supported(C, V, d)) return false;
+  const TcLayout L = tc_layout(C, V, d, device_sms());
+  return L.G >= 1 && L.n1 >= 1;
+}
 
 bool tc_schedule_info(int C, int V, int d, int sms, int32_t* out) {
   if (!tc_supported(C, V, d) || sms < 2) return false;
@@ -1482,7 +1314,7 @@ size_t tc_workspace_bytes(int C, int V, int d) { return tc_layout(C, V, d, devic
 
 size_t tc_draw_bytes(int C, int V, int) { return sizeof(TcSamp) * (size_t)C * 2 * (V / tc::BN); }
 
-int tc_launches(const TcPlan&) { return 1; }
+int tc_launches(const TcPlan&) { return 2; }
 
 template <int CG, bool DRAW>
 cudaError_t launch_kernel(cudaStream_t s, int units, const CUtensorMap* maps, const tc::Params& prm) {
@@ -1558,6 +1390,11 @@ int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, void* w
   E = static_cast<const __nv_bfloat16*>(E) + (size_t)v0 * d;
   p->num_sms = device_sms();
   TcLayout L = tc_layout(C, V, d, p->num_sms);
+  if (L.G < 1 || L.n1 < 1) {
+    snprintf(err, errn, "the tensor-core kernels need more SMs than this device offers (%d)",
+             p->num_sms);
+    return -5;
+  }
   p->grid = L.n1 + L.n2;
   p->ws = ws;
   char* base = static_cast<char*>(ws);
@@ -1587,23 +1424,26 @@ void tc_plan_free(TcPlan* p) { p->ready = false; }
 void tc_counters(const TcPlan& p, unsigned** ptr, int* count) {
   TcLayout L = tc_layout(p.C, p.V, p.d, p.num_sms);
   *ptr = reinterpret_cast<unsigned*>(static_cast<char*>(p.ws) + L.counters);
-  *count = 2 * L.n_vt + 64;
+  *count = 2 * (2 * L.n_vt + 64);
 }
 
 tc::Params base_params(const TcPlan& pl, const TcLayout& L, DevState* st, const float* mref,
                        const float* scale_tab, int S, TileStat* tstats, void* ws,
                        const DrawArgs& draw, float* H, int32_t* argmax, RowStat* rowstat,
-                       float redo_gap, const SamplerArgs& sa) {
+                       float redo_gap, const SamplerArgs& sa, int pass = 0) {
   char* base = static_cast<char*>(ws);
   tc::Params prm;
   prm.C = pl.C; prm.V = pl.Vg; prm.d = pl.d; prm.RB = L.RB; prm.n_vt = L.n_vt;
   prm.n_ranges = L.n_ranges; prm.n_dt = L.n_dt; prm.G = L.G; prm.n1 = L.n1; prm.W2 = L.W2;
   prm.tiles_per_range = tc::KV2 / tc::BN; prm.S = S;
-  prm.mref = mref; prm.scale_tab = scale_tab;
+  prm.mref = const_cast<float*>(mref); prm.scale_tab = scale_tab;
   prm.tstats2 = reinterpret_cast<TcStat*>(tstats);
   prm.Opart = reinterpret_cast<float*>(base + L.Opart);
   prm.P = reinterpret_cast<__nv_bfloat16*>(base + L.P);
-  unsigned* ctr = reinterpret_cast<unsigned*>(base + L.counters);
+  unsigned* ctr0 = reinterpret_cast<unsigned*>(base + L.counters);
+  unsigned* ctr = ctr0 + (size_t)pass * (2 * L.n_vt + 64);     // this pass's counter set
+  prm.pass = pass;
+  prm.redo_in = reinterpret_cast<const int*>(ctr0 + 2 * L.n_vt + 5);   // the first pass's flag
   prm.ready = ctr;
   prm.consumed = ctr + L.n_vt;
   prm.abort_flag = reinterpret_cast<int*>(ctr + 2 * L.n_vt);
@@ -1625,6 +1465,8 @@ tc::Params base_params(const TcPlan& pl, const TcLayout& L, DevState* st, const 
   prm.partial = 0;
   prm.pzs = nullptr;
   prm.pkeys = nullptr;
+  prm.timeout_ns = pl.timeout_ns ? pl.timeout_ns : tc::TIMEOUT_NS;
+  prm.stall = pl.stall;
   return prm;
 }
 
@@ -1647,8 +1489,13 @@ cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, 
   (void)h; (void)E;
   TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
   const tc::Params prm = base_params(pl, L, st, mref, scale_tab, S, tstats, ws, draw, H, argmax,
-                                     rowstat, redo_gap, sa);
-  return launch_params(s, pl, L, prm);
+                                     rowstat, redo_gap, sa, 0);
+  cudaError_t e = launch_params(s, pl, L, prm);
+  if (e != cudaSuccess) return e;
+  // the redo pass (returns at once unless a row's reference was too low)
+  const tc::Params prm2 = base_params(pl, L, st, mref, scale_tab, S, tstats, ws, draw, H, argmax,
+                                      rowstat, redo_gap, sa, 1);
+  return launch_params(s, pl, L, prm2);
 }
 
 size_t tc_partials_bytes(int C, int d) {

@@ -17,9 +17,18 @@ struct TcPlan {
   int num_sms = 0;
   int grid = 0;
   void* ws = nullptr;
+  // Failure-path testing (dg_inject_stall): 0 = the default 2 s wait limit.
+  unsigned long long timeout_ns = 0;
+  unsigned stall = 0;
 };
 
 bool tc_supported(int C, int V, int d);
+// A 2-D tensor map (map: 128 bytes, 64-byte aligned) over a row-major bf16
+// [outer][inner] array, box [box_outer][box_inner], 128-byte swizzle.
+bool tc_encode_2d_bf16(void* map, const void* base, uint64_t inner, uint64_t outer,
+                       uint32_t box_inner, uint32_t box_outer);
+// tc_supported, and the current device has SMs enough for both CTA roles.
+bool tc_fits_device(int C, int V, int d);
 // The work split tc_layout picks on a GPU with `sms` SMs, in the order
 // dg_tc_schedule documents; false if the kernels do not cover the shape.
 constexpr int kTcScheduleValues = 11;
@@ -31,9 +40,13 @@ int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, void* w
                  size_t errn, int v0, int Vg);
 void tc_plan_free(TcPlan* p);
 int tc_launches(const TcPlan& p);   // kernels per launch_tc_attention call
-// The attention kernel; its G1 CTAs also merge the rows' statistics into H,
-// argmax and rowstat and run the sampler, unless a row needs the exact
-// recomputation (then the merge kernel does both).
+// The attention kernel, launched twice: the first pass's G1 CTAs also merge
+// the rows' statistics into H, argmax and rowstat and run the sampler, unless
+// a row's largest logit overshot its reference m_ref; then they raise that
+// row's m_ref to its exact maximum and the second launch (the redo pass, which
+// otherwise returns at once) runs the step again and samples. Only rows whose
+// sums are still not finite after that go to the merge kernel's CUDA-core
+// recomputation.
 cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& p, DevState* st, const void* h,
                                 const void* E, const float* mref, const float* scale_tab,
                                 int S, TileStat* tstats, void* ws,
@@ -72,6 +85,13 @@ cudaError_t launch_tc_finish(cudaStream_t s, const TcPlan& p, DevState* st,
                              float* sc, float redo_gap, const void* h, const void* E,
                              const float* scale_tab, int S, const SamplerArgs& sa,
                              const NextStandin& nx);
+// Self-conditioning network (dg_ffn.cu): emb += W2 gelu(W1 sc + b1) + b2 on
+// tensor cores; scratch holds sc as bf16 [C][d] and the hidden activations
+// [C][dff] (ffn_scratch_bytes). Needs d and dff multiples of 128.
+size_t ffn_scratch_bytes(int C, int d, int dff);
+cudaError_t launch_self_condition(cudaStream_t s, int C, int d, int dff, const float* sc,
+                                  const void* W1, const float* b1, const void* W2, const float* b2,
+                                  void* emb, int emb_bf16, void* scratch, int* status);
 // Hand-off counters the prologue zeroes before every step.
 void tc_counters(const TcPlan& p, unsigned** ptr, int* count);
 // Per-range-group partials of O = P E that the merge sums.
