@@ -123,3 +123,13 @@ def test_null_context_calls_fail_cleanly(lib):
     assert lib.dg_denoise_step(None, None) == dg.DG_EINVAL
     assert lib.dg_read(None, 0, None) == dg.DG_EINVAL
     assert lib.dg_free(None) == dg.DG_OK
+    assert lib.dg_inject_stall(None, 0, 0) == dg.DG_EINVAL
+    assert lib.dg_self_condition(None, 128, None, None, None, None, None, 0, None) == dg.DG_EINVAL
+
+
+def test_self_condition_scratch_bytes(lib):
+    assert dg.dg_self_condition_scratch_bytes(_cfg(), 256) == 0            # d = 64
+    cfg = _cfg(d=1024)
+    assert dg.dg_self_condition_scratch_bytes(cfg, 100) == 0               # d_ff % 128 != 0
+    n = dg.dg_self_condition_scratch_bytes(cfg, 256)
+    assert n >= cfg.C * cfg.d * 2 + cfg.C * 256 * 2 and n % 256 == 0

@@ -121,3 +121,71 @@ def test_vocab_parallel_exchange_two_gloo_ranks():
     a, b = _partials(0), _partials(1)
     dg.reduce_partials_local([a, b], C_X, D_X)
     assert torch.equal(a, got) and torch.equal(b, got)
+
+
+# --- bench.py --parallel vocab: the per-step orchestration on two gloo ranks ---------
+class _FakeShard:
+    """Stands in for a vocabulary-shard Denoiser: its partial step writes this
+    rank's partial row results, its finish records what the exchange left."""
+
+    def __init__(self, rank):
+        self.rank = rank
+        self.calls = []
+        self.seen = None
+
+    def step_partial(self, buf):
+        self.calls.append("partial")
+        buf.copy_(_partials(self.rank))
+
+    def step_finish(self, buf):
+        self.calls.append("finish")
+        self.seen = buf.clone()
+
+
+def _vocab_loop_rank(rank, world, port, q):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        den = _FakeShard(rank)
+        buf = torch.zeros_like(_partials(0))
+        for _ in range(2):
+            bench.vocab_parallel_loop(den, buf, C_X, D_X)
+        q.put((rank, den.calls, den.seen.tolist()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_vocab_parallel_bench_loop_two_gloo_ranks():
+    """Each step: the shard's partial step, the exchange, then the finish, on every
+    rank; the finish sees the reduction of both ranks' partials."""
+    import torch
+
+    import uniform_state_text_b200 as dg
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_vocab_loop_rank, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = {r: (calls, seen) for r, calls, seen in (q.get(timeout=10) for _ in range(world))}
+    for r in range(world):
+        assert res[r][0] == ["partial", "finish"] * 2
+    assert res[0][1] == res[1][1]
+    a, b = _partials(0), _partials(1)
+    dg.reduce_partials_local([a, b], C_X, D_X)
+    assert torch.equal(torch.tensor(res[0][1], dtype=torch.int64), a)
+
+
+def test_strong_scaling_rate():
+    import bench
+    assert bench.shared_canvas_rate(100, 50.0) == pytest.approx(2000.0)

@@ -15,7 +15,7 @@ import synthetic
 import uniform_state_text_b200 as dg
 from oracle import method as M
 from parity import (Tally, check_sampler_exact, compare_attention, compare_draw, h_agreement,
-                    near_tie_flags)
+                    near_tie_flags, standin_terms)
 
 pytestmark = pytest.mark.gpu
 
@@ -59,7 +59,14 @@ def _np(t):
         else t.detach().cpu().numpy()
 
 
-def step_and_compare(den, w, E32, tally: Tally, prev_amax=None):
+def step_and_compare(den, w, E32, tally: Tally, prev_amax=None, do_step=None, peers=(),
+                     h_given=None):
+    """One GPU step (den.step(), or do_step()) compared with the oracle.
+
+    peers: other contexts stepped by do_step (vocabulary shards) that must end
+    in exactly den's state. h_given: the step's hidden state was supplied by the
+    caller (compared bit for bit) instead of the stand-in.
+    """
     st0 = den.state()
     if st0["done"]:
         return False
@@ -69,7 +76,10 @@ def step_and_compare(den, w, E32, tally: Tally, prev_amax=None):
     canvas_in = _np(den.read(dg.DG_CANVAS)).astype(np.int64)
     sc_in = _np(den.read(dg.DG_SC)).astype(np.float64)
     target = _np(den.read(dg.DG_TARGET)).astype(np.int64)
-    den.step()
+    if do_step is None:
+        den.step()
+    else:
+        do_step()
     h = _np(den.read(dg.DG_HIDDEN)).astype(np.float64)
     H = _np(den.read(dg.DG_ENTROPY))
     amax = _np(den.read(dg.DG_ARGMAX)).astype(np.int64)
@@ -81,9 +91,19 @@ def step_and_compare(den, w, E32, tally: Tally, prev_amax=None):
     st1 = den.state()
     out["state"] = st1
     assert st1["status"] == 0
+    for peer in peers:
+        assert peer.state() == st1
+        for k in (dg.DG_HIDDEN, dg.DG_ENTROPY, dg.DG_ARGMAX, dg.DG_SC, dg.DG_CANVAS, dg.DG_ACCEPT,
+                  dg.DG_ORDER, dg.DG_PREFIX, dg.DG_CANVAS_STATE, dg.DG_EMIT):
+            assert np.array_equal(_np(peer.read(k)), _np(den.read(k))), k
+        if multinomial:
+            assert np.array_equal(_np(peer.read(dg.DG_SAMPLED)), sampled)
     t, b = st0["t"], st0["block"]
-    h_orc = M.standin_hidden(w, E32, target, canvas_in, sc_in, b, t)
-    assert h_agreement(w, h, h_orc) < 2e-3
+    if h_given is None:
+        h_orc = M.standin_hidden(w, E32, target, canvas_in, sc_in, b, t)
+        assert h_agreement(w, h, h_orc, standin_terms(w, E32, target, canvas_in, sc_in, h_orc)) < 2e-3
+    else:
+        assert np.array_equal(h, np.asarray(h_given, np.float64))
     T = M.temperature(t, w.max_steps, w.T_start, w.T_end)
     if multinomial:
         att = M.vocab_attention(h, E32, w.logit_scale / T, gumbel_key=(w.seed, b, t))
@@ -133,18 +153,34 @@ def step_and_compare(den, w, E32, tally: Tally, prev_amax=None):
     return True
 
 
-def run_teacher_forced(den, w, E32, max_steps=None):
+def run_teacher_forced(den, w, E32, max_steps=None, do_step=None, peers=()):
     tally = Tally()
     n = 0
     while max_steps is None or n < max_steps:
         if den.state()["done"]:
             break
         pre = _np(den.read(dg.DG_ARGMAX)).astype(np.int64) if den.state()["has_prev"] else None
-        if not step_and_compare(den, w, E32, tally, pre):
+        if not step_and_compare(den, w, E32, tally, pre, do_step=do_step, peers=peers):
             break
         n += 1
     tally.check_budget()
     return tally
+
+
+def shard_stepper(shards, bufs, w):
+    """One step of a vocabulary-parallel canvas: every shard's partial step, the
+    exchange (reduced in-process here; a multi-GPU run does it with NCCL), then
+    every shard's finish."""
+    def do_step():
+        for s, b in zip(shards, bufs):
+            s.step_partial(b)
+            s.stream.synchronize()
+        dg.reduce_partials_local(bufs, w.C, w.d)
+        torch.cuda.synchronize()
+        for s, b in zip(shards, bufs):
+            s.step_finish(b)
+            s.stream.synchronize()
+    return do_step
 
 
 # ----------------------------------------------------------------------------
@@ -231,7 +267,10 @@ def test_batched_canvases_teacher_forced(impl, canvases):
 def test_batched_canvases_with_draw_and_shards():
     """Two canvases per step under the multinomial rule, stepped as two
     vocabulary shards: the options compose (per-canvas sampler after the
-    cross-shard reduction), against the oracle."""
+    cross-shard reduction). Every step is compared with the oracle like a
+    whole-vocabulary step (hidden state, entropy, argmax, sc, draw, sort,
+    prefix sums, accept mask, canvas, per-canvas stop), and both shards must end
+    in the same state bit for bit."""
     w = synthetic.STRESS_PARTIAL.replace(canvases=2, tau=0.5 * 128 * np.log(2), token_rule=1,
                                          max_steps=4, fixed_steps=1)
     Eg, E32 = embedding(w)
@@ -239,27 +278,9 @@ def test_batched_canvases_with_draw_and_shards():
     shards = [dg.Denoiser(w, Eg, impl=dg.DG_IMPL_TC, shard=(0, half)),
               dg.Denoiser(w, Eg, impl=dg.DG_IMPL_TC, shard=(half, half))]
     bufs = [s.partials() for s in shards]
-    st = M.begin_block(w, 0)
-    for _ in range(w.max_steps):
-        for s, b in zip(shards, bufs):
-            s.step_partial(b)
-            s.stream.synchronize()
-        dg.reduce_partials_local(bufs, w.C, w.d)
-        torch.cuda.synchronize()
-        for s, b in zip(shards, bufs):
-            s.step_finish(b)
-            s.stream.synchronize()
-        h = _np(shards[0].read(dg.DG_HIDDEN)).astype(np.float64)
-        rec = M.step(w, E32, st, h=h)
-        canvas = _np(shards[0].read(dg.DG_CANVAS)).astype(np.int64)
-        assert np.array_equal(canvas, _np(shards[1].read(dg.DG_CANVAS)))
-        # the trajectory is teacher-forced through h; tokens agree except on near-ties
-        ties = (rec.att.smargin < 1e-3) | (rec.att.margin < 1e-3)
-        bad = np.flatnonzero((canvas != rec.canvas_out) & ~ties)
-        assert bad.size <= max(1, w.C // 1000), bad[:8]
-        st.canvas = canvas
-        cst = _np(shards[0].read(dg.DG_CANVAS_STATE)).reshape(3, 2)
-        assert np.array_equal(cst[1] != 0, st.done_c)
+    tally = run_teacher_forced(shards[0], w, E32, do_step=shard_stepper(shards, bufs, w),
+                               peers=shards[1:])
+    assert tally.steps == w.max_steps and tally.draws_off_mode > 0
     for s in shards:
         s.close()
 
@@ -384,22 +405,61 @@ def test_block_diffusion_full_size(impl):
     den.close()
 
 
+def _external_h(w, Eg, canvas, seed):
+    """A hidden state that is not the stand-in's: row i leans on a random token
+    with a strength rising from 0 to 12 along the canvas, plus isotropic noise,
+    so the rows range from nearly uniform softmaxes to nearly one-hot ones and
+    the canvas token's logit (the tensor-core path's reference) is often far
+    below the row's largest logit."""
+    g = torch.Generator().manual_seed(seed)
+    tok = torch.randint(0, w.V, (w.C,), generator=g)
+    lean = torch.linspace(0.0, 12.0, w.C)[:, None]
+    noise = torch.randn(w.C, w.d, generator=g) * (0.5 / np.sqrt(w.d))
+    h = lean * Eg[tok.cuda()].float().cpu() + noise
+    return h.to(torch.bfloat16).contiguous()
+
+
 @pytest.mark.parametrize("impl", IMPLS)
-def test_external_hidden_state_from_host(impl):
-    """dg_denoise_step_h with the hidden state in pinned host memory equals the stand-in step."""
-    w = synthetic.SMALL
+@pytest.mark.parametrize("name", ["canvas_c256_v32768_d1024_bf16",
+                                  "canvas_c256_v262144_d2048_bf16"])
+def test_external_hidden_state_from_host(impl, name):
+    """dg_denoise_step_h with a caller's hidden state (not the stand-in) in
+    pinned host memory, two steps, against the oracle: entropy, argmax and sc
+    of that h, then the sampler (sort, prefix sums, acceptance, re-noise), the
+    canvas copied back to pinned host memory, and the stop state."""
+    w = synthetic.WORKLOADS[name].replace(fixed_steps=1)
     den, E32 = make(w, impl)
-    den.step()
-    h = den.read(dg.DG_HIDDEN)
-    ref = {k: _np(den.read(k)) for k in (dg.DG_ENTROPY, dg.DG_ARGMAX, dg.DG_CANVAS, dg.DG_SC)}
-    den.begin_block(0)
-    host_h = h.cpu().pin_memory()
+    Eg, _ = embedding(w)
+    tally = Tally()
     canvas_host = torch.empty(w.C, dtype=torch.int32).pin_memory()
-    done = den.step_h(host_h, canvas_host=canvas_host, want_done=True)
-    assert done in (0, 1)
-    assert np.array_equal(canvas_host.numpy(), ref[dg.DG_CANVAS])
-    assert np.array_equal(_np(den.read(dg.DG_ARGMAX)), ref[dg.DG_ARGMAX])
-    np.testing.assert_array_equal(_np(den.read(dg.DG_ENTROPY)), ref[dg.DG_ENTROPY])
+    for step in range(2):
+        canvas = _np(den.read(dg.DG_CANVAS)).astype(np.int64)
+        h = _external_h(w, Eg, canvas, 1234 + step).pin_memory()
+        pre = _np(den.read(dg.DG_ARGMAX)).astype(np.int64) if den.state()["has_prev"] else None
+        do_step = lambda: den.step_h(h, canvas_host=canvas_host)   # noqa: E731
+        assert step_and_compare(den, w, E32, tally, pre, do_step=do_step,
+                                h_given=h.float().numpy())
+        assert np.array_equal(canvas_host.numpy(), _np(den.read(dg.DG_CANVAS)))
+    tally.check_budget()
+    den.close()
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("variant", ["minus_max", "argmax_stop", "tau0"])
+def test_sampler_rules_teacher_forced(impl, variant):
+    """The acceptance and stop options on the 256-position partial-acceptance
+    stress set, on both kernel families (the tensor-core path runs the sampler
+    at the end of its attention kernel): "sum so far minus the largest" acceptance,
+    the argmax-stability stop, and a zero entropy budget (nothing accepted)."""
+    base = synthetic.STRESS_PARTIAL
+    w = {"minus_max": base.replace(accept_rule=dg.DG_ACCEPT_MINUS_MAX, fixed_steps=1, max_steps=4),
+         "argmax_stop": base.replace(stop_rule=dg.DG_STOP_ARGMAX, max_steps=8),
+         "tau0": base.replace(tau=0.0, max_steps=3)}[variant]
+    den, E32 = make(w, impl)
+    tally = run_teacher_forced(den, w, E32)
+    assert tally.steps >= 2
+    if variant == "argmax_stop":
+        assert den.state()["done"] == 1
     den.close()
 
 
@@ -453,6 +513,75 @@ def test_device_status_word_is_reported():
     den.close()
 
 
+@pytest.mark.parametrize("emb_dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("shape", [(256, 32768, 1024, 1024), (200, 4096, 512, 256),
+                                   (128, 8192, 2048, 1536)])
+def test_self_condition_network(shape, emb_dtype):
+    """dg_self_condition: the context's sc after a step goes through the
+    two-layer network (tensor cores) and is added to the caller's next-step
+    token embeddings; compared with the oracle's network on the same sc,
+    weights and embeddings (ragged canvas included: 200 rows)."""
+    C, V, d, dff = shape
+    w = synthetic.SMALL.replace(C=C, V=V, d=d, tau=0.5 * C * np.log(2), max_steps=2,
+                                fixed_steps=1, coef_target=1.0, coef_canvas=0.5, logit_scale=2.0)
+    den, E32 = make(w, dg.DG_IMPL_AUTO)
+    Eg, _ = embedding(w)
+    den.step()
+    sc = _np(den.read(dg.DG_SC)).astype(np.float64)
+    canvas = _np(den.read(dg.DG_CANVAS)).astype(np.int64)
+    g = torch.Generator().manual_seed(11)
+    W1 = torch.randn(dff, d, generator=g).to(torch.bfloat16)
+    b1 = torch.randn(dff, generator=g) * 0.1
+    W2 = (torch.randn(d, dff, generator=g) / np.sqrt(dff)).to(torch.bfloat16)
+    b2 = torch.randn(d, generator=g) * 0.1
+    tdt = torch.bfloat16 if emb_dtype == "bf16" else torch.float32
+    emb0 = Eg[torch.from_numpy(canvas).cuda()].to(tdt).contiguous()
+    emb = emb0.clone()
+    den.self_condition(W1.cuda(), b1.cuda(), W2.cuda(), b2.cuda(), emb)
+    assert den.state()["status"] == 0
+    y = M.self_condition_ffnn(sc, W1.float().numpy(), b1.numpy(), W2.float().numpy(), b2.numpy())
+    want = M.add_to_embeddings(_np(emb0).astype(np.float64), y, emb_dtype)
+    got = _np(emb).astype(np.float64)
+    if emb_dtype == "bf16":
+        # the sum is rounded to bf16 on both sides; one bf16 ulp of the result,
+        # plus the fp32-vs-fp64 accumulation (far below it)
+        e = np.frexp(np.maximum(np.abs(want), np.abs(got)))[1]
+        tol = np.ldexp(1.0, e - 8) + 1e-4 * np.abs(y).max()
+        assert np.all(np.abs(got - want) <= tol), float(np.abs(got - want).max())
+    else:
+        rel = np.linalg.norm(got - want, axis=1) / np.linalg.norm(want, axis=1)
+        assert rel.max() < 1e-3, rel.max()
+    den.close()
+
+
+def test_device_wait_timeout_is_reported_and_recovered():
+    """A bounded wait of the attention kernel runs out (a hand-off target that
+    no step reaches, with a 20 ms limit): the kernel returns on its own, the
+    next synchronising call reports DG_ETIMEOUT, and after dg_begin_block the
+    context steps correctly again (checked against the oracle)."""
+    import time
+    w = synthetic.STRESS_PARTIAL.replace(V=8192, d=512, max_steps=3, fixed_steps=1)
+    den, E32 = make(w, dg.DG_IMPL_TC)
+    den.step()
+    assert den.state()["status"] == 0
+    with pytest.raises(dg.DgError):
+        dg.dg_inject_stall(den.ctx, -1, 0)
+    dg.dg_inject_stall(den.ctx, 20_000_000, 1)
+    t0 = time.perf_counter()
+    with pytest.raises(dg.DgError) as e:
+        den.step(want_done=True)
+    waited = time.perf_counter() - t0
+    assert e.value.code == dg.DG_ETIMEOUT
+    assert waited < 1.5, waited            # well under the default 2 s limit
+    assert den.state()["status"] == dg.DG_ETIMEOUT
+    dg.dg_inject_stall(den.ctx, 0, 0)
+    den.begin_block(0)
+    assert den.state()["status"] == 0
+    tally = run_teacher_forced(den, w, E32)
+    assert tally.steps == w.max_steps
+    den.close()
+
+
 def test_block_loop_needs_a_stream():
     w = synthetic.TINY
     Eg, _ = embedding(w)
@@ -477,38 +606,9 @@ def test_vocab_parallel_shards(token_rule):
     with pytest.raises(dg.DgError):
         shards[0].step()                          # a shard alone cannot run a whole step
     bufs = [s.partials() for s in shards]
-    tally = Tally()
-    for _ in range(w.max_steps):
-        st0 = shards[0].state()
-        canvas_in = _np(shards[0].read(dg.DG_CANVAS)).astype(np.int64)
-        for s, b in zip(shards, bufs):
-            s.step_partial(b)
-            s.stream.synchronize()
-        dg.reduce_partials_local(bufs, w.C, w.d)
-        torch.cuda.synchronize()
-        for s, b in zip(shards, bufs):
-            s.step_finish(b)
-            s.stream.synchronize()
-        outs = []
-        for s in shards:
-            outs.append({k: _np(s.read(k)) for k in (dg.DG_HIDDEN, dg.DG_ENTROPY, dg.DG_ARGMAX,
-                                                     dg.DG_SC, dg.DG_CANVAS, dg.DG_ACCEPT)})
-            assert s.state()["status"] == 0
-        for k in outs[0]:
-            assert np.array_equal(outs[0][k], outs[1][k]), k
-        t, b = st0["t"], st0["block"]
-        h = outs[0][dg.DG_HIDDEN].astype(np.float64)
-        T = M.temperature(t, w.max_steps, w.T_start, w.T_end)
-        att = M.vocab_attention(h, E32, w.logit_scale / T,
-                                gumbel_key=(w.seed, b, t) if token_rule else None)
-        acc = M.entropy_bounded_accept(att.H.astype(np.float32), w.tau, w.accept_rule)
-        flags = near_tie_flags(att, acc, w.tau, w.accept_rule)
-        compare_attention(tally, att, outs[0][dg.DG_ENTROPY], outs[0][dg.DG_ARGMAX].astype(np.int64),
-                          outs[0][dg.DG_SC].astype(np.float64), flags)
-        if token_rule:
-            compare_draw(tally, att, _np(shards[0].read(dg.DG_SAMPLED)).astype(np.int64))
-        tally.positions += w.C
-    tally.check_budget()
+    tally = run_teacher_forced(shards[0], w, E32, do_step=shard_stepper(shards, bufs, w),
+                               peers=shards[1:])
+    assert tally.steps == w.max_steps
     assert shards[0].state()["done"] == 1
     for s in shards:
         s.close()
