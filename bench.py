@@ -8,20 +8,31 @@ the fixed-step timing mode (adaptive stop off; each block runs its S=32 steps
 and the next block starts). E (1.07 GB) is larger than L2 and is streamed from
 HBM every step, so no L2 flush is needed between steps.
 
-  value  device-timed throughput with inputs resident (CUDA events around K
-         steps on the context's stream, max over ranks).
-  e2e    the same metric through dg_denoise_step_h: every step copies that
-         step's hidden state from pinned host memory and the updated canvas
-         back to pinned host memory; CUDA events on the context's stream
-         bracket all of it (one synchronisation after the last step).
-  roofline  the vocabulary-attention kernels (the dominant kernel) against the
-         tensor roofline: 4*C*d*V flops per step over their event-timed duration.
-  cpu_baseline  the CPU oracle (fp64 numpy) on a bounded sample of rows.
+The JSON line (rank 0) carries:
+  value     device-timed throughput with inputs resident (CUDA events around K
+            steps on the context's stream, max over ranks).
+  e2e       the same metric through dg_denoise_step_h with host buffers: every
+            step copies its hidden state from pinned host memory (on the
+            library's copy stream, overlapping the step before) and the updated
+            canvas back to pinned host memory; host wall clock around K steps
+            with a synchronisation on both sides.
+  roofline  the vocabulary-attention kernel (the dominant kernel) against the
+            tensor roofline: 4*C*d*V flops per step over its event-timed
+            duration. The peak is the measured burst bf16 figure when the timed
+            region is short (under 2 s), the sustained one otherwise; both
+            fractions, the region's length and the sampled clock are given.
+  cpu_baseline  the CPU oracle (fp64 numpy) on whole steps of the workload.
+  workloads the other configurations: the tiny fp32 check (latency), the small
+            and latency-sensitive canvases (throughput and roofline), and four
+            sequential headline blocks to their adaptive stop (end-to-end
+            tokens/s over all 1024 tokens, emitted tokens copied to the host).
 
---impl reference runs the CPU oracle as the reference arm.
-Multi-GPU (torchrun): independent canvases per rank (replicas, seed = rank),
-no collective on the data path; value sums all ranks' steps over the slowest
-rank's time.
+--impl reference runs the CPU oracle as the reference arm (whole steps).
+Multi-GPU (torchrun): by default independent canvases per rank (replicas, seed
+= rank), no collective on the data path; value sums all ranks' steps over the
+slowest rank's time. --parallel vocab instead splits one canvas's vocabulary
+over the ranks (dg_denoise_step_partial, an NCCL exchange of the partial row
+results, dg_denoise_step_finish): value is that canvas's steps/s.
 """
 from __future__ import annotations
 
@@ -43,16 +54,48 @@ sys.path.insert(0, ROOT)
 import synthetic  # noqa: E402
 
 METRIC = "denoise steps/s & canvas tok/s at C=256,V=262k,d=2048; % of step roofline"
+BURST_MAX_S = 2.0          # timed regions shorter than this are burst measurements
 
 
 def measured_peaks():
+    """Peaks from MEASURED_PEAKS.json (HBM GB/s, bf16 TFLOP/s burst and sustained).
+
+    Also returns any clock figures the file records (keys naming MHz), which
+    the roofline uses to state the clock its peaks were taken at.
+    """
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
+        clocks = {}
+
+        def walk(obj, pre=""):
+            if isinstance(obj, dict):
+                for k, v in obj.items():
+                    walk(v, f"{pre}{k}.")
+            elif isinstance(obj, (int, float)) and "mhz" in pre.lower():
+                clocks[pre[:-1]] = float(obj)
+        walk(p)
         return dict(hbm=float(p["hbm_gbs"]), tflops=float(p["bf16_tflops"]),
-                    tflops_sustained=float(p["bf16_tflops_sustained"]), src="measured")
+                    tflops_sustained=float(p["bf16_tflops_sustained"]), src="measured",
+                    clocks=clocks)
     except Exception:
-        return dict(hbm=6650.0, tflops=1590.0, tflops_sustained=1400.0, src="fallback")
+        return dict(hbm=6650.0, tflops=1590.0, tflops_sustained=1400.0, src="fallback",
+                    clocks={})
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_threads() -> int:
+    return int(os.environ.get("OPENBLAS_NUM_THREADS", len(os.sched_getaffinity(0))))
 
 
 class Clocks:
@@ -110,30 +153,34 @@ class Clocks:
                 "samples": len(sm)}
 
 
-def cpu_baseline(w, E32, rows: int, seed_steps: int = 1):
-    """The oracle, as it stands, on `rows` canvas rows of one step; scaled to steps/s.
+def cpu_baseline(w, E32, steps: int = 1, budget_s: float | None = None):
+    """The oracle, as it stands, on whole denoise steps of workload w.
 
-    The sample is the first `rows` rows: their stand-in hidden state, the
-    vocabulary attention (and draw) and the acceptance over them.
+    Runs one untimed step first (it pages E in and warms the BLAS threads),
+    then `steps` timed steps (fewer if budget_s runs out after at least one).
+    Returns the line's cpu_baseline object plus the seconds per step.
     """
     from oracle import method as M
 
     st = M.begin_block(w, 0)
-    wr = w.replace(C=rows, canvases=1)
-    T = M.temperature(0, w.max_steps, w.T_start, w.T_end)
-    key = (w.seed, 0, 0) if getattr(w, "token_rule", 0) == 1 else None
-    t0 = time.perf_counter()
-    for _ in range(seed_steps):
-        h = M.standin_hidden(wr, E32, st.target[:rows], st.canvas[:rows], st.sc[:rows], 0, 0)
-        att = M.vocab_attention(h, E32, w.logit_scale / T, gumbel_key=key)
-        M.entropy_bounded_accept(att.H.astype(np.float32), w.tau, w.accept_rule)
-    dt = (time.perf_counter() - t0) / seed_steps
-    step_s = dt * w.C / rows
-    threads = int(os.environ.get("OPENBLAS_NUM_THREADS", len(os.sched_getaffinity(0))))
-    return {"value": 1.0 / step_s, "unit": "steps/s", "cores": threads, "kind": "oracle",
-            "sample": f"{rows} of {w.C} canvas rows of one step (fp64 numpy, {dt:.1f} s), "
-                      f"scaled by {w.C}/{rows}",
-            "tok_per_s": w.C / step_s}
+    M.step(w, E32, st)
+    times = []
+    t_start = time.perf_counter()
+    for _ in range(steps):
+        if st.done:
+            st = M.begin_block(w, st.block + 1)
+        t0 = time.perf_counter()
+        M.step(w, E32, st)
+        times.append(time.perf_counter() - t0)
+        if budget_s is not None and time.perf_counter() - t_start > budget_s:
+            break
+    step_s = float(np.mean(times))
+    return {"value": 1.0 / step_s, "unit": "steps/s", "cores": cpu_threads(), "kind": "oracle",
+            "cpu_model": cpu_model(), "steps_timed": len(times),
+            "sample": f"{len(times)} whole step(s) of all {w.C} canvas rows (fp64 numpy oracle: "
+                      f"stand-in h, vocabulary attention, sampler, stop test), "
+                      f"{step_s:.2f} s per step, after one untimed step",
+            "tok_per_s": w.C / step_s}, step_s
 
 
 def max_over_ranks(x: float, dist=None, device="cpu") -> float:
@@ -151,54 +198,70 @@ def whole_job_rate(steps_per_rank: int, world: int, slowest_ms: float) -> float:
     return steps_per_rank * world / (slowest_ms / 1e3)
 
 
-def roofline_time(w, pk, sustained=True):
+def shared_canvas_rate(steps: int, slowest_ms: float) -> float:
+    """Strong scaling: all ranks step one canvas together; its steps over the slowest rank's time."""
+    return steps / (slowest_ms / 1e3)
+
+
+def step_roofline(w, pk):
+    """Roofline time of one step as the workload's definition states it:
+    max(4 C d V / P_bf16, 2 V d 2 / B_HBM), burst and sustained."""
     flops = 4.0 * w.C * w.d * w.V
-    t_c = flops / ((pk["tflops_sustained"] if sustained else pk["tflops"]) * 1e12)
     t_m = 2.0 * w.V * w.d * 2 / (pk["hbm"] * 1e9)
-    return max(t_c, t_m), flops
+    return (max(flops / (pk["tflops"] * 1e12), t_m),
+            max(flops / (pk["tflops_sustained"] * 1e12), t_m), flops)
 
 
-def run_reference(args, w):
-    """Reference arm: the CPU oracle on the host cores, same metric and config."""
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
-        return 0
-    E32 = synthetic.make_embedding_f32(w.V, w.d, w.e_seed)
-    if w.dtype == "bf16":
-        import torch
-        E32 = torch.from_numpy(E32).to(torch.bfloat16).float().numpy()
-    # Each timed step is a sample of --ref-rows rows (enough to amortise the
-    # oracle's fixed per-call cost: it widens all of E to fp64 in chunks). At
-    # most as many samples as fit in about two minutes are timed, so a large
-    # --steps still ends in bounded time; "steps" reports how many ran.
-    rows = max(1, min(w.C, args.ref_rows))
-    first = cpu_baseline(w, E32, rows)                       # warm-up and calibration
-    sample_s = rows / (w.C * first["value"])        # seconds per sample
-    n = int(max(1, min(args.steps, 120.0 // max(sample_s, 1e-9))))
-    times = []
-    for _ in range(max(0, min(args.warmup, n) - 1)):
-        cpu_baseline(w, E32, rows)
-    for _ in range(n):
-        times.append(1.0 / cpu_baseline(w, E32, rows)["value"])
-    step_s = float(np.mean(times))
-    cb = cpu_baseline(w, E32, rows)
-    args.steps = n
-    val = 1.0 / step_s
-    line = {"metric": METRIC, "value": val, "unit": "steps/s", "impl": "reference",
-            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "tok_per_s": w.C * val,
-            "config": {"workload": w.name, "C": w.C, "V": w.V, "d": w.d,
-                       "canvases": w.canvases,
-                       "token_rule": "multinomial" if w.token_rule == 1 else "argmax",
-                       "mode": "fixed_steps"},
-            "cpu_baseline": {"value": val, "unit": "steps/s", "cores": cb["cores"],
-                             "kind": "oracle", "sample": cb["sample"]},
-            "e2e": {"value": val, "unit": "steps/s", "h2d_bytes_per_step": 0,
-                    "d2h_bytes_per_step": 0}}
-    print(json.dumps(line), flush=True)
-    return 0
+def choose_peak(timed_s: float, clk) -> str:
+    """'burst' for a timed region shorter than BURST_MAX_S, else 'sustained'.
+
+    A region of a few milliseconds ends before the power cap acts on the clock
+    (and nvidia-smi's 200 ms samples then mostly see the idle GPU around it),
+    so its length decides; the sampled clock is reported beside the result.
+    """
+    return "burst" if timed_s < BURST_MAX_S else "sustained"
+
+
+def kernel_roofline(w, pk, kernel_s: float, timed_s: float, clk, kernel: str):
+    """Roofline object of the vocabulary-attention kernel at one launch per step.
+
+    Algorithmic work per launch: 4 C d V flops (both contractions) and V d b_E
+    bytes of E (read once). The bound is whichever takes longer at the peaks.
+    """
+    esz = 2 if w.dtype == "bf16" else 4
+    flops = 4.0 * w.C * w.d * w.V
+    bytes_ = float(w.V) * w.d * esz + w.C * w.d * (esz + 4)
+    which = choose_peak(timed_s, clk)
+    P = pk["tflops"] if which == "burst" else pk["tflops_sustained"]
+    tensor_bound = flops / (P * 1e12) >= bytes_ / (pk["hbm"] * 1e9)
+    if tensor_bound:
+        achieved = flops / kernel_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": P, "unit": "TFLOP/s",
+                "frac": achieved / P,
+                "frac_burst": achieved / pk["tflops"],
+                "frac_sustained": achieved / pk["tflops_sustained"]}
+    else:
+        achieved = bytes_ / kernel_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": achieved / pk["hbm"]}
+    roof.update({
+        "kernel": kernel, "kernel_us_per_launch": kernel_s * 1e6,
+        "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": bytes_,
+        "peak_choice": which,
+        "peak_src": f"{pk['src']} ({'bf16 burst' if which == 'burst' else 'bf16 sustained'}"
+                    f"{'' if tensor_bound else '; HBM copy'}); timed region {timed_s:.3f} s at "
+                    f"median {clk['sm_mhz'] if clk else '?'} MHz (max "
+                    f"{clk['sm_max_mhz'] if clk else '?'})",
+        "timed_region_s": timed_s,
+        "sm_mhz_median": clk["sm_mhz"] if clk else None,
+    })
+    if clk and clk.get("sm_max_mhz") and tensor_bound:
+        # the same kernel time scaled to the maximum clock, against the burst peak
+        roof["frac_burst_at_max_clock"] = roof["frac_burst"] * clk["sm_max_mhz"] / clk["sm_mhz"] \
+            if clk["sm_mhz"] else None
+    if pk.get("clocks"):
+        roof["peak_clocks"] = pk["clocks"]
+    return roof
 
 
 # DRAM bytes (read + write) per launch of the tensor-core kernel, from the ncu
@@ -211,6 +274,403 @@ DRAM_TRAFFIC = {
 }
 
 
+def run_reference(args, w):
+    """Reference arm: the CPU oracle on the host cores, same metric and config.
+
+    Each timed step is one whole step of the workload. As many steps as
+    --steps asks for are timed, but no more than fit in about two minutes (at
+    least one); "steps" reports how many ran, "warmup" the one untimed step.
+    """
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    E32 = synthetic.make_embedding_f32(w.V, w.d, w.e_seed)
+    if w.dtype == "bf16":
+        import torch
+        E32 = torch.from_numpy(E32).to(torch.bfloat16).float().numpy()
+    cb, step_s = cpu_baseline(w, E32, steps=max(1, args.steps), budget_s=120.0)
+    n = cb["steps_timed"]
+    val = 1.0 / step_s
+    line = {"metric": METRIC, "value": val, "unit": "steps/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": n, "warmup": 1,
+            "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "tok_per_s": w.C * val,
+            "steps_requested": args.steps, "warmup_requested": args.warmup,
+            "config": {"workload": w.name, "C": w.C, "V": w.V, "d": w.d,
+                       "canvases": w.canvases,
+                       "token_rule": "multinomial" if w.token_rule == 1 else "argmax",
+                       "mode": "fixed_steps"},
+            "cpu_baseline": {"value": val, "unit": "steps/s", "cores": cb["cores"],
+                             "kind": "oracle", "sample": cb["sample"], "cpu_model": cb["cpu_model"]},
+            "e2e": {"value": val, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------
+# GPU legs.
+# ----------------------------------------------------------------------------
+class FixedStepLoop:
+    """Steps of one context in the fixed-step mode: a new block after every S steps."""
+
+    def __init__(self, den, S):
+        self.den, self.S, self.t, self.block = den, S, 0, 0
+
+    def __call__(self):
+        if self.t == self.S:
+            self.block += 1
+            self.den.begin_block(self.block)
+            self.t = 0
+        self.den.step()
+        self.t += 1
+
+
+def timed_steps(den, step, steps: int, warmup: int, local: int, dist=None):
+    """Device-timed region of `steps` calls of step() on den's stream.
+
+    Returns (ms of the region, max over ranks), (attention-kernel ms, steps
+    timed, kernels launched) from dg_profile, the sampled clocks and the
+    region's length in seconds.
+    """
+    import torch
+
+    import uniform_state_text_b200 as dg
+    for _ in range(warmup):
+        step()
+    den.stream.synchronize()
+    clocks = Clocks(local)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    dg.dg_profile(den.ctx, True)
+    ev0.record(den.stream)
+    for _ in range(steps):
+        step()
+    ev1.record(den.stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    prof = dg.dg_profile_read(den.ctx)
+    dg.dg_profile(den.ctx, False)
+    clk = clocks.stop()
+    st = den.state()
+    if st["status"] != 0:
+        raise RuntimeError(f"device status {st['status']}")
+    return max_over_ranks(ms, dist, "cuda"), prof, clk, ms / 1e3
+
+
+def e2e_leg(den, w, steps: int, dist=None):
+    """Wall clock of `steps` dg_denoise_step_h calls with host buffers.
+
+    Every step copies a hidden state [C][d] in from pinned host memory (two
+    alternating host buffers) and the updated canvas out to pinned host memory;
+    the host is synchronised before the first call and after the last.
+    """
+    import torch
+
+    import uniform_state_text_b200 as dg
+    den.begin_block(0)
+    den.step()
+    h0 = den.read(dg.DG_HIDDEN).cpu()
+    h_host = [h0.clone().pin_memory(), h0.clone().pin_memory()]
+    canvas_host = torch.empty(w.C, dtype=torch.int32).pin_memory()
+    S = w.max_steps
+
+    def run(n):
+        done_steps = 0
+        for i in range(n):
+            if done_steps == S:
+                den.begin_block(0)
+                done_steps = 0
+            den.step_h(h_host[i % 2], canvas_host=canvas_host)
+            done_steps += 1
+
+    den.begin_block(0)
+    run(3)
+    torch.cuda.synchronize()
+    den.begin_block(0)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    run(steps)
+    torch.cuda.synchronize()
+    el = time.perf_counter() - t0
+    if den.state()["status"] != 0:
+        raise RuntimeError("device status after the e2e leg")
+    return max_over_ranks(el, dist, "cuda"), int(h0.numel() * h0.element_size()), int(w.C * 4)
+
+
+def redo_leg(den, w, E, steps: int):
+    """Cost of the redo pass: device time per step of dg_denoise_step_h with
+    caller hidden states h = 30 E[token] whose largest logits overshoot the
+    rows' references (the logits of the previous step's tokens) on no row, on
+    1% of the rows, and on every row. Steps alternate between two hidden
+    states; in the 'none' case both are the same, so after the untimed first
+    step every reference is exact."""
+    import torch
+
+    import uniform_state_text_b200 as dg
+    g = torch.Generator().manual_seed(7)
+    tok_a = torch.randint(0, w.V, (w.C,), generator=g)
+    tok_b = torch.randint(0, w.V, (w.C,), generator=g)
+    few = tok_a.clone()
+    k = max(1, w.C // 100)
+    few[:k] = tok_b[:k]
+
+    def hid(tok):
+        return (30.0 * E[tok.to(E.device)].float()).to(E.dtype).contiguous()
+
+    h_a = hid(tok_a)
+    cases = {"none": h_a, "1pct": hid(few), "all": hid(tok_b)}
+    n = max(2, min(steps, w.max_steps - 1))
+    out = {"steps": n, "rows": w.C,
+           "path": "dg_denoise_step_h with device hidden states, CUDA events on the stream"}
+    for name, h_b in cases.items():
+        den.begin_block(0)
+        den.step_h(h_a)                                   # step 0: every reference is low
+        r0 = den.state()["redo"]
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(den.stream)
+        for i in range(n):
+            den.step_h(h_b if i % 2 == 0 else h_a)
+        ev1.record(den.stream)
+        torch.cuda.synchronize()
+        st = den.state()
+        if st["status"] != 0:
+            raise RuntimeError("device status after the redo leg")
+        out[name] = {"us_per_step": 1e3 * ev0.elapsed_time(ev1) / n,
+                     "rows_redone_per_step": (st["redo"] - r0) / n}
+    out["all_over_none"] = out["all"]["us_per_step"] / out["none"]["us_per_step"]
+    return out
+
+
+def headline_line(args, w, world, rank, local, dist):
+    import torch
+
+    import uniform_state_text_b200 as dg
+
+    impl = {"auto": dg.DG_IMPL_AUTO, "simt": dg.DG_IMPL_SIMT, "tc": dg.DG_IMPL_TC}[args.kernels]
+    E_cpu = synthetic.make_embedding(w)
+    E = E_cpu.to(f"cuda:{local}")
+    den = dg.Denoiser(w, E, impl=impl)
+    kern = "tcgen05" if den.impl == dg.DG_IMPL_TC else "CUDA-core"
+    ms, (attn_ms, attn_steps, launches), clk, timed_s = timed_steps(
+        den, FixedStepLoop(den, w.max_steps), args.steps, args.warmup, local, dist)
+    value = whole_job_rate(args.steps, world, ms)
+    ms_per_step = ms / args.steps
+
+    e2e = None
+    if not args.no_e2e:
+        el, bi, bo = e2e_leg(den, w, args.steps, dist)
+        e2e = {"value": args.steps * world / el, "unit": "steps/s",
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+               "tok_per_s": w.C * args.steps * world / el, "steps": args.steps,
+               "path": "dg_denoise_step_h: hidden state from pinned host memory (copy stream, "
+                       "overlapping the step before), canvas to pinned host memory; host wall "
+                       "clock with a synchronisation on both sides"}
+
+    redo = None
+    if den.impl == dg.DG_IMPL_TC and not args.no_workloads:
+        redo = redo_leg(den, w, E, args.steps)
+
+    pk = measured_peaks()
+    t_b, t_s, _ = step_roofline(w, pk)
+    roof = kernel_roofline(w, pk, (attn_ms / 1e3) / max(attn_steps, 1), timed_s, clk,
+                           f"vocabulary attention ({kern})")
+    traffic = DRAM_TRAFFIC.get(w.name) if den.impl == dg.DG_IMPL_TC else None
+    roof["traffic"] = traffic[0] if traffic else None
+    roof["traffic_src"] = traffic[1] if traffic else None
+    roof.update({"step_roofline_us": t_b * 1e6, "step_roofline_us_sustained": t_s * 1e6,
+                 "step_roofline_pct": 100.0 * t_b / (ms_per_step / 1e3),
+                 "step_roofline_pct_sustained": 100.0 * t_s / (ms_per_step / 1e3)})
+    den.close()
+    del E
+    torch.cuda.empty_cache()
+    line = {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32",
+            "data": "synthetic (seeded E ~ N(0, I/d), stand-in hidden state)",
+            "tok_per_s": w.C * value,
+            "roofline_pct": roof["step_roofline_pct"],
+            "config": {"workload": w.name, "C": w.C, "V": w.V, "d": w.d,
+                       "canvases": w.canvases,
+                       "token_rule": "multinomial" if w.token_rule == 1 else "argmax",
+                       "max_steps": w.max_steps, "mode": "fixed_steps (adaptive stop off)",
+                       "kernels": "tc" if den.impl == dg.DG_IMPL_TC else "simt",
+                       "l2": "no flush: E (%.2f GB) exceeds the 126 MB L2 and is streamed every step"
+                             % (w.e_bytes / 1e9),
+                       "parallelism": f"replicas x{world}"},
+            "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+            "redo_cost": redo}
+    return line, E_cpu
+
+
+def workload_throughput(w, steps, warmup, local, with_cpu: bool):
+    """Device-timed fixed-step throughput of one more workload, with its roofline."""
+    import torch
+
+    import uniform_state_text_b200 as dg
+    E_cpu = synthetic.make_embedding(w)
+    E = E_cpu.cuda()
+    den = dg.Denoiser(w, E)
+    kern = "tcgen05" if den.impl == dg.DG_IMPL_TC else "CUDA-core"
+    ms, (attn_ms, attn_steps, launches), clk, timed_s = timed_steps(
+        den, FixedStepLoop(den, w.max_steps), steps, warmup, local)
+    pk = measured_peaks()
+    t_b, t_s, _ = step_roofline(w, pk)
+    ms_step = ms / steps
+    out = {"workload": w.name, "C": w.C, "V": w.V, "d": w.d, "dtype": w.dtype,
+           "mode": "fixed_steps", "steps": steps, "warmup": warmup,
+           "value": 1e3 / ms_step, "unit": "steps/s", "ms_per_step": ms_step,
+           "tok_per_s": w.C * 1e3 / ms_step, "gpu_launches": launches, "clocks": clk,
+           "step_roofline_us": t_b * 1e6,
+           "step_roofline_pct": 100.0 * t_b / (ms_step / 1e3),
+           "step_roofline_pct_sustained": 100.0 * t_s / (ms_step / 1e3),
+           "roofline": kernel_roofline(w, pk, (attn_ms / 1e3) / max(attn_steps, 1), timed_s, clk,
+                                       f"vocabulary attention ({kern})")}
+    den.close()
+    del E
+    torch.cuda.empty_cache()
+    if with_cpu:
+        out["cpu_baseline"], _ = cpu_baseline(w, synthetic.embedding_as_f32(E_cpu), steps=1)
+    return out
+
+
+def tiny_latency(local, reps: int = 200):
+    """The tiny fp32 check: latency of one step and of a whole adaptive block."""
+    import torch
+
+    import uniform_state_text_b200 as dg
+    w = synthetic.TINY
+    E = synthetic.make_embedding(w).cuda()
+    wf = w.replace(fixed_steps=1)
+    den = dg.Denoiser(wf, E)
+    ms, (attn_ms, attn_steps, launches), clk, _ = timed_steps(
+        den, FixedStepLoop(den, wf.max_steps), reps, 5, local)
+    den.close()
+    den = dg.Denoiser(w, E)
+    out = torch.empty(w.C, dtype=torch.int32, device="cuda")
+    host = torch.empty(w.C, dtype=torch.int32).pin_memory()
+    for b in range(3):
+        den.block(b, out=out)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    steps = 0
+    for b in range(reps):
+        steps += den.block(b, out=out)[1]
+        host.copy_(out, non_blocking=True)
+        den.stream.synchronize()
+    el = time.perf_counter() - t0
+    den.close()
+    return {"workload": w.name, "C": w.C, "V": w.V, "d": w.d, "dtype": w.dtype,
+            "step_latency_us": 1e3 * ms / reps, "value": reps / (ms / 1e3), "unit": "steps/s",
+            "kernels": "CUDA-core (fp32)", "gpu_launches_per_step": launches / reps,
+            "block_latency_us": 1e6 * el / reps, "block_steps_mean": steps / reps,
+            "block_tok_per_s": w.C * reps / el,
+            "block_path": "dg_denoise_block (graph loop to the adaptive stop) + emitted tokens to "
+                          "pinned host memory, host wall clock per block",
+            "roofline": None, "bound": "launch/latency (2.1 MFLOP per step)"}
+
+
+def blocks_e2e(w, E_cpu, reps: int = 3):
+    """Four sequential headline blocks to their adaptive stop, tokens to the host."""
+    import torch
+
+    import uniform_state_text_b200 as dg
+    E = E_cpu.cuda()
+    den = dg.Denoiser(w, E)
+    buf = torch.empty(w.blocks * w.C, dtype=torch.int32, device="cuda")
+    host = torch.empty(w.blocks * w.C, dtype=torch.int32).pin_memory()
+
+    def run():
+        steps = []
+        for b in range(w.blocks):
+            _, s = den.block(b, out=buf[b * w.C:(b + 1) * w.C])
+            steps.append(s)
+            host[b * w.C:(b + 1) * w.C].copy_(buf[b * w.C:(b + 1) * w.C], non_blocking=True)
+        den.stream.synchronize()
+        return steps
+
+    run()
+    torch.cuda.synchronize()
+    times, steps = [], None
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        steps = run()
+        times.append(time.perf_counter() - t0)
+    den.close()
+    del E
+    torch.cuda.empty_cache()
+    el = float(np.median(times))
+    return {"workload": w.name, "blocks": w.blocks, "C": w.C, "V": w.V, "d": w.d,
+            "dtype": w.dtype, "mode": "adaptive stop", "steps_per_block": steps,
+            "value": w.blocks * w.C / el, "unit": "tok/s", "seconds": el,
+            "path": "dg_denoise_block per block (graph loop to the adaptive stop), emitted tokens "
+                    "copied to pinned host memory; host wall clock, median of %d runs" % reps,
+            "d2h_bytes": w.blocks * w.C * 4}
+
+
+def vocab_parallel_loop(den, buf, C, d, group=None):
+    """One step of a canvas whose vocabulary is split over the ranks: the
+    shard's partial step, the exchange of the partial row results (one sum and
+    one max all-reduce), then the shard's finish (identical on every rank)."""
+    import uniform_state_text_b200 as dg
+    den.step_partial(buf)
+    dg.allreduce_partials(buf, C, d, group=group)
+    den.step_finish(buf)
+
+
+def vocab_parallel_line(args, w, world, rank, local, dist):
+    import torch
+
+    import uniform_state_text_b200 as dg
+    if w.V % (256 * world):
+        raise SystemExit(f"V={w.V} does not split into {world} shards of 256-entry tiles")
+    nv = w.V // world
+    E = synthetic.make_embedding(w).to(f"cuda:{local}")
+    den = dg.Denoiser(w, E, impl=dg.DG_IMPL_TC, shard=(rank * nv, nv))
+    buf = den.partials()
+    state = {"t": 0, "block": 0}
+
+    def step():
+        if state["t"] == w.max_steps:
+            state["block"] += 1
+            den.begin_block(state["block"])
+            state["t"] = 0
+        with torch.cuda.stream(den.stream):
+            vocab_parallel_loop(den, buf, w.C, w.d)
+        state["t"] += 1
+
+    ms, (attn_ms, attn_steps, launches), clk, timed_s = timed_steps(
+        den, step, args.steps, args.warmup, local, dist)
+    value = shared_canvas_rate(args.steps, ms)
+    den.close()
+    if rank == 0:
+        return {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+                "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic (seeded E ~ N(0, I/d), stand-in hidden state)",
+                "tok_per_s": w.C * value,
+                "config": {"workload": w.name, "C": w.C, "V": w.V, "d": w.d,
+                           "mode": "fixed_steps (adaptive stop off)", "kernels": "tc",
+                           "parallelism": f"vocabulary-parallel x{world} (NCCL sum+max exchange)",
+                           "shard_entries": nv},
+                "attention_ms_per_step_rank0": attn_ms / max(attn_steps, 1),
+                "gpu_launches": launches, "clocks": clk, "e2e": None, "roofline": None,
+                "cpu_baseline": None}
+    return None
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -219,15 +679,18 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=synthetic.HEADLINE.name, choices=sorted(synthetic.WORKLOADS))
     ap.add_argument("--kernels", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--parallel", default="replicas", choices=["replicas", "vocab"],
+                    help="multi-GPU mode: independent canvases per rank, or one canvas's "
+                         "vocabulary split over the ranks")
     ap.add_argument("--token-rule", default="argmax", choices=["argmax", "multinomial"],
                     help="token an accepted position takes")
     ap.add_argument("--canvases", type=int, default=0,
                     help="split the workload's C positions into this many independent "
                          "canvases (tau scaled per canvas); 0 keeps the workload's own")
-    ap.add_argument("--cpu-rows", type=int, default=32, help="rows of the oracle baseline sample")
-    ap.add_argument("--ref-rows", type=int, default=16, help="rows per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other workloads (tiny, small, latency, blocks)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -262,141 +725,33 @@ def main():
     if dist:
         dist.barrier()
     dg.lib()
-    w = w.replace(seed=rank)
-    impl = {"auto": dg.DG_IMPL_AUTO, "simt": dg.DG_IMPL_SIMT, "tc": dg.DG_IMPL_TC}[args.kernels]
 
-    E_cpu = synthetic.make_embedding(w)
-    E = E_cpu.to(f"cuda:{local}")
-    den = dg.Denoiser(w, E, impl=impl)
-    stream = den.stream
-    S = w.max_steps
-
-    state = {"t": 0, "block": 0}
-
-    def one_step():
-        if state["t"] == S:
-            state["block"] += 1
-            den.begin_block(state["block"])
-            state["t"] = 0
-        den.step()
-        state["t"] += 1
-
-    for _ in range(args.warmup):
-        one_step()
-    stream.synchronize()
-
-    # --- device-timed region -------------------------------------------------
-    clocks = Clocks(local)
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
-    dg.dg_profile(den.ctx, True)
-    ev0.record(stream)
-    for _ in range(args.steps):
-        one_step()
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    ms = ev0.elapsed_time(ev1)
-    attn_ms, attn_steps, launches = dg.dg_profile_read(den.ctx)
-    dg.dg_profile(den.ctx, False)
-    clk = clocks.stop()
-    st = den.state()
-    if st["status"] != 0:
-        raise RuntimeError(f"device status {st['status']}")
-    ms = max_over_ranks(ms, dist, "cuda")
-    value = whole_job_rate(args.steps, world, ms)
-    ms_per_step = ms / args.steps
-
-    # --- end to end through host buffers ----------------------------------------
-    e2e = None
-    if not args.no_e2e:
-        den.begin_block(0)
-        den.step()
-        h_host = den.read(dg.DG_HIDDEN).cpu().pin_memory()
-        canvas_host = torch.empty(w.C, dtype=torch.int32).pin_memory()
-        den.begin_block(0)
-        n_e2e = max(8, args.steps // 2)
-        for _ in range(3):
-            den.step_h(h_host, canvas_host=canvas_host)
-        torch.cuda.synchronize()
-        den.begin_block(0)
+    if args.parallel == "vocab":
+        line = vocab_parallel_line(args, w, world, rank, local, dist)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
         if dist:
-            dist.barrier()
-        torch.cuda.synchronize()
-        # Device-timed on the library's stream: the events bracket every copy
-        # and kernel, and any gap the host leaves between steps. Each step
-        # copies h in from pinned memory and the canvas back out (the canvas
-        # read-back is asynchronous; the stream is synchronised once, after).
-        e2e0 = torch.cuda.Event(enable_timing=True)
-        e2e1 = torch.cuda.Event(enable_timing=True)
-        e2e0.record(stream)
-        done_steps = 0
-        for i in range(n_e2e):
-            if done_steps == S:
-                den.begin_block(0)
-                done_steps = 0
-            den.step_h(h_host, canvas_host=canvas_host)
-            done_steps += 1
-        e2e1.record(stream)
-        torch.cuda.synchronize()
-        el = e2e0.elapsed_time(e2e1) / 1e3
-        el = max_over_ranks(el, dist, "cuda")
-        e2e = {"value": n_e2e * world / el, "unit": "steps/s",
-               "h2d_bytes_per_step": int(h_host.numel() * h_host.element_size()),
-               "d2h_bytes_per_step": int(w.C * 4),
-               "tok_per_s": w.C * n_e2e * world / el,
-               "path": "dg_denoise_step_h, hidden state from pinned host memory"}
+            dist.destroy_process_group()
+        return 0
 
-    pk = measured_peaks()
-    t_roof, flops = roofline_time(w, pk, sustained=True)
-    t_roof_burst, _ = roofline_time(w, pk, sustained=False)
-    attn_s = (attn_ms / 1e3) / max(attn_steps, 1)
-    achieved_tflops = flops / attn_s / 1e12
-    peak = pk["tflops_sustained"]
-    traffic = DRAM_TRAFFIC.get(w.name) if den.impl == dg.DG_IMPL_TC else None
-    roof = {"bound": "tensor", "achieved": achieved_tflops, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved_tflops / peak,
-            "traffic": traffic[0] if traffic else None,
-            "traffic_src": traffic[1] if traffic else None,
-            "kernel": "vocabulary attention (" + ("tcgen05" if den.impl == dg.DG_IMPL_TC else "CUDA-core") + ")",
-            "kernel_ms_per_step": attn_s * 1e3,
-            "peak_src": f"{pk['src']} bf16 sustained (kernel timed inside a long step loop)",
-            "algorithmic_flops_per_step": flops,
-            "step_roofline_pct_sustained": 100.0 * t_roof / (ms_per_step / 1e3),
-            "step_roofline_us_sustained": t_roof * 1e6,
-            "step_roofline_pct": 100.0 * t_roof_burst / (ms_per_step / 1e3),
-            "step_roofline_us": t_roof_burst * 1e6}
-
-    cb = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        E32 = synthetic.embedding_as_f32(E_cpu)
-        cb = cpu_baseline(w, E32, max(1, min(w.C, args.cpu_rows)))
-
+    w = w.replace(seed=rank)
+    line, E_cpu = headline_line(args, w, world, rank, local, dist)
+    if rank == 0 and world == 1:
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"], _ = cpu_baseline(w, synthetic.embedding_as_f32(E_cpu), steps=1)
+        else:
+            line["cpu_baseline"] = None
+        if not args.no_workloads and args.workload == synthetic.HEADLINE.name:
+            wl = [tiny_latency(local)]
+            for wk in (synthetic.SMALL, synthetic.LATENCY):
+                wl.append(workload_throughput(wk.replace(fixed_steps=1), max(args.steps, 200),
+                                              args.warmup, local, not args.no_cpu_baseline))
+            wl.append(blocks_e2e(synthetic.BLOCKS, E_cpu))
+            line["workloads"] = wl
+    else:
+        line["cpu_baseline"] = None
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "bf16" if w.dtype == "bf16" else "f32",
-                "data": "synthetic (seeded E ~ N(0, I/d), stand-in hidden state)",
-                "tok_per_s": w.C * value,
-                "roofline_pct": roof["step_roofline_pct"],
-                "config": {"workload": w.name, "C": w.C, "V": w.V, "d": w.d,
-                           "canvases": w.canvases,
-                           "token_rule": "multinomial" if w.token_rule == 1 else "argmax",
-                           "max_steps": S, "mode": "fixed_steps (adaptive stop off)",
-                           "kernels": "tc" if den.impl == dg.DG_IMPL_TC else "simt",
-                           "l2": "no flush: E (%.2f GB) exceeds the 126 MB L2 and is streamed every step" % (w.e_bytes / 1e9),
-                           "parallelism": f"replicas x{world}"},
-                "roofline": roof, "e2e": e2e, "gpu_launches": launches,
-                "clocks": clk, "cpu_baseline": cb}
         print(json.dumps(line), flush=True)
-    den.close()
     if dist:
         dist.destroy_process_group()
     return 0
