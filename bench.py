@@ -227,19 +227,24 @@ def kernel_roofline(w, pk, kernel_s: float, timed_s: float, clk, kernel: str):
 
     Algorithmic work per launch: 4 C d V flops (both contractions) and V d b_E
     bytes of E (read once). The bound is whichever takes longer at the peaks.
+    With narrow E (e4m3 codes) the operands are 8-bit: E is V d bytes plus a
+    4-byte exponent per row, and the tensor peak is the measured bf16 peak
+    times the nominal fp8/bf16 ratio (4.5 / 2.25 PFLOP/s dense).
     """
-    esz = 2 if w.dtype == "bf16" else 4
+    fp8 = getattr(w, "e_format", 0) == 1
+    esz = 1 if fp8 else (2 if w.dtype == "bf16" else 4)
     flops = 4.0 * w.C * w.d * w.V
-    bytes_ = float(w.V) * w.d * esz + w.C * w.d * (esz + 4)
+    bytes_ = float(w.V) * w.d * esz + (4.0 * w.V if fp8 else 0.0) + w.C * w.d * (esz + 4)
     which = choose_peak(timed_s, clk)
-    P = pk["tflops"] if which == "burst" else pk["tflops_sustained"]
+    ratio = 2.0 if fp8 else 1.0
+    P = ratio * (pk["tflops"] if which == "burst" else pk["tflops_sustained"])
     tensor_bound = flops / (P * 1e12) >= bytes_ / (pk["hbm"] * 1e9)
     if tensor_bound:
         achieved = flops / kernel_s / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": P, "unit": "TFLOP/s",
                 "frac": achieved / P,
-                "frac_burst": achieved / pk["tflops"],
-                "frac_sustained": achieved / pk["tflops_sustained"]}
+                "frac_burst": achieved / (ratio * pk["tflops"]),
+                "frac_sustained": achieved / (ratio * pk["tflops_sustained"])}
     else:
         achieved = bytes_ / kernel_s / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
@@ -249,6 +254,7 @@ def kernel_roofline(w, pk, kernel_s: float, timed_s: float, clk, kernel: str):
         "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": bytes_,
         "peak_choice": which,
         "peak_src": f"{pk['src']} ({'bf16 burst' if which == 'burst' else 'bf16 sustained'}"
+                    f"{' x 2 (fp8/bf16 nominal ratio)' if fp8 else ''}"
                     f"{'' if tensor_bound else '; HBM copy'}); timed region {timed_s:.3f} s at "
                     f"median {clk['sm_mhz'] if clk else '?'} MHz (max "
                     f"{clk['sm_max_mhz'] if clk else '?'})",
@@ -498,12 +504,14 @@ def headline_line(args, w, world, rank, local, dist):
     line = {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if w.dtype == "bf16" else "f32",
+            "dtype": ("e4m3/e5m2" if w.e_format == 1 else "bf16") if w.dtype == "bf16" else "f32",
             "data": "synthetic (seeded E ~ N(0, I/d), stand-in hidden state)",
             "tok_per_s": w.C * value,
             "roofline_pct": roof["step_roofline_pct"],
             "config": {"workload": w.name, "C": w.C, "V": w.V, "d": w.d,
                        "canvases": w.canvases,
+                       "e_format": "e4m3 codes, power-of-two scale per row" if w.e_format == 1
+                                   else "bf16",
                        "token_rule": "multinomial" if w.token_rule == 1 else "argmax",
                        "max_steps": w.max_steps, "mode": "fixed_steps (adaptive stop off)",
                        "kernels": "tc" if den.impl == dg.DG_IMPL_TC else "simt",
@@ -530,6 +538,7 @@ def workload_throughput(w, steps, warmup, local, with_cpu: bool):
     t_b, t_s, _ = step_roofline(w, pk)
     ms_step = ms / steps
     out = {"workload": w.name, "C": w.C, "V": w.V, "d": w.d, "dtype": w.dtype,
+           "e_format": "e4m3 codes, power-of-two scale per row" if w.e_format == 1 else "bf16",
            "mode": "fixed_steps", "steps": steps, "warmup": warmup,
            "value": 1e3 / ms_step, "unit": "steps/s", "ms_per_step": ms_step,
            "tok_per_s": w.C * 1e3 / ms_step, "gpu_launches": launches, "clocks": clk,
@@ -682,6 +691,8 @@ def main():
     ap.add_argument("--parallel", default="replicas", choices=["replicas", "vocab"],
                     help="multi-GPU mode: independent canvases per rank, or one canvas's "
                          "vocabulary split over the ranks")
+    ap.add_argument("--e-format", default="native", choices=["native", "fp8"],
+                    help="E as given (bf16), or e4m3 codes with a power-of-two scale per row")
     ap.add_argument("--token-rule", default="argmax", choices=["argmax", "multinomial"],
                     help="token an accepted position takes")
     ap.add_argument("--canvases", type=int, default=0,
@@ -697,6 +708,8 @@ def main():
     w = synthetic.WORKLOADS[args.workload].replace(fixed_steps=1)
     if args.token_rule == "multinomial":
         w = w.replace(token_rule=1)
+    if args.e_format == "fp8":
+        w = w.replace(e_format=1)
     if args.canvases > 0:
         w = w.replace(canvases=args.canvases, tau=w.tau * w.canvases / args.canvases)
     if args.impl == "reference":
@@ -746,6 +759,10 @@ def main():
             for wk in (synthetic.SMALL, synthetic.LATENCY):
                 wl.append(workload_throughput(wk.replace(fixed_steps=1), max(args.steps, 200),
                                               args.warmup, local, not args.no_cpu_baseline))
+            # narrow E (e4m3 codes): the memory-bound latency canvas and the headline
+            for wk in (synthetic.LATENCY, synthetic.HEADLINE):
+                wl.append(workload_throughput(wk.replace(fixed_steps=1, e_format=1),
+                                              max(args.steps, 200), args.warmup, local, False))
             wl.append(blocks_e2e(synthetic.BLOCKS, E_cpu))
             line["workloads"] = wl
     else:

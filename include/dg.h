@@ -70,6 +70,11 @@ extern "C" {
                                  /* Gumbel-max argmax_v (z_v + G_v), G_v keyed on */
                                  /* (seed, block, 2^61 + step, pos * V + v)       */
 
+/* How the tensor-core kernels hold E (dg_config.e_format). */
+#define DG_E_NATIVE  0       /* E as given (dtype)                             */
+#define DG_E_FP8     1       /* e4m3 codes, one power-of-two scale per row     */
+                             /* (see dg_init)                                  */
+
 /* Kernel family for the vocabulary-attention step. */
 #define DG_IMPL_AUTO  0      /* tensor-core path when the shape allows it     */
 #define DG_IMPL_SIMT  1      /* CUDA-core kernels (any shape, f32 or bf16)    */
@@ -100,6 +105,7 @@ typedef struct dg_config {
   int32_t  shard_v0;        /* vocabulary-parallel step: this context's share  */
   int32_t  shard_nv;        /* is entries [shard_v0, shard_v0 + shard_nv) of E */
                             /* (both multiples of 256; shard_nv = 0: all V)    */
+  int32_t  e_format;        /* DG_E_NATIVE or DG_E_FP8 (tensor-core path, bf16) */
 } dg_config;
 
 typedef struct dg_ctx dg_ctx;
@@ -119,7 +125,7 @@ typedef struct dg_ctx dg_ctx;
 #define DG_SAMPLED  11   /* int32 [C]   multinomial draw of the last step       */
                          /*             (DG_TOKEN_MULTINOMIAL only; read-only) */
 #define DG_EMIT     12   /* int32 [C]   each canvas's prediction at its own     */
-                         /*             stop (read-only)                       */
+                         /*             stop, 0 before it (read-only)          */
 #define DG_CANVAS_STATE 13 /* int32 [3*canvases]: unchanged steps, stopped   */
                            /* (0/1), steps run, per canvas (read-only)       */
 

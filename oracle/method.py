@@ -376,15 +376,25 @@ def begin_block(w, block: int) -> State:
                  steps_c=np.zeros(B, dtype=np.int64), emit=np.zeros(w.C, dtype=np.int64))
 
 
-def step(w, E: np.ndarray, st: State, h: np.ndarray | None = None) -> StepRecord:
-    """One denoise step from state st (mutated in place). h overrides the stand-in."""
+def step(w, E: np.ndarray, st: State, h: np.ndarray | None = None, narrow=None) -> StepRecord:
+    """One denoise step from state st (mutated in place). h overrides the stand-in.
+
+    narrow: an fp8.NarrowE for a workload with narrow E (E must then be its
+    E_deq); the attention then follows fp8.narrow_attention.
+    """
     t = st.t
     T = temperature(t, w.max_steps, w.T_start, w.T_end)
     if h is None:
         h = standin_hidden(w, E, st.target, st.canvas, st.sc, st.block, t)
     multinomial = getattr(w, "token_rule", 0) == 1
-    if multinomial:
-        att = vocab_attention(h, E, w.logit_scale / T, gumbel_key=(w.seed, st.block, t))
+    gkey = (w.seed, st.block, t) if multinomial else None
+    if narrow is not None:
+        from . import fp8
+        prev = st.argmax_prev if st.argmax_prev is not None else st.canvas
+        att, _ = fp8.narrow_attention(narrow, h, w.logit_scale / T, st.canvas, prev,
+                                      gumbel_key=gkey)
+    elif multinomial:
+        att = vocab_attention(h, E, w.logit_scale / T, gumbel_key=gkey)
     else:
         att = vocab_attention(h, E, w.logit_scale / T)
     H32 = att.H.astype(np.float32)
@@ -436,7 +446,7 @@ def step(w, E: np.ndarray, st: State, h: np.ndarray | None = None) -> StepRecord
     return rec
 
 
-def denoise_block(w, E: np.ndarray, block: int):
+def denoise_block(w, E: np.ndarray, block: int, narrow=None):
     """Run the block's canvases to their stops.
 
     Returns (emitted tokens -- each canvas's argmax at its own final step --,
@@ -445,7 +455,7 @@ def denoise_block(w, E: np.ndarray, block: int):
     st = begin_block(w, block)
     records = []
     while not st.done:
-        records.append(step(w, E, st))
+        records.append(step(w, E, st, narrow=narrow))
     return st.emit.copy(), st.steps_done, records
 
 

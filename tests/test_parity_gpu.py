@@ -13,6 +13,7 @@ import torch
 
 import synthetic
 import uniform_state_text_b200 as dg
+from oracle import fp8 as F8
 from oracle import method as M
 from parity import (Tally, check_sampler_exact, compare_attention, compare_draw, h_agreement,
                     near_tie_flags, standin_terms)
@@ -60,12 +61,14 @@ def _np(t):
 
 
 def step_and_compare(den, w, E32, tally: Tally, prev_amax=None, do_step=None, peers=(),
-                     h_given=None):
+                     h_given=None, narrow=None):
     """One GPU step (den.step(), or do_step()) compared with the oracle.
 
     peers: other contexts stepped by do_step (vocabulary shards) that must end
     in exactly den's state. h_given: the step's hidden state was supplied by the
-    caller (compared bit for bit) instead of the stand-in.
+    caller (compared bit for bit) instead of the stand-in. narrow: the oracle's
+    F8.NarrowE of a narrow-E context (E32 is then its E_deq); the attention is
+    the oracle's narrow_attention with the GPU's own row references.
     """
     st0 = den.state()
     if st0["done"]:
@@ -105,8 +108,13 @@ def step_and_compare(den, w, E32, tally: Tally, prev_amax=None, do_step=None, pe
     else:
         assert np.array_equal(h, np.asarray(h_given, np.float64))
     T = M.temperature(t, w.max_steps, w.T_start, w.T_end)
-    if multinomial:
-        att = M.vocab_attention(h, E32, w.logit_scale / T, gumbel_key=(w.seed, b, t))
+    gkey = (w.seed, b, t) if multinomial else None
+    if narrow is not None:
+        m_ref = _np(den.read(dg.DG_MREF)).astype(np.float64)
+        att, _ = F8.narrow_attention(narrow, h, w.logit_scale / T, canvas_in, canvas_in,
+                                     gumbel_key=gkey, m_ref=m_ref)
+    elif multinomial:
+        att = M.vocab_attention(h, E32, w.logit_scale / T, gumbel_key=gkey)
     else:
         att = M.vocab_attention(h, E32, w.logit_scale / T)
     Cc = w.C // B
@@ -153,14 +161,15 @@ def step_and_compare(den, w, E32, tally: Tally, prev_amax=None, do_step=None, pe
     return True
 
 
-def run_teacher_forced(den, w, E32, max_steps=None, do_step=None, peers=()):
+def run_teacher_forced(den, w, E32, max_steps=None, do_step=None, peers=(), narrow=None):
     tally = Tally()
     n = 0
     while max_steps is None or n < max_steps:
         if den.state()["done"]:
             break
         pre = _np(den.read(dg.DG_ARGMAX)).astype(np.int64) if den.state()["has_prev"] else None
-        if not step_and_compare(den, w, E32, tally, pre, do_step=do_step, peers=peers):
+        if not step_and_compare(den, w, E32, tally, pre, do_step=do_step, peers=peers,
+                                narrow=narrow):
             break
         n += 1
     tally.check_budget()
@@ -551,6 +560,61 @@ def test_self_condition_network(shape, emb_dtype):
     else:
         rel = np.linalg.norm(got - want, axis=1) / np.linalg.norm(want, axis=1)
         assert rel.max() < 1e-3, rel.max()
+    den.close()
+
+
+_NARROW = {}
+
+
+def narrow_embedding(w):
+    """The oracle's narrow E (e4m3 codes, per-row exponents) of the workload's E."""
+    key = (w.V, w.d, w.e_seed)
+    if key not in _NARROW:
+        _NARROW.clear()
+        _NARROW[key] = F8.NarrowE(embedding(w)[1])
+    return _NARROW[key]
+
+
+SMALL128 = synthetic.SMALL.replace(name="c128_v16384_d768", C=128, V=16384, d=768,
+                                   tau=0.5 * 128 * np.log(2), coef_target=1.0, coef_canvas=0.5,
+                                   logit_scale=2.0)
+
+
+@pytest.mark.parametrize("name,steps,token_rule", [
+    ("stress_partial_c256_v32768_d1024_bf16", 4, 0),
+    ("stress_partial_c256_v32768_d1024_bf16", 2, 1),
+    ("c128_v16384_d768", 3, 0),
+    ("canvas_c256_v262144_d2048_bf16", 2, 0),
+    ("canvas_c128_v262144_d2816_bf16", 2, 0)])
+def test_fp8_embedding_teacher_forced(name, steps, token_rule):
+    """Narrow E (e4m3 codes with a power-of-two scale per row, h quantised per
+    row, probabilities rounded to e5m2 for p.E): every step against the
+    oracle's narrow-E attention of the GPU's own hidden state and references,
+    on CTA pairs (256 rows) and single CTAs (128 rows), with both token rules."""
+    base = SMALL128 if name == "c128_v16384_d768" else synthetic.WORKLOADS[name]
+    w = base.replace(e_format=dg.DG_E_FP8, fixed_steps=1, token_rule=token_rule)
+    den, _ = make(w, dg.DG_IMPL_TC)
+    nE = narrow_embedding(w)
+    tally = run_teacher_forced(den, w, nE.E_deq, max_steps=steps, narrow=nE)
+    assert tally.steps == steps
+    den.close()
+
+
+def test_fp8_embedding_block_through_the_graph_loop():
+    """A whole adaptive block with narrow E through the captured loop: the
+    emitted tokens and the step count equal the oracle's narrow-E run (its own
+    reference and redo rule)."""
+    w = synthetic.SMALL.replace(e_format=dg.DG_E_FP8, max_steps=8)
+    den, _ = make(w, dg.DG_IMPL_TC)
+    nE = narrow_embedding(w)
+    out, steps = den.block(0)
+    want, want_steps, recs = M.denoise_block(w, nE.E_deq, 0, narrow=nE)
+    assert steps == want_steps
+    ties = np.zeros(w.C, dtype=bool)
+    for r in recs:
+        ties |= r.att.margin < 1e-3
+    bad = np.flatnonzero((_np(out) != want) & ~ties)
+    assert bad.size == 0, bad[:8]
     den.close()
 
 

@@ -24,6 +24,7 @@ DG_STOP_CANVAS, DG_STOP_ARGMAX = 0, 1
 DG_ACCEPT_CUMSUM, DG_ACCEPT_MINUS_MAX = 0, 1
 DG_IMPL_AUTO, DG_IMPL_SIMT, DG_IMPL_TC = 0, 1, 2
 DG_TOKEN_ARGMAX, DG_TOKEN_MULTINOMIAL = 0, 1
+DG_E_NATIVE, DG_E_FP8 = 0, 1
 (DG_CANVAS, DG_ARGMAX, DG_ENTROPY, DG_ACCEPT, DG_SC, DG_HIDDEN, DG_TARGET, DG_ORDER, DG_PREFIX,
  DG_STATE, DG_MREF, DG_SAMPLED, DG_EMIT, DG_CANVAS_STATE) = range(14)
 DG_ST_T, DG_ST_BLOCK, DG_ST_UNCHANGED, DG_ST_DONE, DG_ST_STEPS, DG_ST_K, DG_ST_STATUS, \
@@ -43,6 +44,7 @@ class dg_config(ctypes.Structure):
         ("canvases", ctypes.c_int32),
         ("seed", ctypes.c_uint64),
         ("shard_v0", ctypes.c_int32), ("shard_nv", ctypes.c_int32),
+        ("e_format", ctypes.c_int32),
     ]
 
 
@@ -125,7 +127,7 @@ def make_config(w, impl: int = DG_IMPL_AUTO, shard=None) -> dg_config:
                      fixed_steps=w.fixed_steps, impl=impl,
                      token_rule=getattr(w, "token_rule", 0),
                      canvases=getattr(w, "canvases", 1), seed=w.seed,
-                     shard_v0=v0, shard_nv=nv)
+                     shard_v0=v0, shard_nv=nv, e_format=getattr(w, "e_format", 0))
 
 
 # ----------------------------------------------------------------------------

@@ -25,6 +25,12 @@ thread_local char g_init_err[512] = "";
 
 constexpr size_t kAlign = 256;
 constexpr float kRedoGap = 64.0f;   // largest logit minus reference that P may carry
+// With narrow E, P' = P 2^(Ee[v] - u) must stay within e5m2's range: the
+// reference may lag the row's maximum by at most 4 nats (P <= e^4), and the
+// step exponent u = (largest row exponent of E) - kFp8UOffset then keeps
+// e^4 2^(Ee[v] - u) <= 54.6 * 2^10 < 57344.
+constexpr float kRedoGapFp8 = 4.0f;
+constexpr int kFp8UOffset = 10;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -35,7 +41,9 @@ struct Layout {
   size_t state = 0, scale = 0, target = 0, canvas = 0, argmax = 0, argmax_prev = 0, accept = 0,
          order = 0, prefix = 0, H = 0, mref = 0, rowstat = 0, h = 0, sc = 0,
          tstats = 0, zbuf = 0, partial = 0, tc = 0, sampled = 0, tsamp = 0, h_last = 0,
-         mref_last = 0, cstate = 0, emit = 0, stage[2] = {0, 0}, total = 0;
+         mref_last = 0, cstate = 0, emit = 0, stage[2] = {0, 0}, Eq = 0, Ee = 0, hq = 0, he = 0,
+         emax = 0, total = 0;
+  bool fp8 = false;
   int canvases = 1;
   size_t tc_bytes = 0;
 };
@@ -52,6 +60,10 @@ int check_config(const dg_config* c, char* why, size_t n) {
     snprintf(why, n, "d=%d must be a multiple of 8 in 8..65536", c->d); return DG_EINVAL;
   }
   if (c->dtype != DG_F32 && c->dtype != DG_BF16) { snprintf(why, n, "bad dtype"); return DG_EINVAL; }
+  if (c->e_format != DG_E_NATIVE && c->e_format != DG_E_FP8) { snprintf(why, n, "bad e_format"); return DG_EINVAL; }
+  if (c->e_format == DG_E_FP8 && c->dtype != DG_BF16) {
+    snprintf(why, n, "DG_E_FP8 quantises a bf16 E"); return DG_EINVAL;
+  }
   if (c->max_steps < 1 || c->max_steps > (1 << 20)) { snprintf(why, n, "bad max_steps"); return DG_EINVAL; }
   if (!(c->T_start > 0.f) || !(c->T_end > 0.f) || !std::isfinite(c->T_start) ||
       !std::isfinite(c->T_end)) { snprintf(why, n, "temperatures must be finite and > 0"); return DG_EINVAL; }
@@ -91,6 +103,13 @@ int resolve_impl(const dg_config* c, char* why, size_t n) {
     if (!tc_ok || c->impl == DG_IMPL_SIMT) {
       snprintf(why, n, "a vocabulary shard needs the tensor-core path (bf16, C in {128, 256}, "
                "d %% 256 == 0)");
+      return -1;
+    }
+    return DG_IMPL_TC;
+  }
+  if (c->e_format == DG_E_FP8) {
+    if (!tc_ok || c->impl == DG_IMPL_SIMT) {
+      snprintf(why, n, "DG_E_FP8 needs the tensor-core path (bf16, C in {128, 256}, d %% 256 == 0)");
       return -1;
     }
     return DG_IMPL_TC;
@@ -151,11 +170,21 @@ int make_layout(const dg_config* c, Layout* L, char* why, size_t n) {
     const int nv = shard_nv(c);             // the vocabulary this context's kernels cover
     L->ntiles = tc_stat_tiles(c->C, nv, c->d);
     L->tstats = take(sizeof(TileStat) * C * L->ntiles);
-    L->tc_bytes = tc_workspace_bytes(c->C, nv, c->d);
+    L->fp8 = c->e_format == DG_E_FP8;
+    L->tc_bytes = tc_workspace_bytes(c->C, nv, c->d, L->fp8);
     L->tc = take(L->tc_bytes);
     L->h_last = take(esz * C * d);
     L->mref_last = take(4 * C);
     if (c->token_rule == DG_TOKEN_MULTINOMIAL) L->tsamp = take(tc_draw_bytes(c->C, nv, c->d));
+    if (L->fp8) {
+      // e4m3 codes of all of E (the stand-in gathers rows anywhere in it) and
+      // of h, their per-row exponents, and the largest exponent of E
+      L->Eq = take(V * d);
+      L->Ee = take(4 * V);
+      L->hq = take(C * d);
+      L->he = take(4 * C);
+      L->emax = take(4);
+    }
   }
   L->total = off;
   return DG_OK;
@@ -195,6 +224,9 @@ struct dg_ctx {
   // host-to-device copies of external hidden states: a copy stream, and per
   // staging slot an event when its copy landed and one when its last reader ran
   cudaStream_t copy_stream = nullptr;
+  // narrow E: the step exponent of P and the largest reference lag before a redo
+  int fp8_u = 0;
+  float redo_gap = kRedoGap;
   cudaEvent_t ev_copied[2] = {nullptr, nullptr}, ev_free[2] = {nullptr, nullptr};
   int stage_slot = 0;
   // profiling
@@ -250,6 +282,8 @@ NextStandin next_standin(dg_ctx* ctx) {
   tc_counters(ctx->tc_plan, &nx.zero, &nx.nzero);
   nx.h_last = at<void>(ctx, ctx->L.h_last);
   nx.mref_last = at<float>(ctx, ctx->L.mref_last);
+  nx.fp8 = ctx->L.fp8 ? 1 : 0;
+  nx.sc_scale = ctx->L.fp8 ? std::ldexp(1.0f, ctx->fp8_u) : 1.0f;
   return nx;
 }
 
@@ -261,6 +295,16 @@ int prologue_if_needed(dg_ctx* ctx, bool standin, bool use_cond, const void* hsr
   unsigned* zero = nullptr;
   int nzero = 0;
   if (tc) tc_counters(ctx->tc_plan, &zero, &nzero);
+  if (ctx->L.fp8) {
+    // narrow E: h (stand-in or the caller's), its e4m3 codes and m_ref, every step
+    DG_CK(launch_prologue_fp8(ctx->stream, ctx->st, at<uint8_t>(ctx, ctx->L.Eq),
+                              at<int32_t>(ctx, ctx->L.Ee), ctx->target, ctx->canvas, ctx->sc,
+                              ctx->h, hsrc, at<uint8_t>(ctx, ctx->L.hq), at<int32_t>(ctx, ctx->L.he),
+                              ctx->mref, c.C, c.V, c.d, c.seed, c.coef_target, c.coef_canvas,
+                              standin_sigma(c), standin ? 1 : 0, ctx->scale_tab, c.max_steps,
+                              ctx->argmax_prev, zero, nzero));
+    return 1;
+  }
   // After a tensor-core step the merge kernel has already written this step's
   // stand-in h and m_ref (DevState::h_ready); a stepwise call then skips the
   // prologue launch. The captured block loop has none: dg_denoise_block runs
@@ -297,12 +341,12 @@ int launch_step(dg_ctx* ctx, bool standin, bool use_cond, const void* hsrc = nul
   if (tc) {
     DG_CK(launch_tc_attention(s, ctx->tc_plan, ctx->st, ctx->h, ctx->E, ctx->mref, ctx->scale_tab,
                               c.max_steps, ctx->tstats, ctx->tc, ctx->draw, ctx->H,
-                              ctx->argmax, ctx->rowstat, kRedoGap, sa));
+                              ctx->argmax, ctx->rowstat, ctx->redo_gap, sa));
     if (e1) DG_CK(cudaEventRecord(e1, s));
     // sc, the next step's h (and, if a row needs the exact recomputation, the
     // rows' merge and the sampler)
     DG_CK(launch_tc_merge(s, ctx->tc_plan, ctx->st, ctx->tstats, ctx->mref, ctx->rowstat, ctx->H,
-                          ctx->argmax, ctx->sc, kRedoGap, ctx->h, ctx->E,
+                          ctx->argmax, ctx->sc, ctx->redo_gap, ctx->h, ctx->E,
                           ctx->scale_tab, c.max_steps, sa, ctx->draw, next_standin(ctx)));
     // the merge prepares the next step's h unless the block stopped, and then
     // nothing more runs until dg_begin_block
@@ -417,9 +461,34 @@ int dg_init(const dg_config* cfg, const void* E, void* workspace, size_t ws_byte
     ctx->partial = at<float>(ctx, L.partial);
   } else {
     ctx->tc = at<void>(ctx, L.tc);
+    TcFp8 f8;
+    if (L.fp8) {
+      // quantise E once: e4m3 codes with a power-of-two scale per row
+      int* emax = at<int>(ctx, L.emax);
+      int emax_h = 0;
+      cudaError_t e = cudaMemsetAsync(emax, 0x80, sizeof(int), ctx->stream);   // very negative
+      if (e == cudaSuccess)
+        e = launch_quantize_e(ctx->stream, E, cfg->V, cfg->d, at<uint8_t>(ctx, L.Eq),
+                              at<int32_t>(ctx, L.Ee), emax);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(&emax_h, emax, sizeof(int), cudaMemcpyDeviceToHost, ctx->stream);
+      if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->stream);
+      if (e != cudaSuccess) {
+        fail(nullptr, DG_ECUDA, "quantising E: %s", cudaGetErrorString(e));
+        delete ctx;
+        return DG_ECUDA;
+      }
+      ctx->fp8_u = emax_h - kFp8UOffset;
+      ctx->redo_gap = kRedoGapFp8;
+      f8.Eq = at<uint8_t>(ctx, L.Eq);
+      f8.Ee = at<int32_t>(ctx, L.Ee);
+      f8.hq = at<uint8_t>(ctx, L.hq);
+      f8.he = at<int32_t>(ctx, L.he);
+      f8.u = ctx->fp8_u;
+    }
     rc = tc_plan_init(&ctx->tc_plan, cfg->C, shard_nv(cfg), cfg->d, E, ctx->h, ctx->tc,
                       ctx->err, sizeof(ctx->err),
-                      sharded(cfg) ? cfg->shard_v0 : 0, cfg->V);
+                      sharded(cfg) ? cfg->shard_v0 : 0, cfg->V, L.fp8 ? &f8 : nullptr);
     if (rc) {
       snprintf(g_init_err, sizeof(g_init_err), "%s", ctx->err);
       delete ctx;
@@ -458,7 +527,8 @@ int dg_begin_block(dg_ctx* ctx, int32_t block) {
   if (block < 0) return fail(ctx, DG_EINVAL, "block must be >= 0");
   const dg_config& c = ctx->cfg;
   DG_CK(launch_begin_block(ctx->stream, ctx->st, ctx->target, ctx->canvas, ctx->sc, c.C, c.d, c.V,
-                           c.seed, block, at<int32_t>(ctx, ctx->L.cstate), 3 * ctx->L.canvases));
+                           c.seed, block, at<int32_t>(ctx, ctx->L.cstate), 3 * ctx->L.canvases,
+                           at<int32_t>(ctx, ctx->L.emit)));
   ctx->launches += 1;
   ctx->h_ready = false;
   return DG_OK;
@@ -536,8 +606,9 @@ int dg_denoise_block(dg_ctx* ctx, int32_t block, int32_t* out_dev, int32_t* step
   int rc = dg_begin_block(ctx, block);
   if (rc) return rc;
   // The tensor-core loop's first step needs the stand-in h and m_ref; the
-  // merge of each step prepares the next one's.
-  if (ctx->L.impl == DG_IMPL_TC) {
+  // merge of each step prepares the next one's (narrow E: the loop runs its
+  // own prologue every step).
+  if (ctx->L.impl == DG_IMPL_TC && !ctx->L.fp8) {
     rc = prologue_if_needed(ctx, true, false);
     if (rc < 0) return rc;
     ctx->launches += rc;
@@ -616,7 +687,7 @@ int dg_denoise_step_finish(dg_ctx* ctx, const void* partials) {
   const dg_config& c = ctx->cfg;
   ctx->launches += 2;
   DG_CK(launch_tc_finish(ctx->stream, ctx->tc_plan, ctx->st, partials, ctx->tstats, ctx->draw,
-                         ctx->mref, ctx->rowstat, ctx->H, ctx->argmax, ctx->sc, kRedoGap, ctx->h,
+                         ctx->mref, ctx->rowstat, ctx->H, ctx->argmax, ctx->sc, ctx->redo_gap, ctx->h,
                          ctx->E, ctx->scale_tab, c.max_steps, sampler_args(ctx, false),
                          next_standin(ctx)));
   ctx->h_ready = true;

@@ -27,7 +27,7 @@ namespace dg {
 // ---------------------------------------------------------------------------
 __global__ void k_begin_block(DevState* st, int32_t* target, int32_t* canvas, float* sc,
                               int C, int d, int V, uint64_t seed, int block, int32_t* cstate,
-                              int ncstate) {
+                              int ncstate, int32_t* emit) {
   const uint64_t sb = seed + (uint64_t)(uint32_t)block;
   const uint64_t pt = key_prefix(sb, 0, kTagTarget);
   const uint64_t pc = key_prefix(sb, 0, kTagInitCanvas);
@@ -38,6 +38,7 @@ __global__ void k_begin_block(DevState* st, int32_t* target, int32_t* canvas, fl
     if (i < (size_t)C) {
       target[i] = (int32_t)(sm64(pt ^ (uint64_t)i) & (uint64_t)(V - 1));
       canvas[i] = (int32_t)(sm64(pc ^ (uint64_t)i) & (uint64_t)(V - 1));
+      emit[i] = 0;                       // no canvas has stopped in this block yet
     }
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -370,13 +371,13 @@ __global__ void __launch_bounds__(1024) k_sampler(SamplerArgs a) {
 // ---------------------------------------------------------------------------
 cudaError_t launch_begin_block(cudaStream_t s, DevState* st, int32_t* target, int32_t* canvas,
                                float* sc, int C, int d, int V, uint64_t seed, int block,
-                               int32_t* cstate, int ncstate) {
+                               int32_t* cstate, int ncstate, int32_t* emit) {
   const size_t n = (size_t)C * d;
   int grid = (int)((n + 255) / 256);
   if (grid > 4096) grid = 4096;
   if (grid < 1) grid = 1;
   k_begin_block<<<grid, 256, 0, s>>>(st, target, canvas, sc, C, d, V, seed, block, cstate,
-                                     ncstate);
+                                     ncstate, emit);
   return cudaGetLastError();
 }
 

@@ -68,6 +68,10 @@ struct NextStandin {
   int nzero = 0;
   void* h_last = nullptr;                 // [C][d] bf16: copy of the step's own h
   float* mref_last = nullptr;             // [C]: copy of the step's own m_ref
+  // Narrow E: the next step's h, its codes and m_ref come from the narrow-E
+  // prologue instead, and the P.E sums carry a factor 2^-u (sc_scale = 2^u).
+  int fp8 = 0;
+  float sc_scale = 1.f;
 };
 
 // Multinomial token draw (DG_TOKEN_MULTINOMIAL): where the per-row draws go.
@@ -80,7 +84,7 @@ struct DrawArgs {
 
 cudaError_t launch_begin_block(cudaStream_t s, DevState* st, int32_t* target, int32_t* canvas,
                                float* sc, int C, int d, int V, uint64_t seed, int block,
-                               int32_t* cstate, int ncstate);
+                               int32_t* cstate, int ncstate, int32_t* emit);
 
 cudaError_t launch_prologue(cudaStream_t s, int dtype, const DevState* st, const void* E,
                             const int32_t* target, const int32_t* canvas, const float* sc,

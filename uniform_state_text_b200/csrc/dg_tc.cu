@@ -45,6 +45,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -87,7 +88,7 @@ struct Params {
   float* mref;                 // per-row logit reference; the first pass raises a low one
   const float* scale_tab;
   float* Opart;              // [G][C][d]
-  __nv_bfloat16* P;          // [RING][C][BN]: ring of P tiles
+  void* P;                   // [RING][C][BN]: ring of P tiles (bf16, or e5m2 codes for F8)
   unsigned* ready;           // [n_vt]: epilogue warps that finished a tile
   unsigned* consumed;        // [n_vt]: G2 CTAs that finished loading a tile
   int* abort_flag;
@@ -103,6 +104,12 @@ struct Params {
   // pass raised its redo flag (redo_in) and then uses its own counter set.
   int pass;
   const int* redo_in;
+  // Narrow E (e4m3 codes, F8 instantiations): per-row exponents of E (global
+  // row index) and of h, and the step exponent u: P' = P 2^(Ee[v] - u) is
+  // rounded to e5m2 for the P.E contraction, whose sums are 2^-u sc Z.
+  const int32_t* Ee;
+  const int32_t* he;
+  int u;
   TcStat* tstats2;             // [C][2 * n_vt] half-tile statistics
   TcSamp* tsamp;               // [C][2 * n_vt] best z + G (multinomial draw), or nullptr
   uint64_t seed;               // keys the draw's Gumbel variates
@@ -355,9 +362,50 @@ __device__ __noinline__ void g1_finish(const Params& p, int ng1, unsigned char* 
   }
 }
 
+// Elements per 128-byte operand row, and per MMA instruction along K.
+template <bool F8> struct Fmt {
+  static constexpr int BKE = F8 ? 128 : 64;   // K elements per pipeline stage
+  static constexpr int KPI = F8 ? 32 : 16;    // K elements per tcgen05.mma
+  static constexpr int TPS = BN / BKE;        // G2 stages per 256-entry tile
+  static constexpr int BOXC = F8 ? 128 : 64;  // columns of d per E box of the P.E operand
+};
+
+template <int CG, bool F8>
+__device__ __forceinline__ void mma_k(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                      uint32_t accumulate) {
+  if constexpr (!F8) {
+    mma<CG>(d_tmem, a, b, idesc, accumulate);
+  } else if constexpr (CG == 2) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
+}
+
+// Instruction descriptor of kind::f8f6f4 with fp32 accumulation: A and B
+// formats (0 = e4m3, 1 = e5m2), B K- or MN-major.
+__host__ __device__ constexpr uint32_t idesc_f8(int M, int N, int a_fmt, int b_fmt, int b_mn_major) {
+  return (1u << 4) | ((uint32_t)a_fmt << 7) | ((uint32_t)b_fmt << 10) |
+         ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// A power of two 2^e as a float (e in [-126, 127]).
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
+
 // DRAW: the multinomial rule's Gumbel-max draw in the G1 epilogue (a separate
-// instantiation, so the argmax kernel keeps its register budget).
-template <int CG, bool DRAW>
+// instantiation, so the argmax kernel keeps its register budget). F8: operands
+// are 8-bit (h and E as e4m3 codes, P as e5m2), see Params::Ee.
+template <int CG, bool DRAW, bool F8>
 __global__ void __launch_bounds__(THREADS, 1)
     k_vocab_attention(const __grid_constant__ CUtensorMap tm_h,
                       const __grid_constant__ CUtensorMap tm_ek,
@@ -441,6 +489,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   // after the wait. No early trigger: merge CTAs waiting beside this kernel
   // for its whole duration cost more than their launch saves (measured).
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // The first pass lets the redo pass launch now: its CTAs (as large as these)
+  // can only take SMs this grid has left, and wait there for it to complete,
+  // so that its check of the redo flag follows this pass without a launch gap.
+  if (p.pass == 0) asm volatile("griddepcontrol.launch_dependents;");
   const bool skip = p.st->done != 0;                     // uniform over the grid
   // CTA 0 is a G1 CTA: this reset precedes its g1_done release, so it is
   // ordered before the sampler sets the flag again at the end of G1. A skipped
@@ -451,8 +503,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   // cover both row blocks with M = 256).
   const int RBI = CG == 2 ? 1 : p.RB;
   const int n_items1 = RBI * p.n_vt;
-  const int nk1 = p.d / BK;
-  const int nk2 = KV2 / BK;
+  constexpr int BKE = Fmt<F8>::BKE, KPI = Fmt<F8>::KPI, TPS = Fmt<F8>::TPS, BOXC = Fmt<F8>::BOXC;
+  const int nk1 = p.d / BKE;
+  const int nk2 = KV2 / BKE;
   int g = 0, rb2 = 0, dt = 0;
   if (!is_g1) {
     const int o = unit - p.n1;
@@ -501,8 +554,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             TR_ADD(w_empty);
             unsigned char* st = smem + s * STAGE_BYTES;
             if (leader) mbar_expect_tx(&full[s], STAGE_BYTES * CG);
-            tma_load<CG>(st, &tm_h, &full[s], kc * BK, rb * BM, keep);
-            tma_load<CG>(st + A_BYTES, &tm_ek, &full[s], kc * BK, vt * BN + (int)rank * NB_ROWS, keep);
+            tma_load<CG>(st, &tm_h, &full[s], kc * BKE, rb * BM, keep);
+            tma_load<CG>(st + A_BYTES, &tm_ek, &full[s], kc * BKE, vt * BN + (int)rank * NB_ROWS, keep);
             ++issued;
             if (++s == STAGES) { s = 0; ph ^= 1; }
           }
@@ -510,8 +563,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       } else {
         for (int r = g; ok && r < p.n_ranges; r += p.G) {
           for (int kc = 0; kc < nk2; ++kc) {
-            const int vt = r * p.tiles_per_range + kc / (BN / BK);
-            if (kc % (BN / BK) == 0) {
+            const int vt = r * p.tiles_per_range + kc / TPS;
+            if (kc % TPS == 0) {
               TR_T0();
               if (!counter_wait(&p.ready[vt], ready_target + p.stall, p)) { ok = false; break; }
               TR_ADD(w_ctr);
@@ -522,14 +575,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             TR_ADD(w_empty);
             unsigned char* st = smem + s * STAGE_BYTES;
             if (leader) mbar_expect_tx(&full[s], STAGE_BYTES * CG);
-            tma_load<CG>(st, &tm_p, &full[s], (kc % (BN / BK)) * BK, (vt % RING) * p.C + rb2 * BM,
+            tma_load<CG>(st, &tm_p, &full[s], (kc % TPS) * BKE, (vt % RING) * p.C + rb2 * BM,
                          keep);
+            // E as the MN-major B operand: boxes of BOXC columns of d (128 bytes)
+            // by BKE vocabulary rows
             for (int b = 0; b < p.W2; ++b)
 #pragma unroll
-              for (int j = 0; j < NB_ROWS / 64; ++j)
-                tma_load<CG>(st + A_BYTES + (b * (NB_ROWS / 64) + j) * (64 * BK * 2), &tm_emn,
-                             &full[s], (dt * p.W2 + b) * BN + (int)rank * NB_ROWS + j * 64,
-                             r * KV2 + kc * BK, drop);
+              for (int j = 0; j < NB_ROWS / BOXC; ++j)
+                tma_load<CG>(st + A_BYTES + (b * (NB_ROWS / BOXC) + j) * (128 * BKE), &tm_emn,
+                             &full[s], (dt * p.W2 + b) * BN + (int)rank * NB_ROWS + j * BOXC,
+                             r * KV2 + kc * BKE, drop);
             ++issued;
             if (++s == STAGES) { s = 0; ph ^= 1; }
           }
@@ -554,7 +609,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t ph = 0;
       bool ok = true;
       if (is_g1) {
-        const uint32_t idesc = idesc_bf16(BM * CG, BN, 0);
+        const uint32_t idesc = F8 ? idesc_f8(BM * CG, BN, 0, 0, 0) : idesc_bf16(BM * CG, BN, 0);
         for (int n = 0; ok; ++n) {
           int it;
           if (!item_take<CG>(n, &it, item_full, item_empty, item_q, true, p)) { ok = false; break; }
@@ -575,10 +630,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
             const uint32_t b0 = a0 + A_BYTES;
 #pragma unroll
-            for (int k = 0; k < BK / 16; ++k) {
+            for (int k = 0; k < BKE / KPI; ++k) {      // 32 bytes of K per instruction
               const uint64_t ad = sdesc(a0 + k * 32, 16, 1024);
               const uint64_t bd = sdesc(b0 + k * 32, 16, 1024);
-              mma<CG>(d_tmem, ad, bd, idesc, (kc | k) ? 1u : 0u);
+              mma_k<CG, F8>(d_tmem, ad, bd, idesc, (kc | k) ? 1u : 0u);
             }
             commit<CG>(&empty[s]);
             if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -587,7 +642,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           commit<CG>(&acc_full[buf]);
         }
       } else {
-        const uint32_t idesc = idesc_bf16(BM * CG, BN, 1);
+        const uint32_t idesc = F8 ? idesc_f8(BM * CG, BN, 1, 0, 1) : idesc_bf16(BM * CG, BN, 1);
         bool first = true;
         for (int r = g; ok && r < p.n_ranges; r += p.G) {
           for (int kc = 0; kc < nk2; ++kc) {
@@ -595,18 +650,19 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (!mbar_wait(&full[s], ph, p)) { ok = false; break; }
             TR_ADD(w_full);
             tc_fence_after();
-            if (kc % (BN / BK) == BN / BK - 1)      // the tile's P is now in shared memory
-              red_relaxed_add(&p.consumed[r * p.tiles_per_range + kc / (BN / BK)], 1u);
+            if (kc % TPS == TPS - 1)                 // the tile's P is now in shared memory
+              red_relaxed_add(&p.consumed[r * p.tiles_per_range + kc / TPS], 1u);
             const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
             const uint32_t b0 = a0 + A_BYTES;
 #pragma unroll
-            for (int k = 0; k < BK / 16; ++k) {
+            for (int k = 0; k < BKE / KPI; ++k) {
               const uint64_t ad = sdesc(a0 + k * 32, 16, 1024);
               for (int b = 0; b < p.W2; ++b) {
-                // MN-major B: 64-column blocks 8 KB apart (LBO), 8-row K groups 1 KB apart (SBO)
-                const uint64_t bd = sdesc(b0 + b * (NB_ROWS / 64) * (64 * BK * 2) + k * (16 * 128),
-                                          64 * BK * 2, 1024);
-                mma<CG>(tmem + b * BN, ad, bd, idesc, first ? 0u : 1u);
+                // MN-major B: 128-byte column blocks (one box each) 128 * BKE bytes
+                // apart (LBO), 8-row K groups 1 KB apart (SBO); KPI rows per instruction
+                const uint64_t bd = sdesc(b0 + b * (NB_ROWS / BOXC) * (128 * BKE) + k * (KPI * 128),
+                                          128 * BKE, 1024);
+                mma_k<CG, F8>(tmem + b * BN, ad, bd, idesc, first ? 0u : 1u);
               }
               first = false;
             }
@@ -672,12 +728,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int row = rb * BM + r_local;
         const float mref = p.mref[row];
         const float k0 = -mref * 1.4426950408889634f;
+        const int he_row = F8 ? p.he[row] : 0;     // the row's exponent of h (F8)
         // P = 2^(k1 v + k0) = e^(z - mref); Z = sum P; S2 = sum P (z - mref) log2(e).
         float Z = 0.f, S2 = 0.f, vbest = -INFINITY;
         int arg = 0x7fffffff;
         float gbest = -INFINITY;    // multinomial draw: best z + G, first index on ties
         int garg = 0x7fffffff;
-        __nv_bfloat16* prow = p.P + ((size_t)((vt % RING) * p.C + row)) * BN + c0;
+        unsigned char* prow = static_cast<unsigned char*>(p.P) +
+                              (((size_t)(vt % RING) * p.C + row) * BN + c0) * (F8 ? 1 : 2);
 #pragma unroll 1
         for (int c = 0; c < HALF / 32; ++c) {
           float v[32];
@@ -693,6 +751,18 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (lane == 0) mbar_arrive_remote_relaxed(acc_empty_addr + buf * 8);
           }
           TR_T0();
+          int eev[32];              // F8: exponents of the chunk's 32 vocabulary rows
+          if constexpr (F8) {
+            const int4* ep = reinterpret_cast<const int4*>(p.Ee + p.v0 + vt * BN + c0 + c * 32);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int4 q4 = __ldg(ep + j);
+              eev[4 * j] = q4.x; eev[4 * j + 1] = q4.y; eev[4 * j + 2] = q4.z; eev[4 * j + 3] = q4.w;
+            }
+            // the tensor cores summed code products: scale back to h_deq . E_deq
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] *= pow2f(eev[j] + he_row);
+          }
           float cm = v[0];
 #pragma unroll
           for (int j = 1; j < 32; ++j) cm = fmaxf(cm, v[j]);
@@ -725,15 +795,30 @@ __global__ void __launch_bounds__(THREADS, 1)
             const float e0 = ex2(x0), e1 = ex2(x1);
             Z += e0 + e1;
             S2 = fmaf(e0, x0, fmaf(e1, x1, S2));
-            pk[j >> 1] = pack_bf16(e0, e1);
+            if constexpr (F8) {
+              // P' = P 2^(Ee[v] - u) as e5m2 (lower byte: the lower column)
+              const uint32_t two = __nv_cvt_float2_to_fp8x2(
+                  make_float2(e0 * pow2f(eev[j] - p.u), e1 * pow2f(eev[j + 1] - p.u)),
+                  __NV_SATFINITE, __NV_E5M2);
+              if (j & 2) pk[j >> 2] |= two << 16;
+              else pk[j >> 2] = two;
+            } else {
+              pk[j >> 1] = pack_bf16(e0, e1);
+            }
           }
           TR_ADD(t_math);
           {
             TR_T0();
-            uint4* dst = reinterpret_cast<uint4*>(prow + c * 32);
+            if constexpr (F8) {
+              uint4* dst = reinterpret_cast<uint4*>(prow + c * 32);
+              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(prow + c * 64);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+              for (int j = 0; j < 4; ++j)
+                dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            }
             TR_ADD(t_st);
           }
         }
@@ -870,7 +955,7 @@ __device__ __forceinline__ void merge_fast_tail(DevState* st, const float* Opart
     int S, const int32_t* argmax, const int32_t* canvas, float* mref, const float* inv_row,
     const NextStandin& nx, int i0) {
   __shared__ float red[kMergeRows * kMergeThreadsPerRow / 32][2 * kMergeRows];
-  const bool prep = *(volatile int*)&st->done == 0;
+  const bool prep = !nx.fp8 && *(volatile int*)&st->done == 0;
   const int t1 = *(volatile int*)&st->t;                 // the next step (the sampler advanced it)
   const uint64_t pre = key_prefix(nx.seed, (uint64_t)(uint32_t)*(volatile int*)&st->block,
                                   kTagNoise + (uint64_t)t1);
@@ -893,7 +978,7 @@ __device__ __forceinline__ void merge_fast_tail(DevState* st, const float* Opart
       const float4 o = *reinterpret_cast<const float4*>(Opart + g * pstride + off);
       acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
     }
-    const float inv = inv_row[q];
+    const float inv = inv_row[q] * nx.sc_scale;
     const float s4[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
     *reinterpret_cast<float4*>(sc + off) = make_float4(s4[0], s4[1], s4[2], s4[3]);
     const uint2 hold = *reinterpret_cast<const uint2*>(h + off);
@@ -1068,7 +1153,7 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
       if (redo) atomicAdd(&st->redo, 1);
     }
     sh_redo[r] = redo;
-    sh_inv[r] = 1.0f / Z;
+    sh_inv[r] = nx.sc_scale / Z;
     sh_best[r] = best;
   }
   __syncthreads();
@@ -1152,7 +1237,7 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
         }
       }
     }
-    sh_go = go && !*(volatile int*)&st->done;
+    sh_go = go && !nx.fp8 && !*(volatile int*)&st->done;
   }
   __syncthreads();
   if (blockIdx.x == 0) {
@@ -1212,7 +1297,7 @@ int device_sms() {
   return 148;
 }
 
-TcLayout tc_layout(int C, int V, int d, int sms) {
+TcLayout tc_layout(int C, int V, int d, int sms, bool fp8 = false) {
   TcLayout L;
   L.CG = C == 256 ? 2 : 1;
   L.W2 = (L.CG == 2 && d % (2 * tc::BN) == 0) ? 2 : 1;
@@ -1244,7 +1329,7 @@ TcLayout tc_layout(int C, int V, int d, int sms) {
   size_t off = 0;
   // two sets of hand-off counters: the first pass's and the redo pass's
   L.counters = off; off = al(off + sizeof(unsigned) * 2 * (2 * (size_t)L.n_vt + 64));
-  L.P = off; off = al(off + (size_t)tc::RING * C * tc::BN * 2);
+  L.P = off; off = al(off + (size_t)tc::RING * C * tc::BN * (fp8 ? 1 : 2));
   L.Opart = off; off = al(off + (size_t)(L.G > 0 ? L.G : 1) * C * d * 4);
   L.trace = off; off = al(off + (size_t)256 * 32 * 8);
   L.total = off;
@@ -1267,14 +1352,14 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
 }
 
 bool encode(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
-            uint32_t box_outer) {
+            uint32_t box_outer, bool bytes = false) {
   auto fn = get_encoder();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * 2};
+  cuuint64_t strides[1] = {inner * (bytes ? 1 : 2)};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+  CUresult r = fn(m, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -1310,13 +1395,15 @@ bool tc_schedule_info(int C, int V, int d, int sms, int32_t* out) {
   return true;
 }
 
-size_t tc_workspace_bytes(int C, int V, int d) { return tc_layout(C, V, d, device_sms()).total; }
+size_t tc_workspace_bytes(int C, int V, int d, bool fp8) {
+  return tc_layout(C, V, d, device_sms(), fp8).total;
+}
 
 size_t tc_draw_bytes(int C, int V, int) { return sizeof(TcSamp) * (size_t)C * 2 * (V / tc::BN); }
 
 int tc_launches(const TcPlan&) { return 2; }
 
-template <int CG, bool DRAW>
+template <int CG, bool DRAW, bool F8>
 cudaError_t launch_kernel(cudaStream_t s, int units, const CUtensorMap* maps, const tc::Params& prm) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(units * CG);
@@ -1340,14 +1427,14 @@ cudaError_t launch_kernel(cudaStream_t s, int units, const CUtensorMap* maps, co
     attr[0].val.cooperative = 1;
     cfg.numAttrs = 1;
   }
-  return cudaLaunchKernelEx(&cfg, tc::k_vocab_attention<CG, DRAW>, maps[0], maps[1], maps[2],
+  return cudaLaunchKernelEx(&cfg, tc::k_vocab_attention<CG, DRAW, F8>, maps[0], maps[1], maps[2],
                             maps[3], prm);
 }
 
 // Every unit of the persistent grid must be resident at once (they wait on one another).
-template <int CG, bool DRAW>
+template <int CG, bool DRAW, bool F8>
 int check_residency(int units, int sms, char* err, size_t errn) {
-  cudaError_t e = cudaFuncSetAttribute(tc::k_vocab_attention<CG, DRAW>,
+  cudaError_t e = cudaFuncSetAttribute(tc::k_vocab_attention<CG, DRAW, F8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)tc::Pipe<CG>::SMEM);
   if (e != cudaSuccess) {
@@ -1367,10 +1454,10 @@ int check_residency(int units, int sms, char* err, size_t errn) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaOccupancyMaxActiveClusters(&fit, tc::k_vocab_attention<CG, DRAW>, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&fit, tc::k_vocab_attention<CG, DRAW, F8>, &cfg);
   } else {
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tc::k_vocab_attention<CG, DRAW>,
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tc::k_vocab_attention<CG, DRAW, F8>,
                                                       tc::THREADS, tc::Pipe<CG>::SMEM);
     fit = per_sm * sms;
   }
@@ -1383,13 +1470,22 @@ int check_residency(int units, int sms, char* err, size_t errn) {
 }
 
 int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, void* ws, char* err,
-                 size_t errn, int v0, int Vg) {
+                 size_t errn, int v0, int Vg, const TcFp8* f8) {
   p->C = C; p->V = V; p->d = d;
   p->v0 = v0; p->Vg = Vg;
+  p->fp8 = f8 != nullptr;
+  if (f8) {
+    // the kernels read the e4m3 codes of E and h instead of the bf16 arrays
+    E = f8->Eq;
+    h = const_cast<uint8_t*>(f8->hq);
+    p->Ee = f8->Ee;
+    p->he = f8->he;
+    p->u = f8->u;
+  }
   // the kernels' E tensor maps start at the shard's first row
-  E = static_cast<const __nv_bfloat16*>(E) + (size_t)v0 * d;
+  E = static_cast<const unsigned char*>(E) + (size_t)v0 * d * (f8 ? 1 : 2);
   p->num_sms = device_sms();
-  TcLayout L = tc_layout(C, V, d, p->num_sms);
+  TcLayout L = tc_layout(C, V, d, p->num_sms, p->fp8);
   if (L.G < 1 || L.n1 < 1) {
     snprintf(err, errn, "the tensor-core kernels need more SMs than this device offers (%d)",
              p->num_sms);
@@ -1400,20 +1496,32 @@ int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, void* w
   char* base = static_cast<char*>(ws);
   static_assert(sizeof(CUtensorMap) <= 128, "tensor map size");
   CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(p->maps);
-  bool ok = encode(&maps[0], h, (uint64_t)d, (uint64_t)C, tc::BK, tc::BM) &&
-            encode(&maps[1], E, (uint64_t)d, (uint64_t)V, tc::BK, tc::BN / L.CG) &&
-            encode(&maps[2], E, (uint64_t)d, (uint64_t)V, tc::BK, 64) &&
-            encode(&maps[3], base + L.P, (uint64_t)tc::BN, (uint64_t)tc::RING * C, tc::BK, tc::BM);
+  // every box row is 128 bytes: 64 bf16 or 128 e4m3/e5m2 elements
+  const uint32_t bk = p->fp8 ? 128 : tc::BK, boxc = p->fp8 ? 128 : 64;
+  const bool b8 = p->fp8;
+  bool ok = encode(&maps[0], h, (uint64_t)d, (uint64_t)C, bk, tc::BM, b8) &&
+            encode(&maps[1], E, (uint64_t)d, (uint64_t)V, bk, tc::BN / L.CG, b8) &&
+            encode(&maps[2], E, (uint64_t)d, (uint64_t)V, boxc, bk, b8) &&
+            encode(&maps[3], base + L.P, (uint64_t)tc::BN, (uint64_t)tc::RING * C, bk, tc::BM, b8);
   if (!ok) {
     snprintf(err, errn, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
     return -3;
   }
   // both instantiations (argmax rule, multinomial draw) must fit
-  int rc = L.CG == 2 ? check_residency<2, false>(p->grid, p->num_sms, err, errn)
-                     : check_residency<1, false>(p->grid, p->num_sms, err, errn);
-  if (!rc)
-    rc = L.CG == 2 ? check_residency<2, true>(p->grid, p->num_sms, err, errn)
-                   : check_residency<1, true>(p->grid, p->num_sms, err, errn);
+  int rc;
+  if (p->fp8) {
+    rc = L.CG == 2 ? check_residency<2, false, true>(p->grid, p->num_sms, err, errn)
+                   : check_residency<1, false, true>(p->grid, p->num_sms, err, errn);
+    if (!rc)
+      rc = L.CG == 2 ? check_residency<2, true, true>(p->grid, p->num_sms, err, errn)
+                     : check_residency<1, true, true>(p->grid, p->num_sms, err, errn);
+  } else {
+    rc = L.CG == 2 ? check_residency<2, false, false>(p->grid, p->num_sms, err, errn)
+                   : check_residency<1, false, false>(p->grid, p->num_sms, err, errn);
+    if (!rc)
+      rc = L.CG == 2 ? check_residency<2, true, false>(p->grid, p->num_sms, err, errn)
+                     : check_residency<1, true, false>(p->grid, p->num_sms, err, errn);
+  }
   if (rc) return rc;
   p->ready = true;
   return 0;
@@ -1422,7 +1530,7 @@ int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, void* w
 void tc_plan_free(TcPlan* p) { p->ready = false; }
 
 void tc_counters(const TcPlan& p, unsigned** ptr, int* count) {
-  TcLayout L = tc_layout(p.C, p.V, p.d, p.num_sms);
+  TcLayout L = tc_layout(p.C, p.V, p.d, p.num_sms, p.fp8);
   *ptr = reinterpret_cast<unsigned*>(static_cast<char*>(p.ws) + L.counters);
   *count = 2 * (2 * L.n_vt + 64);
 }
@@ -1439,7 +1547,10 @@ tc::Params base_params(const TcPlan& pl, const TcLayout& L, DevState* st, const 
   prm.mref = const_cast<float*>(mref); prm.scale_tab = scale_tab;
   prm.tstats2 = reinterpret_cast<TcStat*>(tstats);
   prm.Opart = reinterpret_cast<float*>(base + L.Opart);
-  prm.P = reinterpret_cast<__nv_bfloat16*>(base + L.P);
+  prm.P = base + L.P;
+  prm.Ee = pl.Ee;
+  prm.he = pl.he;
+  prm.u = pl.u;
   unsigned* ctr0 = reinterpret_cast<unsigned*>(base + L.counters);
   unsigned* ctr = ctr0 + (size_t)pass * (2 * L.n_vt + 64);     // this pass's counter set
   prm.pass = pass;
@@ -1474,11 +1585,18 @@ cudaError_t launch_params(cudaStream_t s, const TcPlan& pl, const TcLayout& L,
                           const tc::Params& prm) {
   const CUtensorMap* maps = reinterpret_cast<const CUtensorMap*>(pl.maps);
   const int units = L.n1 + L.n2;
+  if (pl.fp8) {
+    if (prm.tsamp)
+      return L.CG == 2 ? launch_kernel<2, true, true>(s, units, maps, prm)
+                       : launch_kernel<1, true, true>(s, units, maps, prm);
+    return L.CG == 2 ? launch_kernel<2, false, true>(s, units, maps, prm)
+                     : launch_kernel<1, false, true>(s, units, maps, prm);
+  }
   if (prm.tsamp)
-    return L.CG == 2 ? launch_kernel<2, true>(s, units, maps, prm)
-                     : launch_kernel<1, true>(s, units, maps, prm);
-  return L.CG == 2 ? launch_kernel<2, false>(s, units, maps, prm)
-                   : launch_kernel<1, false>(s, units, maps, prm);
+    return L.CG == 2 ? launch_kernel<2, true, false>(s, units, maps, prm)
+                     : launch_kernel<1, true, false>(s, units, maps, prm);
+  return L.CG == 2 ? launch_kernel<2, false, false>(s, units, maps, prm)
+                   : launch_kernel<1, false, false>(s, units, maps, prm);
 }
 
 cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, const void* h,
@@ -1487,7 +1605,7 @@ cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, 
                                 const DrawArgs& draw, float* H, int32_t* argmax,
                                 RowStat* rowstat, float redo_gap, const SamplerArgs& sa) {
   (void)h; (void)E;
-  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
+  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms, pl.fp8);
   const tc::Params prm = base_params(pl, L, st, mref, scale_tab, S, tstats, ws, draw, H, argmax,
                                      rowstat, redo_gap, sa, 0);
   cudaError_t e = launch_params(s, pl, L, prm);
@@ -1543,7 +1661,7 @@ cudaError_t launch_tc_partial(cudaStream_t s, const TcPlan& pl, DevState* st, co
                               const void* E, const float* mref, const float* scale_tab, int S,
                               TileStat* tstats, void* ws, const DrawArgs& draw, void* partials) {
   (void)h; (void)E;
-  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
+  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms, pl.fp8);
   SamplerArgs none = {};
   tc::Params prm = base_params(pl, L, st, mref, scale_tab, S, tstats, ws, draw, nullptr, nullptr,
                                nullptr, 0.f, none);
@@ -1572,7 +1690,7 @@ cudaError_t launch_tc_merge(cudaStream_t s, const TcPlan& pl, DevState* st, cons
                             float* sc, float redo_gap, const void* h,
                             const void* E, const float* scale_tab, int S,
                             const SamplerArgs& sa, const DrawArgs& draw, const NextStandin& nx) {
-  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
+  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms, pl.fp8);
   const float* Opart = reinterpret_cast<const float*>(static_cast<const char*>(pl.ws) + L.Opart);
   return merge_launch(s, pl, st, reinterpret_cast<const TcStat*>(tstats), 2 * L.n_vt, Opart, L.G,
                       draw.sampled ? static_cast<const TcSamp*>(draw.tsamp) : nullptr, mref,
@@ -1605,7 +1723,7 @@ cudaError_t merge_launch(cudaStream_t s, const TcPlan& pl, DevState* st, const T
                          float* sc, float redo_gap, const void* h, const void* E,
                          const float* scale_tab, int S, const SamplerArgs& sa,
                          const DrawArgs& draw, const NextStandin& nx) {
-  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
+  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms, pl.fp8);
   // the sampler runs on one row's threads of the last CTA
   if (pl.C > tc::kMergeThreadsPerRow) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
@@ -1627,7 +1745,7 @@ cudaError_t merge_launch(cudaStream_t s, const TcPlan& pl, DevState* st, const T
 }
 
 void tc_partials(const TcPlan& pl, const float** Opart, int* nO) {
-  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms);
+  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms, pl.fp8);
   *Opart = reinterpret_cast<const float*>(static_cast<const char*>(pl.ws) + L.Opart);
   *nO = L.G;
 }

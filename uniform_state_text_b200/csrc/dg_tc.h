@@ -17,6 +17,12 @@ struct TcPlan {
   int num_sms = 0;
   int grid = 0;
   void* ws = nullptr;
+  // Narrow E (DG_E_FP8): the kernels read e4m3 codes of E and h with per-row
+  // exponents Ee (global vocabulary row) and he; u is the step exponent of P.
+  bool fp8 = false;
+  const int32_t* Ee = nullptr;
+  const int32_t* he = nullptr;
+  int u = 0;
   // Failure-path testing (dg_inject_stall): 0 = the default 2 s wait limit.
   unsigned long long timeout_ns = 0;
   unsigned stall = 0;
@@ -34,10 +40,32 @@ bool tc_fits_device(int C, int V, int d);
 constexpr int kTcScheduleValues = 11;
 bool tc_schedule_info(int C, int V, int d, int sms, int32_t* out);
 int tc_stat_tiles(int C, int V, int d);
-size_t tc_workspace_bytes(int C, int V, int d);
-// E: the whole [Vg][d] table; the kernels cover entries [v0, v0 + V).
+size_t tc_workspace_bytes(int C, int V, int d, bool fp8 = false);
+// The narrow-E arrays of a context (all device, in its workspace).
+struct TcFp8 {
+  const uint8_t* Eq = nullptr;   // [Vg][d] e4m3 codes of E
+  const int32_t* Ee = nullptr;   // [Vg] row exponents: E_deq[v] = Eq[v] 2^Ee[v]
+  const uint8_t* hq = nullptr;   // [C][d] e4m3 codes of h
+  const int32_t* he = nullptr;   // [C] row exponents of h
+  int u = 0;                     // step exponent: P' = P 2^(Ee[v] - u) as e5m2
+};
+// E: the whole [Vg][d] table; the kernels cover entries [v0, v0 + V). f8: the
+// narrow-E arrays (DG_E_FP8), or nullptr for bf16 operands.
 int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, void* ws, char* err,
-                 size_t errn, int v0, int Vg);
+                 size_t errn, int v0, int Vg, const TcFp8* f8 = nullptr);
+// Narrow E (dg_fp8.cu): quantise rows of a bf16 [rows][d] array to e4m3 codes
+// with per-row power-of-two exponents; the largest exponent goes to *emax.
+cudaError_t launch_quantize_e(cudaStream_t s, const void* E, int rows, int d, uint8_t* Eq,
+                              int32_t* Ee, int* emax);
+// The step's prologue for narrow E: stand-in (or caller's) h in bf16, its e4m3
+// codes and exponent, and m_ref from the dequantised h and E rows.
+cudaError_t launch_prologue_fp8(cudaStream_t s, const DevState* st, const uint8_t* Eq,
+                                const int32_t* Ee, const int32_t* target, const int32_t* canvas,
+                                const float* sc, void* h, const void* hsrc, uint8_t* hq,
+                                int32_t* he, float* mref, int C, int V, int d, uint64_t seed,
+                                float A, float B, float sigma, int standin,
+                                const float* scale_tab, int S, const int32_t* argmax_prev,
+                                unsigned* zero, int nzero);
 void tc_plan_free(TcPlan* p);
 int tc_launches(const TcPlan& p);   // kernels per launch_tc_attention call
 // The attention kernel, launched twice: the first pass's G1 CTAs also merge
