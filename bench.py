@@ -318,6 +318,19 @@ def run_reference(args, w):
 # ----------------------------------------------------------------------------
 # GPU legs.
 # ----------------------------------------------------------------------------
+_E_CPU = {}
+
+
+def embedding_cpu(w):
+    """The workload's E on the host, made once per (V, d, dtype, seed) in a run."""
+    key = (w.V, w.d, w.dtype, w.e_seed)
+    if key not in _E_CPU:
+        if len(_E_CPU) >= 3:
+            _E_CPU.pop(next(iter(_E_CPU)))
+        _E_CPU[key] = synthetic.make_embedding(w)
+    return _E_CPU[key]
+
+
 class FixedStepLoop:
     """Steps of one context in the fixed-step mode: a new block after every S steps."""
 
@@ -465,7 +478,7 @@ def headline_line(args, w, world, rank, local, dist):
     import uniform_state_text_b200 as dg
 
     impl = {"auto": dg.DG_IMPL_AUTO, "simt": dg.DG_IMPL_SIMT, "tc": dg.DG_IMPL_TC}[args.kernels]
-    E_cpu = synthetic.make_embedding(w)
+    E_cpu = embedding_cpu(w)
     E = E_cpu.to(f"cuda:{local}")
     den = dg.Denoiser(w, E, impl=impl)
     kern = "tcgen05" if den.impl == dg.DG_IMPL_TC else "CUDA-core"
@@ -528,7 +541,7 @@ def workload_throughput(w, steps, warmup, local, with_cpu: bool):
     import torch
 
     import uniform_state_text_b200 as dg
-    E_cpu = synthetic.make_embedding(w)
+    E_cpu = embedding_cpu(w)
     E = E_cpu.cuda()
     den = dg.Denoiser(w, E)
     kern = "tcgen05" if den.impl == dg.DG_IMPL_TC else "CUDA-core"
@@ -646,7 +659,7 @@ def vocab_parallel_line(args, w, world, rank, local, dist):
     if w.V % (256 * world):
         raise SystemExit(f"V={w.V} does not split into {world} shards of 256-entry tiles")
     nv = w.V // world
-    E = synthetic.make_embedding(w).to(f"cuda:{local}")
+    E = embedding_cpu(w).to(f"cuda:{local}")
     den = dg.Denoiser(w, E, impl=dg.DG_IMPL_TC, shard=(rank * nv, nv))
     buf = den.partials()
     state = {"t": 0, "block": 0}

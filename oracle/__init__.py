@@ -12,13 +12,17 @@ the confidence threshold), which is stated at each such place.
 Modules:
   rng     -- SplitMix64 counter hash, uniform tokens, Gaussian draws.
   method  -- temperature schedule, stand-in hidden state, vocabulary
-             softmax/entropy/argmax/self-conditioning, entropy-bounded
-             sampler, re-noise, adaptive stop, the step and the block loop.
+             softmax/entropy/argmax/self-conditioning, the self-conditioning
+             feed-forward network, entropy-bounded sampler, re-noise,
+             adaptive stop, the step and the block loop.
+  fp8     -- e4m3/e5m2 rounding, per-row power-of-two scaling and the step's
+             vocabulary attention with a narrow (e4m3) embedding.
 
 Parity status: every function is pinned by tests/test_oracle_*.py against
-closed forms, brute force in long double, a published SplitMix64 vector and a
-hand-worked acceptance example. The pages' end-to-end quality behaviour
+closed forms, brute force in long double, a published SplitMix64 vector, a
+hand-worked acceptance example, every code of the 8-bit formats and a library
+conversion. The pages' end-to-end quality behaviour
 (quality versus step count, the Sudoku experiment) needs the trained model and
 is not part of this oracle.
 """
-from . import rng, method  # noqa: F401
+from . import rng, method, fp8  # noqa: F401
