@@ -128,6 +128,11 @@ typedef struct dg_ctx dg_ctx;
                          /*             stop, 0 before it (read-only)          */
 #define DG_CANVAS_STATE 13 /* int32 [3*canvases]: unchanged steps, stopped   */
                            /* (0/1), steps run, per canvas (read-only)       */
+#define DG_TC_TRACE_COUNTERS 14 /* int64 [256][32]: per-CTA wait counters of */
+                           /* the last tensor-core attention launch, in ns  */
+                           /* (slot 0 start, 1 end, 2-12 waits and busy     */
+                           /* times; see dg_tc.cu); written only by a build */
+                           /* with -DDG_TC_TRACE (read-only)                */
 
 /* Indices into the DG_STATE array. */
 #define DG_ST_T          0  /* next step index within the block               */

@@ -156,3 +156,23 @@ def standin_terms(w, E32, target, canvas, sc, h_orc):
     # bf16 workloads h_orc is already rounded, which only adds to |noise| here
     n = np.asarray(h_orc, np.float64) - a - b - s
     return np.abs(a) + np.abs(b) + np.abs(s) + np.abs(n)
+
+
+def reduce_partials_local(bufs, C: int, d: int) -> None:
+    """The cross-shard reduction of vocabulary-parallel partials over buffers of
+    one process (every buffer gets the result): the same sums and maxima the
+    multi-GPU exchange (uniform_state_text_b200.allreduce_partials, NCCL) takes,
+    for tests that run several shard contexts on one GPU or on the CPU. Test
+    plumbing: eager torch ops, not part of the library's path."""
+    import torch
+
+    import uniform_state_text_b200 as dg
+    views = [dg.partials_views(b, C, d) for b in bufs]
+    fs = views[0][0].clone()
+    for f, _ in views[1:]:
+        fs += f
+    ks = torch.stack([k.bitwise_xor(-(1 << 63)) for _, k in views]).amax(dim=0)
+    ks.bitwise_xor_(-(1 << 63))
+    for f, k in views:
+        f.copy_(fs)
+        k.copy_(ks)

@@ -11,6 +11,8 @@ import socket
 import pytest
 import torch.multiprocessing as mp
 
+from parity import reduce_partials_local
+
 
 def _free_port():
     with socket.socket() as s:
@@ -119,7 +121,7 @@ def test_vocab_parallel_exchange_two_gloo_ranks():
     assert [v % (1 << 64) for v in k.tolist()] == want
     # the single-process helper gives the same buffers
     a, b = _partials(0), _partials(1)
-    dg.reduce_partials_local([a, b], C_X, D_X)
+    reduce_partials_local([a, b], C_X, D_X)
     assert torch.equal(a, got) and torch.equal(b, got)
 
 
@@ -182,7 +184,7 @@ def test_vocab_parallel_bench_loop_two_gloo_ranks():
         assert res[r][0] == ["partial", "finish"] * 2
     assert res[0][1] == res[1][1]
     a, b = _partials(0), _partials(1)
-    dg.reduce_partials_local([a, b], C_X, D_X)
+    reduce_partials_local([a, b], C_X, D_X)
     assert torch.equal(torch.tensor(res[0][1], dtype=torch.int64), a)
 
 

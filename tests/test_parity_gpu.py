@@ -16,7 +16,7 @@ import uniform_state_text_b200 as dg
 from oracle import fp8 as F8
 from oracle import method as M
 from parity import (Tally, check_sampler_exact, compare_attention, compare_draw, h_agreement,
-                    near_tie_flags, standin_terms)
+                    near_tie_flags, reduce_partials_local, standin_terms)
 
 pytestmark = pytest.mark.gpu
 
@@ -184,7 +184,7 @@ def shard_stepper(shards, bufs, w):
         for s, b in zip(shards, bufs):
             s.step_partial(b)
             s.stream.synchronize()
-        dg.reduce_partials_local(bufs, w.C, w.d)
+        reduce_partials_local(bufs, w.C, w.d)
         torch.cuda.synchronize()
         for s, b in zip(shards, bufs):
             s.step_finish(b)

@@ -26,7 +26,7 @@ DG_IMPL_AUTO, DG_IMPL_SIMT, DG_IMPL_TC = 0, 1, 2
 DG_TOKEN_ARGMAX, DG_TOKEN_MULTINOMIAL = 0, 1
 DG_E_NATIVE, DG_E_FP8 = 0, 1
 (DG_CANVAS, DG_ARGMAX, DG_ENTROPY, DG_ACCEPT, DG_SC, DG_HIDDEN, DG_TARGET, DG_ORDER, DG_PREFIX,
- DG_STATE, DG_MREF, DG_SAMPLED, DG_EMIT, DG_CANVAS_STATE) = range(14)
+ DG_STATE, DG_MREF, DG_SAMPLED, DG_EMIT, DG_CANVAS_STATE, DG_TC_TRACE_COUNTERS) = range(15)
 DG_ST_T, DG_ST_BLOCK, DG_ST_UNCHANGED, DG_ST_DONE, DG_ST_STEPS, DG_ST_K, DG_ST_STATUS, \
     DG_ST_HASPREV, DG_ST_REDO = range(9)
 
@@ -293,7 +293,8 @@ class Denoiser:
                 DG_PREFIX: ((C,), torch.float32), DG_STATE: ((16,), torch.int32),
                 DG_MREF: ((C,), torch.float32), DG_SAMPLED: ((C,), torch.int32),
                 DG_EMIT: ((C,), torch.int32),
-                DG_CANVAS_STATE: ((3 * getattr(self.w, "canvases", 1),), torch.int32)}[what]
+                DG_CANVAS_STATE: ((3 * getattr(self.w, "canvases", 1),), torch.int32),
+                DG_TC_TRACE_COUNTERS: ((256, 32), torch.int64)}[what]
 
     def read(self, what):
         import torch
@@ -413,18 +414,3 @@ def allreduce_partials(buf, C: int, d: int, group=None) -> None:
     keys.bitwise_xor_(-(1 << 63))
     dist.all_reduce(keys, op=dist.ReduceOp.MAX, group=group)
     keys.bitwise_xor_(-(1 << 63))
-
-
-def reduce_partials_local(bufs, C: int, d: int) -> None:
-    """The same reduction over buffers of one process (every buffer gets the result)."""
-    import torch
-
-    views = [partials_views(b, C, d) for b in bufs]
-    fs = views[0][0].clone()
-    for f, _ in views[1:]:
-        fs += f
-    ks = torch.stack([k.bitwise_xor(-(1 << 63)) for _, k in views]).amax(dim=0)
-    ks.bitwise_xor_(-(1 << 63))
-    for f, k in views:
-        f.copy_(fs)
-        k.copy_(ks)

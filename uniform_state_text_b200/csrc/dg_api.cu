@@ -727,6 +727,10 @@ int dg_read(dg_ctx* ctx, int32_t what, void* dst) {
       src = at<int32_t>(ctx, ctx->L.cstate);
       bytes = 4 * 3 * (size_t)ctx->L.canvases;
       break;
+    case DG_TC_TRACE_COUNTERS:
+      if (ctx->L.impl != DG_IMPL_TC) return fail(ctx, DG_EUNSUPPORTED, "no tensor-core kernels");
+      src = tc_trace(ctx->tc_plan, &bytes);
+      break;
     default: return fail(ctx, DG_EINVAL, "unknown item %d", what);
   }
   DG_CK(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, ctx->stream));

@@ -1744,6 +1744,12 @@ cudaError_t merge_launch(cudaStream_t s, const TcPlan& pl, DevState* st, const T
       tsamp, draw.sampled, nx, sa);
 }
 
+const void* tc_trace(const TcPlan& pl, size_t* bytes) {
+  TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms, pl.fp8);
+  *bytes = (size_t)256 * 32 * 8;
+  return static_cast<const char*>(pl.ws) + L.trace;
+}
+
 void tc_partials(const TcPlan& pl, const float** Opart, int* nO) {
   TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms, pl.fp8);
   *Opart = reinterpret_cast<const float*>(static_cast<const char*>(pl.ws) + L.Opart);

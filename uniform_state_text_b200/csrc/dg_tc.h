@@ -122,6 +122,9 @@ cudaError_t launch_self_condition(cudaStream_t s, int C, int d, int dff, const f
                                   void* emb, int emb_bf16, void* scratch, int* status);
 // Hand-off counters the prologue zeroes before every step.
 void tc_counters(const TcPlan& p, unsigned** ptr, int* count);
+// The attention kernel's per-CTA wait counters ([256][32] int64; written only
+// by a build with -DDG_TC_TRACE).
+const void* tc_trace(const TcPlan& p, size_t* bytes);
 // Per-range-group partials of O = P E that the merge sums.
 void tc_partials(const TcPlan& p, const float** Opart, int* nO);
 
