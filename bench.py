@@ -450,24 +450,31 @@ def redo_leg(den, w, E, steps: int):
     h_a = hid(tok_a)
     cases = {"none": h_a, "1pct": hid(few), "all": hid(tok_b)}
     n = max(2, min(steps, w.max_steps - 1))
-    out = {"steps": n, "rows": w.C,
-           "path": "dg_denoise_step_h with device hidden states, CUDA events on the stream"}
-    for name, h_b in cases.items():
-        den.begin_block(0)
-        den.step_h(h_a)                                   # step 0: every reference is low
-        r0 = den.state()["redo"]
-        ev0 = torch.cuda.Event(enable_timing=True)
-        ev1 = torch.cuda.Event(enable_timing=True)
-        ev0.record(den.stream)
-        for i in range(n):
-            den.step_h(h_b if i % 2 == 0 else h_a)
-        ev1.record(den.stream)
-        torch.cuda.synchronize()
-        st = den.state()
-        if st["status"] != 0:
-            raise RuntimeError("device status after the redo leg")
-        out[name] = {"us_per_step": 1e3 * ev0.elapsed_time(ev1) / n,
-                     "rows_redone_per_step": (st["redo"] - r0) / n}
+    out = {"steps": n, "rows": w.C, "rounds": 3,
+           "path": "dg_denoise_step_h with device hidden states, CUDA events on the stream; "
+                   "the cases interleaved over 3 rounds, median per case"}
+    times = {k: [] for k in cases}
+    redone = {}
+    for _ in range(3):
+        for name, h_b in cases.items():
+            den.begin_block(0)
+            den.step_h(h_a)                               # step 0: every reference is low
+            r0 = den.state()["redo"]
+            ev0 = torch.cuda.Event(enable_timing=True)
+            ev1 = torch.cuda.Event(enable_timing=True)
+            ev0.record(den.stream)
+            for i in range(n):
+                den.step_h(h_b if i % 2 == 0 else h_a)
+            ev1.record(den.stream)
+            torch.cuda.synchronize()
+            st = den.state()
+            if st["status"] != 0:
+                raise RuntimeError("device status after the redo leg")
+            times[name].append(1e3 * ev0.elapsed_time(ev1) / n)
+            redone[name] = (st["redo"] - r0) / n
+    for name in cases:
+        out[name] = {"us_per_step": float(np.median(times[name])),
+                     "rows_redone_per_step": redone[name]}
     out["all_over_none"] = out["all"]["us_per_step"] / out["none"]["us_per_step"]
     return out
 

@@ -533,7 +533,8 @@ def test_self_condition_network(shape, emb_dtype):
     C, V, d, dff = shape
     w = synthetic.SMALL.replace(C=C, V=V, d=d, tau=0.5 * C * np.log(2), max_steps=2,
                                 fixed_steps=1, coef_target=1.0, coef_canvas=0.5, logit_scale=2.0)
-    den, E32 = make(w, dg.DG_IMPL_AUTO)
+    impl = dg.DG_IMPL_TC if C in (128, 256) else dg.DG_IMPL_SIMT
+    den, E32 = make(w, impl)
     Eg, _ = embedding(w)
     den.step()
     sc = _np(den.read(dg.DG_SC)).astype(np.float64)
