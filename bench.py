@@ -274,9 +274,12 @@ def kernel_roofline(w, pk, kernel_s: float, timed_s: float, clk, kernel: str):
 # capture summarised under profiles/ (taken on the V=65536 profiling shape and
 # scaled by the vocabulary, since E and the P ring both grow with V).
 DRAM_TRAFFIC = {
-    synthetic.HEADLINE.name: (4 * (286.7264e6 + 6.975744e6),
-                              "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at "
-                              "C=256, V=65536, d=2048, scaled by 4 to V=262144"),
+    (synthetic.HEADLINE.name, 0): (4 * (291.04384e6 + 8.018432e6),
+                                   "ncu dram__bytes_read.sum + dram__bytes_write.sum of one first-pass "
+                                   "launch at C=256, V=65536, d=2048, scaled by 4 to V=262144"),
+    (synthetic.HEADLINE.name, 1): (4 * (135.387648e6 + 4.126464e6),
+                                   "ncu dram__bytes_read.sum + dram__bytes_write.sum of one first-pass "
+                                   "launch (narrow E) at C=256, V=65536, d=2048, scaled by 4"),
 }
 
 
@@ -512,7 +515,7 @@ def headline_line(args, w, world, rank, local, dist):
     t_b, t_s, _ = step_roofline(w, pk)
     roof = kernel_roofline(w, pk, (attn_ms / 1e3) / max(attn_steps, 1), timed_s, clk,
                            f"vocabulary attention ({kern})")
-    traffic = DRAM_TRAFFIC.get(w.name) if den.impl == dg.DG_IMPL_TC else None
+    traffic = DRAM_TRAFFIC.get((w.name, w.e_format)) if den.impl == dg.DG_IMPL_TC else None
     roof["traffic"] = traffic[0] if traffic else None
     roof["traffic_src"] = traffic[1] if traffic else None
     roof.update({"step_roofline_us": t_b * 1e6, "step_roofline_us_sustained": t_s * 1e6,
@@ -567,6 +570,8 @@ def workload_throughput(w, steps, warmup, local, with_cpu: bool):
            "step_roofline_pct_sustained": 100.0 * t_s / (ms_step / 1e3),
            "roofline": kernel_roofline(w, pk, (attn_ms / 1e3) / max(attn_steps, 1), timed_s, clk,
                                        f"vocabulary attention ({kern})")}
+    tr = DRAM_TRAFFIC.get((w.name, w.e_format)) if den.impl == dg.DG_IMPL_TC else None
+    out["roofline"]["traffic"] = tr[0] if tr else None
     den.close()
     del E
     torch.cuda.empty_cache()
