@@ -152,7 +152,9 @@ __device__ __forceinline__ void max_key_decode(unsigned long long key, float* v,
 // Slots: 0 start, 1 end, 2 producer waits on free stages, 3 producer waits on
 // counters, 4 MMA waits on full stages, 5 MMA waits on free accumulators,
 // 6 epilogue waits on full accumulators, 7 items, 8 epilogue busy, and within
-// it 9 TMEM loads, 10 softmax arithmetic, 11 P stores, 12 publishing the tile.
+// it 9 TMEM loads, 10 softmax arithmetic, 11 P stores, 12 publishing the tile;
+// 13 and 14 the SM clock counter at the CTA's start and end (with slots 0 and
+// 1, the clock the kernel ran at).
 // The block of [grid][32] int64 lies in the tensor-core workspace after the
 // counters, the P ring and the O partials.
 #ifdef DG_TC_TRACE
@@ -449,7 +451,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const bool leader = rank == 0;
   const int unit = blockIdx.x / CG;                    // pair (or CTA) index
   const bool is_g1 = unit < p.n1;
-  if (threadIdx.x == 0) TR_STORE(0, gtimer());
+  if (threadIdx.x == 0) { TR_STORE(0, gtimer()); TR_STORE(13, clock64()); }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -878,7 +880,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   __syncthreads();
   if constexpr (CG == 2) cluster_sync();    // no remote arrivals after this point
-  if (threadIdx.x == 0) TR_STORE(1, gtimer());
+  if (threadIdx.x == 0) { TR_STORE(1, gtimer()); TR_STORE(14, clock64()); }
   if (warp == 1) {
     tc_fence_after();
     if constexpr (CG == 2)
