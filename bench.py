@@ -261,10 +261,14 @@ def kernel_roofline(w, pk, kernel_s: float, timed_s: float, clk, kernel: str):
         "timed_region_s": timed_s,
         "sm_mhz_median": clk["sm_mhz"] if clk else None,
     })
-    if clk and clk.get("sm_max_mhz") and tensor_bound:
-        # the same kernel time scaled to the maximum clock, against the burst peak
-        roof["frac_burst_at_max_clock"] = roof["frac_burst"] * clk["sm_max_mhz"] / clk["sm_mhz"] \
-            if clk["sm_mhz"] else None
+    kmhz = clk.get("kernel_sm_mhz") if clk else None
+    if kmhz and tensor_bound:
+        # the clock the kernel itself ran at (clock64 over %globaltimer of one
+        # CTA), and the fraction of the nominal dense tensor peak at that clock
+        # (148 SMs x 8192 bf16 flop per clock, x 2 for 8-bit operands)
+        nominal = 148 * 8192 * ratio * kmhz * 1e6 / 1e12
+        roof["kernel_sm_mhz"] = kmhz
+        roof["frac_nominal_at_kernel_clock"] = achieved / nominal
     if pk.get("clocks"):
         roof["peak_clocks"] = pk["clocks"]
     return roof
@@ -349,6 +353,17 @@ class FixedStepLoop:
         self.t += 1
 
 
+def kernel_clock_mhz(den):
+    """The SM clock the last attention launch ran at: clock64 over %globaltimer
+    of one CTA across its lifetime (tensor-core contexts), or None."""
+    import uniform_state_text_b200 as dg
+    if den.impl != dg.DG_IMPL_TC:
+        return None
+    r = den.read(dg.DG_TC_TRACE_COUNTERS)[255].cpu().tolist()
+    dt = r[2] - r[0]
+    return 1e3 * (r[3] - r[1]) / dt if dt > 0 else None
+
+
 def timed_steps(den, step, steps: int, warmup: int, local: int, dist=None):
     """Device-timed region of `steps` calls of step() on den's stream.
 
@@ -385,6 +400,8 @@ def timed_steps(den, step, steps: int, warmup: int, local: int, dist=None):
     st = den.state()
     if st["status"] != 0:
         raise RuntimeError(f"device status {st['status']}")
+    if clk is not None:
+        clk["kernel_sm_mhz"] = kernel_clock_mhz(den)
     return max_over_ranks(ms, dist, "cuda"), prof, clk, ms / 1e3
 
 

@@ -131,8 +131,11 @@ typedef struct dg_ctx dg_ctx;
 #define DG_TC_TRACE_COUNTERS 14 /* int64 [256][32]: per-CTA wait counters of */
                            /* the last tensor-core attention launch, in ns  */
                            /* (slot 0 start, 1 end, 2-12 waits and busy     */
-                           /* times; see dg_tc.cu); written only by a build */
-                           /* with -DDG_TC_TRACE (read-only)                */
+                           /* times; see dg_tc.cu), written only by a build */
+                           /* with -DDG_TC_TRACE; in every build row 255    */
+                           /* holds CTA 0's %globaltimer and clock64 at its */
+                           /* start (0, 1) and end (2, 3): the SM clock the */
+                           /* kernel ran at (read-only)                     */
 
 /* Indices into the DG_STATE array. */
 #define DG_ST_T          0  /* next step index within the block               */

@@ -154,7 +154,9 @@ __device__ __forceinline__ void max_key_decode(unsigned long long key, float* v,
 // 6 epilogue waits on full accumulators, 7 items, 8 epilogue busy, and within
 // it 9 TMEM loads, 10 softmax arithmetic, 11 P stores, 12 publishing the tile;
 // 13 and 14 the SM clock counter at the CTA's start and end (with slots 0 and
-// 1, the clock the kernel ran at).
+// 1, the clock the kernel ran at). In every build, row 255 holds CTA 0's
+// timer and clock counter at its start (slots 0, 1) and end (2, 3) of the
+// last first-pass launch: the SM clock the kernel actually ran at.
 // The block of [grid][32] int64 lies in the tensor-core workspace after the
 // counters, the P ring and the O partials.
 #ifdef DG_TC_TRACE
@@ -452,6 +454,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int unit = blockIdx.x / CG;                    // pair (or CTA) index
   const bool is_g1 = unit < p.n1;
   if (threadIdx.x == 0) { TR_STORE(0, gtimer()); TR_STORE(13, clock64()); }
+  if (blockIdx.x == 0 && threadIdx.x == 0 && p.pass == 0) {
+    p.trace[255 * 32 + 0] = gtimer();
+    p.trace[255 * 32 + 1] = clock64();
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -881,6 +887,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   if constexpr (CG == 2) cluster_sync();    // no remote arrivals after this point
   if (threadIdx.x == 0) { TR_STORE(1, gtimer()); TR_STORE(14, clock64()); }
+  if (blockIdx.x == 0 && threadIdx.x == 0 && p.pass == 0) {
+    p.trace[255 * 32 + 2] = gtimer();
+    p.trace[255 * 32 + 3] = clock64();
+  }
   if (warp == 1) {
     tc_fence_after();
     if constexpr (CG == 2)
