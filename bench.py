@@ -228,7 +228,7 @@ def kernel_roofline(w, pk, kernel_s: float, timed_s: float, clk, kernel: str):
     Algorithmic work per launch: 4 C d V flops (both contractions) and V d b_E
     bytes of E (read once). The bound is whichever takes longer at the peaks.
     With narrow E (e4m3 codes) the operands are 8-bit: E is V d bytes plus a
-    4-byte exponent per row, and the tensor peak is the measured bf16 peak
+    4-byte exponent per row (one per 256-row block, stored per row), and the tensor peak is the measured bf16 peak
     times the nominal fp8/bf16 ratio (4.5 / 2.25 PFLOP/s dense).
     """
     fp8 = getattr(w, "e_format", 0) == 1
@@ -550,7 +550,7 @@ def headline_line(args, w, world, rank, local, dist):
             "roofline_pct": roof["step_roofline_pct"],
             "config": {"workload": w.name, "C": w.C, "V": w.V, "d": w.d,
                        "canvases": w.canvases,
-                       "e_format": "e4m3 codes, power-of-two scale per row" if w.e_format == 1
+                       "e_format": "e4m3 codes, power-of-two scale per 256-row block" if w.e_format == 1
                                    else "bf16",
                        "token_rule": "multinomial" if w.token_rule == 1 else "argmax",
                        "max_steps": w.max_steps, "mode": "fixed_steps (adaptive stop off)",
@@ -578,7 +578,7 @@ def workload_throughput(w, steps, warmup, local, with_cpu: bool):
     t_b, t_s, _ = step_roofline(w, pk)
     ms_step = ms / steps
     out = {"workload": w.name, "C": w.C, "V": w.V, "d": w.d, "dtype": w.dtype,
-           "e_format": "e4m3 codes, power-of-two scale per row" if w.e_format == 1 else "bf16",
+           "e_format": "e4m3 codes, power-of-two scale per 256-row block" if w.e_format == 1 else "bf16",
            "mode": "fixed_steps", "steps": steps, "warmup": warmup,
            "value": 1e3 / ms_step, "unit": "steps/s", "ms_per_step": ms_step,
            "tok_per_s": w.C * 1e3 / ms_step, "gpu_launches": launches, "clocks": clk,
@@ -734,7 +734,7 @@ def main():
                     help="multi-GPU mode: independent canvases per rank, or one canvas's "
                          "vocabulary split over the ranks")
     ap.add_argument("--e-format", default="native", choices=["native", "fp8"],
-                    help="E as given (bf16), or e4m3 codes with a power-of-two scale per row")
+                    help="E as given (bf16), or e4m3 codes with a power-of-two scale per 256-row block")
     ap.add_argument("--token-rule", default="argmax", choices=["argmax", "multinomial"],
                     help="token an accepted position takes")
     ap.add_argument("--canvases", type=int, default=0,

@@ -72,8 +72,8 @@ extern "C" {
 
 /* How the tensor-core kernels hold E (dg_config.e_format). */
 #define DG_E_NATIVE  0       /* E as given (dtype)                             */
-#define DG_E_FP8     1       /* e4m3 codes, one power-of-two scale per row     */
-                             /* (see dg_init)                                  */
+#define DG_E_FP8     1       /* e4m3 codes, one power-of-two scale per block   */
+                             /* of 256 vocabulary rows (see dg_init)           */
 
 /* Kernel family for the vocabulary-attention step. */
 #define DG_IMPL_AUTO  0      /* tensor-core path when the shape allows it     */
@@ -171,6 +171,17 @@ size_t dg_workspace_bytes(const dg_config* cfg);
  * does not cover: it needs dtype bf16, C = 128 or 256, d a multiple of 256,
  * V a multiple of 256), DG_ECUDA. The context starts at block 0 (as if
  * dg_begin_block(ctx, 0) had run).
+ *
+ * Narrow E (cfg->e_format = DG_E_FP8; bf16 E, tensor-core path): dg_init
+ * quantises E once, in the workspace, to e4m3 codes with one power-of-two
+ * scale per block of 256 vocabulary rows (the smallest that brings the
+ * block's largest magnitude within 448; rounding to nearest even, saturated),
+ * and synchronises the stream. Every step then uses the dequantised E: the
+ * stand-in gathers its rows, h is quantised per canvas row the same way, both
+ * contractions run on 8-bit tensor cores, and the probabilities p.E takes are
+ * rounded to e5m2. After dg_init, E itself is read only by the CUDA-core
+ * fallback for a row whose sums are not finite even after the redo pass
+ * (non-finite hidden states), which then uses the unquantised values.
  */
 int dg_init(const dg_config* cfg, const void* E, void* workspace, size_t ws_bytes,
             void* stream, dg_ctx** out);

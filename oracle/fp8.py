@@ -8,12 +8,17 @@ in NVFP4 fits an 18 GB GPU; "A Visual Guide to DiffusionGemma" on the roofline
 of the step). They give no format details. The reading here, for the step's
 own arithmetic:
 
-  * E is stored as e4m3 codes with one power-of-two scale per vocabulary row:
-    E_deq[v] = q[v] * 2^e[v], e[v] the smallest exponent with
-    max_k |E[v, k]| * 2^-e[v] <= 448 (the e4m3 maximum). One scale per row
-    (not per 32-element block along d) because the second contraction,
-    p.E, runs over the vocabulary: a scale that varies along d cannot be
-    taken out of that sum, a per-row one folds into p exactly.
+  * E is stored as e4m3 codes with one power-of-two scale per block of
+    GROUP = 256 consecutive vocabulary rows: E_deq[v] = q[v] * 2^e[v], e[v]
+    the smallest exponent with max |E[block of v]| * 2^-e[v] <= 448 (the
+    e4m3 maximum), the same for every row of the block. Blocks run along the
+    vocabulary, not along d (as 32-element MX blocks would), because the
+    second contraction, p.E, sums over the vocabulary: a scale that varies
+    along d cannot be taken out of that sum, one per vocabulary block folds
+    into p exactly. e4m3 is a floating-point format: entries down to
+    2^-6 / 448 (about 2^-14.8) of their block's largest keep its relative
+    precision of 2^-4, so rows smaller than their block's largest lose
+    little.
   * h is quantised the same way per canvas row (e4m3, power-of-two scale).
   * The logits, entropy, argmax and the partition sum are those of h_deq and
     E_deq (fp32 accumulation on the device, fp64 here).
@@ -66,13 +71,19 @@ def row_scale_exponent(amax, fmt: str = "e4m3") -> np.ndarray:
     return np.where(amax > 0, e, 0).astype(np.int64)
 
 
-def quantize_rows(X, fmt: str = "e4m3"):
-    """Per-row power-of-two scaling and rounding: returns (codes as values, exponents).
+def quantize_rows(X, fmt: str = "e4m3", group: int = 1):
+    """Power-of-two scaling per block of `group` consecutive rows, and rounding:
+    returns (codes as values, one exponent per row, equal within a block).
 
     X[r] ~= codes[r] * 2^exps[r]; codes lie in the format's range.
     """
     X = np.asarray(X, dtype=np.float64)
-    e = row_scale_exponent(np.abs(X).max(axis=1), fmt)
+    amax = np.abs(X).max(axis=1)
+    if group > 1:
+        n = X.shape[0]
+        assert n % group == 0
+        amax = np.repeat(amax.reshape(n // group, group).max(axis=1), group)
+    e = row_scale_exponent(amax, fmt)
     return fp8_round(np.ldexp(X, -e[:, None]), fmt), e
 
 
@@ -105,6 +116,7 @@ def sc_from_quantized_p(z, m_ref, E_codes, E_exps, u: int) -> np.ndarray:
 # e^REDO_GAP 2^(e[v] - u) <= 54.6 * 2^10 within e5m2's range.
 REDO_GAP = 4.0
 U_OFFSET = 10
+GROUP = 256          # vocabulary rows per scale of E
 
 
 def step_exponent(E_exps) -> int:
@@ -112,15 +124,16 @@ def step_exponent(E_exps) -> int:
 
 
 class NarrowE:
-    """E held as e4m3 codes with per-row power-of-two exponents (see the module
-    docstring); E_deq is the embedding every other part of the step uses."""
+    """E held as e4m3 codes with one power-of-two exponent per block of GROUP
+    vocabulary rows (see the module docstring; exps holds it for every row);
+    E_deq is the embedding every other part of the step uses."""
 
     def __init__(self, E):
         V, d = E.shape
         self.codes = np.empty((V, d), dtype=np.float32)   # exact: e4m3 values are fp32 values
         self.exps = np.empty(V, dtype=np.int64)
         for r0 in range(0, V, 8192):                     # row chunks bound the fp64 temporaries
-            q, e = quantize_rows(E[r0:r0 + 8192], "e4m3")
+            q, e = quantize_rows(E[r0:r0 + 8192], "e4m3", group=min(GROUP, V))
             self.codes[r0:r0 + 8192] = q
             self.exps[r0:r0 + 8192] = e
         self.E_deq = np.ldexp(self.codes, self.exps[:, None]).astype(np.float32)   # exact as well
@@ -130,7 +143,8 @@ class NarrowE:
 def narrow_attention(nE: NarrowE, h, scale, canvas, prev, gumbel_key=None, m_ref=None):
     """Entropy, argmax, draw and sc of a step with narrow E.
 
-    h (the stand-in or the caller's, already bf16) is quantised per row; the
+    h (the stand-in or the caller's, already bf16) is quantised per row (one
+    exponent per canvas row); the
     logits are those of h_deq and E_deq. The reference of row i is the logit of
     its canvas token or previous prediction, whichever is larger (prev = canvas
     on the block's first step), raised to the row's largest logit when it lags

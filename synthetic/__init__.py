@@ -68,7 +68,7 @@ class Workload:
     accept_rule: int = 0    # 0: cumulative sum, 1: cumulative sum minus max
     token_rule: int = 0     # 0: argmax, 1: multinomial draw (Gumbel-max)
     canvases: int = 1       # independent canvases of C / canvases positions per step
-    e_format: int = 0       # 0: E as dtype; 1: e4m3 codes with a power-of-two scale per row
+    e_format: int = 0       # 0: E as dtype; 1: e4m3 codes, a power-of-two scale per 256 rows
     fixed_steps: int = 0    # 1: run exactly max_steps (timing mode)
     seed: int = 0
     blocks: int = 1

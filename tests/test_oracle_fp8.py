@@ -172,3 +172,21 @@ def test_narrow_sc_is_close_to_the_plain_sc_of_the_dequantised_values():
     rel = np.linalg.norm(att.sc - plain.sc, axis=1) / np.linalg.norm(plain.sc, axis=1)
     assert rel.max() < 0.05
     np.testing.assert_allclose(att.H, plain.H)
+
+
+def test_block_scale_is_shared_by_the_block_and_fits_its_largest_row():
+    """One exponent per block of GROUP vocabulary rows: the smallest that brings
+    the block's largest magnitude within e4m3's range; a row a thousand times
+    smaller than its block's largest keeps e4m3's relative precision as a
+    vector (its entries lie within e4m3's normal range, 2^-6 .. 448)."""
+    g = np.random.default_rng(7)
+    V, d = 2 * F.GROUP, 16
+    E = g.standard_normal((V, d)) * np.repeat([0.01, 3.0], F.GROUP)[:, None]
+    E[5] *= 1e-3                                    # a much smaller row in block 0
+    nE = F.NarrowE(E)
+    for b in range(2):
+        blk = slice(b * F.GROUP, (b + 1) * F.GROUP)
+        assert len(set(nE.exps[blk].tolist())) == 1
+        assert nE.exps[blk][0] == F.row_scale_exponent(np.abs(E[blk]).max(), "e4m3")
+    rel = np.linalg.norm(nE.E_deq[5] - E[5]) / np.linalg.norm(E[5])
+    assert rel <= 2.0 ** -4

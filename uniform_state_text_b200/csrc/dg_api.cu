@@ -463,7 +463,7 @@ int dg_init(const dg_config* cfg, const void* E, void* workspace, size_t ws_byte
     ctx->tc = at<void>(ctx, L.tc);
     TcFp8 f8;
     if (L.fp8) {
-      // quantise E once: e4m3 codes with a power-of-two scale per row
+      // quantise E once: e4m3 codes with a power-of-two scale per 256-row block
       int* emax = at<int>(ctx, L.emax);
       int emax_h = 0;
       cudaError_t e = cudaMemsetAsync(emax, 0x80, sizeof(int), ctx->stream);   // very negative

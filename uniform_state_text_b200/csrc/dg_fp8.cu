@@ -2,11 +2,14 @@
 // DG_E_FP8). The pages name a quantised model for the smaller GPUs
 // ("DiffusionGemma: from autoregressive to diffusion denoising", throughput
 // table) without format details; the reading used here:
-//   * E is held as e4m3 codes with one power-of-two scale per vocabulary row,
-//     E_deq[v] = q[v] 2^e[v], e[v] the smallest exponent that brings the row's
-//     largest magnitude within 448. One scale per row (not per block along d)
-//     because the second contraction sums over the vocabulary: a per-row
-//     scale folds into the probabilities exactly.
+//   * E is held as e4m3 codes with one power-of-two scale per block of 256
+//     vocabulary rows (the kernels' vocabulary tile), E_deq[v] = q[v] 2^e[v],
+//     e[v] the smallest exponent that brings the block's largest magnitude
+//     within 448. Blocks run along the vocabulary, not along d, because the
+//     second contraction sums over the vocabulary: a scale per vocabulary block
+//     folds into the probabilities exactly; and one per tile costs the
+//     attention kernel's epilogue one constant per tile instead of one per
+//     logit.
 //   * The hidden state is quantised the same way per canvas row, after it has
 //     been formed in bf16 (the stand-in, or the caller's h).
 //   * The stand-in gathers its rows from E_deq, and the per-row logit
@@ -68,29 +71,29 @@ __device__ __forceinline__ float2 block_sum2(float a, float b, float* red) {
   return make_float2(x, y);
 }
 
-// One CTA per row of a bf16 [rows][d] array: codes and the row's exponent;
-// the largest exponent of all rows goes to *emax (atomic).
-__global__ void __launch_bounds__(256) k_quantize_rows_e4m3(const __nv_bfloat16* X, uint8_t* Q,
-                                                            int32_t* ex, int d, int* emax) {
+// One CTA per block of `group` rows of a bf16 [rows][d] array: the codes of
+// the block with its common exponent, written for each of its rows; the
+// largest exponent of all blocks goes to *emax (atomic).
+__global__ void __launch_bounds__(256) k_quantize_blocks_e4m3(const __nv_bfloat16* X, uint8_t* Q,
+                                                              int32_t* ex, int d, int group,
+                                                              int* emax) {
   __shared__ float red[64];
-  const size_t r = blockIdx.x;
-  const __nv_bfloat16* xr = X + r * d;
+  const size_t n = (size_t)group * d;
+  const __nv_bfloat16* xb = X + (size_t)blockIdx.x * n;
   float a = 0.f;
-  for (int k = threadIdx.x * 2; k < d; k += blockDim.x * 2) {
-    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(xr + k);
+  for (size_t k = threadIdx.x * 2; k < n; k += blockDim.x * 2) {
+    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(xb + k);
     a = fmaxf(a, fmaxf(fabsf(__bfloat162float(v.x)), fabsf(__bfloat162float(v.y))));
   }
   const int e = e4m3_row_exponent(block_max(a, red));
-  uint8_t* qr = Q + r * d;
-  for (int k = threadIdx.x * 2; k < d; k += blockDim.x * 2) {
-    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(xr + k);
-    *reinterpret_cast<uint16_t*>(qr + k) =
+  uint8_t* qb = Q + (size_t)blockIdx.x * n;
+  for (size_t k = threadIdx.x * 2; k < n; k += blockDim.x * 2) {
+    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(xb + k);
+    *reinterpret_cast<uint16_t*>(qb + k) =
         f32x2_to_e4m3(ldexpf(__bfloat162float(v.x), -e), ldexpf(__bfloat162float(v.y), -e));
   }
-  if (threadIdx.x == 0) {
-    ex[r] = e;
-    atomicMax(emax, e);
-  }
+  for (int r = threadIdx.x; r < group; r += blockDim.x) ex[(size_t)blockIdx.x * group + r] = e;
+  if (threadIdx.x == 0) atomicMax(emax, e);
 }
 
 // The step's prologue in the narrow-E form, one CTA per canvas row:
@@ -168,8 +171,10 @@ __global__ void __launch_bounds__(256) k_prologue_fp8(
 
 cudaError_t launch_quantize_e(cudaStream_t s, const void* E, int rows, int d, uint8_t* Eq,
                               int32_t* Ee, int* emax) {
-  k_quantize_rows_e4m3<<<rows, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(E), Eq, Ee, d,
-                                             emax);
+  constexpr int kGroup = 256;                 // the kernels' vocabulary tile
+  if (rows % kGroup) return cudaErrorInvalidValue;
+  k_quantize_blocks_e4m3<<<rows / kGroup, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(E), Eq,
+                                                        Ee, d, kGroup, emax);
   return cudaGetLastError();
 }
 

@@ -104,9 +104,10 @@ struct Params {
   // pass raised its redo flag (redo_in) and then uses its own counter set.
   int pass;
   const int* redo_in;
-  // Narrow E (e4m3 codes, F8 instantiations): per-row exponents of E (global
-  // row index) and of h, and the step exponent u: P' = P 2^(Ee[v] - u) is
-  // rounded to e5m2 for the P.E contraction, whose sums are 2^-u sc Z.
+  // Narrow E (e4m3 codes, F8 instantiations): exponents of E per row (global
+  // row index; equal within each 256-row vocabulary tile) and of h per row,
+  // and the step exponent u: P' = P 2^(Ee[v] - u) is rounded to e5m2 for the
+  // P.E contraction, whose sums are 2^-u sc Z.
   const int32_t* Ee;
   const int32_t* he;
   int u;
@@ -736,7 +737,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int row = rb * BM + r_local;
         const float mref = p.mref[row];
         const float k0 = -mref * 1.4426950408889634f;
-        const int he_row = F8 ? p.he[row] : 0;     // the row's exponent of h (F8)
+        // F8: the tensor cores summed code products; the tile's exponent of E
+        // and the row's of h bring them back to h_deq . E_deq (folded into the
+        // logit scale), and P' = P 2^(Ee - u) is the probability the P.E
+        // contraction takes
+        float k1i = k1, scalei = scale, pq = 1.f;
+        if constexpr (F8) {
+          const int et = __ldg(p.Ee + p.v0 + vt * BN);
+          const float s8 = pow2f(et + p.he[row]);
+          k1i = k1 * s8;
+          scalei = scale * s8;
+          pq = pow2f(et - p.u);
+        }
         // P = 2^(k1 v + k0) = e^(z - mref); Z = sum P; S2 = sum P (z - mref) log2(e).
         float Z = 0.f, S2 = 0.f, vbest = -INFINITY;
         int arg = 0x7fffffff;
@@ -759,18 +771,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (lane == 0) mbar_arrive_remote_relaxed(acc_empty_addr + buf * 8);
           }
           TR_T0();
-          int eev[32];              // F8: exponents of the chunk's 32 vocabulary rows
-          if constexpr (F8) {
-            const int4* ep = reinterpret_cast<const int4*>(p.Ee + p.v0 + vt * BN + c0 + c * 32);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int4 q4 = __ldg(ep + j);
-              eev[4 * j] = q4.x; eev[4 * j + 1] = q4.y; eev[4 * j + 2] = q4.z; eev[4 * j + 3] = q4.w;
-            }
-            // the tensor cores summed code products: scale back to h_deq . E_deq
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] *= pow2f(eev[j] + he_row);
-          }
           float cm = v[0];
 #pragma unroll
           for (int j = 1; j < 32; ++j) cm = fmaxf(cm, v[j]);
@@ -786,12 +786,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           // cannot win: such chunks are skipped (1.0 of slack covers the
           // rounding differences between mref and these logits).
           if constexpr (DRAW) {
-            if (cm * scale >= mref - 20.5f) {
+            if (cm * scalei >= mref - 20.5f) {
               const int col0 = p.v0 + vt * BN + c0 + c * 32;
               const uint64_t rbase = (uint64_t)row * (uint64_t)p.V + (uint64_t)col0;
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
-                const float g = v[j] * scale + gumbel_from_key(sm64(gpre ^ (rbase + (uint64_t)j)));
+                const float g = v[j] * scalei + gumbel_from_key(sm64(gpre ^ (rbase + (uint64_t)j)));
                 if (g > gbest) { gbest = g; garg = col0 + j; }
               }
             }
@@ -799,15 +799,14 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
-            const float x0 = fmaf(v[j], k1, k0), x1 = fmaf(v[j + 1], k1, k0);
+            const float x0 = fmaf(v[j], k1i, k0), x1 = fmaf(v[j + 1], k1i, k0);
             const float e0 = ex2(x0), e1 = ex2(x1);
             Z += e0 + e1;
             S2 = fmaf(e0, x0, fmaf(e1, x1, S2));
             if constexpr (F8) {
               // P' = P 2^(Ee[v] - u) as e5m2 (lower byte: the lower column)
-              const uint32_t two = __nv_cvt_float2_to_fp8x2(
-                  make_float2(e0 * pow2f(eev[j] - p.u), e1 * pow2f(eev[j + 1] - p.u)),
-                  __NV_SATFINITE, __NV_E5M2);
+              const uint32_t two = __nv_cvt_float2_to_fp8x2(make_float2(e0 * pq, e1 * pq),
+                                                            __NV_SATFINITE, __NV_E5M2);
               if (j & 2) pk[j >> 2] |= two << 16;
               else pk[j >> 2] = two;
             } else {
@@ -833,7 +832,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         TcStat ts;
         ts.Z = Z;
         ts.S1 = S2 * 0.6931471805599453f;
-        ts.best = vbest * scale;
+        ts.best = vbest * scalei;
         ts.arg = arg;
         p.tstats2[(size_t)row * (2 * p.n_vt) + 2 * vt + half] = ts;
         if constexpr (DRAW) {

@@ -54,7 +54,8 @@ struct TcFp8 {
 int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, void* ws, char* err,
                  size_t errn, int v0, int Vg, const TcFp8* f8 = nullptr);
 // Narrow E (dg_fp8.cu): quantise rows of a bf16 [rows][d] array to e4m3 codes
-// with per-row power-of-two exponents; the largest exponent goes to *emax.
+// with one power-of-two exponent per 256-row block (stored for every row);
+// the largest exponent goes to *emax.
 cudaError_t launch_quantize_e(cudaStream_t s, const void* E, int rows, int d, uint8_t* Eq,
                               int32_t* Ee, int* emax);
 // The step's prologue for narrow E: stand-in (or caller's) h in bf16, its e4m3
