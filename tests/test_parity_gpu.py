@@ -647,6 +647,24 @@ def test_device_wait_timeout_is_reported_and_recovered():
     den.close()
 
 
+def test_attention_kernel_clock_stamps():
+    """Every tensor-core step stamps one CTA's %globaltimer and clock counter at
+    its start and end (row 255 of DG_TC_TRACE_COUNTERS): the SM clock the kernel
+    ran at comes out between 0.3 and 3 GHz, and the stamps move with each step."""
+    w = synthetic.SMALL.replace(fixed_steps=1)
+    den, _ = make(w, dg.DG_IMPL_TC)
+    den.step()
+    r1 = den.read(dg.DG_TC_TRACE_COUNTERS)[255].cpu().tolist()
+    den.step()
+    r2 = den.read(dg.DG_TC_TRACE_COUNTERS)[255].cpu().tolist()
+    for r in (r1, r2):
+        assert r[2] > r[0] and r[3] > r[1]
+        ghz = (r[3] - r[1]) / (r[2] - r[0])
+        assert 0.3 < ghz < 3.0, ghz
+    assert r2[0] > r1[2]
+    den.close()
+
+
 def test_block_loop_needs_a_stream():
     w = synthetic.TINY
     Eg, _ = embedding(w)
