@@ -76,9 +76,17 @@ constexpr uint32_t B_BYTES = BN * BK * 2;
 template <int CG> struct Pipe {
   static constexpr int STAGES = CG == 2 ? 6 : 4;
   static constexpr uint32_t STAGE = A_BYTES + B_BYTES / CG;
-  static constexpr int STAGES_W2 = 4;
+  static constexpr int STAGES_W2 = CG == 2 ? 4 : 0;   // single CTAs never take W2 = 2
   static constexpr uint32_t STAGE_W2 = A_BYTES + 2 * (B_BYTES / CG);
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 512;
+  // The stage region holds either role's ring; the barriers sit after the
+  // larger of the two, so that neither ring can reach them.
+  static constexpr size_t RING_BYTES =
+      (size_t)STAGES * STAGE > (size_t)STAGES_W2 * STAGE_W2 ? (size_t)STAGES * STAGE
+                                                            : (size_t)STAGES_W2 * STAGE_W2;
+  static constexpr size_t SMEM = 1024 + RING_BYTES + 512;
+  static_assert(RING_BYTES >= (size_t)STAGES * STAGE && RING_BYTES >= (size_t)STAGES_W2 * STAGE_W2,
+                "stage region smaller than a role's ring");
+  static_assert(SMEM <= 227 * 1024, "stage region exceeds the per-CTA shared memory limit");
 };
 constexpr unsigned long long TIMEOUT_NS = 2000000000ull;   // 2 s: the default wait limit
 
@@ -418,6 +426,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                       const __grid_constant__ CUtensorMap tm_p,
                       const __grid_constant__ Params p) {
   constexpr int NSTAGE_MAX = Pipe<CG>::STAGES;         // barrier array size
+  static_assert(Pipe<CG>::STAGES_W2 <= NSTAGE_MAX, "barrier arrays sized for the G1 ring");
+  static_assert((2 * NSTAGE_MAX + 6 + 2 * QN) * 8 + QN * 4 <= 512, "barrier area overflows");
   constexpr int NB_ROWS = BN / CG;                      // B rows (G1) / columns (G2) per CTA
   // G1 CTAs and single-accumulator G2 CTAs: Pipe::STAGES stages of A + B/CG;
   // two-accumulator G2 CTAs: Pipe::STAGES_W2 stages of A + 2B/CG.
@@ -438,7 +448,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Pipe<CG>::STAGES * Pipe<CG>::STAGE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Pipe<CG>::RING_BYTES);
   uint64_t* full = bars;                        // [STAGES] (leader's counts both CTAs' bytes)
   uint64_t* empty = bars + NSTAGE_MAX;          // [STAGES]
   uint64_t* acc_full = bars + 2 * NSTAGE_MAX;   // [2]
