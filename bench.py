@@ -10,7 +10,9 @@ HBM every step, so no L2 flush is needed between steps.
 
 The JSON line (rank 0) carries:
   value     device-timed throughput with inputs resident (CUDA events around K
-            steps on the context's stream, max over ranks).
+            steps on the context's stream, max over ranks; no event inside a
+            step, where one would end the kernels' programmatic dependent
+            launches).
   e2e       the same metric through dg_denoise_step_h with host buffers: every
             step copies its hidden state from pinned host memory (on the
             library's copy stream, overlapping the step before) and the updated
@@ -18,9 +20,12 @@ The JSON line (rank 0) carries:
             with a synchronisation on both sides.
   roofline  the vocabulary-attention kernel (the dominant kernel) against the
             tensor roofline: 4*C*d*V flops per step over its event-timed
-            duration. The peak is the measured burst bf16 figure when the timed
+            duration (events around its launches in a second run of the same
+            K steps). The peak is the measured burst bf16 figure when the timed
             region is short (under 2 s), the sustained one otherwise; both
             fractions, the region's length and the sampled clock are given.
+  step_timeline_us  the last timed step's kernel boundaries from in-kernel
+            %globaltimer stamps, after the previous step's merge ended.
   cpu_baseline  the CPU oracle (fp64 numpy) on whole steps of the workload.
   workloads the other configurations: the tiny fp32 check (latency), the small
             and latency-sensitive canvases (throughput and roofline), and four
@@ -222,7 +227,7 @@ def choose_peak(timed_s: float, clk) -> str:
     return "burst" if timed_s < BURST_MAX_S else "sustained"
 
 
-def kernel_roofline(w, pk, kernel_s: float, timed_s: float, clk, kernel: str):
+def kernel_roofline(w, pk, kernel_s: float, timed_s: float, clk, kernel: str, timeline=None):
     """Roofline object of the vocabulary-attention kernel at one launch per step.
 
     Algorithmic work per launch: 4 C d V flops (both contractions) and V d b_E
@@ -251,6 +256,10 @@ def kernel_roofline(w, pk, kernel_s: float, timed_s: float, clk, kernel: str):
                 "frac": achieved / pk["hbm"]}
     roof.update({
         "kernel": kernel, "kernel_us_per_launch": kernel_s * 1e6,
+        "kernel_time_src": "CUDA events on the context's stream around each step's first "
+                           "attention launch (the redo pass, which returns at once, is outside), "
+                           "over a second run of the same steps; the step rate comes from the "
+                           "run without them",
         "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": bytes_,
         "peak_choice": which,
         "peak_src": f"{pk['src']} ({'bf16 burst' if which == 'burst' else 'bf16 sustained'}"
@@ -269,6 +278,13 @@ def kernel_roofline(w, pk, kernel_s: float, timed_s: float, clk, kernel: str):
         nominal = 148 * 8192 * ratio * kmhz * 1e6 / 1e12
         roof["kernel_sm_mhz"] = kmhz
         roof["frac_nominal_at_kernel_clock"] = achieved / nominal
+    if timeline and tensor_bound:
+        # the same kernel in the run without events, from its own stamps: from
+        # its dependency wait to the redo pass finding it complete
+        ks = (timeline["first_pass_done"] - timeline["attention_past_wait"]) * 1e-6
+        if ks > 0:
+            roof["kernel_us_timeline"] = ks * 1e6
+            roof["frac_timeline"] = flops / ks / 1e12 / P
     if pk.get("clocks"):
         roof["peak_clocks"] = pk["clocks"]
     return roof
@@ -364,12 +380,35 @@ def kernel_clock_mhz(den):
     return 1e3 * (r[3] - r[1]) / dt if dt > 0 else None
 
 
+def step_timeline(den):
+    """The last step's timeline from the kernels' %globaltimer stamps (row 255
+    of DG_TC_TRACE_COUNTERS, each by CTA 0 of its kernel), in us after the
+    previous step's merge kernel ended; None for CUDA-core contexts."""
+    import uniform_state_text_b200 as dg
+    if den.impl != dg.DG_IMPL_TC:
+        return None
+    r = den.read(dg.DG_TC_TRACE_COUNTERS)[255].cpu().tolist()
+    if not (r[9] > 0 and r[8] >= r[9]):
+        return None
+    keys = (("attention_started", 0), ("attention_past_wait", 4), ("first_pass_done", 5),
+            ("merge_started", 6), ("merge_past_wait", 7), ("merge_done", 8))
+    return {k: (r[j] - r[9]) / 1e3 for k, j in keys}
+
+
 def timed_steps(den, step, steps: int, warmup: int, local: int, dist=None):
     """Device-timed region of `steps` calls of step() on den's stream.
 
-    Returns (ms of the region, max over ranks), (attention-kernel ms, steps
-    timed, kernels launched) from dg_profile, the sampled clocks and the
-    region's length in seconds.
+    The region itself has no event inside a step: an event recorded between two
+    kernels ends their programmatic dependent launch, and the two per step that
+    timing the attention kernel needs added about 10 us of gaps per step
+    (measured). So the same `steps` calls run twice: first bare, for the step
+    time; then with dg_profile's events around each attention launch, for that
+    kernel's duration and the launch count.
+
+    Returns (ms of the bare region, max over ranks), (attention-kernel ms,
+    steps timed, kernels launched) from the profiled pass, the clocks sampled
+    during the bare region, its length in seconds and the timeline of its last
+    step (step_timeline).
     """
     import torch
 
@@ -385,7 +424,6 @@ def timed_steps(den, step, steps: int, warmup: int, local: int, dist=None):
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.3)
-    dg.dg_profile(den.ctx, True)
     ev0.record(den.stream)
     for _ in range(steps):
         step()
@@ -394,15 +432,22 @@ def timed_steps(den, step, steps: int, warmup: int, local: int, dist=None):
     if dist:
         dist.barrier()
     ms = ev0.elapsed_time(ev1)
+    clk = clocks.stop()
+    kclk = kernel_clock_mhz(den)
+    tl = step_timeline(den)
+    dg.dg_profile(den.ctx, True)
+    for _ in range(steps):
+        step()
     prof = dg.dg_profile_read(den.ctx)
     dg.dg_profile(den.ctx, False)
-    clk = clocks.stop()
+    if dist:
+        dist.barrier()
     st = den.state()
     if st["status"] != 0:
         raise RuntimeError(f"device status {st['status']}")
     if clk is not None:
-        clk["kernel_sm_mhz"] = kernel_clock_mhz(den)
-    return max_over_ranks(ms, dist, "cuda"), prof, clk, ms / 1e3
+        clk["kernel_sm_mhz"] = kclk
+    return max_over_ranks(ms, dist, "cuda"), prof, clk, ms / 1e3, tl
 
 
 def e2e_leg(den, w, steps: int, dist=None):
@@ -509,7 +554,7 @@ def headline_line(args, w, world, rank, local, dist):
     E = E_cpu.to(f"cuda:{local}")
     den = dg.Denoiser(w, E, impl=impl)
     kern = "tcgen05" if den.impl == dg.DG_IMPL_TC else "CUDA-core"
-    ms, (attn_ms, attn_steps, launches), clk, timed_s = timed_steps(
+    ms, (attn_ms, attn_steps, launches), clk, timed_s, timeline = timed_steps(
         den, FixedStepLoop(den, w.max_steps), args.steps, args.warmup, local, dist)
     value = whole_job_rate(args.steps, world, ms)
     ms_per_step = ms / args.steps
@@ -531,7 +576,7 @@ def headline_line(args, w, world, rank, local, dist):
     pk = measured_peaks()
     t_b, t_s, _ = step_roofline(w, pk)
     roof = kernel_roofline(w, pk, (attn_ms / 1e3) / max(attn_steps, 1), timed_s, clk,
-                           f"vocabulary attention ({kern})")
+                           f"vocabulary attention ({kern})", timeline)
     traffic = DRAM_TRAFFIC.get((w.name, w.e_format)) if den.impl == dg.DG_IMPL_TC else None
     roof["traffic"] = traffic[0] if traffic else None
     roof["traffic_src"] = traffic[1] if traffic else None
@@ -559,7 +604,7 @@ def headline_line(args, w, world, rank, local, dist):
                              % (w.e_bytes / 1e9),
                        "parallelism": f"replicas x{world}"},
             "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
-            "redo_cost": redo}
+            "step_timeline_us": timeline, "redo_cost": redo}
     return line, E_cpu
 
 
@@ -572,7 +617,7 @@ def workload_throughput(w, steps, warmup, local, with_cpu: bool):
     E = E_cpu.cuda()
     den = dg.Denoiser(w, E)
     kern = "tcgen05" if den.impl == dg.DG_IMPL_TC else "CUDA-core"
-    ms, (attn_ms, attn_steps, launches), clk, timed_s = timed_steps(
+    ms, (attn_ms, attn_steps, launches), clk, timed_s, timeline = timed_steps(
         den, FixedStepLoop(den, w.max_steps), steps, warmup, local)
     pk = measured_peaks()
     t_b, t_s, _ = step_roofline(w, pk)
@@ -582,11 +627,11 @@ def workload_throughput(w, steps, warmup, local, with_cpu: bool):
            "mode": "fixed_steps", "steps": steps, "warmup": warmup,
            "value": 1e3 / ms_step, "unit": "steps/s", "ms_per_step": ms_step,
            "tok_per_s": w.C * 1e3 / ms_step, "gpu_launches": launches, "clocks": clk,
-           "step_roofline_us": t_b * 1e6,
+           "step_timeline_us": timeline, "step_roofline_us": t_b * 1e6,
            "step_roofline_pct": 100.0 * t_b / (ms_step / 1e3),
            "step_roofline_pct_sustained": 100.0 * t_s / (ms_step / 1e3),
            "roofline": kernel_roofline(w, pk, (attn_ms / 1e3) / max(attn_steps, 1), timed_s, clk,
-                                       f"vocabulary attention ({kern})")}
+                                       f"vocabulary attention ({kern})", timeline)}
     tr = DRAM_TRAFFIC.get((w.name, w.e_format)) if den.impl == dg.DG_IMPL_TC else None
     out["roofline"]["traffic"] = tr[0] if tr else None
     den.close()
@@ -606,7 +651,7 @@ def tiny_latency(local, reps: int = 200):
     E = synthetic.make_embedding(w).cuda()
     wf = w.replace(fixed_steps=1)
     den = dg.Denoiser(wf, E)
-    ms, (attn_ms, attn_steps, launches), clk, _ = timed_steps(
+    ms, (attn_ms, attn_steps, launches), clk, _, _ = timed_steps(
         den, FixedStepLoop(den, wf.max_steps), reps, 5, local)
     den.close()
     den = dg.Denoiser(w, E)
@@ -702,7 +747,7 @@ def vocab_parallel_line(args, w, world, rank, local, dist):
             vocab_parallel_loop(den, buf, w.C, w.d)
         state["t"] += 1
 
-    ms, (attn_ms, attn_steps, launches), clk, timed_s = timed_steps(
+    ms, (attn_ms, attn_steps, launches), clk, timed_s, timeline = timed_steps(
         den, step, args.steps, args.warmup, local, dist)
     value = shared_canvas_rate(args.steps, ms)
     den.close()

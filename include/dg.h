@@ -135,7 +135,12 @@ typedef struct dg_ctx dg_ctx;
                            /* with -DDG_TC_TRACE; in every build row 255    */
                            /* holds CTA 0's %globaltimer and clock64 at its */
                            /* start (0, 1) and end (2, 3): the SM clock the */
-                           /* kernel ran at (read-only)                     */
+                           /* kernel ran at; and %globaltimer stamps of the */
+                           /* step's timeline, each by CTA 0: 4 first pass  */
+                           /* past its dependency wait, 5 redo pass past    */
+                           /* its wait, 6 merge kernel started, 7 merge     */
+                           /* past its wait, 8 merge done (fast path), 9    */
+                           /* the previous step's stamp 8 (read-only)       */
 
 /* Indices into the DG_STATE array. */
 #define DG_ST_T          0  /* next step index within the block               */
@@ -293,8 +298,10 @@ int dg_write(dg_ctx* ctx, int32_t what, const void* src_dev);
 
 /*
  * Per-step timing of the vocabulary-attention kernel(s) (the tensor-core
- * kernel alone on that path; the CUDA-core attention kernels otherwise), for
- * measurement:
+ * kernel's first launch, the one that does the step's work, on that path; the
+ * CUDA-core attention kernels otherwise), for measurement. The events sit
+ * between kernels that otherwise overlap their launches, so a profiled step
+ * runs a little slower than one without:
  * enable != 0 records CUDA events around them on the context's stream in every
  * dg_denoise_step / dg_denoise_step_h and resets the counters;
  * dg_profile_read synchronises and returns the total milliseconds and number
@@ -343,6 +350,7 @@ int dg_inject_stall(dg_ctx* ctx, int64_t wait_limit_ns, int32_t stall);
  *   [2] RB: 128-row blocks   [3] n_vt: 256-entry tiles   [4] n_ranges
  *   [5] n_dt: slices of d    [6] G: range groups         [7] n1: G1 units
  *   [8] n2: G2 units         [9] ring: P tiles resident  [10] CTAs launched
+ *   (the ring holds every tile when n_vt <= 128, else 72 of them).
  * Returns 11, DG_EUNSUPPORTED if the tensor-core kernels do not cover the
  * shape, or DG_EINVAL (NULL out, n < 11, sms < 2); dg_last_error(NULL) gives
  * the message.

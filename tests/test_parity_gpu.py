@@ -453,6 +453,39 @@ def test_external_hidden_state_from_host(impl, name):
     den.close()
 
 
+def test_full_size_redo_pass():
+    """The redo pass at the headline size. Caller hidden states h = 30 E[token]
+    put a row's largest logit far above its reference (the logit of its canvas
+    token, or of its previous argmax) unless that token is the row's argmax
+    already: step 0 overshoots on every row, step 1 (the same tokens except on
+    1% of the rows) on those rows only. Both steps are redone by the second
+    tensor-core pass and must equal the oracle's step."""
+    w = synthetic.HEADLINE.replace(fixed_steps=1, max_steps=4)
+    den, E32 = make(w, dg.DG_IMPL_TC)
+    Eg, _ = embedding(w)
+    g = torch.Generator().manual_seed(11)
+    tok_a = torch.randint(0, w.V, (w.C,), generator=g)
+    tok_b = tok_a.clone()
+    k = max(1, w.C // 100)
+    tok_b[:k] = torch.randint(0, w.V, (k,), generator=g)
+
+    def hid(tok):
+        return (30.0 * Eg[tok.cuda()].float()).to(torch.bfloat16).contiguous()
+
+    tally = Tally()
+    redone = []
+    for h in (hid(tok_a), hid(tok_b)):
+        r0 = den.state()["redo"]
+        pre = _np(den.read(dg.DG_ARGMAX)).astype(np.int64) if den.state()["has_prev"] else None
+        assert step_and_compare(den, w, E32, tally, pre, do_step=lambda: den.step_h(h),
+                                h_given=_np(h))
+        redone.append(den.state()["redo"] - r0)
+    assert redone[0] >= w.C - 2, redone      # all rows (bar a canvas token equal to the row's)
+    assert redone[1] == k, redone
+    tally.check_budget()
+    den.close()
+
+
 @pytest.mark.parametrize("impl", IMPLS)
 @pytest.mark.parametrize("variant", ["minus_max", "argmax_stop", "tau0"])
 def test_sampler_rules_teacher_forced(impl, variant):
@@ -650,7 +683,8 @@ def test_device_wait_timeout_is_reported_and_recovered():
 def test_attention_kernel_clock_stamps():
     """Every tensor-core step stamps one CTA's %globaltimer and clock counter at
     its start and end (row 255 of DG_TC_TRACE_COUNTERS): the SM clock the kernel
-    ran at comes out between 0.3 and 3 GHz, and the stamps move with each step."""
+    ran at comes out between 0.3 and 3 GHz, and the stamps move with each step.
+    The timeline stamps of the redo pass and the merge kernel are in causal order."""
     w = synthetic.SMALL.replace(fixed_steps=1)
     den, _ = make(w, dg.DG_IMPL_TC)
     den.step()
@@ -661,7 +695,10 @@ def test_attention_kernel_clock_stamps():
         assert r[2] > r[0] and r[3] > r[1]
         ghz = (r[3] - r[1]) / (r[2] - r[0])
         assert 0.3 < ghz < 3.0, ghz
+        # the step's timeline: each stamp follows the completion it waits for
+        assert r[0] <= r[4] <= r[5] <= r[7] <= r[8] and r[6] <= r[7], r[:10]
     assert r2[0] > r1[2]
+    assert r2[9] == r1[8] and r2[9] <= r2[4]        # the previous merge's end, kept
     den.close()
 
 

@@ -55,6 +55,7 @@ def check_shape(C, V, d, sms=148):
     assert len(cover) == s["n_ranges"] * RB * s["n_dt"]
     # progress of the hand-off
     ring, n_vt = s["ring"], s["n_vt"]
+    assert ring == (n_vt if n_vt <= 128 else 72)   # every tile resident up to 128 tiles
     consumers = RBI * s["n_dt"]               # G2 units that load each tile
     ready = [0] * n_vt                        # row blocks of the tile written
     consumed = [0] * n_vt

@@ -341,8 +341,7 @@ int launch_step(dg_ctx* ctx, bool standin, bool use_cond, const void* hsrc = nul
   if (tc) {
     DG_CK(launch_tc_attention(s, ctx->tc_plan, ctx->st, ctx->h, ctx->E, ctx->mref, ctx->scale_tab,
                               c.max_steps, ctx->tstats, ctx->tc, ctx->draw, ctx->H,
-                              ctx->argmax, ctx->rowstat, ctx->redo_gap, sa));
-    if (e1) DG_CK(cudaEventRecord(e1, s));
+                              ctx->argmax, ctx->rowstat, ctx->redo_gap, sa, e1));
     // sc, the next step's h (and, if a row needs the exact recomputation, the
     // rows' merge and the sampler)
     DG_CK(launch_tc_merge(s, ctx->tc_plan, ctx->st, ctx->tstats, ctx->mref, ctx->rowstat, ctx->H,

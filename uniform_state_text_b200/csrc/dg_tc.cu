@@ -64,7 +64,12 @@ constexpr int BK = 64;         // K per pipeline stage (one 128-byte swizzle row
 constexpr int KV2 = 256;       // vocabulary entries per range (unit of G2 ownership): one tile,
                                // so range group g owns tiles g, g+G, ... and all groups
                                // advance through the ring together
-constexpr int RING = 72;       // P tiles (256 vocabulary entries each) resident at once
+// P tiles (256 vocabulary entries each) resident at once: every tile when the
+// vocabulary has at most RING_ALL tiles, else RING. A ring of 72 measured best
+// at 1024 tiles (56 and 96 were slower: E rows wait longer in L2 between their
+// two reads); at 128 tiles holding them all took the ring waits out of G1.
+constexpr int RING = 72;
+constexpr int RING_ALL = 128;
 constexpr int THREADS = 320;    // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr int EPI_WARPS = 8;
 constexpr int QN = 8;          // G1 item queue depth (tile indices handed to the CTA's warps)
@@ -96,7 +101,8 @@ struct Params {
   float* mref;                 // per-row logit reference; the first pass raises a low one
   const float* scale_tab;
   float* Opart;              // [G][C][d]
-  void* P;                   // [RING][C][BN]: ring of P tiles (bf16, or e5m2 codes for F8)
+  void* P;                   // [ring][C][BN]: ring of P tiles (bf16, or e5m2 codes for F8)
+  int ring;                  // P tiles in the ring
   unsigned* ready;           // [n_vt]: epilogue warps that finished a tile
   unsigned* consumed;        // [n_vt]: G2 CTAs that finished loading a tile
   int* abort_flag;
@@ -440,6 +446,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // its redo flag; with no row to redo the whole grid returns before any
     // set-up, and lets the next kernel launch at once.
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (blockIdx.x == 0 && threadIdx.x == 0) p.trace[255 * 32 + 5] = gtimer();
     if (*(volatile const int*)p.redo_in == 0) {
       asm volatile("griddepcontrol.launch_dependents;");
       return;
@@ -512,6 +519,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   // can only take SMs this grid has left, and wait there for it to complete,
   // so that its check of the redo flag follows this pass without a launch gap.
   if (p.pass == 0) asm volatile("griddepcontrol.launch_dependents;");
+  if (blockIdx.x == 0 && threadIdx.x == 0 && p.pass == 0) {
+    // the previous step's merge has completed: keep its end stamp
+    p.trace[255 * 32 + 9] = p.trace[255 * 32 + 8];
+    p.trace[255 * 32 + 4] = gtimer();
+  }
   const bool skip = p.st->done != 0;                     // uniform over the grid
   // CTA 0 is a G1 CTA: this reset precedes its g1_done release, so it is
   // ordered before the sampler sets the flag again at the end of G1. A skipped
@@ -562,9 +574,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (it < 0) break;
           const int vt = it / RBI;
           const int rb = CG == 2 ? (int)rank : it % RBI;
-          if (vt >= RING) {
+          if (vt >= p.ring) {
             TR_T0();
-            if (!counter_wait(&p.consumed[vt - RING], consumed_target, p)) { ok = false; break; }
+            if (!counter_wait(&p.consumed[vt - p.ring], consumed_target, p)) { ok = false; break; }
             TR_ADD(w_ctr);
           }
           for (int kc = 0; kc < nk1; ++kc) {
@@ -594,7 +606,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             TR_ADD(w_empty);
             unsigned char* st = smem + s * STAGE_BYTES;
             if (leader) mbar_expect_tx(&full[s], STAGE_BYTES * CG);
-            tma_load<CG>(st, &tm_p, &full[s], (kc % TPS) * BKE, (vt % RING) * p.C + rb2 * BM,
+            tma_load<CG>(st, &tm_p, &full[s], (kc % TPS) * BKE, (vt % p.ring) * p.C + rb2 * BM,
                          keep);
             // E as the MN-major B operand: boxes of BOXC columns of d (128 bytes)
             // by BKE vocabulary rows
@@ -765,7 +777,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         float gbest = -INFINITY;    // multinomial draw: best z + G, first index on ties
         int garg = 0x7fffffff;
         unsigned char* prow = static_cast<unsigned char*>(p.P) +
-                              (((size_t)(vt % RING) * p.C + row) * BN + c0) * (F8 ? 1 : 2);
+                              (((size_t)(vt % p.ring) * p.C + row) * BN + c0) * (F8 ? 1 : 2);
 #pragma unroll 1
         for (int c = 0; c < HALF / 32; ++c) {
           float v[32];
@@ -1065,11 +1077,14 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
     RowStat* rowstat, float* H, int32_t* argmax, float* sc, float redo_gap,
     __nv_bfloat16* h, const __nv_bfloat16* E, const float* scale_tab, int S,
     unsigned* ticket, const TcSamp* tsamp, int32_t* sampled, const NextStandin nx,
-    const SamplerArgs sa) {
+    const SamplerArgs sa, unsigned long long* stamp) {
   // Programmatic dependent launch: wait for the attention kernel's results.
   // No early trigger: the next kernel is usually the next step's attention
   // kernel, and its CTAs waiting beside this grid slowed it (measured).
+  const bool stamper = blockIdx.x == 0 && threadIdx.x == 0;
+  if (stamper) stamp[6] = gtimer();
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (stamper) stamp[7] = gtimer();
   // The attention kernel's G1 CTAs normally merged the rows and ran the
   // sampler already (tc_sampled); then only sc, the copies of this step's h
   // and the next step's h remain -- sc even when that sampler stopped the
@@ -1105,6 +1120,7 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
     __syncthreads();
     merge_fast_tail(st, Opart, nO, C, V, d, sc, h, E, scale_tab, S, argmax, sa.canvas, mref,
                     sh_inv, nx, i0);
+    if (stamper) stamp[8] = gtimer();
     return;
   } else {
   if (threadIdx.x == 0) sh_epoch0 = *(volatile int*)&st->epoch;   // before this CTA's ticket
@@ -1305,6 +1321,7 @@ struct TcLayout {
   int CG = 1;              // CTAs per MMA group (2: CTA pairs, M = 256)
   int W2 = 1;              // accumulators per G2 unit (2: a 512-column slice of d)
   int RB = 0, n_vt = 0, n_ranges = 0, n_dt = 0, G = 0, n1 = 0, n2 = 0;   // n1, n2 in groups
+  int ring = 0;            // P tiles in the ring
 };
 
 size_t al(size_t x) { return (x + 255) / 256 * 256; }
@@ -1326,6 +1343,7 @@ TcLayout tc_layout(int C, int V, int d, int sms, bool fp8 = false) {
   L.n_vt = V / tc::BN;
   L.n_ranges = V / tc::KV2;
   L.n_dt = d / (tc::BN * L.W2);
+  L.ring = L.n_vt <= tc::RING_ALL ? L.n_vt : tc::RING;
   // Choose the number of range groups G: G2 units = RBI * n_dt * G, G1 units take
   // the rest; minimise the larger of the two roles' per-unit work.
   const int units = sms / L.CG;
@@ -1350,7 +1368,7 @@ TcLayout tc_layout(int C, int V, int d, int sms, bool fp8 = false) {
   size_t off = 0;
   // two sets of hand-off counters: the first pass's and the redo pass's
   L.counters = off; off = al(off + sizeof(unsigned) * 2 * (2 * (size_t)L.n_vt + 64));
-  L.P = off; off = al(off + (size_t)tc::RING * C * tc::BN * (fp8 ? 1 : 2));
+  L.P = off; off = al(off + (size_t)L.ring * C * tc::BN * (fp8 ? 1 : 2));
   L.Opart = off; off = al(off + (size_t)(L.G > 0 ? L.G : 1) * C * d * 4);
   L.trace = off; off = al(off + (size_t)256 * 32 * 8);
   L.total = off;
@@ -1411,7 +1429,7 @@ bool tc_schedule_info(int C, int V, int d, int sms, int32_t* out) {
   const TcLayout L = tc_layout(C, V, d, sms);
   if (L.G < 1 || L.n1 < 1) return false;
   const int32_t v[kTcScheduleValues] = {L.CG, L.W2, L.RB, L.n_vt, L.n_ranges, L.n_dt, L.G,
-                                        L.n1, L.n2, tc::RING, L.CG * (L.n1 + L.n2)};
+                                        L.n1, L.n2, L.ring, L.CG * (L.n1 + L.n2)};
   for (int i = 0; i < kTcScheduleValues; ++i) out[i] = v[i];
   return true;
 }
@@ -1523,7 +1541,7 @@ int tc_plan_init(TcPlan* p, int C, int V, int d, const void* E, void* h, void* w
   bool ok = encode(&maps[0], h, (uint64_t)d, (uint64_t)C, bk, tc::BM, b8) &&
             encode(&maps[1], E, (uint64_t)d, (uint64_t)V, bk, tc::BN / L.CG, b8) &&
             encode(&maps[2], E, (uint64_t)d, (uint64_t)V, boxc, bk, b8) &&
-            encode(&maps[3], base + L.P, (uint64_t)tc::BN, (uint64_t)tc::RING * C, bk, tc::BM, b8);
+            encode(&maps[3], base + L.P, (uint64_t)tc::BN, (uint64_t)L.ring * C, bk, tc::BM, b8);
   if (!ok) {
     snprintf(err, errn, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
     return -3;
@@ -1564,7 +1582,7 @@ tc::Params base_params(const TcPlan& pl, const TcLayout& L, DevState* st, const 
   tc::Params prm;
   prm.C = pl.C; prm.V = pl.Vg; prm.d = pl.d; prm.RB = L.RB; prm.n_vt = L.n_vt;
   prm.n_ranges = L.n_ranges; prm.n_dt = L.n_dt; prm.G = L.G; prm.n1 = L.n1; prm.W2 = L.W2;
-  prm.tiles_per_range = tc::KV2 / tc::BN; prm.S = S;
+  prm.tiles_per_range = tc::KV2 / tc::BN; prm.S = S; prm.ring = L.ring;
   prm.mref = const_cast<float*>(mref); prm.scale_tab = scale_tab;
   prm.tstats2 = reinterpret_cast<TcStat*>(tstats);
   prm.Opart = reinterpret_cast<float*>(base + L.Opart);
@@ -1624,13 +1642,15 @@ cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& pl, DevState* st, 
                                 const void* E, const float* mref, const float* scale_tab,
                                 int S, TileStat* tstats, void* ws,
                                 const DrawArgs& draw, float* H, int32_t* argmax,
-                                RowStat* rowstat, float redo_gap, const SamplerArgs& sa) {
+                                RowStat* rowstat, float redo_gap, const SamplerArgs& sa,
+                                cudaEvent_t after_first) {
   (void)h; (void)E;
   TcLayout L = tc_layout(pl.C, pl.V, pl.d, pl.num_sms, pl.fp8);
   const tc::Params prm = base_params(pl, L, st, mref, scale_tab, S, tstats, ws, draw, H, argmax,
                                      rowstat, redo_gap, sa, 0);
   cudaError_t e = launch_params(s, pl, L, prm);
   if (e != cudaSuccess) return e;
+  if (after_first && (e = cudaEventRecord(after_first, s)) != cudaSuccess) return e;
   // the redo pass (returns at once unless a row's reference was too low)
   const tc::Params prm2 = base_params(pl, L, st, mref, scale_tab, S, tstats, ws, draw, H, argmax,
                                       rowstat, redo_gap, sa, 1);
@@ -1762,7 +1782,8 @@ cudaError_t merge_launch(cudaStream_t s, const TcPlan& pl, DevState* st, const T
       rowstat, H, argmax, sc, redo_gap, static_cast<__nv_bfloat16*>(const_cast<void*>(h)),
       static_cast<const __nv_bfloat16*>(E), scale_tab, S,
       reinterpret_cast<unsigned*>(static_cast<char*>(pl.ws) + L.counters) + 2 * L.n_vt + 2,
-      tsamp, draw.sampled, nx, sa);
+      tsamp, draw.sampled, nx, sa,
+      reinterpret_cast<unsigned long long*>(static_cast<char*>(pl.ws) + L.trace) + 255 * 32);
 }
 
 const void* tc_trace(const TcPlan& pl, size_t* bytes) {

@@ -80,7 +80,9 @@ cudaError_t launch_tc_attention(cudaStream_t s, const TcPlan& p, DevState* st, c
                                 const void* E, const float* mref, const float* scale_tab,
                                 int S, TileStat* tstats, void* ws,
                                 const DrawArgs& draw, float* H, int32_t* argmax,
-                                RowStat* rowstat, float redo_gap, const SamplerArgs& sa);
+                                RowStat* rowstat, float redo_gap, const SamplerArgs& sa,
+                                cudaEvent_t after_first = nullptr);
+// (after_first: recorded between the two launches when given, to time the first.)
 // Per-row merge of the kernel's statistics and partials into sc, H and argmax
 // (rows whose maximum overshot the reference are recomputed exactly); the last
 // CTA then runs the sampler and stop test for the whole canvas, after which
