@@ -566,8 +566,9 @@ def headline_line(args, w, world, rank, local, dist):
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
                "tok_per_s": w.C * args.steps * world / el, "steps": args.steps,
                "path": "dg_denoise_step_h: hidden state from pinned host memory (copy stream, "
-                       "overlapping the step before), canvas to pinned host memory; host wall "
-                       "clock with a synchronisation on both sides"}
+                       "overlapping the step before), canvas to pinned host memory (written by "
+                       "the step's merge kernel, no copy in the stream); host wall clock with a "
+                       "synchronisation on both sides"}
 
     redo = None
     if den.impl == dg.DG_IMPL_TC and not args.no_workloads:

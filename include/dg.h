@@ -219,8 +219,12 @@ int dg_denoise_step(dg_ctx* ctx, int32_t* done_host);
  * before; the step itself waits for its copy on the context's stream. The
  * caller keeps h_src unchanged until the context's stream has passed this
  * step. canvas_host (nullable, pinned) receives the updated canvas, int32 [C],
- * asynchronously: it is valid once the stream has reached it. done_host
- * (nullable) receives the done flag; a non-NULL done_host synchronises.
+ * asynchronously: it is valid once the stream has passed this step. On the
+ * tensor-core path a page-locked canvas_host that the device can address (any
+ * cudaHostAlloc / cudaMallocHost buffer under unified addressing) is written
+ * by the step's last kernel directly, with no copy in the stream; other
+ * buffers are copied after the step. done_host (nullable) receives the done
+ * flag; a non-NULL done_host synchronises.
  */
 int dg_denoise_step_h(dg_ctx* ctx, const void* h_src, int32_t h_on_host,
                       int32_t* canvas_host, int32_t* done_host);

@@ -453,6 +453,27 @@ def test_external_hidden_state_from_host(impl, name):
     den.close()
 
 
+def test_canvas_to_host_buffers():
+    """dg_denoise_step_h's canvas_host on the tensor-core path: a pinned buffer
+    (written by the merge kernel itself), a pageable one (copied after the
+    step), and a fresh pinned one after the block has stopped (the merge
+    kernel's early return writes it too) all equal the context's canvas."""
+    w = synthetic.SMALL.replace(max_steps=2, fixed_steps=1)
+    den, _ = make(w, dg.DG_IMPL_TC)
+    Eg, _ = embedding(w)
+    for kind in ("pinned", "pageable", "pinned after stop"):
+        canvas = _np(den.read(dg.DG_CANVAS)).astype(np.int64)
+        h = _external_h(w, Eg, canvas, 99).cuda()
+        buf = torch.full((w.C,), -1, dtype=torch.int32)
+        if kind != "pageable":
+            buf = buf.pin_memory()
+        den.step_h(h, canvas_host=buf)
+        den.stream.synchronize()
+        assert np.array_equal(buf.numpy(), _np(den.read(dg.DG_CANVAS))), kind
+    assert den.state()["done"] == 1
+    den.close()
+
+
 def test_full_size_redo_pass():
     """The redo pass at the headline size. Caller hidden states h = 30 E[token]
     put a row's largest logit far above its reference (the logit of its canvas

@@ -235,6 +235,7 @@ struct dg_ctx {
   std::vector<cudaEvent_t> ev;
   size_t ev_used = 0;
   long long launches = 0;   // kernels launched since the last dg_profile call
+  int32_t* canvas_out = nullptr;   // set only while dg_denoise_step_h launches its step
   char err[512] = "";
 };
 
@@ -284,6 +285,7 @@ NextStandin next_standin(dg_ctx* ctx) {
   nx.mref_last = at<float>(ctx, ctx->L.mref_last);
   nx.fp8 = ctx->L.fp8 ? 1 : 0;
   nx.sc_scale = ctx->L.fp8 ? std::ldexp(1.0f, ctx->fp8_u) : 1.0f;
+  nx.canvas_out = ctx->canvas_out;
   return nx;
 }
 
@@ -557,6 +559,18 @@ int dg_denoise_step_h(dg_ctx* ctx, const void* h_src, int32_t h_on_host, int32_t
   const dg_config& c = ctx->cfg;
   const size_t bytes = (size_t)c.C * c.d * (c.dtype == DG_F32 ? 4 : 2);
   int rc;
+  // A pinned canvas_host that the device can address is written by the merge
+  // kernel itself (tensor-core path); anything else is copied after the step.
+  // The pointer reaches the kernels only through this call's launch_step.
+  int32_t* direct = nullptr;
+  if (canvas_host && ctx->L.impl == DG_IMPL_TC) {
+    cudaPointerAttributes pa;
+    if (cudaPointerGetAttributes(&pa, canvas_host) == cudaSuccess && pa.type == cudaMemoryTypeHost &&
+        pa.devicePointer)
+      direct = static_cast<int32_t*>(pa.devicePointer);
+    else
+      cudaGetLastError();
+  }
   if (h_on_host) {
     // The copy runs on the context's copy stream into a staging slot, so that
     // it overlaps the previous step's kernels; the step waits for it, and the
@@ -577,15 +591,19 @@ int dg_denoise_step_h(dg_ctx* ctx, const void* h_src, int32_t h_on_host, int32_t
     DG_CK(cudaMemcpyAsync(stage, h_src, bytes, cudaMemcpyHostToDevice, ctx->copy_stream));
     DG_CK(cudaEventRecord(ctx->ev_copied[slot], ctx->copy_stream));
     DG_CK(cudaStreamWaitEvent(ctx->stream, ctx->ev_copied[slot], 0));
+    ctx->canvas_out = direct;
     rc = launch_step(ctx, false, false, stage);
+    ctx->canvas_out = nullptr;
     if (rc) return rc;
     DG_CK(cudaEventRecord(ctx->ev_free[slot], ctx->stream));
   } else {
     DG_CK(cudaMemcpyAsync(ctx->h, h_src, bytes, cudaMemcpyDeviceToDevice, ctx->stream));
+    ctx->canvas_out = direct;
     rc = launch_step(ctx, false, false);
+    ctx->canvas_out = nullptr;
     if (rc) return rc;
   }
-  if (canvas_host)
+  if (canvas_host && !direct)
     DG_CK(cudaMemcpyAsync(canvas_host, ctx->canvas, sizeof(int32_t) * c.C, cudaMemcpyDeviceToHost,
                           ctx->stream));
   if (done_host) {

@@ -72,6 +72,10 @@ struct NextStandin {
   // prologue instead, and the P.E sums carry a factor 2^-u (sc_scale = 2^u).
   int fp8 = 0;
   float sc_scale = 1.f;
+  // Pinned host memory mapped into the device ([C]), or null: the merge kernel
+  // writes the step's canvas there itself (dg_denoise_step_h's canvas_host),
+  // so that no copy sits between this step's kernels and the next step's.
+  int32_t* canvas_out = nullptr;
 };
 
 // Multinomial token draw (DG_TOKEN_MULTINOMIAL): where the per-row draws go.

@@ -1095,6 +1095,8 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
   const bool fast = *(volatile int*)&st->tc_sampled != 0;
   if (!fast && st->done) {
     if (sa.use_cond && blockIdx.x == 0 && threadIdx.x == 0) cudaGraphSetConditional(sa.cond, 0);
+    if (nx.canvas_out && threadIdx.x < kMergeRows && blockIdx.x * kMergeRows + threadIdx.x < C)
+      nx.canvas_out[blockIdx.x * kMergeRows + threadIdx.x] = sa.canvas[blockIdx.x * kMergeRows + threadIdx.x];
     return;
   }
   __shared__ SamplerSmem sm;
@@ -1123,6 +1125,8 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
     __syncthreads();
     merge_fast_tail(st, Opart, nO, C, V, d, sc, h, E, scale_tab, S, argmax, sa.canvas, mref,
                     sh_inv, nx, i0);
+    if (nx.canvas_out && threadIdx.x < kMergeRows && i0 + (int)threadIdx.x < C)
+      nx.canvas_out[i0 + threadIdx.x] = sa.canvas[i0 + threadIdx.x];
     if (stamper) stamp[8] = gtimer();
     return;
   } else {
@@ -1221,6 +1225,8 @@ __global__ void __launch_bounds__(kMergeRows * kMergeThreadsPerRow) k_merge_tc(D
   if (last) {
     if (threadIdx.x < nsamp) {
       sample_and_stop(sa, sm, nsamp);
+      // thread i wrote position i of the canvas
+      if (nx.canvas_out && (int)threadIdx.x < C) nx.canvas_out[threadIdx.x] = sa.canvas[threadIdx.x];
       sum_sc = false;
     }
     x0 = threadIdx.x - nsamp;
