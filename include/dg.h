@@ -354,8 +354,8 @@ int dg_inject_stall(dg_ctx* ctx, int64_t wait_limit_ns, int32_t stall);
  *   [2] RB: 128-row blocks   [3] n_vt: 256-entry tiles   [4] n_ranges
  *   [5] n_dt: slices of d    [6] G: range groups         [7] n1: G1 units
  *   [8] n2: G2 units         [9] ring: P tiles resident  [10] CTAs launched
- *   (the ring holds every tile when n_vt <= 128, else 72 of them; a context
- *   with DG_E_FP8 holds 144).
+ *   (the ring holds every tile when n_vt <= 128, else 72 of them for CTA
+ *   pairs and 84 for single CTAs; a context with DG_E_FP8 holds 144).
  * Returns 11, DG_EUNSUPPORTED if the tensor-core kernels do not cover the
  * shape, or DG_EINVAL (NULL out, n < 11, sms < 2); dg_last_error(NULL) gives
  * the message.

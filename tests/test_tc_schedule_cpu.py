@@ -55,7 +55,8 @@ def check_shape(C, V, d, sms=148):
     assert len(cover) == s["n_ranges"] * RB * s["n_dt"]
     # progress of the hand-off
     ring, n_vt = s["ring"], s["n_vt"]
-    assert ring == (n_vt if n_vt <= 128 else 72)   # every tile resident up to 128 tiles
+    # every tile resident up to 128 tiles, else 72 (CTA pairs) or 84 (single CTAs)
+    assert ring == (n_vt if n_vt <= 128 else min(n_vt, 72 if CG == 2 else 84))
     consumers = RBI * s["n_dt"]               # G2 units that load each tile
     ready = [0] * n_vt                        # row blocks of the tile written
     consumed = [0] * n_vt

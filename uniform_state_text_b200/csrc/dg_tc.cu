@@ -66,12 +66,15 @@ constexpr int KV2 = 256;       // vocabulary entries per range (unit of G2 owner
                                // so range group g owns tiles g, g+G, ... and all groups
                                // advance through the ring together
 // P tiles (256 vocabulary entries each) resident at once: every tile when the
-// vocabulary has at most RING_ALL tiles, else RING (twice that with 8-bit E,
-// whose tiles take half the bytes). A ring of 72 measured best at 1024 tiles
-// with bf16 E (56 and 96 were slower: E rows wait longer in L2 between their
-// two reads), 144 with e4m3 E (72 and 96 left G1 waiting for slots, 192 was
-// slower); at 128 tiles holding them all took the ring waits out of G1.
+// vocabulary has at most RING_ALL tiles, else RING for CTA pairs with bf16 E,
+// RING_SINGLE for single CTAs (128-row canvases) with bf16 E, and RING_F8 with
+// e4m3 E. Measured at 1024 tiles: pairs 72 (56, 84, 96, 120 slower: E rows
+// wait longer in L2 between their two reads, and the clock drops), single CTAs
+// 84 (72 and 96 slower at d = 2816), e4m3 144 (72, 96, 168, 192 slower); at
+// 128 tiles holding them all took the ring waits out of G1.
 constexpr int RING = 72;
+constexpr int RING_SINGLE = 84;
+constexpr int RING_F8 = 144;
 constexpr int RING_ALL = 128;
 constexpr int THREADS = 320;    // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr int EPI_WARPS = 8;
@@ -1361,7 +1364,9 @@ TcLayout tc_layout(int C, int V, int d, int sms, bool fp8 = false) {
   L.n_vt = V / tc::BN;
   L.n_ranges = V / tc::KV2;
   L.n_dt = d / (tc::BN * L.W2);
-  L.ring = L.n_vt <= tc::RING_ALL ? L.n_vt : std::min(L.n_vt, tc::RING * (fp8 ? 2 : 1));
+  L.ring = L.n_vt <= tc::RING_ALL
+               ? L.n_vt
+               : std::min(L.n_vt, fp8 ? tc::RING_F8 : (L.CG == 2 ? tc::RING : tc::RING_SINGLE));
   // Choose the number of range groups G: G2 units = RBI * n_dt * G, G1 units take
   // the rest; minimise the larger of the two roles' per-unit work.
   const int units = sms / L.CG;
