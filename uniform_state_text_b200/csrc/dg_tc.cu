@@ -760,6 +760,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int vt = it / RBI;
         const int rb = CG == 2 ? (int)rank : it % RBI;
         const int buf = n & 1;
+        // The tile's row values are read before the wait for its accumulator,
+        // so that their latency overlaps the MMAs rather than the epilogue.
+        const int row = rb * BM + r_local;
+        const float mref = p.mref[row];
+        int et = 0, her = 0;
+        if constexpr (F8) {
+          et = __ldg(p.Ee + p.v0 + vt * BN);
+          her = p.he[row];
+        }
         {
           TR_T0();
           // every lane waits; the warp goes on only if all of them saw the
@@ -771,8 +780,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         TR_T0();
         tc_fence_after();
-        const int row = rb * BM + r_local;
-        const float mref = p.mref[row];
         const float k0 = -mref * 1.4426950408889634f;
         // F8: the tensor cores summed code products; the tile's exponent of E
         // and the row's of h bring them back to h_deq . E_deq (folded into the
@@ -780,8 +787,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // contraction takes
         float k1i = k1, scalei = scale, pq = 1.f;
         if constexpr (F8) {
-          const int et = __ldg(p.Ee + p.v0 + vt * BN);
-          const float s8 = pow2f(et + p.he[row]);
+          const float s8 = pow2f(et + her);
           k1i = k1 * s8;
           scalei = scale * s8;
           pq = pow2f(et - p.u);
@@ -793,15 +799,24 @@ __global__ void __launch_bounds__(THREADS, 1)
         int garg = 0x7fffffff;
         unsigned char* prow = static_cast<unsigned char*>(p.P) +
                               (((size_t)(vt % p.ring) * p.C + row) * BN + c0) * (F8 ? 1 : 2);
+        // Each chunk's TMEM load is issued before the previous chunk's math,
+        // and waited for after it.
+        const uint32_t tchunk = tmem + lane_addr + buf * BN + c0;
+        uint32_t rld[32];
+        tmem_ld32_issue(tchunk, rld);
 #pragma unroll 1
         for (int c = 0; c < HALF / 32; ++c) {
           float v[32];
           {
             TR_T0();
-            tmem_ld32(tmem + lane_addr + buf * BN + c0 + c * 32, v);
+            tmem_ld_wait(rld);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(rld[j]);
             TR_ADD(t_ld);
           }
-          if (c == HALF / 32 - 1) {
+          if (c + 1 < HALF / 32) {
+            tmem_ld32_issue(tchunk + (c + 1) * 32, rld);
+          } else {
             // Last read of this accumulator buffer: hand it back to the MMA warp.
             tc_fence_before();
             __syncwarp();
