@@ -294,10 +294,10 @@ def kernel_roofline(w, pk, kernel_s: float, timed_s: float, clk, kernel: str, ti
 # capture summarised under profiles/ (taken on the V=65536 profiling shape and
 # scaled by the vocabulary, since E and the P ring both grow with V).
 DRAM_TRAFFIC = {
-    (synthetic.HEADLINE.name, 0): (4 * (290.516992e6 + 8.263680e6),
+    (synthetic.HEADLINE.name, 0): (4 * (291.782144e6 + 9.212928e6),
                                    "ncu dram__bytes_read.sum + dram__bytes_write.sum of one first-pass "
                                    "launch at C=256, V=65536, d=2048, scaled by 4 to V=262144"),
-    (synthetic.HEADLINE.name, 1): (4 * (137.454080e6 + 5.851904e6),
+    (synthetic.HEADLINE.name, 1): (4 * (136.710912e6 + 6.254592e6),
                                    "ncu dram__bytes_read.sum + dram__bytes_write.sum of one first-pass "
                                    "launch (narrow E) at C=256, V=65536, d=2048, scaled by 4"),
 }
