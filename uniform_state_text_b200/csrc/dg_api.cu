@@ -285,6 +285,12 @@ NextStandin next_standin(dg_ctx* ctx) {
   nx.mref_last = at<float>(ctx, ctx->L.mref_last);
   nx.fp8 = ctx->L.fp8 ? 1 : 0;
   nx.sc_scale = ctx->L.fp8 ? std::ldexp(1.0f, ctx->fp8_u) : 1.0f;
+  if (ctx->L.fp8) {
+    nx.Eq = at<uint8_t>(ctx, ctx->L.Eq);
+    nx.Ee = at<int32_t>(ctx, ctx->L.Ee);
+    nx.hq = at<uint8_t>(ctx, ctx->L.hq);
+    nx.he = at<int32_t>(ctx, ctx->L.he);
+  }
   nx.canvas_out = ctx->canvas_out;
   return nx;
 }
@@ -298,7 +304,10 @@ int prologue_if_needed(dg_ctx* ctx, bool standin, bool use_cond, const void* hsr
   int nzero = 0;
   if (tc) tc_counters(ctx->tc_plan, &zero, &nzero);
   if (ctx->L.fp8) {
-    // narrow E: h (stand-in or the caller's), its e4m3 codes and m_ref, every step
+    // narrow E: h (stand-in or the caller's), its e4m3 codes and m_ref. The
+    // launch stays in every step (and in the captured loop): the merge kernel
+    // prepares them only on its usual path, and the kernel returns at once
+    // when it did (DevState::h_ready).
     DG_CK(launch_prologue_fp8(ctx->stream, ctx->st, at<uint8_t>(ctx, ctx->L.Eq),
                               at<int32_t>(ctx, ctx->L.Ee), ctx->target, ctx->canvas, ctx->sc,
                               ctx->h, hsrc, at<uint8_t>(ctx, ctx->L.hq), at<int32_t>(ctx, ctx->L.he),
@@ -623,8 +632,8 @@ int dg_denoise_block(dg_ctx* ctx, int32_t block, int32_t* out_dev, int32_t* step
   int rc = dg_begin_block(ctx, block);
   if (rc) return rc;
   // The tensor-core loop's first step needs the stand-in h and m_ref; the
-  // merge of each step prepares the next one's (narrow E: the loop runs its
-  // own prologue every step).
+  // merge of each step prepares the next one's (narrow E: the loop keeps a
+  // prologue node in every step, which returns at once when the merge did).
   if (ctx->L.impl == DG_IMPL_TC && !ctx->L.fp8) {
     rc = prologue_if_needed(ctx, true, false);
     if (rc < 0) return rc;

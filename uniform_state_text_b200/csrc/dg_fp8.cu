@@ -20,31 +20,12 @@
 #include <cuda_fp8.h>
 
 #include "dg_common.cuh"
+#include "dg_fp8.cuh"
 #include "dg_kernels.h"
 #include "dg_tc.h"
 
 namespace dg {
 namespace {
-
-__device__ __forceinline__ float e4m3_to_f32(uint8_t c) {
-  __nv_fp8_e4m3 v;
-  v.__x = c;
-  return static_cast<float>(v);
-}
-
-// Two floats to two e4m3 codes (x in the lower byte), nearest even, saturated.
-__device__ __forceinline__ uint16_t f32x2_to_e4m3(float x, float y) {
-  return (uint16_t)__nv_cvt_float2_to_fp8x2(make_float2(x, y), __NV_SATFINITE, __NV_E4M3);
-}
-
-// Smallest e with amax 2^-e <= 448 = 0.875 2^9: amax = m 2^x, m in [0.5, 1),
-// e = x - 9, plus one when m > 0.875 (0 for amax = 0).
-__device__ __forceinline__ int e4m3_row_exponent(float amax) {
-  if (!(amax > 0.f)) return 0;
-  int x;
-  const float m = frexpf(amax, &x);
-  return x - 9 + (m > 0.875f ? 1 : 0);
-}
 
 __device__ __forceinline__ float block_max(float v, float* red) {
   for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -116,6 +97,9 @@ __global__ void __launch_bounds__(256) k_prologue_fp8(
   const int tgt = target[i] & (V - 1), can = canvas[i] & (V - 1);
   const int prev_raw = argmax_prev[i] & (V - 1);
   if (st->done) return;
+  // The tensor-core merge of the previous step already wrote this step's
+  // stand-in h, its codes, m_ref and zeroed counters.
+  if (standin && st->h_ready) return;
   if (zero && blockIdx.x == 0)
     for (int j = threadIdx.x; j < nzero; j += blockDim.x) zero[j] = 0u;
   const int t = st->t;

@@ -72,6 +72,10 @@ struct NextStandin {
   // prologue instead, and the P.E sums carry a factor 2^-u (sc_scale = 2^u).
   int fp8 = 0;
   float sc_scale = 1.f;
+  const uint8_t* Eq = nullptr;            // narrow E: e4m3 codes of E [V][d]
+  const int32_t* Ee = nullptr;            //   and their exponents [V]
+  uint8_t* hq = nullptr;                  //   the next h's codes [C][d]
+  int32_t* he = nullptr;                  //   and its row exponents [C]
   // Pinned host memory mapped into the device ([C]), or null: the merge kernel
   // writes the step's canvas there itself (dg_denoise_step_h's canvas_host),
   // so that no copy sits between this step's kernels and the next step's.

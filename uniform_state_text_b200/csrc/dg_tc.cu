@@ -53,6 +53,7 @@
 
 #include "dg_tc.h"
 #include "dg_tcgen05.cuh"
+#include "dg_fp8.cuh"
 #include "dg_sampler.cuh"
 #include "dg_standin.cuh"
 
@@ -1013,12 +1014,18 @@ __device__ __noinline__ void merge_recompute(int i, int V, int d, const __nv_bfl
 // element over the CTA's rows does sc = (sum of the G2 partials) / Z, keeps the
 // step's h, writes the next step's stand-in h (the prologue's arithmetic, in
 // the same order) and accumulates the two dot products of the next m_ref.
+// With narrow E the stand-in is formed from the dequantised E rows, and a
+// second pass, once the rows' largest magnitudes are known, writes h's e4m3
+// codes and takes m_ref from the dequantised h and E rows (the narrow-E
+// prologue's arithmetic).
 __device__ __forceinline__ void merge_fast_tail(DevState* st, const float* Opart, int nO, int C,
     int V, int d, float* sc, __nv_bfloat16* h, const __nv_bfloat16* E, const float* scale_tab,
     int S, const int32_t* argmax, const int32_t* canvas, float* mref, const float* inv_row,
     const NextStandin& nx, int i0) {
   __shared__ float red[kMergeRows * kMergeThreadsPerRow / 32][2 * kMergeRows];
-  const bool prep = !nx.fp8 && *(volatile int*)&st->done == 0;
+  const bool going = *(volatile int*)&st->done == 0;
+  const bool prep = !nx.fp8 && going;
+  const bool prep8 = nx.fp8 && going;
   const int t1 = *(volatile int*)&st->t;                 // the next step (the sampler advanced it)
   const uint64_t pre = key_prefix(nx.seed, (uint64_t)(uint32_t)*(volatile int*)&st->block,
                                   kTagNoise + (uint64_t)t1);
@@ -1029,6 +1036,12 @@ __device__ __forceinline__ void merge_fast_tail(DevState* st, const float* Opart
   const int can0 = canvas[i0] & (V - 1), can1 = canvas[r1] & (V - 1);
   const int prev0 = argmax[i0] & (V - 1), prev1 = argmax[r1] & (V - 1);   // next step's previous argmax
   float dc0 = 0.f, dp0 = 0.f, dc1 = 0.f, dp1 = 0.f;
+  float am0 = 0.f, am1 = 0.f;                            // narrow E: the rows' largest |h|
+  float st0 = 1.f, st1 = 1.f, sc0 = 1.f, sc1 = 1.f;      //   and the E rows' scales
+  if (prep8) {
+    st0 = pow2f(nx.Ee[tgt0]); st1 = pow2f(nx.Ee[tgt1]);
+    sc0 = pow2f(nx.Ee[can0]); sc1 = pow2f(nx.Ee[can1]);
+  }
   const size_t pstride = (size_t)C * d;
   const int d4 = d / 4;
   __nv_bfloat16* hl = static_cast<__nv_bfloat16*>(nx.h_last);
@@ -1046,6 +1059,28 @@ __device__ __forceinline__ void merge_fast_tail(DevState* st, const float* Opart
     *reinterpret_cast<float4*>(sc + off) = make_float4(s4[0], s4[1], s4[2], s4[3]);
     const uint2 hold = *reinterpret_cast<const uint2*>(h + off);
     *reinterpret_cast<uint2*>(hl + off) = hold;
+    if (prep8) {
+      const uint32_t qt4 = *reinterpret_cast<const uint32_t*>(nx.Eq + (size_t)(q ? tgt1 : tgt0) * d + k);
+      const uint32_t qc4 = *reinterpret_cast<const uint32_t*>(nx.Eq + (size_t)(q ? can1 : can0) * d + k);
+      const float st_ = q ? st1 : st0, sc_ = q ? sc1 : sc0;
+      float hv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint64_t idx = (uint64_t)(i0 + q) * (uint64_t)d + (uint64_t)(k + e);
+        float v = nx.A * (e4m3_to_f32((uint8_t)(qt4 >> (8 * e))) * st_) +
+                  nx.B * (e4m3_to_f32((uint8_t)(qc4 >> (8 * e))) * sc_);
+        v = v + s4[e];
+        v = v + nx.sigma * gauss_from_key(sm64(pre ^ idx));
+        hv[e] = __bfloat162float(__float2bfloat16_rn(v));
+      }
+      const float am = fmaxf(fmaxf(fabsf(hv[0]), fabsf(hv[1])), fmaxf(fabsf(hv[2]), fabsf(hv[3])));
+      if (q) am1 = fmaxf(am1, am); else am0 = fmaxf(am0, am);
+      const __nv_bfloat162 b01 = __floats2bfloat162_rn(hv[0], hv[1]);
+      const __nv_bfloat162 b23 = __floats2bfloat162_rn(hv[2], hv[3]);
+      *reinterpret_cast<uint2*>(h + off) = make_uint2(*reinterpret_cast<const uint32_t*>(&b01),
+                                                      *reinterpret_cast<const uint32_t*>(&b23));
+      continue;
+    }
     if (!prep) continue;
     const uint2 ut = *reinterpret_cast<const uint2*>(E + (size_t)(q ? tgt1 : tgt0) * d + k);
     const uint2 uc = *reinterpret_cast<const uint2*>(E + (size_t)(q ? can1 : can0) * d + k);
@@ -1081,6 +1116,51 @@ __device__ __forceinline__ void merge_fast_tail(DevState* st, const float* Opart
     if (q) { dc1 += pc; dp1 += pp; } else { dc0 += pc; dp0 += pp; }
   }
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (prep8) {
+    // the rows' exponents from their largest magnitudes, then h's codes and
+    // the dot products of the dequantised rows (each thread re-reads the h
+    // elements it wrote above)
+    __shared__ int sh_e[kMergeRows];
+    for (int o = 16; o; o >>= 1) {
+      am0 = fmaxf(am0, __shfl_xor_sync(0xffffffffu, am0, o));
+      am1 = fmaxf(am1, __shfl_xor_sync(0xffffffffu, am1, o));
+    }
+    if (l == 0) { red[w][0] = am0; red[w][1] = am1; }
+    __syncthreads();
+    if (threadIdx.x < nrows) {
+      float a = 0.f;
+      for (int j = 0; j < (int)(blockDim.x >> 5); ++j) a = fmaxf(a, red[j][threadIdx.x]);
+      sh_e[threadIdx.x] = e4m3_row_exponent(a);
+      nx.he[i0 + threadIdx.x] = sh_e[threadIdx.x];
+    }
+    __syncthreads();
+    const float sp0 = pow2f(nx.Ee[prev0]), sp1 = pow2f(nx.Ee[prev1]);
+    for (int x = threadIdx.x; x < nrows * d4; x += blockDim.x) {
+      const int q = x / d4, k = (x % d4) * 4;
+      const size_t off = (size_t)(i0 + q) * d + k;
+      const int e = sh_e[q];
+      const float he_ = pow2f(e), rinv = pow2f(-e);
+      const uint2 hb = *reinterpret_cast<const uint2*>(h + off);
+      const float hv[4] = {__uint_as_float(hb.x << 16), __uint_as_float(hb.x & 0xFFFF0000u),
+                           __uint_as_float(hb.y << 16), __uint_as_float(hb.y & 0xFFFF0000u)};
+      const uint32_t c01 = f32x2_to_e4m3(hv[0] * rinv, hv[1] * rinv);
+      const uint32_t c23 = f32x2_to_e4m3(hv[2] * rinv, hv[3] * rinv);
+      const uint32_t codes = c01 | (c23 << 16);
+      *reinterpret_cast<uint32_t*>(nx.hq + off) = codes;
+      const uint32_t qc4 = *reinterpret_cast<const uint32_t*>(nx.Eq + (size_t)(q ? can1 : can0) * d + k);
+      const uint32_t qp4 = *reinterpret_cast<const uint32_t*>(nx.Eq + (size_t)(q ? prev1 : prev0) * d + k);
+      const float sc_ = q ? sc1 : sc0, sp_ = q ? sp1 : sp0;
+      float pc = 0.f, pp = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float hd = e4m3_to_f32((uint8_t)(codes >> (8 * j))) * he_;
+        pc = fmaf(hd, e4m3_to_f32((uint8_t)(qc4 >> (8 * j))) * sc_, pc);
+        pp = fmaf(hd, e4m3_to_f32((uint8_t)(qp4 >> (8 * j))) * sp_, pp);
+      }
+      if (q) { dc1 += pc; dp1 += pp; } else { dc0 += pc; dp0 += pp; }
+    }
+    __syncthreads();                       // red is reused below
+  }
   for (int o = 16; o; o >>= 1) {
     dc0 += __shfl_xor_sync(0xffffffffu, dc0, o);
     dp0 += __shfl_xor_sync(0xffffffffu, dp0, o);
@@ -1092,9 +1172,9 @@ __device__ __forceinline__ void merge_fast_tail(DevState* st, const float* Opart
   if (blockIdx.x == 0) {
     // the attention kernel has completed: its counters start the next step at zero
     for (int j = threadIdx.x; j < nx.nzero; j += blockDim.x) nx.zero[j] = 0u;
-    if (threadIdx.x == 0) st->h_ready = prep ? 1 : 0;
+    if (threadIdx.x == 0) st->h_ready = (prep || prep8) ? 1 : 0;
   }
-  if (threadIdx.x < nrows && prep) {
+  if (threadIdx.x < nrows && (prep || prep8)) {
     const int q = threadIdx.x;
     float a = 0.f, b = 0.f;
     for (int j = 0; j < (int)(blockDim.x >> 5); ++j) { a += red[j][2 * q]; b += red[j][2 * q + 1]; }
