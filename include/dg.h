@@ -235,7 +235,9 @@ int dg_denoise_step_h(dg_ctx* ctx, const void* h_src, int32_t h_on_host,
  * [VG] 5.1/5.3 by vocabulary rows). Every rank holds the whole E and the same
  * canvas state, so the stand-in h and the logit reference m_ref are computed
  * identically everywhere; each rank's context (cfg.shard_v0, shard_nv) covers
- * its share of the vocabulary. Tensor-core path only (DG_EUNSUPPORTED else).
+ * its share of the vocabulary. Tensor-core path with E as given only
+ * (DG_E_NATIVE; a shard with DG_E_FP8 has no workspace size and dg_init
+ * returns DG_EUNSUPPORTED).
  *   dg_partials_bytes  bytes of one partials buffer (device, caller-owned,
  *                      16-byte aligned); 0 if the configuration has no
  *                      vocabulary-parallel step.

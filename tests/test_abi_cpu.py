@@ -104,6 +104,14 @@ def test_vocabulary_shard_needs_tensor_cores(lib):
     assert dg.dg_partials_bytes(dg.make_config(w, dg.DG_IMPL_SIMT)) == 0
 
 
+def test_vocabulary_shard_takes_e_as_given(lib):
+    w = synthetic.SMALL.replace(C=128, V=4096, d=256)
+    assert dg.dg_workspace_bytes(dg.make_config(w, dg.DG_IMPL_TC, shard=(0, 1024))) > 0
+    w8 = w.replace(e_format=dg.DG_E_FP8)
+    assert dg.dg_workspace_bytes(dg.make_config(w8, dg.DG_IMPL_TC)) > 0
+    assert dg.dg_workspace_bytes(dg.make_config(w8, dg.DG_IMPL_TC, shard=(0, 1024))) == 0
+
+
 def test_tensor_core_request_on_unsupported_shape(lib):
     cfg = dg.make_config(synthetic.TINY, dg.DG_IMPL_TC)     # fp32, C=16: not covered
     assert dg.dg_workspace_bytes(cfg) == 0

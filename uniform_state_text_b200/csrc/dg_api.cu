@@ -105,6 +105,12 @@ int resolve_impl(const dg_config* c, char* why, size_t n) {
                "d %% 256 == 0)");
       return -1;
     }
+    // The shard path's exact recomputation of a row (after the exchange) reads
+    // E as given, not the narrow codes, so the two are not combined.
+    if (c->e_format == DG_E_FP8) {
+      snprintf(why, n, "a vocabulary shard takes E as given (DG_E_NATIVE)");
+      return -1;
+    }
     return DG_IMPL_TC;
   }
   if (c->e_format == DG_E_FP8) {
