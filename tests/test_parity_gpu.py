@@ -655,6 +655,31 @@ def test_fp8_embedding_teacher_forced(name, steps, token_rule):
     den.close()
 
 
+def test_fp8_external_hidden_state_from_host():
+    """Narrow E with a caller's hidden state from pinned host memory, two
+    steps: the narrow-E prologue quantises the caller's h, rows whose largest
+    logit overshoots the reference (the redo gap is 4 nats here) take the redo
+    pass, and the step equals the oracle's narrow-E step; the canvas reaches
+    the caller's pinned buffer."""
+    w = synthetic.SMALL.replace(e_format=dg.DG_E_FP8, fixed_steps=1)
+    den, _ = make(w, dg.DG_IMPL_TC)
+    Eg, _ = embedding(w)
+    nE = narrow_embedding(w)
+    tally = Tally()
+    canvas_host = torch.empty(w.C, dtype=torch.int32).pin_memory()
+    for step in range(2):
+        canvas = _np(den.read(dg.DG_CANVAS)).astype(np.int64)
+        h = _external_h(w, Eg, canvas, 4321 + step).pin_memory()
+        pre = _np(den.read(dg.DG_ARGMAX)).astype(np.int64) if den.state()["has_prev"] else None
+        do_step = lambda: den.step_h(h, canvas_host=canvas_host)   # noqa: E731
+        assert step_and_compare(den, w, nE.E_deq, tally, pre, do_step=do_step,
+                                h_given=h.float().numpy(), narrow=nE)
+        assert np.array_equal(canvas_host.numpy(), _np(den.read(dg.DG_CANVAS)))
+    assert den.state()["redo"] > 0
+    tally.check_budget()
+    den.close()
+
+
 def test_fp8_embedding_block_through_the_graph_loop():
     """A whole adaptive block with narrow E through the captured loop: the
     emitted tokens and the step count equal the oracle's narrow-E run (its own
